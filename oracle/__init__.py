@@ -1,0 +1,262 @@
+"""CPU oracle for the NVFP4 W4A4 Gated DeltaNet layer forward.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package; the product library
+never does, and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C: exact float32 for the
+quantiser, float64 elsewhere); this module only marshals numpy arrays and
+composes the steps in the order the pages give them:
+
+1. online NVFP4 quantisation of the activations (review page "Why Gated
+   DeltaNet Survives 4-Bit Quantization", background / paper sec.1);
+2. block-scaled FP4 x FP4 GEMM for the fused q|k|v|z|a|b projection with one
+   harmonised weight scale (review page, paper sec.6; abstract page);
+3. gates, Eq.(1) (review page, paper sec.2) and q/k L2 normalisation;
+4. the delta-rule recurrence, Eq.(2) (review page, paper sec.1), then the
+   NVFP4 out_proj.
+
+Every function states the reading it follows where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+FORM_PAGES = 0
+FORM_STANDARD = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c with gcc (no fast-math, no FMA contraction)."""
+    src = os.path.join(_HERE, "oracle.c")
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(src):
+        subprocess.check_call([
+            "gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
+            "-shared", "-fPIC", src, "-o", _LIB_PATH, "-lm"])
+    return _LIB_PATH
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        i64, i32, f32, f64, u8 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_double, ctypes.c_uint8
+        lib.orc_e2m1_decode.argtypes = [u8]; lib.orc_e2m1_decode.restype = f64
+        lib.orc_e2m1_encode.argtypes = [f32]; lib.orc_e2m1_encode.restype = u8
+        lib.orc_e4m3_decode.argtypes = [u8]; lib.orc_e4m3_decode.restype = f64
+        lib.orc_e4m3_encode.argtypes = [f32]; lib.orc_e4m3_encode.restype = u8
+        lib.orc_global_scale.argtypes = [P, i64]; lib.orc_global_scale.restype = f32
+        lib.orc_quantize.argtypes = [P, i64, i64, f32, P, P]; lib.orc_quantize.restype = None
+        lib.orc_dequantize.argtypes = [P, P, f32, i64, i64, P]; lib.orc_dequantize.restype = None
+        lib.orc_sf_linear_to_mma.argtypes = [P, i64, i64, P]; lib.orc_sf_linear_to_mma.restype = None
+        lib.orc_gemm_nt.argtypes = [P, P, i64, i64, i64, P]; lib.orc_gemm_nt.restype = None
+        lib.orc_softplus.argtypes = [f64]; lib.orc_softplus.restype = f64
+        lib.orc_gates.argtypes = [P, P, P, P, i64, i32, P, P]; lib.orc_gates.restype = None
+        lib.orc_l2norm.argtypes = [P, i64, i32, f64]; lib.orc_l2norm.restype = None
+        lib.orc_scan.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, f64, i32, P, P, P]
+        lib.orc_scan.restype = None
+        lib.orc_scan_chunked.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, f64, i32, i32,
+                                         P, P, P]
+        lib.orc_scan_chunked.restype = None
+        lib.orc_num_threads.argtypes = []; lib.orc_num_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_threads() -> int:
+    return int(_L().orc_num_threads())
+
+
+# ---------------------------------------------------------------- formats --
+def e2m1_decode(code: int) -> float:
+    return float(_L().orc_e2m1_decode(int(code)))
+
+
+def e2m1_encode(y: float) -> int:
+    return int(_L().orc_e2m1_encode(float(y)))
+
+
+def e4m3_decode(b: int) -> float:
+    return float(_L().orc_e4m3_decode(int(b)))
+
+
+def e4m3_encode(s: float) -> int:
+    return int(_L().orc_e4m3_encode(float(s)))
+
+
+# -------------------------------------------------------------- quantiser --
+def global_scale(x: np.ndarray) -> np.float32:
+    """S = fl32(amax/2688), or 1 when amax < 2^-100 (reading Q1)."""
+    x = _c(x, np.float32)
+    return np.float32(_L().orc_global_scale(_p(x), x.size))
+
+
+def quantize(x: np.ndarray, S: float | None = None):
+    """NVFP4-quantise a float32 matrix [rows x cols] (cols % 16 == 0).
+
+    Returns (codes uint8 [rows, cols/2], sf uint8 [rows, cols/16] linear, S).
+    ``S`` given = use that global scale (harmonised weights); else computed
+    from the tensor's amax.
+    """
+    x = _c(x, np.float32)
+    rows, cols = x.shape
+    assert cols % 16 == 0
+    if S is None:
+        S = global_scale(x)
+    S = np.float32(S)
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    sf = np.zeros((rows, cols // 16), np.uint8)
+    _L().orc_quantize(_p(x), rows, cols, float(S), _p(codes), _p(sf))
+    return codes, sf, S
+
+
+def dequantize(codes: np.ndarray, sf: np.ndarray, S: float) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    sf = _c(sf, np.uint8)
+    rows = codes.shape[0]
+    cols = codes.shape[1] * 2
+    out = np.empty((rows, cols), np.float64)
+    _L().orc_dequantize(_p(codes), _p(sf), float(np.float32(S)), rows, cols, _p(out))
+    return out
+
+
+def sf_linear_to_mma(sf: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Permute linear block scales into the tensor-core atom layout (rows
+    padded to a multiple of 128 with zero bytes).  Returns a flat uint8 array."""
+    sf = _c(sf, np.uint8)
+    prow = (rows + 127) // 128 * 128
+    out = np.empty(prow * (cols // 16), np.uint8)
+    _L().orc_sf_linear_to_mma(_p(sf), rows, cols, _p(out))
+    return out
+
+
+# -------------------------------------------------------------------- GEMM --
+def gemm_nt(A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """C = A @ B^T in float64 (triple loop in C)."""
+    A = _c(A, np.float64)
+    B = _c(B, np.float64)
+    M, K = A.shape
+    N = B.shape[0]
+    C = np.empty((M, N), np.float64)
+    _L().orc_gemm_nt(_p(A), _p(B), M, N, K, _p(C))
+    return C
+
+
+def w4a4_gemm(Aq, Bq) -> np.ndarray:
+    """Block-scaled FP4 GEMM reference: dequantise both operands exactly, then
+    float64 C = A_hat @ B_hat^T (the product of S_A S_B and the block-scaled
+    sums)."""
+    A = dequantize(*Aq)
+    B = dequantize(*Bq)
+    return gemm_nt(A, B)
+
+
+# -------------------------------------------------------------------- gates --
+def softplus(u: float) -> float:
+    return float(_L().orc_softplus(float(u)))
+
+
+def gates(a: np.ndarray, b: np.ndarray, A_log: np.ndarray, dt_bias: np.ndarray):
+    """Eq.(1): g = -exp(A_log) softplus(a + dt_bias), alpha = e^g, beta = sigmoid(b).
+    a, b: [n, Hv].  Returns (g, beta) float64."""
+    a = _c(a, np.float64)
+    b = _c(b, np.float64)
+    n, Hv = a.shape
+    g = np.empty_like(a)
+    beta = np.empty_like(a)
+    _L().orc_gates(_p(a), _p(b), _p(_c(A_log, np.float64)), _p(_c(dt_bias, np.float64)), n, Hv,
+                   _p(g), _p(beta))
+    return g, beta
+
+
+def l2norm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """x / sqrt(sum x^2 + eps) along the last axis (reading G2)."""
+    y = np.array(x, dtype=np.float64, order="C", copy=True)
+    D = y.shape[-1]
+    _L().orc_l2norm(_p(y), y.size // D, D, eps)
+    return y
+
+
+# --------------------------------------------------------------------- scan --
+def scan(q, k, v, g, beta, scale=None, form=FORM_PAGES, S0=None):
+    """Eq.(2) token by token.  q, k: [B,T,Hk,K]; v: [B,T,Hv,V]; g, beta: [B,T,Hv];
+    S0: [B,Hv,K,V] or None.  Returns (o [B,T,Hv,V], S [B,Hv,K,V])."""
+    q, k, v = _c(q, np.float64), _c(k, np.float64), _c(v, np.float64)
+    g, beta = _c(g, np.float64), _c(beta, np.float64)
+    B, T, Hk, K = q.shape
+    Hv, V = v.shape[2], v.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(K)
+    S = np.empty((B, Hv, K, V), np.float64)
+    o = np.empty((B, T, Hv, V), np.float64)
+    s0 = None if S0 is None else _c(S0, np.float64)
+    _L().orc_scan(_p(q), _p(k), _p(v), _p(g), _p(beta), B, T, Hk, Hv, K, V, float(scale), int(form),
+                  None if s0 is None else _p(s0), _p(S), _p(o))
+    return o, S
+
+
+def scan_chunked(q, k, v, g, beta, chunk=64, scale=None, form=FORM_PAGES, S0=None):
+    """Chunked restatement of Eq.(2) (pins the GPU kernel's derivation)."""
+    q, k, v = _c(q, np.float64), _c(k, np.float64), _c(v, np.float64)
+    g, beta = _c(g, np.float64), _c(beta, np.float64)
+    B, T, Hk, K = q.shape
+    Hv, V = v.shape[2], v.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(K)
+    S = np.empty((B, Hv, K, V), np.float64)
+    o = np.empty((B, T, Hv, V), np.float64)
+    s0 = None if S0 is None else _c(S0, np.float64)
+    _L().orc_scan_chunked(_p(q), _p(k), _p(v), _p(g), _p(beta), B, T, Hk, Hv, K, V, float(scale),
+                          int(form), int(chunk), None if s0 is None else _p(s0), _p(S), _p(o))
+    return o, S
+
+
+# -------------------------------------------------------------------- layer --
+def split_projection(P: np.ndarray, Hk: int, Hv: int, K: int, V: int):
+    """Column slices of the fused projection, in the order q | k | v | z | a | b."""
+    widths = [Hk * K, Hk * K, Hv * V, Hv * V, Hv, Hv]
+    out, c = [], 0
+    for w in widths:
+        out.append(P[..., c:c + w])
+        c += w
+    return out
+
+
+def layer_forward(x: np.ndarray, W_in_q, W_out_q, A_log, dt_bias, B: int, T: int, Hk: int, Hv: int,
+                  K: int, V: int, form=FORM_PAGES, S0=None, stages: bool = False):
+    """The four steps composed.  x: float32 [B*T, H] (bf16 values);
+    W_in_q, W_out_q: (codes, sf_linear, S) of the fused in_proj [N_in, H] and
+    out_proj [H, Hv*V].  Returns y [B*T, H] float64 and the final state (and
+    every intermediate when ``stages``)."""
+    xq = quantize(x)                                            # step 1
+    P = w4a4_gemm(xq, W_in_q)                                   # step 2
+    q, k, v, _z, a, b = split_projection(P, Hk, Hv, K, V)
+    g, beta = gates(a, b, A_log, dt_bias)                       # step 3
+    qh = l2norm(q.reshape(B, T, Hk, K))
+    kh = l2norm(k.reshape(B, T, Hk, K))
+    o, S = scan(qh, kh, v.reshape(B, T, Hv, V), g.reshape(B, T, Hv), beta.reshape(B, T, Hv),
+                form=form, S0=S0)                               # step 4
+    o2 = o.reshape(B * T, Hv * V).astype(np.float32)            # the out_proj reads fp32 o
+    oq = quantize(o2)
+    y = w4a4_gemm(oq, W_out_q)
+    if stages:
+        return dict(xq=xq, P=P, g=g, beta=beta, q_hat=qh, k_hat=kh, o=o, S=S, oq=oq, y=y)
+    return y, S

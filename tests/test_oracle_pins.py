@@ -1,0 +1,416 @@
+"""Pins of the CPU oracle against facts fixed outside it: the pages' printed
+format facts and bounds, closed forms, library routines (torch float8,
+numpy) and brute force on tiny inputs.  CPU only."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gdn_synth
+from conftest import read_golden
+
+E2M1_MAGS = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+# ----------------------------------------------------------------- formats --
+def test_e2m1_grid_matches_golden():
+    for code_s, val_s in read_golden("e2m1_grid.txt"):
+        code, val = int(code_s, 16), float(val_s)
+        got = oracle.e2m1_decode(code)
+        assert got == val and math.copysign(1, got) == math.copysign(1, val), (code, got, val)
+        assert oracle.e2m1_encode(val) == code
+
+
+def _e2m1_bruteforce(y):
+    """Nearest grid magnitude; on a tie the one with an even mantissa bit
+    (code index even); above 6 saturate."""
+    a = abs(y)
+    dists = [abs(a - m) for m in E2M1_MAGS]
+    best = min(dists)
+    cands = [i for i, d in enumerate(dists) if d == best]
+    if len(cands) > 1:
+        cands = [i for i in cands if i % 2 == 0]
+    idx = cands[0]
+    if a >= 6.0:
+        idx = 7
+    return (8 if math.copysign(1, y) < 0 else 0) | idx
+
+
+def test_e2m1_rounding_bruteforce():
+    ys = list(np.linspace(-8, 8, 4001, dtype=np.float32))
+    ties = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0]
+    for t in ties:
+        for s in (1, -1):
+            ys += [np.float32(s * t), np.nextafter(np.float32(s * t), np.float32(0)),
+                   np.nextafter(np.float32(s * t), np.float32(s * 100))]
+    ys += [np.float32(-0.0), np.float32(1e-30), np.float32(-1e-30), np.float32(1e30), np.float32(-1e30)]
+    for y in ys:
+        assert oracle.e2m1_encode(float(y)) == _e2m1_bruteforce(float(y)), y
+
+
+def test_e2m1_ties_spot_values():
+    # ties to the even mantissa: 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4
+    want = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0, 6.5: 6.0, 100.0: 6.0}
+    for y, v in want.items():
+        assert oracle.e2m1_decode(oracle.e2m1_encode(y)) == v
+
+
+def test_e4m3_decode_matches_torch_float8():
+    bits = torch.arange(256, dtype=torch.uint8)
+    ref = bits.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for b in range(256):
+        got = oracle.e4m3_decode(b)
+        if np.isnan(ref[b]):
+            assert np.isnan(got)
+        else:
+            assert got == ref[b], (b, got, ref[b])
+
+
+def test_e4m3_encode_matches_torch_float8():
+    g = gdn_synth.rng(123)
+    vals = np.exp(g.uniform(np.log(2.0 ** -12), np.log(447.0), 20000)).astype(np.float32)
+    # exact ties between neighbouring E4M3 values and the subnormal range
+    reps = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mids = ((reps[1:] + reps[:-1]) / 2).astype(np.float32)
+    vals = np.concatenate([vals, mids, reps.astype(np.float32), np.float32([2.0 ** -10, 2.0 ** -11, 3e-3])])
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for v, r in zip(vals, ref):
+        assert oracle.e4m3_encode(float(v)) == int(r), (v, oracle.e4m3_encode(float(v)), r)
+
+
+def test_e4m3_encode_saturates():
+    for v in (448.0, 449.0, 464.0, 500.0, 1e6, 3e38):
+        assert oracle.e4m3_encode(v) == 0x7E
+    assert oracle.e4m3_encode(0.0) == 0
+
+
+# --------------------------------------------------------------- quantiser --
+def test_roundtrip_exact_on_scaled_grid():
+    """Values already of the form code * E4M3 * S with S a power of two, every
+    block containing a +-6 and one block at scale 448, come back bit-exactly."""
+    g = gdn_synth.rng(7)
+    rows, cols = 8, 64
+    S = np.float32(2.0 ** -3)
+    nb = cols // 16
+    sbs = g.integers(0x08, 0x7F, size=(rows, nb)).astype(np.uint8)   # normal E4M3 scales, no NaN
+    sbs[3, 2] = 0x7E                                                  # 448
+    codes_lin = g.integers(0, 16, size=(rows, cols)).astype(np.uint8)
+    codes_lin[:, ::16] = 0x7                                          # a +6 in every block
+    codes_lin[:, 5::16] = 0xF                                         # and a -6
+    vals = np.array([[float(v) for v in row] for row in np.vectorize(oracle.e2m1_decode)(codes_lin)])
+    scl = np.vectorize(oracle.e4m3_decode)(sbs)
+    x = (vals * np.repeat(scl, 16, axis=1) * float(S)).astype(np.float32)
+    assert np.all(x.astype(np.float64) == vals * np.repeat(scl, 16, axis=1) * float(S))
+    codes, sf, S2 = oracle.quantize(x)
+    assert S2 == S
+    assert np.array_equal(sf, sbs)
+    packed = (codes_lin[:, 0::2] | (codes_lin[:, 1::2] << 4)).astype(np.uint8)
+    # -0 codes cannot arise here except for code 8 itself, which decodes to -0 and re-encodes as 8
+    assert np.array_equal(codes, packed)
+
+
+def test_block_bound_max_over_rms():
+    rows = {r[0]: float(r[1]) for r in read_golden("block_bound.txt")}
+    bs, bound = int(rows["block_size"]), rows["max_over_rms_bound"]
+    assert bound == math.sqrt(bs)
+    _, x = gdn_synth.activations(11, 64, 512, hot="percent")
+    codes, sf, S = oracle.quantize(x)
+    xd = oracle.dequantize(codes, sf, S)
+    for arr in (x.astype(np.float64), xd):
+        blk = arr.reshape(-1, bs)
+        nz = np.any(blk != 0, axis=1)
+        ratio = np.abs(blk[nz]).max(1) / np.sqrt((blk[nz] ** 2).mean(1))
+        assert np.all(ratio <= bound * (1 + 1e-12))
+    # one-hot blocks reach the bound exactly, before and after quantisation
+    oh = np.zeros((4, 64), np.float32)
+    oh[np.arange(4), [0, 17, 34, 63]] = [1.0, -2.5, 3.0, 0.75]
+    c, s, S = oracle.quantize(oh)
+    d = oracle.dequantize(c, s, S).reshape(-1, bs)
+    nz = np.any(d != 0, axis=1)
+    ratio = np.abs(d[nz]).max(1) / np.sqrt((d[nz] ** 2).mean(1))
+    assert np.allclose(ratio, bound, rtol=0, atol=1e-12)
+
+
+def test_outlier_localised_to_its_block():
+    rows = {r[0]: float(r[1]) for r in read_golden("block_bound.txt")}
+    nnb = int(rows["neighbours_degraded"])
+    _, x = gdn_synth.activations(12, 16, 256, hot="none")
+    c0, s0, S0 = oracle.quantize(x)
+    # (i) an outlier that does not raise the tensor amax changes only its own block
+    x1 = x.copy()
+    amax = np.abs(x).max()
+    r, col = 5, 37
+    x1[r, col] = np.float32(amax * 0.99)
+    c1, s1, S1 = oracle.quantize(x1)
+    assert S1 == S0
+    blk = col // 16
+    diff_sf = np.argwhere(s1 != s0)
+    assert all(tuple(d) == (r, blk) for d in diff_sf)
+    diff_c = np.argwhere(c1 != c0)
+    assert all(d[0] == r and d[1] // 8 == blk for d in diff_c)
+    # (ii) an outlier 100x the amax: its block's other 15 values collapse, the rest keep
+    # their usual error level
+    x2 = x.copy()
+    x2[r, col] = np.float32(amax * 100)
+    c2, s2, S2 = oracle.quantize(x2)
+    d2 = oracle.dequantize(c2, s2, S2)
+    err = np.abs(d2 - x2)
+    hot = np.zeros_like(x2, bool)
+    hot[r, blk * 16:(blk + 1) * 16] = True
+    hot[r, col] = False
+    assert hot.sum() == nnb
+    rel_hot = np.linalg.norm(err[hot]) / np.linalg.norm(x2[hot])
+    rel_rest = np.linalg.norm(err[~hot & (np.arange(256)[None] != col)]) / np.linalg.norm(x2[~hot & (np.arange(256)[None] != col)])
+    assert rel_hot > 0.5
+    assert rel_rest < 0.2
+
+
+def test_zero_and_tiny_tensors():
+    x = np.zeros((4, 32), np.float32)
+    c, s, S = oracle.quantize(x)
+    assert S == 1.0 and not c.any() and not s.any()
+    x[1, 3] = 1e-35
+    c, s, S = oracle.quantize(x)
+    assert S == 1.0 and not c.any() and not s.any()
+    x = np.full((2, 16), -1e-3, np.float32)
+    x[0, 0] = 1.0
+    c, s, S = oracle.quantize(x)
+    # row 1 is 1e-3 of the amax: scale 1e-3*448 ~ 0.45 -> representable, codes = -6 -> 0xF
+    assert s[1, 0] != 0 and np.all(c[1] == 0xFF)
+
+
+def test_sf_layout_is_the_atom_permutation():
+    rows, cols = 300, 512
+    g = gdn_synth.rng(5)
+    sf = g.integers(0, 256, size=(rows, cols // 16)).astype(np.uint8)
+    out = oracle.sf_linear_to_mma(sf, rows, cols)
+    # independent construction: pad, then reshape [rb, 4 (row/32), 32 (row%32), kb, 4] and
+    # reorder to [rb, kb, 32, 4, 4]
+    prow = (rows + 127) // 128 * 128
+    pad = np.zeros((prow, cols // 16), np.uint8)
+    pad[:rows] = sf
+    t = pad.reshape(prow // 128, 4, 32, cols // 64, 4).transpose(0, 3, 2, 1, 4)
+    assert np.array_equal(out, t.reshape(-1))
+
+
+# -------------------------------------------------------------------- GEMM --
+def test_dequantize_is_code_times_scale_times_S():
+    _, x = gdn_synth.activations(13, 8, 64, hot="fixed")
+    c, s, S = oracle.quantize(x)
+    d = oracle.dequantize(c, s, S)
+    grid = {int(a, 16): float(b) for a, b in read_golden("e2m1_grid.txt")}
+    sfv = torch.from_numpy(s.copy()).view(torch.float8_e4m3fn).double().numpy()
+    for r in range(8):
+        for col in range(64):
+            byte = c[r, col // 2]
+            code = (byte >> 4) if col % 2 else (byte & 15)
+            assert d[r, col] == grid[int(code)] * sfv[r, col // 16] * float(S)
+
+
+def test_gemm_matches_numpy_and_bruteforce():
+    g = gdn_synth.rng(9)
+    A = g.standard_normal((7, 48))
+    B = g.standard_normal((5, 48))
+    C = oracle.gemm_nt(A, B)
+    assert np.allclose(C, A @ B.T, rtol=1e-13, atol=1e-13)
+    for i in range(7):
+        for j in range(5):
+            assert abs(C[i, j] - sum(A[i, k] * B[j, k] for k in range(48))) < 1e-12
+
+
+def test_harmonised_fused_gemm_equals_per_slice():
+    """One weight scale for the fused tensor: the fused GEMM equals the
+    concatenation of per-slice GEMMs run under that shared scale; with
+    per-module scales applied through one fused scale, slice m is off by
+    S_0 / S_m (the mismatch the pages repair; review page sec.6, abstract)."""
+    sl, gain = (32, 32, 64), (1.0, 4.0, 2.0)
+    W = gdn_synth.weights(21, sum(sl), 128, slice_rows=sl, slice_gain=gain)
+    _, x = gdn_synth.activations(22, 16, 128, hot="fixed")
+    xq = oracle.quantize(x)
+    Wq = oracle.quantize(W)                       # harmonised: one amax over the fused tensor
+    fused = oracle.w4a4_gemm(xq, Wq)
+    r0, parts, own = 0, [], []
+    for n in sl:
+        part = oracle.quantize(W[r0:r0 + n], S=Wq[2])
+        assert np.array_equal(part[0], Wq[0][r0:r0 + n]) and np.array_equal(part[1], Wq[1][r0:r0 + n])
+        parts.append(oracle.w4a4_gemm(xq, part))
+        own.append(oracle.quantize(W[r0:r0 + n]))
+        r0 += n
+    assert np.array_equal(fused, np.concatenate(parts, axis=1))
+    # negative control: per-module codes/scales served with module 0's global scale
+    S0 = own[0][2]
+    bad = np.concatenate([oracle.w4a4_gemm(xq, (c, s, S0)) for c, s, _ in own], axis=1)
+    good = np.concatenate([oracle.w4a4_gemm(xq, o) for o in own], axis=1)
+    r0 = 0
+    for (c, s, Sm), n in zip(own, sl):
+        ratio = float(S0) / float(Sm)
+        assert np.allclose(bad[:, r0:r0 + n], good[:, r0:r0 + n] * ratio, rtol=1e-12, atol=0)
+        r0 += n
+    rel = np.linalg.norm(bad[:, 32:64] - good[:, 32:64]) / np.linalg.norm(good[:, 32:64])
+    assert rel > 0.5
+
+
+# ------------------------------------------------------------------- gates --
+def test_softplus_closed_forms():
+    assert abs(oracle.softplus(0.0) - math.log(2.0)) < 1e-15
+    for u in (-30.0, -3.0, -0.5, 0.7, 5.0, 40.0):
+        assert abs(oracle.softplus(u) - float(np.logaddexp(0.0, u))) <= 1e-15 * max(1, abs(u))
+    assert oracle.softplus(800.0) == 800.0
+
+
+def test_gates_ranges_and_library_forms():
+    g = gdn_synth.rng(31)
+    a = g.standard_normal((50, 4)) * 5
+    b = g.standard_normal((50, 4)) * 5
+    A_log, dt_bias = gdn_synth.gate_params(32, 4)
+    gg, beta = oracle.gates(a, b, A_log, dt_bias)
+    alpha = np.exp(gg)
+    assert np.all((alpha > 0) & (alpha < 1)) and np.all((beta > 0) & (beta < 1))
+    ref_g = -np.exp(A_log.astype(np.float64)) * np.logaddexp(0.0, a + dt_bias.astype(np.float64))
+    assert np.allclose(gg, ref_g, rtol=1e-13, atol=0)
+    from scipy.special import expit
+    assert np.allclose(beta, expit(b), rtol=1e-14, atol=0)
+
+
+def test_l2norm_unit_rows():
+    x = gdn_synth.gaussian(33, (10, 3, 64))
+    y = oracle.l2norm(x)
+    n = np.linalg.norm(x.astype(np.float64), axis=-1, keepdims=True)
+    assert np.allclose(y, x / np.sqrt(n ** 2 + 1e-6), rtol=1e-14)
+    assert np.allclose(np.linalg.norm(y, axis=-1), 1.0, atol=1e-6)
+
+
+# -------------------------------------------------------------------- scan --
+def _orthonormal(seed, n, K):
+    g = gdn_synth.rng(seed)
+    Q, _ = np.linalg.qr(g.standard_normal((K, K)))
+    return Q[:, :n].T.copy()
+
+
+@pytest.mark.parametrize("form", [oracle.FORM_PAGES, oracle.FORM_STANDARD])
+def test_delta_rule_overwrite_retrieves_values(form):
+    """alpha = beta = 1 with orthonormal keys: each write overwrites the state
+    along its key, so S_n^T k_i = v_i and querying with k_i returns
+    v_i / sqrt(K) (review page, mechanism step 3, paper sec.5.3)."""
+    K = V = 16
+    n = 10
+    keys = _orthonormal(40, n, K)
+    g = gdn_synth.rng(41)
+    v = g.standard_normal((1, n, 1, V))
+    k = keys.reshape(1, n, 1, K)
+    q = keys[::-1].reshape(1, n, 1, K).copy()
+    S0 = g.standard_normal((1, 1, K, V))
+    zeros = np.zeros((1, n, 1))
+    o, S = oracle.scan(q, k, v, zeros, np.ones((1, n, 1)), form=form, S0=S0)
+    for i in range(n):
+        assert np.allclose(S[0, 0].T @ keys[i], v[0, i, 0], atol=1e-12)
+    # the last query is k_0, read after all writes
+    assert np.allclose(o[0, n - 1, 0], v[0, 0, 0] / np.sqrt(K), atol=1e-12)
+
+
+def test_beta_zero_is_pure_decay():
+    B, T, Hk, Hv, K, V = 1, 9, 1, 2, 8, 8
+    q, k, v, g, beta = gdn_synth.scan_inputs(50, B, T, Hk, Hv, K, V)
+    S0 = gdn_synth.gaussian(51, (B, Hv, K, V))
+    o, S = oracle.scan(q, k, v, g, np.zeros_like(beta), S0=S0)
+    G = np.cumsum(g.astype(np.float64), axis=1)
+    for h in range(Hv):
+        assert np.allclose(S[0, h], np.exp(G[0, -1, h]) * S0[0, h], rtol=1e-13)
+        for t in range(T):
+            want = np.exp(G[0, t, h]) * S0[0, h].T @ q[0, t, 0] / np.sqrt(K)
+            assert np.allclose(o[0, t, h], want, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("form", [oracle.FORM_PAGES, oracle.FORM_STANDARD])
+def test_scan_matches_matrix_product_form(form):
+    """PAGES: S_t = (alpha I - beta k k^T) S + beta k v^T; STANDARD (the usual
+    Gated DeltaNet form): S_t = alpha (I - beta k k^T) S + beta k v^T; built
+    here with numpy matrix products.  GQA: value head h reads key head h*Hk//Hv."""
+    B, T, Hk, Hv, K, V = 2, 7, 2, 4, 6, 5
+    q, k, v, g, beta = gdn_synth.scan_inputs(60, B, T, Hk, Hv, K, V, alpha_lo=0.5)
+    S0 = gdn_synth.gaussian(61, (B, Hv, K, V))
+    o, S = oracle.scan(q, k, v, g, beta, form=form, S0=S0, scale=0.37)
+    for bb in range(B):
+        for h in range(Hv):
+            hk = h * Hk // Hv
+            St = S0[bb, h].astype(np.float64)
+            for t in range(T):
+                kt = k[bb, t, hk].astype(np.float64)
+                a, bt = math.exp(g[bb, t, h]), float(beta[bb, t, h])
+                if form == oracle.FORM_PAGES:
+                    St = (a * np.eye(K) - bt * np.outer(kt, kt)) @ St + bt * np.outer(kt, v[bb, t, h])
+                else:
+                    St = a * (np.eye(K) - bt * np.outer(kt, kt)) @ St + bt * np.outer(kt, v[bb, t, h])
+                assert np.allclose(o[bb, t, h], 0.37 * St.T @ q[bb, t, hk], rtol=1e-12, atol=1e-12)
+            assert np.allclose(S[bb, h], St, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("form", [oracle.FORM_PAGES, oracle.FORM_STANDARD])
+@pytest.mark.parametrize("T,C", [(100, 16), (64, 64), (5, 8), (33, 32)])
+def test_chunked_form_equals_recurrence(form, T, C):
+    B, Hk, Hv, K, V = 1, 1, 2, 8, 6
+    q, k, v, g, beta = gdn_synth.scan_inputs(70 + T, B, T, Hk, Hv, K, V, alpha_lo=0.3)
+    S0 = gdn_synth.gaussian(71, (B, Hv, K, V))
+    o1, S1 = oracle.scan(q, k, v, g, beta, form=form, S0=S0)
+    o2, S2 = oracle.scan_chunked(q, k, v, g, beta, chunk=C, form=form, S0=S0)
+    assert np.max(np.abs(o1 - o2)) < 1e-12 * max(1, np.abs(o1).max())
+    assert np.max(np.abs(S1 - S2)) < 1e-12 * max(1, np.abs(S1).max())
+
+
+def test_chunked_handles_underflowing_decay():
+    B, T, Hk, Hv, K, V = 1, 40, 1, 1, 8, 4
+    q, k, v, g, beta = gdn_synth.scan_inputs(80, B, T, Hk, Hv, K, V)
+    g[:] = -400.0       # alpha = e^-400: the cumulative decay underflows double
+    o1, S1 = oracle.scan(q, k, v, g, beta)
+    o2, S2 = oracle.scan_chunked(q, k, v, g, beta, chunk=16)
+    assert np.all(np.isfinite(o2)) and np.allclose(o1, o2, atol=1e-12)
+
+
+def test_state_chaining_is_exact():
+    B, T, Hk, Hv, K, V = 1, 50, 1, 2, 8, 8
+    q, k, v, g, beta = gdn_synth.scan_inputs(90, B, T, Hk, Hv, K, V)
+    o, S = oracle.scan(q, k, v, g, beta)
+    t = 23
+    oa, Sa = oracle.scan(q[:, :t], k[:, :t], v[:, :t], g[:, :t], beta[:, :t])
+    ob, Sb = oracle.scan(q[:, t:], k[:, t:], v[:, t:], g[:, t:], beta[:, t:], S0=Sa)
+    assert np.array_equal(np.concatenate([oa, ob], 1), o) and np.array_equal(Sb, S)
+
+
+def test_impulse_propagates_linearly():
+    """The recurrence is affine in the state: a state impulse D evolves as
+    D_t = (alpha_t I - beta_t k k^T) D_{t-1} (PAGES form), whatever v is
+    (review page, mechanism step 3, impulse study, Fig.1b)."""
+    B, T, Hk, Hv, K, V = 1, 30, 1, 1, 8, 8
+    q, k, v, g, beta = gdn_synth.scan_inputs(95, B, T, Hk, Hv, K, V, alpha_lo=0.8)
+    S0 = gdn_synth.gaussian(96, (B, Hv, K, V))
+    D0 = gdn_synth.gaussian(97, (B, Hv, K, V), std=0.01)
+    _, Sa = oracle.scan(q, k, v, g, beta, S0=S0)
+    _, Sb = oracle.scan(q, k, v, g, beta, S0=S0.astype(np.float64) + D0.astype(np.float64))
+    D = D0[0, 0].astype(np.float64)
+    for t in range(T):
+        kt = k[0, t, 0].astype(np.float64)
+        D = (math.exp(g[0, t, 0]) * np.eye(K) - beta[0, t, 0] * np.outer(kt, kt)) @ D
+    assert np.allclose(Sb[0, 0] - Sa[0, 0], D, atol=1e-13)
+
+
+def test_layer_oracle_composes_on_tiny_shapes():
+    sh = gdn_synth.TINY
+    _, x = gdn_synth.activations(0, 64, sh.H, hot="fixed")
+    W_in = gdn_synth.weights(100, sh.n_in, sh.H)
+    W_out = gdn_synth.weights(101, sh.H, sh.Hv * sh.V)
+    A_log, dt_bias = gdn_synth.gate_params(102, sh.Hv)
+    st = oracle.layer_forward(x, oracle.quantize(W_in), oracle.quantize(W_out), A_log, dt_bias,
+                              1, 64, sh.Hk, sh.Hv, sh.K, sh.V, stages=True)
+    assert st["P"].shape == (64, sh.n_in) and st["y"].shape == (64, sh.H)
+    assert np.all(np.isfinite(st["y"]))
+    # the W4A4 layer output sits near the float64 unquantised layer output (A4/W4 noise level)
+    P = x.astype(np.float64) @ W_in.astype(np.float64).T
+    q, k, v, _z, a, b = oracle.split_projection(P, sh.Hk, sh.Hv, sh.K, sh.V)
+    g, beta = oracle.gates(a, b, A_log, dt_bias)
+    o, _ = oracle.scan(oracle.l2norm(q.reshape(1, 64, sh.Hk, sh.K)), oracle.l2norm(k.reshape(1, 64, sh.Hk, sh.K)),
+                       v.reshape(1, 64, sh.Hv, sh.V), g.reshape(1, 64, sh.Hv), beta.reshape(1, 64, sh.Hv))
+    y = o.reshape(64, -1) @ W_out.astype(np.float64).T
+    rel = np.linalg.norm(st["y"] - y) / np.linalg.norm(y)
+    assert rel < 0.5
