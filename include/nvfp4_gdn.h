@@ -1,0 +1,213 @@
+/*
+ * nvfp4_gdn.h -- C ABI of the B200 (sm_100a) NVFP4 W4A4 Gated DeltaNet layer forward.
+ *
+ * The method is the one described by the web pages on "Why Gated DeltaNet
+ * Survives 4-Bit Quantization: NVFP4 W4A4 for the Recurrent Half of a Hybrid
+ * 27B LLM" (a review page at jaehun.me and the paper's abstract):
+ *   - NVFP4: E2M1 4-bit values, one E4M3 scale per 16-element block and one
+ *     FP32 scale per tensor (review page, background section, paper sec.1);
+ *   - W4A4 linear layers, the GDN in_proj fused into one GEMM whose modules
+ *     share one global weight scale (review page, paper sec.6; abstract);
+ *   - gates, Eq.(1): g = -exp(A_log) softplus(a + dt_bias), alpha = e^g,
+ *     beta = sigmoid(b) (review page, paper sec.2);
+ *   - the delta rule, Eq.(2): S_t = alpha_t S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T,
+ *     o_t = S_t^T (q_t / sqrt(K)) (review page, background, paper sec.1).
+ *
+ * Conventions shared by every call:
+ *   - Pointers named in a call are DEVICE pointers owned by the caller unless
+ *     the comment says host; the library allocates no device memory.  Scratch
+ *     ("workspace") is sized by the matching *_workspace_size() call and
+ *     passed in; it must stay valid until the stream reaches the call.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and launches only this library's kernels (plus
+ *     cudaMemsetAsync of workspace words).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and returns a non-OK status.  The
+ *     message of the last failure on the calling host thread is returned by
+ *     nvfp4_last_error().  Nothing throws across this ABI.
+ *   - Device-side failures (a bounded wait that ran out) set a device error
+ *     word; nvfp4_check_device_error() synchronises the stream and reports
+ *     (and clears) it.
+ *   - Row-major matrices; `ld` arguments are in elements.
+ */
+#ifndef NVFP4_GDN_H
+#define NVFP4_GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, negative or zero size, bad enum */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside what the kernels cover */
+    NVFP4_ERR_MISALIGNED = 3,        /* pointer or leading dimension not 16-byte aligned */
+    NVFP4_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+    NVFP4_ERR_TIMEOUT = 5,           /* a kernel's bounded wait ran out (device error word) */
+    NVFP4_ERR_WORKSPACE = 6          /* workspace missing or smaller than required */
+} nvfp4_status;
+
+typedef void* nvfp4_stream_t; /* cudaStream_t */
+
+enum { NVFP4_DTYPE_BF16 = 0, NVFP4_DTYPE_FP32 = 1 };
+enum { NVFP4_QUANT_COMPUTE_SCALE = 0, NVFP4_QUANT_GIVEN_SCALE = 1 };
+enum { GDN_FORM_PAGES = 0, GDN_FORM_STANDARD = 1 };
+enum { GDN_SCAN_AUTO = 0, GDN_SCAN_RECURRENT = 1, GDN_SCAN_CHUNKED = 2 };
+
+/* An NVFP4 matrix [rows x cols] (cols % 64 == 0).
+ *   codes: rows * cols / 2 bytes, row-major, two E2M1 codes per byte (element
+ *          2i in the low nibble), code bits sign|e1 e0|m.  16-byte aligned.
+ *   sf:    nvfp4_sf_bytes(rows, cols) bytes of E4M3 block scales in the
+ *          tensor-core atom layout: 512-byte atoms covering 128 rows x 4
+ *          blocks (64 columns), atoms ordered (row block, column block) with
+ *          the column block fastest; the byte of (row r, block j) inside an
+ *          atom is at (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4.  Rows are
+ *          padded to a multiple of 128; the quantiser writes 0 in the pad.
+ *   global_scale: one float, the per-tensor dequantisation multiplier S, so
+ *          that x ~ e2m1(code) * e4m3(sf) * S.                              */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* sf;
+    float* global_scale;
+    int64_t rows;
+    int64_t cols;
+} nvfp4_tensor;
+
+/* Head geometry of one GDN layer.  Value head h reads key head h * Hk / Hv. */
+typedef struct {
+    int32_t Hk; /* key heads */
+    int32_t Hv; /* value heads (a multiple of Hk) */
+    int32_t K;  /* key head dim: 64 or 128 */
+    int32_t V;  /* value head dim: 64 or 128 */
+} gdn_dims;
+
+/* ---------------------------------------------------------------- errors -- */
+NVFP4_API const char* nvfp4_last_error(void);
+/* Synchronises `stream`, then returns NVFP4_ERR_TIMEOUT if any kernel of this
+ * library recorded a failed bounded wait on the current device since the last
+ * check (and clears the record), else NVFP4_OK (or NVFP4_ERR_CUDA). */
+NVFP4_API nvfp4_status nvfp4_check_device_error(nvfp4_stream_t stream);
+/* Library version, "major.minor.patch". Host string, static storage. */
+NVFP4_API const char* nvfp4_version(void);
+
+/* ------------------------------------------------------------ quantiser -- */
+/* Bytes of the scale-factor buffer of an NVFP4 [rows x cols] matrix. */
+NVFP4_API size_t nvfp4_sf_bytes(int64_t rows, int64_t cols);
+/* Bytes of workspace nvfp4_quantize needs (one amax word, padded). */
+NVFP4_API size_t nvfp4_quantize_workspace_size(void);
+
+/* Online NVFP4 quantisation of x [rows x cols] (review page, background /
+ * paper sec.1: E2M1 values, E4M3 per-16 scales, FP32 per-tensor scale; the
+ * per-tensor scale is computed from the tensor at run time).
+ *   x:       device, bf16 or fp32 (x_dtype), row pitch `ld` elements; x and
+ *            ld * element size 16-byte aligned; finite values.
+ *   out:     host struct describing device buffers (codes, sf, global_scale);
+ *            out->rows == rows, out->cols == cols.
+ *   flags:   NVFP4_QUANT_COMPUTE_SCALE: S = amax(|x|) / 2688 (S = 1 when
+ *            amax < 2^-100) is computed on the device and written to
+ *            *out->global_scale;  NVFP4_QUANT_GIVEN_SCALE: the value already
+ *            in *out->global_scale is used (harmonised weight scales).
+ *   Per block of 16: sb = E4M3_rn_satfinite(m / (6 S)), m the block amax;
+ *   codes = E2M1_rn_satfinite(x * (1 / (E4M3(sb) * S))), all float32 ops
+ *   rounded to nearest even; blocks whose E4M3(sb) * S is 0 get code 0.
+ *   workspace: device, >= nvfp4_quantize_workspace_size() bytes (required in
+ *            COMPUTE_SCALE mode; may be NULL with GIVEN_SCALE).
+ * Requirements: rows >= 1, cols >= 64, cols % 64 == 0. */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, int64_t ld,
+                            const nvfp4_tensor* out, int32_t flags, void* workspace,
+                            size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* ----------------------------------------------------------------- GEMM -- */
+/* Block-scaled FP4 x FP4 GEMM on the tcgen05 tensor cores (review page, paper
+ * sec.6: the fused in_proj GEMM; the out_proj uses the same call):
+ *   C[M x N] = S_A * S_B * sum_k (e2m1(A) e4m3(sfA))[m,k] (e2m1(B) e4m3(sfB))[n,k]
+ * A: [M x K] NVFP4 (activations), B: [N x K] NVFP4 (weights, K-major rows).
+ * C: device float32, row pitch ldc (ldc >= N, ldc % 4 == 0, C 16-byte aligned).
+ * Requirements: K % 64 == 0, N % 4 == 0, A->cols == B->cols == K. */
+NVFP4_API nvfp4_status w4a4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, float* C, int64_t ldc,
+                       nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------- gates -- */
+/* Gates, Eq.(1) (review page, paper sec.2), and per-head q/k L2 normalisation:
+ *   proj: device float32 [n_tokens x ld_proj], the fused projection with
+ *         column slices q [Hk*K] | k [Hk*K] | v [Hv*V] | z [Hv*V] | a [Hv] | b [Hv].
+ *   q_hat, k_hat: device float32 [n_tokens x Hk x K]: x / sqrt(sum x^2 + 1e-6).
+ *   g:     device float32 [n_tokens x Hv]: -exp(A_log[h]) * softplus(a + dt_bias[h])
+ *          (log of the decay alpha), softplus(u) = max(u,0) + log1p(exp(-|u|)).
+ *   beta:  device float32 [n_tokens x Hv]: 1 / (1 + exp(-b)).
+ *   A_log, dt_bias: device float32 [Hv]. */
+NVFP4_API nvfp4_status gdn_gates(const float* proj, int64_t ld_proj, int64_t n_tokens, const gdn_dims* dims,
+                       const float* A_log, const float* dt_bias, float* q_hat, float* k_hat,
+                       float* g, float* beta, nvfp4_stream_t stream);
+
+/* ----------------------------------------------------------------- scan -- */
+/* Bytes of workspace gdn_scan needs for (B, T, dims, algo). */
+NVFP4_API size_t gdn_scan_workspace_size(int32_t B, int64_t T, const gdn_dims* dims, int32_t algo);
+
+/* Delta-rule recurrence, Eq.(2) (review page, background, paper sec.1), in
+ * float32 with the state carried in float32:
+ *   form GDN_FORM_PAGES:    S_t = a S + b k (v - S^T k)^T   (as the pages write it)
+ *   form GDN_FORM_STANDARD: S_t = a S + b k (v - a S^T k)^T (decay inside the correction)
+ *   o_t = scale * S_t^T q_t.
+ * q_hat, k_hat: device [B x T x Hk x K]; v: device, token (b, t) row at
+ * v + (b*T + t) * ld_v, head h at + h*V; g (log alpha), beta: device [B x T x Hv];
+ * o: device [B x T x Hv x V]; state_in (NULL = zeros), state_out (NULL = not
+ * written): device [B x Hv x K x V].  state_in may equal state_out.
+ * algo: AUTO (chunked for T > 1, recurrent for T == 1), RECURRENT (token by
+ * token), CHUNKED (chunks of 64 tokens, WY/UT form).
+ * workspace: device, >= gdn_scan_workspace_size(B, T, dims, algo) bytes. */
+NVFP4_API nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const float* v, int64_t ld_v,
+                      const float* g, const float* beta, int32_t B, int64_t T, const gdn_dims* dims,
+                      float scale, int32_t form, int32_t algo, const float* state_in,
+                      float* state_out, float* o, void* workspace, size_t workspace_bytes,
+                      nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------- layer -- */
+typedef struct {
+    nvfp4_tensor w_in;    /* [N_in x hidden], N_in = 2*Hk*K + 2*Hv*V + 2*Hv, one global scale */
+    nvfp4_tensor w_out;   /* [hidden x Hv*V] */
+    const float* A_log;   /* device [Hv] */
+    const float* dt_bias; /* device [Hv] */
+    gdn_dims dims;
+    int32_t hidden;
+} gdn_layer_weights;
+
+/* Byte offsets of the intermediates gdn_layer_forward leaves in its
+ * workspace (valid after the stream reaches the call). */
+typedef struct {
+    size_t x_codes, x_sf, x_scale; /* quantised input */
+    size_t proj;                   /* float32 [B*T x N_in] fused projection */
+    size_t q_hat, k_hat, g, beta;  /* gate / normalisation outputs */
+    size_t o;                      /* float32 [B*T x Hv*V] scan output */
+    size_t o_codes, o_sf, o_scale; /* quantised scan output */
+    size_t quant_ws;               /* quantiser scratch */
+    size_t scan_ws;                /* scan scratch */
+    size_t total;                  /* bytes required */
+} gdn_layer_ws_layout;
+
+NVFP4_API nvfp4_status gdn_layer_workspace_layout(const gdn_layer_weights* w, int32_t B, int64_t T,
+                                        gdn_layer_ws_layout* out /* host */);
+
+/* One GDN layer forward under NVFP4 W4A4 (the four steps above, then the
+ * NVFP4 out_proj):
+ *   x_bf16: device bf16 [B*T x hidden]; y: device float32 [B*T x hidden].
+ *   state_in (NULL = zeros) / state_out (NULL = not written): device float32
+ *   [B x Hv x K x V].  form: GDN_FORM_PAGES or GDN_FORM_STANDARD.
+ *   workspace: device, >= the layout's `total` bytes, 256-byte aligned. */
+NVFP4_API nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void* x_bf16, int32_t B, int64_t T,
+                               float* y, const float* state_in, float* state_out, int32_t form,
+                               void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_GDN_H */

@@ -1,0 +1,103 @@
+// api.cu -- status plumbing, device error word, TMA descriptor encoding.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+
+namespace nvg {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+nvfp4_status fail(nvfp4_status st, const std::string& msg) {
+    g_last_error = msg;
+    return st;
+}
+
+nvfp4_status cuda_fail(cudaError_t e, const char* what) {
+    g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return NVFP4_ERR_CUDA;
+}
+
+// One word per device: kernels OR failure codes into it.
+__device__ unsigned int g_device_error_word;
+
+unsigned int* device_error_word() {
+    static std::mutex mu;
+    static unsigned int* ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<unsigned int*>(p);
+    }
+    return ptrs[dev];
+}
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+nvfp4_status make_tmap_u8_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes,
+                                uint32_t box_rows, uint32_t box_bytes) {
+    auto fn = encode_fn();
+    if (!fn) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_bytes, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string(r));
+    return NVFP4_OK;
+}
+
+}  // namespace nvg
+
+extern "C" const char* nvfp4_last_error(void) { return nvg::g_last_error.c_str(); }
+
+extern "C" const char* nvfp4_version(void) { return "0.1.0"; }
+
+extern "C" nvfp4_status nvfp4_check_device_error(nvfp4_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(nvg::as_stream(stream));
+    if (e != cudaSuccess) return nvg::cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int* w = nvg::device_error_word();
+    if (!w) return nvg::fail(NVFP4_ERR_CUDA, "device error word unavailable");
+    unsigned int v = 0;
+    e = cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return nvg::cuda_fail(e, "read device error word");
+    if (v != 0) {
+        unsigned int z = 0;
+        cudaMemcpy(w, &z, sizeof(z), cudaMemcpyHostToDevice);
+        return nvg::fail(NVFP4_ERR_TIMEOUT, "a kernel's bounded wait ran out (code " + std::to_string(v) + ")");
+    }
+    return NVFP4_OK;
+}

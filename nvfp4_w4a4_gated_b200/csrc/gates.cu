@@ -1,0 +1,111 @@
+// gates.cu -- gate parameterisation (Eq.(1) of the review page of "Why Gated
+// DeltaNet Survives 4-Bit Quantization", paper sec.2) and per-head q/k L2
+// normalisation, read straight from the fused projection's column slices.
+//
+//   g     = -exp(A_log) * softplus(a + dt_bias)   (log of alpha, alpha = e^g in (0,1))
+//   beta  = sigmoid(b)
+//   q_hat = q / sqrt(sum q^2 + 1e-6), same for k
+//
+// Element-wise and HBM-bound: one warp per (token, head) row for the
+// normalisation (coalesced 16-byte loads), one thread per (token, value head)
+// for the gates.
+#include "common.cuh"
+
+namespace nvg {
+
+namespace {
+
+template <int D>
+__global__ void __launch_bounds__(256) l2norm_kernel(const float* __restrict__ proj, int64_t ld, int64_t n_tokens,
+                                                     int Hk, float* __restrict__ q_hat, float* __restrict__ k_hat) {
+    constexpr int PER_LANE = D / 32;  // 2 or 4 contiguous floats per lane
+    const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = n_tokens * Hk * 2;
+    if (gw >= rows) return;
+    const int which = static_cast<int>(gw % 2);  // 0 = q, 1 = k
+    const int64_t th = gw / 2;
+    const int64_t t = th / Hk;
+    const int h = static_cast<int>(th - t * Hk);
+    const float* src = proj + t * ld + static_cast<int64_t>(which) * Hk * D + static_cast<int64_t>(h) * D + lane * PER_LANE;
+    float v[PER_LANE];
+    if constexpr (PER_LANE == 4) {
+        const float4 u = *reinterpret_cast<const float4*>(src);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    } else {
+        const float2 u = *reinterpret_cast<const float2*>(src);
+        v[0] = u.x; v[1] = u.y;
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) ss = fmaf(v[i], v[i], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = 1.0f / sqrtf(ss + 1e-6f);
+    float* dst = (which == 0 ? q_hat : k_hat) + th * D + lane * PER_LANE;
+    if constexpr (PER_LANE == 4) {
+        *reinterpret_cast<float4*>(dst) = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+    } else {
+        *reinterpret_cast<float2*>(dst) = make_float2(v[0] * inv, v[1] * inv);
+    }
+}
+
+__global__ void __launch_bounds__(256) gate_kernel(const float* __restrict__ proj, int64_t ld, int64_t n_tokens, int Hv,
+                                                   int64_t col_a, int64_t col_b, const float* __restrict__ A_log,
+                                                   const float* __restrict__ dt_bias, float* __restrict__ g,
+                                                   float* __restrict__ beta) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= n_tokens * Hv) return;
+    const int64_t t = i / Hv;
+    const int h = static_cast<int>(i - t * Hv);
+    const float a = proj[t * ld + col_a + h];
+    const float b = proj[t * ld + col_b + h];
+    const float u = a + dt_bias[h];
+    const float sp = fmaxf(u, 0.0f) + log1pf(expf(-fabsf(u)));
+    g[i] = -expf(A_log[h]) * sp;
+    beta[i] = 1.0f / (1.0f + expf(-b));
+}
+
+}  // namespace
+
+nvfp4_status validate_dims(const gdn_dims* d) {
+    if (!d) return fail(NVFP4_ERR_INVALID_ARG, "dims is null");
+    if (d->Hk < 1 || d->Hv < 1 || d->Hv % d->Hk) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Hv must be a multiple of Hk");
+    if ((d->K != 64 && d->K != 128) || (d->V != 64 && d->V != 128))
+        return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "head dims K, V must be 64 or 128");
+    return NVFP4_OK;
+}
+
+nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
+                          const float* dt_bias, float* q_hat, float* k_hat, float* g, float* beta, cudaStream_t st) {
+    const int64_t warps = n * d.Hk * 2;
+    const unsigned blocks_n = static_cast<unsigned>((warps * 32 + 255) / 256);
+    if (d.K == 128)
+        l2norm_kernel<128><<<blocks_n, 256, 0, st>>>(proj, ld, n, d.Hk, q_hat, k_hat);
+    else
+        l2norm_kernel<64><<<blocks_n, 256, 0, st>>>(proj, ld, n, d.Hk, q_hat, k_hat);
+    const int64_t col_a = 2ll * d.Hk * d.K + 2ll * d.Hv * d.V;
+    const unsigned blocks_g = static_cast<unsigned>((n * d.Hv + 255) / 256);
+    gate_kernel<<<blocks_g, 256, 0, st>>>(proj, ld, n, d.Hv, col_a, col_a + d.Hv, A_log, dt_bias, g, beta);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gates launch");
+    return NVFP4_OK;
+}
+
+}  // namespace nvg
+
+extern "C" nvfp4_status gdn_gates(const float* proj, int64_t ld_proj, int64_t n_tokens, const gdn_dims* dims,
+                                  const float* A_log, const float* dt_bias, float* q_hat, float* k_hat, float* g,
+                                  float* beta, nvfp4_stream_t stream) {
+    using namespace nvg;
+    nvfp4_status s = validate_dims(dims);
+    if (s != NVFP4_OK) return s;
+    if (!proj || !A_log || !dt_bias || !q_hat || !k_hat || !g || !beta)
+        return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+    if (n_tokens < 1) return fail(NVFP4_ERR_INVALID_ARG, "n_tokens < 1");
+    const int64_t n_in = 2ll * dims->Hk * dims->K + 2ll * dims->Hv * dims->V + 2ll * dims->Hv;
+    if (ld_proj < n_in) return fail(NVFP4_ERR_INVALID_ARG, "ld_proj smaller than the fused projection width");
+    if (!aligned16(proj) || ld_proj % 4 || !aligned16(q_hat) || !aligned16(k_hat))
+        return fail(NVFP4_ERR_MISALIGNED, "proj / q_hat / k_hat must be 16-byte aligned, ld_proj % 4 == 0");
+    return gates_launch(proj, ld_proj, n_tokens, *dims, A_log, dt_bias, q_hat, k_hat, g, beta, as_stream(stream));
+}

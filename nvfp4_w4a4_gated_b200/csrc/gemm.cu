@@ -1,0 +1,295 @@
+// gemm.cu -- block-scaled FP4 x FP4 GEMM on the sm_100a tensor cores.
+//
+//   C[M x N] = S_A * S_B * sum_k (e2m1(A) * e4m3(sfA))[m,k] * (e2m1(B) * e4m3(sfB))[n,k]
+//
+// The fused in_proj of the layer (q|k|v|z|a|b under one harmonised weight
+// scale, review page of "Why Gated DeltaNet Survives 4-Bit Quantization",
+// paper sec.6) and the out_proj both run through this kernel.
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: A tile [128 x 256] and B tile [BN x 256] codes
+//               (128-byte swizzle, one 128-byte row per operand row) plus the
+//               matching 512-byte scale atoms (bulk copies) into a STAGES-deep
+//               shared-memory ring guarded by full/empty mbarriers;
+//   warp 1      TMEM owner and MMA issuer: per k-tile, tcgen05.cp moves the
+//               scale atoms into TMEM, then 4 x tcgen05.mma kind::mxf4nvf4
+//               (M=128, N=BN, K=64 each) accumulate in TMEM; tcgen05.commit
+//               frees the stage and, after the last k-tile, signals the tile;
+//   warps 2..5  epilogue: tcgen05.ld of the f32 accumulator (warp w reads
+//               TMEM lanes 32*(w%4)...), scale by S_A*S_B, 16-byte stores.
+// Two accumulator buffers of BN columns; for BN = 256 they overlap in 64
+// columns (TMEM holds 512) and the epilogue drains the shared chunk first, so
+// the next tile's MMAs start after one chunk and the rest of the drain overlaps
+// them.  Every wait is bounded: on expiry the kernel records a code in the
+// device error word and returns.
+#include "common.cuh"
+
+namespace nvg {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int K_TILE_BYTES = 128;  // 256 FP4 values per operand row per stage
+constexpr int TMEM_COLS = 512;
+constexpr int SFA_COL = 448;       // 4 k-blocks x 4 columns
+constexpr int SFB_COL = 464;       // 4 k-blocks x (BN/128 x 4) columns
+
+template <int BN>
+struct Cfg {
+    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int A_BYTES = BM * K_TILE_BYTES;
+    static constexpr int B_BYTES = BN * K_TILE_BYTES;
+    static constexpr int SFA_BYTES = 4 * 512;
+    static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+    static constexpr int ACC_OFF = (2 * BN <= SFA_COL) ? BN : SFA_COL - BN;  // start column of buffer 1
+    static constexpr int NCHUNK = BN / 64;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + BAR_BYTES + 1024;
+    static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
+};
+
+__device__ __forceinline__ void st_global_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const uint8_t* __restrict__ sfA, const uint8_t* __restrict__ sfB,
+                     const float* __restrict__ scaleA, const float* __restrict__ scaleB, float* __restrict__ C,
+                     int64_t ldc, int M, int N, int K, unsigned int* __restrict__ err) {
+    using G = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + G::STAGES * G::A_BYTES;
+    uint8_t* sSFA = sB + G::STAGES * G::B_BYTES;
+    uint8_t* sSFB = sSFA + G::STAGES * G::SFA_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + G::STAGES * G::SFB_BYTES);
+    uint64_t* empty = full + G::STAGES;
+    uint64_t* acc_full = empty + G::STAGES;
+    uint64_t* tmem_free = acc_full + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tmem_free + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int kb_total = K / 64;                 // 64-wide k-blocks = scale atoms along K
+    const int num_kt = (kb_total + 3) / 4;       // 256-wide k-tiles
+    const int sfb_row_blocks = (N + 127) / 128;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < G::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(tmem_free, 4);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------- producer --
+            uint32_t stage = 0, phase = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+                const int m_idx = tile % num_m, n_idx = tile / num_m;
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, err, kErrTimeoutTma)) goto producer_done;
+                    const int nkb = min(4, kb_total - kt * 4);
+                    int nb_valid = 0;
+#pragma unroll
+                    for (int nb = 0; nb < BN / 128; ++nb) nb_valid += (n_idx * (BN / 128) + nb < sfb_row_blocks);
+                    const uint32_t bytes = G::A_BYTES + G::B_BYTES + nkb * 512 * (1 + nb_valid);
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(sA + stage * G::A_BYTES, &tmA, &full[stage], kt * K_TILE_BYTES, m_idx * BM);
+                    tma_load_2d(sB + stage * G::B_BYTES, &tmB, &full[stage], kt * K_TILE_BYTES, n_idx * BN);
+                    bulk_load(sSFA + stage * G::SFA_BYTES, sfA + ((int64_t)m_idx * kb_total + kt * 4) * 512,
+                              nkb * 512, &full[stage]);
+#pragma unroll
+                    for (int nb = 0; nb < BN / 128; ++nb) {
+                        const int rb = n_idx * (BN / 128) + nb;
+                        if (rb < sfb_row_blocks)
+                            bulk_load(sSFB + stage * G::SFB_BYTES + nb * 2048,
+                                      sfB + ((int64_t)rb * kb_total + kt * 4) * 512, nkb * 512, &full[stage]);
+                    }
+                    if (++stage == G::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        producer_done:;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // --------------------------------------------------------- MMA --
+            uint32_t stage = 0, phase = 0;
+            int local = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+                const uint32_t acc = tmem + (local & 1) * G::ACC_OFF;
+                if (local > 0) {
+                    if (!mbar_wait(tmem_free, (local - 1) & 1, err, kErrTimeoutMma)) break;
+                    tc_fence_after();
+                }
+                bool ok = true;
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    if (!mbar_wait(&full[stage], phase, err, kErrTimeoutMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nkb = min(4, kb_total - kt * 4);
+                    const uint32_t a_base = smem_u32(sA + stage * G::A_BYTES);
+                    const uint32_t b_base = smem_u32(sB + stage * G::B_BYTES);
+                    const uint32_t sfa_base = smem_u32(sSFA + stage * G::SFA_BYTES);
+                    const uint32_t sfb_base = smem_u32(sSFB + stage * G::SFB_BYTES);
+                    for (int j = 0; j < nkb; ++j) {
+                        tmem_cp_sf_atom(tmem + SFA_COL + 4 * j, sdesc_sf_atom(sfa_base + j * 512));
+#pragma unroll
+                        for (int nb = 0; nb < BN / 128; ++nb)
+                            tmem_cp_sf_atom(tmem + SFB_COL + j * (BN / 32) + nb * 4,
+                                            sdesc_sf_atom(sfb_base + nb * 2048 + j * 512));
+                    }
+                    for (int j = 0; j < nkb; ++j) {
+                        mma_nvf4(acc, sdesc_kmajor_sw128(a_base + j * 32), sdesc_kmajor_sw128(b_base + j * 32),
+                                 G::IDESC, tmem + SFA_COL + 4 * j, tmem + SFB_COL + j * (BN / 32),
+                                 (kt > 0 || j > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[stage]);
+                    if (++stage == G::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(acc_full);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue --
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const float alpha = __fmul_rn(*scaleA, *scaleB);
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            const int m_idx = tile % num_m, n_idx = tile / num_m;
+            const int buf = local & 1;
+            if (!mbar_wait(acc_full, local & 1, err, kErrTimeoutEpi)) break;
+            tc_fence_after();
+            const int row = m_idx * BM + q * 32 + lane;
+            float* crow = C + (int64_t)row * ldc;
+#pragma unroll 1
+            for (int ci = 0; ci < G::NCHUNK; ++ci) {
+                // buffer 0 of the overlapping pair drains its shared (last) chunk first
+                const int c = (G::ACC_OFF < BN && buf == 0) ? (ci + G::NCHUNK - 1) % G::NCHUNK : ci;
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * G::ACC_OFF + c * 64;
+                uint32_t v0[32], v1[32];
+                tmem_ld_32x32b_x32(taddr, v0);
+                tmem_ld_32x32b_x32(taddr + 32, v1);
+                tmem_wait_ld();
+                if (ci == 0) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tmem_free);
+                }
+                if (row < M) {
+                    const int col0 = n_idx * BN + c * 64;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int col = col0 + 4 * i;
+                        if (col < N)
+                            st_global_v4(crow + col, alpha * __uint_as_float(v0[4 * i]),
+                                         alpha * __uint_as_float(v0[4 * i + 1]), alpha * __uint_as_float(v0[4 * i + 2]),
+                                         alpha * __uint_as_float(v0[4 * i + 3]));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int col = col0 + 32 + 4 * i;
+                        if (col < N)
+                            st_global_v4(crow + col, alpha * __uint_as_float(v1[4 * i]),
+                                         alpha * __uint_as_float(v1[4 * i + 1]), alpha * __uint_as_float(v1[4 * i + 2]),
+                                         alpha * __uint_as_float(v1[4 * i + 3]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int BN>
+nvfp4_status launch_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C, int64_t ldc, cudaStream_t st) {
+    using G = Cfg<BN>;
+    const int M = static_cast<int>(A.rows), N = static_cast<int>(B.rows), K = static_cast<int>(A.cols);
+    CUtensorMap ta, tb;
+    nvfp4_status s = make_tmap_u8_sw128(&ta, A.codes, A.rows, A.cols / 2, BM, K_TILE_BYTES);
+    if (s != NVFP4_OK) return s;
+    s = make_tmap_u8_sw128(&tb, B.codes, B.rows, B.cols / 2, BN, K_TILE_BYTES);
+    if (s != NVFP4_OK) return s;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
+        attr_done[dev] = true;
+    }
+    unsigned int* err = device_error_word();
+    if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    w4a4_gemm_kernel<BN><<<grid, 192, G::SMEM, st>>>(ta, tb, A.sf, B.sf, A.global_scale, B.global_scale, C, ldc, M, N,
+                                                     K, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm launch");
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+nvfp4_status validate_tensor(const nvfp4_tensor* t, const char* name);
+
+nvfp4_status gemm_launch(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C, int64_t ldc, cudaStream_t st) {
+    const int64_t M = A.rows, N = B.rows;
+    const int64_t tiles256 = ((M + BM - 1) / BM) * ((N + 255) / 256);
+    if (N <= 128 || tiles256 < num_sms()) return launch_gemm<128>(A, B, C, ldc, st);
+    return launch_gemm<256>(A, B, C, ldc, st);
+}
+
+}  // namespace nvg
+
+extern "C" nvfp4_status w4a4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, float* C, int64_t ldc,
+                                  nvfp4_stream_t stream) {
+    using namespace nvg;
+    nvfp4_status s = validate_tensor(A, "A");
+    if (s != NVFP4_OK) return s;
+    s = validate_tensor(B, "B");
+    if (s != NVFP4_OK) return s;
+    if (A->cols != B->cols) return fail(NVFP4_ERR_INVALID_ARG, "A and B have different K");
+    if (!C) return fail(NVFP4_ERR_INVALID_ARG, "C is null");
+    if (B->rows % 4) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 4");
+    if (ldc < B->rows) return fail(NVFP4_ERR_INVALID_ARG, "ldc < N");
+    if (!aligned16(C) || ldc % 4) return fail(NVFP4_ERR_MISALIGNED, "C / ldc not 16-byte aligned");
+    if (A->rows > (int64_t(1) << 30) || B->rows > (int64_t(1) << 30))
+        return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M or N too large");
+    return gemm_launch(*A, *B, C, ldc, as_stream(stream));
+}

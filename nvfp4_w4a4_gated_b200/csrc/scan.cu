@@ -1,0 +1,582 @@
+// scan.cu -- the delta-rule recurrence, Eq.(2) of the review page of "Why
+// Gated DeltaNet Survives 4-Bit Quantization" (paper sec.1):
+//
+//   S_t = alpha_t S_{t-1} + beta_t k_t (v_t - c_t S_{t-1}^T k_t)^T,   o_t = scale * S_t^T q_t
+//
+// with c_t = 1 (form PAGES, as the pages write it) or c_t = alpha_t (form
+// STANDARD).  The state is float32 throughout.
+//
+// Two algorithms:
+//  * recurrent: one CTA per (sequence, value head, 32-column slice of V); the
+//    state slice lives in registers (thread = column, K/4 rows per warp), one
+//    token per step.  Used for decode (T = 1) and as a reference path.
+//  * chunked (C = 64 tokens): with G_t the running sum of g = log(alpha)
+//    inside a chunk, the chunk's writes u solve the unit lower-triangular system
+//      u_t + b_t sum_{i<t} e^{Gd_t - G_i} (k_t.k_i) u_i = beta_t v_t - b_t e^{Gd_t} S0^T k_t
+//    (Gd_t = G_{t-1} for PAGES, G_t for STANDARD), i.e. U = U~ - W~ S0 with
+//    U~ = T (beta V), W~ = T (D K), T = (I + L)^-1; then
+//      o_t  = scale (e^{G_t} S0^T q_t + sum_{i<=t} e^{G_t - G_i} (q_t.k_i) u_i)
+//      S_C  = e^{G_C} S0 + sum_i e^{G_C - G_i} k_i u_i^T.
+//    Kernel 1 (parallel over chunk x head) builds W~, U~, the masked decayed
+//    Q K^T and G; kernel 2 (one CTA per head x 32-column V slice) walks the
+//    chunks in order.  Products run on the tensor cores in TF32 with float32
+//    accumulation (mma.sync m16n8k8).
+#include "common.cuh"
+
+namespace nvg {
+
+namespace {
+
+constexpr int CH = 64;  // chunk length
+
+// --------------------------------------------------------------- recurrent --
+template <int K>
+__global__ void __launch_bounds__(128) scan_recurrent_kernel(
+    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, int64_t ld_v,
+    const float* __restrict__ g, const float* __restrict__ beta, int B, int64_t T, int Hk, int Hv, int V, float scale,
+    int form, const float* state_in, float* state_out, float* __restrict__ o) {
+    constexpr int RW = K / 4;
+    const int nslice = V / 32;
+    const int bh = blockIdx.x / nslice, slice = blockIdx.x - bh * nslice;
+    const int b = bh / Hv, h = bh - b * Hv;
+    const int hk = static_cast<int>((static_cast<int64_t>(h) * Hk) / Hv);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = slice * 32 + lane;
+    const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
+
+    float S[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) S[i] = state_in ? state_in[sbase + static_cast<int64_t>(w * RW + i) * V + j] : 0.0f;
+
+    __shared__ float ks[K], qs[K];
+    __shared__ float red1[4][32], red2[4][32];
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t tok = static_cast<int64_t>(b) * T + t;
+        if (threadIdx.x < K) {
+            ks[threadIdx.x] = k[(tok * Hk + hk) * K + threadIdx.x];
+            qs[threadIdx.x] = q[(tok * Hk + hk) * K + threadIdx.x];
+        }
+        const float alpha = expf(g[tok * Hv + h]);
+        const float bt = beta[tok * Hv + h];
+        const float vj = v[tok * ld_v + static_cast<int64_t>(h) * V + j];
+        __syncthreads();
+        float p = 0.0f;
+#pragma unroll
+        for (int i = 0; i < RW; ++i) p = fmaf(S[i], ks[w * RW + i], p);
+        red1[w][lane] = p;
+        __syncthreads();
+        float pred = (red1[0][lane] + red1[1][lane]) + (red1[2][lane] + red1[3][lane]);
+        if (form == GDN_FORM_STANDARD) pred *= alpha;
+        const float u = bt * (vj - pred);
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+            S[i] = fmaf(alpha, S[i], ks[w * RW + i] * u);
+            acc = fmaf(S[i], qs[w * RW + i], acc);
+        }
+        red2[w][lane] = acc;
+        __syncthreads();
+        if (w == 0) o[(tok * Hv + h) * V + j] = scale * ((red2[0][lane] + red2[1][lane]) + (red2[2][lane] + red2[3][lane]));
+    }
+    if (state_out) {
+#pragma unroll
+        for (int i = 0; i < RW; ++i) state_out[sbase + static_cast<int64_t>(w * RW + i) * V + j] = S[i];
+    }
+}
+
+// ------------------------------------------------------------ mma helpers --
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// 3xTF32: a*b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi (float32-level accuracy).
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = to_tf32(x);
+    lo = to_tf32(x - __uint_as_float(hi));
+}
+
+template <bool PREC3>
+__device__ __forceinline__ void mma_f32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
+    if constexpr (PREC3) {
+        uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
+        split_tf32(b[0], bh[0], bl[0]);
+        split_tf32(b[1], bh[1], bl[1]);
+        mma_tf32(d, al, bh);
+        mma_tf32(d, ah, bl);
+        mma_tf32(d, ah, bh);
+    } else {
+        const uint32_t ai[4] = {to_tf32(a[0]), to_tf32(a[1]), to_tf32(a[2]), to_tf32(a[3])};
+        const uint32_t bi[2] = {to_tf32(b[0]), to_tf32(b[1])};
+        mma_tf32(d, ai, bi);
+    }
+}
+
+// ------------------------------------------------------ chunk preparation --
+// One CTA (256 threads) per (sequence, chunk, value head).
+template <int K, int V>
+struct PrepSmem {
+    static constexpr int KS = K + 4;  // row stride of K/Q tiles (== 4 mod 32)
+    float ks[CH * KS];
+    float qs[CH * KS];
+    float L[CH * CH];
+    float gin[CH], gd[CH], bet[CH], graw[CH];
+};
+
+template <int K, int V>
+__global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                                                         const float* __restrict__ v, int64_t ld_v,
+                                                         const float* __restrict__ g, const float* __restrict__ beta,
+                                                         int64_t T, int Hk, int Hv, int form, int NC,
+                                                         float* __restrict__ Wt, float* __restrict__ Ut,
+                                                         float* __restrict__ Mt, float* __restrict__ Gt) {
+    using SM = PrepSmem<K, V>;
+    constexpr int KS = SM::KS;
+    extern __shared__ float4 smem_f4[];
+    SM& sm = *reinterpret_cast<SM*>(smem_f4);
+    const int h = blockIdx.x % Hv;
+    const int c = (blockIdx.x / Hv) % NC;
+    const int b = blockIdx.x / (Hv * NC);
+    const int hk = static_cast<int>((static_cast<int64_t>(h) * Hk) / Hv);
+    const int64_t t0 = static_cast<int64_t>(c) * CH;
+    const int n = static_cast<int>((T - t0) < CH ? (T - t0) : CH);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // load K, Q rows (zero past the end of the sequence), g and beta
+    constexpr int V4 = K / 4;
+    for (int idx = tid; idx < CH * V4; idx += 256) {
+        const int r = idx / V4, c4 = idx - r * V4;
+        float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv;
+        if (r < n) {
+            const int64_t off = ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4;
+            kv = *reinterpret_cast<const float4*>(k + off);
+            qv = *reinterpret_cast<const float4*>(q + off);
+        }
+        *reinterpret_cast<float4*>(&sm.ks[r * KS + c4 * 4]) = kv;
+        *reinterpret_cast<float4*>(&sm.qs[r * KS + c4 * 4]) = qv;
+    }
+    if (tid < CH) {
+        const int64_t gi = (static_cast<int64_t>(b) * T + t0 + tid) * Hv + h;
+        sm.graw[tid] = tid < n ? g[gi] : 0.0f;
+        sm.bet[tid] = tid < n ? beta[gi] : 0.0f;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // inclusive prefix sum of g over the chunk (2 values per lane)
+        float a0 = sm.graw[2 * lane], a1 = sm.graw[2 * lane + 1];
+        float s = a0 + a1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        const float excl = s - (a0 + a1);
+        const float g0 = excl + a0, g1 = s;
+        sm.gin[2 * lane] = g0;
+        sm.gin[2 * lane + 1] = g1;
+        sm.gd[2 * lane] = form == GDN_FORM_STANDARD ? g0 : excl;
+        sm.gd[2 * lane + 1] = form == GDN_FORM_STANDARD ? g1 : g0;
+    }
+    __syncthreads();
+
+    // K K^T (warps 0-3) and Q K^T (warps 4-7), 16 rows per warp, TF32 tensor cores
+    {
+        const int grp = lane >> 2, tig = lane & 3;
+        const float* A = warp < 4 ? sm.ks : sm.qs;
+        const int r0 = (warp & 3) * 16;
+        float acc[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 4
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            const float a[4] = {A[(r0 + grp) * KS + k0 + tig], A[(r0 + grp + 8) * KS + k0 + tig],
+                                A[(r0 + grp) * KS + k0 + tig + 4], A[(r0 + grp + 8) * KS + k0 + tig + 4]};
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const float bb[2] = {sm.ks[(nt * 8 + grp) * KS + k0 + tig], sm.ks[(nt * 8 + grp) * KS + k0 + tig + 4]};
+                mma_f32<false>(acc[nt], a, bb);
+            }
+        }
+        const int64_t mbase = ((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH * CH;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = r0 + grp + (e >> 1) * 8;
+                const int i = nt * 8 + 2 * tig + (e & 1);
+                if (warp < 4) {
+                    sm.L[t * CH + i] = (i < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
+                } else {
+                    Mt[mbase + t * CH + i] = (i <= t) ? expf(sm.gin[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
+                }
+            }
+        }
+    }
+    if (tid < CH) Gt[((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH + tid] = sm.gin[tid];
+    __syncthreads();
+
+    // forward substitution, one right-hand-side column per thread:
+    // columns [0, K) give W~ (rhs b_t e^{Gd_t} k_t), columns [K, K+V) give U~ (rhs beta_t v_t)
+    if (tid < K + V) {
+        const bool isW = tid < K;
+        const int col = isW ? tid : tid - K;
+        float x[CH];
+#pragma unroll
+        for (int t = 0; t < CH; ++t) {
+            float r;
+            if (isW) {
+                r = sm.bet[t] * expf(sm.gd[t]) * sm.ks[t * KS + col];
+            } else {
+                r = t < n ? sm.bet[t] * v[(static_cast<int64_t>(b) * T + t0 + t) * ld_v + static_cast<int64_t>(h) * V + col]
+                          : 0.0f;
+            }
+#pragma unroll
+            for (int i = 0; i < t; ++i) r = fmaf(-sm.L[t * CH + i], x[i], r);
+            x[t] = r;
+        }
+        const int64_t cb = (static_cast<int64_t>(b) * Hv + h) * NC + c;
+        if (isW) {
+#pragma unroll
+            for (int t = 0; t < CH; ++t) Wt[(cb * CH + t) * K + col] = x[t];
+        } else {
+#pragma unroll
+            for (int t = 0; t < CH; ++t) Ut[(cb * CH + t) * V + col] = x[t];
+        }
+    }
+}
+
+// ------------------------------------------------------ sequential chunks --
+template <int K>
+struct SeqSmem {
+    static constexpr int XS = K + 4;   // [W~; Q] tile row stride (== 4 mod 32)
+    static constexpr int KS = K + 8;   // K tile row stride (== 8 mod 32, transposed reads)
+    static constexpr int MS = CH + 4;  // masked Q K^T row stride
+    static constexpr int SS = 40;      // state / U row stride (== 8 mod 32)
+    float x1[2 * CH * XS];
+    float kc[CH * KS];
+    float mc[CH * MS];
+    float s[K * SS];
+    float u[CH * SS];
+    float ud[CH * SS];
+    float gin[CH];
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One CTA (256 threads) per (sequence, value head, 32-column slice of V).
+template <int K, bool PREC3>
+__global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                                                        int64_t T, int Hk, int Hv, int V, float scale, int NC,
+                                                        const float* __restrict__ Wt, const float* __restrict__ Ut,
+                                                        const float* __restrict__ Mt, const float* __restrict__ Gt,
+                                                        const float* state_in, float* state_out, float* __restrict__ o) {
+    using SM = SeqSmem<K>;
+    constexpr int XS = SM::XS, KS = SM::KS, MS = SM::MS, SS = SM::SS;
+    extern __shared__ float4 smem_f4[];
+    SM& sm = *reinterpret_cast<SM*>(smem_f4);
+    const int nslice = V / 32;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % Hv;
+    const int b = blockIdx.x / (nslice * Hv);
+    const int hk = static_cast<int>((static_cast<int64_t>(h) * Hk) / Hv);
+    const int vs0 = slice * 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 2, tig = lane & 3;
+    const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
+    const int64_t hc = (static_cast<int64_t>(b) * Hv + h) * NC;
+
+    for (int idx = tid; idx < K * 32; idx += 256) {
+        const int r = idx >> 5, cc = idx & 31;
+        sm.s[r * SS + cc] = state_in ? state_in[sbase + static_cast<int64_t>(r) * V + vs0 + cc] : 0.0f;
+    }
+
+    auto load_wq = [&](int c) {
+        const int64_t t0 = static_cast<int64_t>(c) * CH;
+        constexpr int V4 = K / 4;
+        for (int idx = tid; idx < CH * V4; idx += 256) {
+            const int r = idx / V4, c4 = idx - r * V4;
+            cp_async16(&sm.x1[r * XS + c4 * 4], Wt + ((hc + c) * CH + r) * K + c4 * 4, true);
+            const bool valid = t0 + r < T;
+            const int64_t qoff = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
+            cp_async16(&sm.x1[(CH + r) * XS + c4 * 4], q + qoff, valid);
+        }
+    };
+    auto load_km = [&](int c) {
+        const int64_t t0 = static_cast<int64_t>(c) * CH;
+        constexpr int V4 = K / 4;
+        for (int idx = tid; idx < CH * V4; idx += 256) {
+            const int r = idx / V4, c4 = idx - r * V4;
+            const bool valid = t0 + r < T;
+            const int64_t koff = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
+            cp_async16(&sm.kc[r * KS + c4 * 4], k + koff, valid);
+        }
+        for (int idx = tid; idx < CH * CH / 4; idx += 256) {
+            const int r = idx >> 4, c4 = idx & 15;
+            cp_async16(&sm.mc[r * MS + c4 * 4], Mt + ((hc + c) * CH + r) * CH + c4 * 4, true);
+        }
+        if (tid < CH / 4) cp_async16(&sm.gin[tid * 4], Gt + (hc + c) * CH + tid * 4, true);
+    };
+
+    load_wq(0);
+    load_km(0);
+    cp_async_commit();
+
+    for (int c = 0; c < NC; ++c) {
+        const int64_t t0 = static_cast<int64_t>(c) * CH;
+        cp_async_wait<0>();
+        __syncthreads();
+
+        // P1: [W~; Q] (128 x K) times S (K x 32); warp w owns rows 16w..16w+15
+        float acc[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        {
+            const int r0 = warp * 16;
+#pragma unroll 4
+            for (int k0 = 0; k0 < K; k0 += 8) {
+                const float a[4] = {sm.x1[(r0 + grp) * XS + k0 + tig], sm.x1[(r0 + grp + 8) * XS + k0 + tig],
+                                    sm.x1[(r0 + grp) * XS + k0 + tig + 4], sm.x1[(r0 + grp + 8) * XS + k0 + tig + 4]};
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const float bb[2] = {sm.s[(k0 + tig) * SS + nt * 8 + grp], sm.s[(k0 + tig + 4) * SS + nt * 8 + grp]};
+                    mma_f32<PREC3>(acc[nt], a, bb);
+                }
+            }
+        }
+        const float glast = sm.gin[CH - 1];
+        if (warp < 4) {
+            // U = U~ - W~ S0; also U scaled by e^{G_C - G_i} for the state update
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = warp * 16 + grp + (e >> 1) * 8;
+                    const int col = nt * 8 + 2 * tig + (e & 1);
+                    const float ut = Ut[((hc + c) * CH + i) * V + vs0 + col];
+                    const float uval = ut - acc[nt][e];
+                    sm.u[i * SS + col] = uval;
+                    sm.ud[i * SS + col] = expf(glast - sm.gin[i]) * uval;
+                }
+            }
+        }
+        __syncthreads();
+        // X1 is free: prefetch the next chunk's W~ and Q while this chunk finishes
+        if (c + 1 < NC) {
+            load_wq(c + 1);
+            cp_async_commit();
+        }
+
+        if (warp >= 4) {
+            // o = scale * (e^{G_t} Q S0 + Mqk U); rows t = 16(w-4)..
+            const int r0 = (warp - 4) * 16;
+            float mu[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) mu[nt][0] = mu[nt][1] = mu[nt][2] = mu[nt][3] = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < CH; k0 += 8) {
+                const float a[4] = {sm.mc[(r0 + grp) * MS + k0 + tig], sm.mc[(r0 + grp + 8) * MS + k0 + tig],
+                                    sm.mc[(r0 + grp) * MS + k0 + tig + 4], sm.mc[(r0 + grp + 8) * MS + k0 + tig + 4]};
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const float bb[2] = {sm.u[(k0 + tig) * SS + nt * 8 + grp], sm.u[(k0 + tig + 4) * SS + nt * 8 + grp]};
+                    mma_f32<false>(mu[nt], a, bb);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int t = r0 + grp + hh * 8;
+                    if (t0 + t < T) {
+                        const float eg = expf(sm.gin[t]);
+                        const int col = nt * 8 + 2 * tig;
+                        const float o0 = scale * fmaf(eg, acc[nt][2 * hh], mu[nt][2 * hh]);
+                        const float o1 = scale * fmaf(eg, acc[nt][2 * hh + 1], mu[nt][2 * hh + 1]);
+                        *reinterpret_cast<float2*>(o + ((static_cast<int64_t>(b) * T + t0 + t) * Hv + h) * V + vs0 + col) =
+                            make_float2(o0, o1);
+                    }
+                }
+            }
+        }
+
+        // S <- e^{G_C} S + K^T (diag(e^{G_C - G}) U); warp w owns state rows 16w..16w+15
+        if (warp * 16 < K) {
+            const int d0 = warp * 16;
+            const float eg = expf(glast);
+            float st[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int col = nt * 8 + 2 * tig;
+                st[nt][0] = eg * sm.s[(d0 + grp) * SS + col];
+                st[nt][1] = eg * sm.s[(d0 + grp) * SS + col + 1];
+                st[nt][2] = eg * sm.s[(d0 + grp + 8) * SS + col];
+                st[nt][3] = eg * sm.s[(d0 + grp + 8) * SS + col + 1];
+            }
+#pragma unroll
+            for (int k0 = 0; k0 < CH; k0 += 8) {
+                const float a[4] = {sm.kc[(k0 + tig) * KS + d0 + grp], sm.kc[(k0 + tig) * KS + d0 + grp + 8],
+                                    sm.kc[(k0 + tig + 4) * KS + d0 + grp], sm.kc[(k0 + tig + 4) * KS + d0 + grp + 8]};
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const float bb[2] = {sm.ud[(k0 + tig) * SS + nt * 8 + grp], sm.ud[(k0 + tig + 4) * SS + nt * 8 + grp]};
+                    mma_f32<PREC3>(st[nt], a, bb);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int col = nt * 8 + 2 * tig;
+                sm.s[(d0 + grp) * SS + col] = st[nt][0];
+                sm.s[(d0 + grp) * SS + col + 1] = st[nt][1];
+                sm.s[(d0 + grp + 8) * SS + col] = st[nt][2];
+                sm.s[(d0 + grp + 8) * SS + col + 1] = st[nt][3];
+            }
+        }
+        __syncthreads();
+        if (c + 1 < NC) {
+            load_km(c + 1);
+            cp_async_commit();
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (state_out) {
+        for (int idx = tid; idx < K * 32; idx += 256) {
+            const int r = idx >> 5, cc = idx & 31;
+            state_out[sbase + static_cast<int64_t>(r) * V + vs0 + cc] = sm.s[r * SS + cc];
+        }
+    }
+}
+
+struct ChunkWs {
+    float *Wt, *Ut, *Mt, *Gt;
+    size_t bytes;
+};
+
+ChunkWs chunk_ws(void* base, int B, int64_t T, const gdn_dims& d) {
+    const int64_t NC = (T + CH - 1) / CH;
+    const int64_t units = static_cast<int64_t>(B) * d.Hv * NC;
+    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t w = al(units * CH * d.K * 4), u = al(units * CH * d.V * 4), m = al(units * CH * CH * 4),
+                 gg = al(units * CH * 4);
+    ChunkWs ws;
+    char* p = static_cast<char*>(base);
+    ws.Wt = reinterpret_cast<float*>(p);
+    ws.Ut = reinterpret_cast<float*>(p + w);
+    ws.Mt = reinterpret_cast<float*>(p + w + u);
+    ws.Gt = reinterpret_cast<float*>(p + w + u + m);
+    ws.bytes = w + u + m + gg;
+    return ws;
+}
+
+template <int K, int V>
+nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
+                               const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form,
+                               const float* s_in, float* s_out, float* o, const ChunkWs& ws, cudaStream_t st) {
+    const int NC = static_cast<int>((T + CH - 1) / CH);
+    const int prep_smem = sizeof(PrepSmem<K, V>);
+    const int seq_smem = sizeof(SeqSmem<K>);
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prep)");
+        e = cudaFuncSetAttribute(chunk_seq_kernel<K, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq)");
+        attr_done[dev] = true;
+    }
+    const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
+    chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, ws.Wt,
+                                                                 ws.Ut, ws.Mt, ws.Gt);
+    const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
+    chunk_seq_kernel<K, false><<<seq_blocks, 256, seq_smem, st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt, ws.Ut,
+                                                                  ws.Mt, ws.Gt, s_in, s_out, o);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+nvfp4_status validate_dims(const gdn_dims* d);
+
+size_t scan_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo) {
+    const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
+    if (!chunked) return 0;
+    return chunk_ws(nullptr, B, T, d).bytes;
+}
+
+nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
+                         const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form, int algo,
+                         const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st) {
+    const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
+    if (!chunked) {
+        const unsigned blocks = static_cast<unsigned>(B * d.Hv * (d.V / 32));
+        if (d.K == 128)
+            scan_recurrent_kernel<128><<<blocks, 128, 0, st>>>(q, k, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form,
+                                                               s_in, s_out, o);
+        else
+            scan_recurrent_kernel<64><<<blocks, 128, 0, st>>>(q, k, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form,
+                                                              s_in, s_out, o);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "recurrent scan launch");
+        return NVFP4_OK;
+    }
+    const ChunkWs cws = chunk_ws(ws, B, T, d);
+    if (d.K == 128 && d.V == 128)
+        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+    if (d.K == 128 && d.V == 64)
+        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+    if (d.K == 64 && d.V == 128)
+        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+}
+
+}  // namespace nvg
+
+extern "C" size_t gdn_scan_workspace_size(int32_t B, int64_t T, const gdn_dims* dims, int32_t algo) {
+    if (!dims || nvg::validate_dims(dims) != NVFP4_OK || B < 1 || T < 1) return 0;
+    return nvg::scan_workspace_bytes(B, T, *dims, algo);
+}
+
+extern "C" nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const float* v, int64_t ld_v, const float* g,
+                                 const float* beta, int32_t B, int64_t T, const gdn_dims* dims, float scale,
+                                 int32_t form, int32_t algo, const float* state_in, float* state_out, float* o,
+                                 void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+    using namespace nvg;
+    nvfp4_status s = validate_dims(dims);
+    if (s != NVFP4_OK) return s;
+    if (!q_hat || !k_hat || !v || !g || !beta || !o) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+    if (B < 1 || T < 1) return fail(NVFP4_ERR_INVALID_ARG, "B and T must be >= 1");
+    if (form != GDN_FORM_PAGES && form != GDN_FORM_STANDARD) return fail(NVFP4_ERR_INVALID_ARG, "bad form");
+    if (algo != GDN_SCAN_AUTO && algo != GDN_SCAN_RECURRENT && algo != GDN_SCAN_CHUNKED)
+        return fail(NVFP4_ERR_INVALID_ARG, "bad algo");
+    if (ld_v < static_cast<int64_t>(dims->Hv) * dims->V) return fail(NVFP4_ERR_INVALID_ARG, "ld_v < Hv*V");
+    if (static_cast<int64_t>(B) * T > (int64_t(1) << 31)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "B*T too large");
+    if (!aligned16(q_hat) || !aligned16(k_hat) || !aligned16(o) || !aligned16(v) || ld_v % 4)
+        return fail(NVFP4_ERR_MISALIGNED, "q_hat, k_hat, v, o must be 16-byte aligned and ld_v % 4 == 0");
+    const size_t need = scan_workspace_bytes(B, T, *dims, algo);
+    if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)))
+        return fail(NVFP4_ERR_WORKSPACE, "scan workspace missing, too small or not 256-byte aligned");
+    return scan_launch(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, algo, state_in, state_out, o,
+                       workspace, as_stream(stream));
+}

@@ -1,0 +1,133 @@
+"""The C-ABI library loads, exports every symbol the header declares, and its
+host-side validation rejects bad arguments before launching anything.  CPU only:
+no call here reaches a kernel launch."""
+import ctypes
+import re
+import os
+
+import pytest
+
+import nvfp4_w4a4_gated_b200 as nv
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "nvfp4_gdn.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_symbols() == sorted(nv.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = nv.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_version_and_sizes():
+    L = nv.lib()
+    assert L.nvfp4_version().decode().count(".") == 2
+    assert L.nvfp4_sf_bytes(1, 64) == 128 * 4
+    assert L.nvfp4_sf_bytes(129, 128) == 256 * 8
+    assert L.nvfp4_sf_bytes(8192, 5120) == 8192 * 320
+    assert L.nvfp4_quantize_workspace_size() >= 4
+    d = nv.GdnDims(16, 32, 128, 128).c()
+    assert L.gdn_scan_workspace_size(1, 1, ctypes.byref(d), nv.SCAN_AUTO) == 0
+    n = L.gdn_scan_workspace_size(1, 4096, ctypes.byref(d), nv.SCAN_CHUNKED)
+    assert n >= 32 * 64 * (64 * 128 * 2 + 64 * 64 + 64) * 4
+    bad = nv.GdnDims(3, 32, 128, 128).c()
+    assert L.gdn_scan_workspace_size(1, 4096, ctypes.byref(bad), nv.SCAN_CHUNKED) == 0
+
+
+def _err(status):
+    return status, nv.lib().nvfp4_last_error().decode()
+
+
+FAKE = 0x10000  # a 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+def _tensor(rows=128, cols=256, codes=FAKE, sf=FAKE, scale=FAKE):
+    return nv._Tensor(codes, sf, scale, rows, cols)
+
+
+def test_quantize_validation():
+    L = nv.lib()
+    t = _tensor()
+    st, msg = _err(L.nvfp4_quantize(None, 0, 128, 256, 256, ctypes.byref(t), 0, FAKE, 256, None))
+    assert st == 1 and "null" in msg
+    st, _ = _err(L.nvfp4_quantize(FAKE, 7, 128, 256, 256, ctypes.byref(t), 0, FAKE, 256, None))
+    assert st == 1
+    t2 = _tensor(cols=100)
+    st, _ = _err(L.nvfp4_quantize(FAKE, 0, 128, 100, 100, ctypes.byref(t2), 0, FAKE, 256, None))
+    assert st == 2
+    st, _ = _err(L.nvfp4_quantize(FAKE + 2, 0, 128, 256, 256, ctypes.byref(t), 0, FAKE, 256, None))
+    assert st == 3
+    st, _ = _err(L.nvfp4_quantize(FAKE, 0, 128, 256, 256, ctypes.byref(t), 0, None, 0, None))
+    assert st == 6
+    st, _ = _err(L.nvfp4_quantize(FAKE, 0, 64, 256, 256, ctypes.byref(t), 0, FAKE, 256, None))
+    assert st == 1  # shape differs from out
+
+
+def test_gemm_validation():
+    L = nv.lib()
+    A, B = _tensor(128, 256), _tensor(64, 512)
+    st, msg = _err(L.w4a4_gemm(ctypes.byref(A), ctypes.byref(B), FAKE, 64, None))
+    assert st == 1 and "K" in msg
+    B = _tensor(66, 256)
+    st, _ = _err(L.w4a4_gemm(ctypes.byref(A), ctypes.byref(B), FAKE, 68, None))
+    assert st == 2
+    B = _tensor(64, 256)
+    st, _ = _err(L.w4a4_gemm(ctypes.byref(A), ctypes.byref(B), FAKE, 62, None))
+    assert st == 1
+    st, _ = _err(L.w4a4_gemm(ctypes.byref(A), ctypes.byref(B), FAKE + 4, 64, None))
+    assert st == 3
+    A = _tensor(128, 256, codes=FAKE + 8)
+    st, _ = _err(L.w4a4_gemm(ctypes.byref(A), ctypes.byref(B), FAKE, 64, None))
+    assert st == 3
+    A = _tensor(128, 256, sf=0)
+    st, _ = _err(L.w4a4_gemm(ctypes.byref(A), ctypes.byref(B), FAKE, 64, None))
+    assert st == 1
+
+
+def test_gates_and_scan_validation():
+    L = nv.lib()
+    d = nv.GdnDims(16, 32, 128, 128).c()
+    n_in = 2 * 16 * 128 + 2 * 32 * 128 + 64
+    st, _ = _err(L.gdn_gates(FAKE, n_in - 4, 10, ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None))
+    assert st == 1
+    bad = nv.GdnDims(16, 32, 96, 128).c()
+    st, _ = _err(L.gdn_gates(FAKE, n_in, 10, ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None))
+    assert st == 2
+    st, _ = _err(L.gdn_scan(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 64, ctypes.byref(d), 0.1, 5, 0, None, None, FAKE,
+                            FAKE, 1 << 30, None))
+    assert st == 1
+    st, _ = _err(L.gdn_scan(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 4096, ctypes.byref(d), 0.1, 0, 2, None, None, FAKE,
+                            None, 0, None))
+    assert st == 6
+    st, _ = _err(L.gdn_scan(FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 64, ctypes.byref(d), 0.1, 0, 0, None, None, FAKE,
+                            FAKE, 1 << 30, None))
+    assert st == 1
+
+
+def test_layer_layout_and_validation():
+    L = nv.lib()
+    dims = nv.GdnDims(16, 32, 128, 128)
+    w_in = nv.NVFP4Matrix(None, None, None, dims.n_in, 5120)
+    lw = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120)
+    lay = nv._Layout()
+    assert L.gdn_layer_workspace_layout(ctypes.byref(lw), 1, 4096, ctypes.byref(lay)) == 0
+    assert lay.proj > lay.x_scale and lay.total > lay.scan_ws
+    assert all(getattr(lay, f) % 256 == 0 for f in nv._LAYOUT_FIELDS)
+    assert lay.q_hat - lay.proj >= 4096 * 12352 * 4
+    lw_bad = nv._LayerWeights(_tensor(dims.n_in - 64, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120)
+    st, msg = _err(L.gdn_layer_workspace_layout(ctypes.byref(lw_bad), 1, 4096, ctypes.byref(lay)))
+    assert st == 1 and "w_in" in msg
+    st, _ = _err(L.gdn_layer_forward(ctypes.byref(lw), FAKE, 1, 4096, FAKE, None, None, 0, FAKE, 10, None))
+    assert st == 6
+    st, _ = _err(L.gdn_layer_forward(ctypes.byref(lw), FAKE, 1, 4096, FAKE, None, None, 3, FAKE, 1 << 40, None))
+    assert st == 1
+    del w_in

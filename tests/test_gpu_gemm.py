@@ -1,0 +1,114 @@
+"""tcgen05 block-scaled FP4 GEMM vs the oracle's float64 product of the
+dequantised operands: relative Frobenius error <= 1e-3 (and no element off by
+more than 1e-3 of the largest output)."""
+import numpy as np
+import pytest
+import torch
+
+import gdn_synth
+import nvfp4_w4a4_gated_b200 as nv
+import oracle
+from gpu_util import rel_fro, upload_oracle_nvfp4
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+def _operands(seed, M, N, K, slices=None, gains=None):
+    _, x = gdn_synth.activations(seed, M, K, hot="percent")
+    W = gdn_synth.weights(seed + 1, N, K, slice_rows=slices, slice_gain=gains)
+    return oracle.quantize(x), oracle.quantize(W)
+
+
+def _run(Aq, Bq, M, N, K, ldc=None):
+    A = upload_oracle_nvfp4(Aq, M, K)
+    B = upload_oracle_nvfp4(Bq, N, K)
+    C = None
+    if ldc is not None:
+        C = torch.full((M, ldc), float("nan"), dtype=torch.float32, device="cuda")
+        nv.w4a4_gemm(A, B, C)
+    else:
+        C = nv.w4a4_gemm(A, B)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    return C.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 256),      # one tile
+    (64, 516, 256),       # tiny in_proj: ragged M, N = 516 (two partial N tiles)
+    (64, 256, 128),       # tiny out_proj: K shorter than one k-tile
+    (200, 1000, 320),     # ragged M, N, K % 256 == 64
+    (384, 768, 1024),     # several tiles in both dimensions
+    (1, 64, 64),          # smallest legal problem
+    (1000, 1536, 640),    # many tiles per CTA
+])
+def test_gemm_matches_oracle(cuda_dev, M, N, K):
+    Aq, Bq = _operands(M + N + K, M, N, K)
+    got = _run(Aq, Bq, M, N, K)
+    ref = oracle.w4a4_gemm(Aq, Bq)
+    assert rel_fro(got, ref) <= TOL
+    assert np.max(np.abs(got - ref)) <= TOL * np.max(np.abs(ref))
+
+
+def test_gemm_writes_only_its_columns(cuda_dev):
+    M, N, K = 130, 260, 256
+    Aq, Bq = _operands(3, M, N, K)
+    got = _run(Aq, Bq, M, N, K, ldc=300)
+    assert np.all(np.isnan(got[:, N:]))
+    ref = oracle.w4a4_gemm(Aq, Bq)
+    assert rel_fro(got[:, :N], ref) <= TOL
+
+
+def test_gemm_harmonised_fused_slices(cuda_dev):
+    """Fused GEMM of a weight quantised as one tensor (one global scale) equals
+    the per-slice GEMMs under that scale; the per-module scale mismatch, if
+    served through the fused kernel, is caught (review page, paper sec.6)."""
+    sl, gain = (128, 128, 256), (1.0, 4.0, 2.0)
+    M, K = 96, 512
+    _, x = gdn_synth.activations(31, M, K, hot="percent")
+    W = gdn_synth.weights(32, sum(sl), K, slice_rows=sl, slice_gain=gain)
+    Aq = oracle.quantize(x)
+    Wq = oracle.quantize(W)
+    fused = _run(Aq, Wq, M, sum(sl), K)
+    r0 = 0
+    for n in sl:
+        part = oracle.quantize(W[r0:r0 + n], S=Wq[2])
+        got = _run(Aq, part, M, n, K)
+        assert rel_fro(got, fused[:, r0:r0 + n]) <= 1e-6
+        r0 += n
+    # mismatch: slice 1 quantised under its own scale but served with slice 0's
+    own0 = oracle.quantize(W[:128])
+    own1 = oracle.quantize(W[128:256])
+    bad = _run(Aq, (own1[0], own1[1], own0[2]), M, 128, K)
+    good = _run(Aq, own1, M, 128, K)
+    assert rel_fro(bad, good) > 0.5
+
+
+def test_gemm_full_size_sampled_rows(cuda_dev):
+    """The standalone workload M=8192, N=12288 (q|k|v|z slices 2048|2048|4096|4096,
+    module amax 4x apart), K=5120, in the launch configuration the benchmark
+    times; 48 sampled rows checked against the float64 oracle."""
+    M, N, K = 8192, 12288, 5120
+    bits, x = gdn_synth.activations(1, M, K, hot="percent")
+    W = gdn_synth.weights(2, N, K, slice_rows=gdn_synth.GEMM_SLICES, slice_gain=gdn_synth.GEMM_SLICE_GAIN)
+    Aq = oracle.quantize(x)
+    Wq = oracle.quantize(W)
+    got = _run(Aq, Wq, M, N, K)
+    rows = np.unique(np.concatenate([np.arange(8), gdn_synth.rng(5).integers(0, M, 32), np.arange(M - 8, M)]))
+    Ad = oracle.dequantize(Aq[0][rows], Aq[1][rows], Aq[2])
+    Bd = oracle.dequantize(*Wq)
+    ref = oracle.gemm_nt(Ad, Bd)
+    assert rel_fro(got[rows], ref) <= TOL
+    assert np.all(np.isfinite(got))
+
+
+def test_gemm_decode_shape(cuda_dev):
+    """Decode-step shape: 64 tokens against the fused in_proj [12352 x 5120]."""
+    sh = gdn_synth.FULL
+    M, N, K = 64, sh.n_in, sh.H
+    Aq, Bq = _operands(44, M, N, K)
+    got = _run(Aq, Bq, M, N, K)
+    ref = oracle.w4a4_gemm(Aq, Bq)
+    assert rel_fro(got, ref) <= TOL
