@@ -1,0 +1,544 @@
+"""Benchmark: one Gated DeltaNet layer forward under NVFP4 W4A4 (prefill).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one "step"): gdn_layer_forward over B=1, T=4096 tokens of a layer
+with hidden 5120, 16 key / 32 value heads, head dims 128 (fused in_proj
+N_in = 12352, out_proj 5120 x 4096), synthetic seeded inputs (outlier-heavy
+bf16 activations, N(0, 0.02) weights quantised once to NVFP4, untimed).  The
+step covers every stage of the path: activation quantisation, fused in_proj
+GEMM, gates + q/k normalisation, chunked delta-rule scan, o quantisation,
+out_proj GEMM.  L2 (126 MB) is flushed by a 256 MB write before every timed
+step; each step is timed with CUDA events on the launching stream.
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
+replica of the workload (the layer does not shard at this size; weak scaling)
+and the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN-layer W4A4 prefill tokens/s; FP4 GEMM TFLOPS and % NVFP4/HBM roofline"
+UNIT = "tokens/s"
+WORKLOAD = "gdn_layer_prefill_B1_T4096_h5120_hk16_hv32_k128_v128"
+NVFP4_OVER_BF16 = 4.0   # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+
+# launches of this library's kernels per gdn_layer_forward (T > 1): quantise x (amax, quant),
+# in_proj GEMM, gates (norm, gate), scan (prep, sequential), quantise o (amax, quant), out_proj GEMM
+LAUNCHES_PER_STEP = 10
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi samples of this GPU's SM clock and throttle reasons."""
+    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) != len(self.FIELDS):
+                continue
+            if self.uuid and f[0] != self.uuid:
+                continue
+            try:
+                sm.append(float(f[1].split()[0]))
+                smax.append(float(f[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- workload -----
+def make_layer(dev, seed):
+    import gdn_synth
+    import nvfp4_w4a4_gated_b200 as nv
+    sh = gdn_synth.FULL
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+    W_in = gdn_synth.weights(seed + 100, sh.n_in, sh.H)
+    W_out = gdn_synth.weights(seed + 101, sh.H, sh.Hv * sh.V)
+    A_log, dt_bias = gdn_synth.gate_params(seed + 102, sh.Hv, 0.0, math.log(16.0))
+    dims = nv.GdnDims(sh.Hk, sh.Hv, sh.K, sh.V)
+    w = nv.LayerWeights(nv.nvfp4_quantize(f32(W_in)), nv.nvfp4_quantize(f32(W_out)), f32(A_log), f32(dt_bias),
+                        dims, sh.H)
+    return w, sh
+
+
+def stage_work(sh, B, T):
+    """Algorithmic work per stage of one step (bytes for HBM-bound stages,
+    flops for the GEMMs): the per-unit figures times the units one launch
+    processes."""
+    BT = B * T
+    HvV, HkK = sh.Hv * sh.V, sh.Hk * sh.K
+    return {
+        "quant_x": ("hbm", BT * sh.H * (2 + 0.5 + 1 / 16)),
+        "gemm_in": ("tensor", 2.0 * BT * sh.n_in * sh.H),
+        "gates": ("hbm", BT * (2 * HkK * 4 + 2 * sh.Hv * 4 + 2 * HkK * 4 + 2 * sh.Hv * 4)),
+        "scan": ("hbm", BT * (2 * HkK * 4 + HvV * 4 + 2 * sh.Hv * 4 + HvV * 4) + 2 * B * sh.Hv * sh.K * sh.V * 4),
+        "quant_o": ("hbm", BT * HvV * (4 + 0.5 + 1 / 16)),
+        "gemm_out": ("tensor", 2.0 * BT * sh.H * HvV),
+    }
+
+
+STAGE_KERNELS = {"quant_x": "quant_kernel<bf16> (+amax)", "gemm_in": "w4a4_gemm_kernel", "gates": "l2norm+gate",
+                 "scan": "chunk_prep_kernel + chunk_seq_kernel", "quant_o": "quant_kernel<f32> (+amax)",
+                 "gemm_out": "w4a4_gemm_kernel"}
+
+
+def run_stages(nv, w, x, B, T, ws, lay, y, stream, events=None):
+    """The layer forward as its six library calls (the same launches, in the
+    same order, as gdn_layer_forward), optionally with an event after each."""
+    import ctypes
+    L = nv.lib()
+    sh = w.dims
+    base = ws.data_ptr()
+    BT, H, HvV = B * T, w.hidden, sh.Hv * sh.V
+    ldp = (sh.n_in + 3) // 4 * 4
+    xq = nv._Tensor(base + lay["x_codes"], base + lay["x_sf"], base + lay["x_scale"], BT, H)
+    oq = nv._Tensor(base + lay["o_codes"], base + lay["o_sf"], base + lay["o_scale"], BT, HvV)
+    s = ctypes.c_void_p(stream.cuda_stream)
+    P = base + lay["proj"]
+    d = sh.c()
+    win, wout = w.w_in.c(), w.w_out.c()
+
+    def ev(i):
+        if events is not None:
+            events[i].record(stream)
+
+    ev(0)
+    nv._check(L.nvfp4_quantize(ctypes.c_void_p(x.data_ptr()), 0, BT, H, H, ctypes.byref(xq), 0,
+                               ctypes.c_void_p(base + lay["quant_ws"]), 256, s))
+    ev(1)
+    nv._check(L.w4a4_gemm(ctypes.byref(xq), ctypes.byref(win), ctypes.c_void_p(P), ldp, s))
+    ev(2)
+    nv._check(L.gdn_gates(ctypes.c_void_p(P), ldp, BT, ctypes.byref(d), ctypes.c_void_p(w.A_log.data_ptr()),
+                          ctypes.c_void_p(w.dt_bias.data_ptr()), ctypes.c_void_p(base + lay["q_hat"]),
+                          ctypes.c_void_p(base + lay["k_hat"]), ctypes.c_void_p(base + lay["g"]),
+                          ctypes.c_void_p(base + lay["beta"]), s))
+    ev(3)
+    scan_ws = L.gdn_scan_workspace_size(B, T, ctypes.byref(d), 0)
+    nv._check(L.gdn_scan(ctypes.c_void_p(base + lay["q_hat"]), ctypes.c_void_p(base + lay["k_hat"]),
+                         ctypes.c_void_p(P + 2 * sh.Hk * sh.K * 4), ldp, ctypes.c_void_p(base + lay["g"]),
+                         ctypes.c_void_p(base + lay["beta"]), B, T, ctypes.byref(d), 1.0 / math.sqrt(sh.K), 0, 0,
+                         None, None, ctypes.c_void_p(base + lay["o"]), ctypes.c_void_p(base + lay["scan_ws"]),
+                         scan_ws, s))
+    ev(4)
+    nv._check(L.nvfp4_quantize(ctypes.c_void_p(base + lay["o"]), 1, BT, HvV, HvV, ctypes.byref(oq), 0,
+                               ctypes.c_void_p(base + lay["quant_ws"]), 256, s))
+    ev(5)
+    nv._check(L.w4a4_gemm(ctypes.byref(oq), ctypes.byref(wout), ctypes.c_void_p(y.data_ptr()), H, s))
+    ev(6)
+
+
+def traffic_for(stage: str):
+    """DRAM bytes per launch of the stage's dominant kernel from the committed
+    ncu summary (profiles/dram_traffic.txt), or None when absent or when the
+    kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src_of = {"gemm_in": "gemm.cu", "gemm_out": "gemm.cu", "scan": "scan.cu", "quant_x": "quantize.cu",
+              "quant_o": "quantize.cu", "gates": "gates.cu"}
+    src = os.path.join(ROOT, "nvfp4_w4a4_gated_b200", "csrc", src_of[stage])
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for ln in open(p):
+        f = ln.split()
+        if len(f) >= 3 and not ln.startswith("#") and f[0] == stage:
+            return float(f[1]) if f[2] == sha else None
+    return None
+
+
+def cpu_baseline(sample_tokens: int, seed: int):
+    """The oracle, as it stands, on a prefix of the same workload's sequence."""
+    import gdn_synth
+    import oracle
+    sh = gdn_synth.FULL
+    W_in = gdn_synth.weights(seed + 100, sh.n_in, sh.H)
+    W_out = gdn_synth.weights(seed + 101, sh.H, sh.Hv * sh.V)
+    A_log, dt_bias = gdn_synth.gate_params(seed + 102, sh.Hv, 0.0, math.log(16.0))
+    Wid = oracle.dequantize(*oracle.quantize(W_in))
+    Wod = oracle.dequantize(*oracle.quantize(W_out))
+    _, x = gdn_synth.activations(seed, 4096, sh.H, hot="percent")
+    xs = x[:sample_tokens]
+    t0 = time.perf_counter()
+    oracle.layer_forward(xs, None, None, A_log, dt_bias, 1, sample_tokens, sh.Hk, sh.Hv, sh.K, sh.V, W_in_deq=Wid,
+                         W_out_deq=Wod)
+    dt = time.perf_counter() - t0
+    return {"value": sample_tokens / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {sample_tokens} of the 4096 tokens (B=1), full layer width, float64 oracle; "
+                      f"weights dequantised before timing", "seconds": dt}
+
+
+# ------------------------------------------------------------- our arm -----
+def run_ours(args, rank, world, local_rank):
+    import nvfp4_w4a4_gated_b200 as nv
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = world > 1
+    seed = 2 + rank
+    B, T = 1, 4096
+    w, sh = make_layer(dev, seed)
+    import gdn_synth
+    bits, _ = gdn_synth.activations(seed, B * T, sh.H, hot="percent")
+    x = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    y = torch.empty((B * T, sh.H), dtype=torch.float32, device=dev)
+    lay = nv.layer_workspace_layout(w, B, T)
+    ws = torch.empty(lay["total"], dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nv.gdn_layer_forward(w, x, B, T, y=y, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    nv.check_device_error()
+
+    # ---- timed region: K steps of gdn_layer_forward, L2 flushed before each
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+
+    # ---- the same step as its six calls, an event after each: per-stage times
+    nstage = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        run_stages(nv, w, x, B, T, ws, lay, y, stream, evs[i])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    nv.check_device_error()
+    names = ["quant_x", "gemm_in", "gates", "scan", "quant_o", "gemm_out"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(names)}
+
+    # ---- standalone GEMM workload (M=8192, N=12288, K=5120), TFLOPS
+    gemm = bench_gemm(nv, dev, args.steps, flush, stream)
+
+    # ---- end to end through the public call with host buffers
+    x_host = torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(x.cpu())
+    y_host = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    x_dev2 = torch.empty_like(x)
+    for i in range(args.steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        x_dev2.copy_(x_host, non_blocking=True)
+        nv.gdn_layer_forward(w, x_dev2, B, T, y=y, workspace=ws, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+
+    # ---- aggregate over ranks: max time
+    tvec = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        torch.distributed.all_reduce(tvec, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms = float(tvec[0]), float(tvec[1])
+    tokens = world * B * T * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    pk = peaks()
+    work = stage_work(sh, B, T)
+    dom = max(stage_ms, key=stage_ms.get)
+    bound, units = work[dom]
+    if bound == "tensor":
+        peak = pk["bf16_tflops"] * NVFP4_OVER_BF16
+        achieved = units / (stage_ms[dom] / 1e3) / 1e12
+        unit, peak_note = "TFLOP/s", f"{pk['source']} bf16 burst x {NVFP4_OVER_BF16:g} (nominal FP4:BF16)"
+    else:
+        peak = pk["hbm_gbs"]
+        achieved = units / (stage_ms[dom] / 1e3) / 1e9
+        unit, peak_note = "GB/s", f"{pk['source']} HBM copy"
+    traffic = traffic_for(dom)
+    stages = {}
+    for n in names:
+        b, u = work[n]
+        if b == "tensor":
+            stages[n] = {"ms": round(stage_ms[n], 4), "TFLOP/s": round(u / (stage_ms[n] / 1e3) / 1e12, 1),
+                         "frac": round(u / (stage_ms[n] / 1e3) / 1e12 / (pk["bf16_tflops"] * NVFP4_OVER_BF16), 3)}
+        else:
+            stages[n] = {"ms": round(stage_ms[n], 4), "GB/s": round(u / (stage_ms[n] / 1e3) / 1e9, 1),
+                         "frac": round(u / (stage_ms[n] / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4(e2m1,e4m3)+f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "T": T, "hidden": sh.H, "Hk": sh.Hk, "Hv": sh.Hv, "K": sh.K,
+                   "V": sh.V, "n_in": sh.n_in, "form": "pages", "scan": "chunked C=64",
+                   "l2": "flushed (256 MB write) before every timed step", "replicas": world},
+        "roofline": {"bound": bound, "kernel": f"{dom}: {STAGE_KERNELS[dom]}", "achieved": round(achieved, 1),
+                     "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_source": peak_note},
+        "stages": stages,
+        "gemm_standalone": gemm,
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk,
+    }
+    return out
+
+
+def bench_gemm(nv, dev, steps, flush, stream):
+    """Standalone block-scaled GEMM, M=8192, N=12288 (q|k|v|z slices with 4x
+    module amax spread, one harmonised scale), K=5120, fp32 C."""
+    import gdn_synth
+    M, N, K = 8192, 12288, 5120
+    bits, _ = gdn_synth.activations(1, M, K, hot="percent")
+    Wt = gdn_synth.weights(2, N, K, slice_rows=gdn_synth.GEMM_SLICES, slice_gain=gdn_synth.GEMM_SLICE_GAIN)
+    xa = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    A = nv.nvfp4_quantize(xa)
+    Bm = nv.nvfp4_quantize(torch.from_numpy(Wt).to(dev))
+    C = torch.empty((M, N), dtype=torch.float32, device=dev)
+    for _ in range(3):
+        nv.w4a4_gemm(A, Bm, C, stream=stream)
+    qa = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ts = []
+    for i in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        nv.w4a4_gemm(A, Bm, C, stream=stream)
+        e.record(stream)
+        ts.append((s, e))
+    # quantiser on the same activation (HBM-bound)
+    qt = []
+    for i in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        nv.nvfp4_quantize(xa, out=A, stream=stream)
+        e.record(stream)
+        qt.append((s, e))
+    torch.cuda.synchronize()
+    ms = statistics.mean(s.elapsed_time(e) for s, e in ts)
+    qms = statistics.mean(s.elapsed_time(e) for s, e in qt)
+    pk = peaks()
+    tflops = 2.0 * M * N * K / (ms / 1e3) / 1e12
+    qgbs = M * K * 2.5625 / (qms / 1e3) / 1e9
+    del qa
+    return {"workload": "gemm_M8192_N12288_K5120_fp32out", "ms": round(ms, 4), "TFLOP/s": round(tflops, 1),
+            "frac_of_nvfp4_peak": round(tflops / (pk["bf16_tflops"] * NVFP4_OVER_BF16), 4),
+            "quantize_8192x5120_bf16": {"ms": round(qms, 4), "GB/s": round(qgbs, 1),
+                                         "frac_of_hbm": round(qgbs / pk["hbm_gbs"], 4)}}
+
+
+# ------------------------------------------------------ reference arm -----
+def run_reference(args):
+    """The oracle as the reference implementation, timed on the host cores:
+    each step is the layer forward over a bounded prefix of the workload."""
+    import gdn_synth
+    import oracle
+    sh = gdn_synth.FULL
+    seed = 2
+    sample = args.ref_tokens
+    W_in = gdn_synth.weights(seed + 100, sh.n_in, sh.H)
+    W_out = gdn_synth.weights(seed + 101, sh.H, sh.Hv * sh.V)
+    A_log, dt_bias = gdn_synth.gate_params(seed + 102, sh.Hv, 0.0, math.log(16.0))
+    Wid = oracle.dequantize(*oracle.quantize(W_in))
+    Wod = oracle.dequantize(*oracle.quantize(W_out))
+    _, x = gdn_synth.activations(seed, 4096, sh.H, hot="percent")
+    xs = x[:sample]
+
+    def step():
+        oracle.layer_forward(xs, None, None, A_log, dt_bias, 1, sample, sh.Hk, sh.Hv, sh.K, sh.V, W_in_deq=Wid,
+                             W_out_deq=Wod)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = sample * args.steps / dt
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (quantiser exact f32)",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": 1, "T": 4096, "hidden": sh.H, "Hk": sh.Hk, "Hv": sh.Hv,
+                       "K": sh.K, "V": sh.V, "sample_tokens_per_step": sample},
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"first {sample} tokens of the T=4096 workload per step"},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def kernel_case(args):
+    """One kernel on a fixed-size case, a few launches, for profiler captures
+    (ncu -k <kernel> -c <n>); prints the mean launch time."""
+    import nvfp4_w4a4_gated_b200 as nv
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    stream = torch.cuda.current_stream(dev)
+    if args.kernel_case == "gemm":
+        M, N, K = args.M, args.N, args.K
+        A = nv.nvfp4_quantize(torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16))
+        Bm = nv.nvfp4_quantize(torch.randn((N, K), generator=g, device=dev) * 0.02)
+        C = torch.empty((M, N), dtype=torch.float32, device=dev)
+        fn = lambda: nv.w4a4_gemm(A, Bm, C)
+    elif args.kernel_case == "quant":
+        x = torch.randn((args.M, args.K), generator=g, device=dev).to(torch.bfloat16)
+        out = nv.NVFP4Matrix.empty(args.M, args.K, dev)
+        fn = lambda: nv.nvfp4_quantize(x, out=out)
+    elif args.kernel_case == "scan":
+        B, T, Hk, Hv, Kd = 1, args.T, 16, 32, 128
+        dims = nv.GdnDims(Hk, Hv, Kd, Kd)
+        qh = torch.nn.functional.normalize(torch.randn((B * T, Hk, Kd), generator=g, device=dev), dim=-1)
+        kh = torch.nn.functional.normalize(torch.randn((B * T, Hk, Kd), generator=g, device=dev), dim=-1)
+        v = torch.randn((B * T, Hv * Kd), generator=g, device=dev)
+        gg = torch.log(torch.rand((B * T, Hv), generator=g, device=dev) * 0.5 + 0.5)
+        bt = torch.rand((B * T, Hv), generator=g, device=dev)
+        o = torch.empty((B * T, Hv, Kd), device=dev)
+        ws = torch.empty(nv.lib().gdn_scan_workspace_size(B, T, __import__("ctypes").byref(dims.c()), 0),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: nv.gdn_scan(qh, kh, v, gg, bt, B, T, dims, o=o, workspace=ws)
+    else:
+        raise SystemExit("unknown kernel case")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    print(json.dumps({"kernel_case": args.kernel_case, "ms_per_launch": s.elapsed_time(e) / args.steps,
+                      "M": args.M, "N": args.N, "K": args.K, "T": args.T}))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    ap.add_argument("--ref-tokens", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan"], default=None,
+                    help="profile helper: run one kernel on a fixed case and exit")
+    ap.add_argument("--M", type=int, default=8192)
+    ap.add_argument("--N", type=int, default=12288)
+    ap.add_argument("--K", type=int, default=5120)
+    ap.add_argument("--T", type=int, default=4096)
+    args = ap.parse_args(argv)
+    if args.kernel_case:
+        kernel_case(args)
+        return 0
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(args.cpu_sample_tokens, 2)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

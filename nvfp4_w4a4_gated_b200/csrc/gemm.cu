@@ -16,7 +16,9 @@
 //               (M=128, N=BN, K=64 each) accumulate in TMEM; tcgen05.commit
 //               frees the stage and, after the last k-tile, signals the tile;
 //   warps 2..5  epilogue: tcgen05.ld of the f32 accumulator (warp w reads
-//               TMEM lanes 32*(w%4)...), scale by S_A*S_B, 16-byte stores.
+//               TMEM lanes 32*(w%4)...), scale by S_A*S_B, write 32 x 32
+//               sub-tiles to shared memory (128-byte swizzle) and TMA-store
+//               them, so every global write is a full 128-byte row segment.
 // Two accumulator buffers of BN columns; for BN = 256 they overlap in 64
 // columns (TMEM holds 512) and the epilogue drains the shared chunk first, so
 // the next tile's MMAs start after one chunk and the rest of the drain overlaps
@@ -36,28 +38,38 @@ constexpr int SFB_COL = 464;       // 4 k-blocks x (BN/128 x 4) columns
 
 template <int BN>
 struct Cfg {
-    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int STAGES = BN == 256 ? 3 : 5;
     static constexpr int A_BYTES = BM * K_TILE_BYTES;
     static constexpr int B_BYTES = BN * K_TILE_BYTES;
     static constexpr int SFA_BYTES = 4 * 512;
     static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
     static constexpr int ACC_OFF = (2 * BN <= SFA_COL) ? BN : SFA_COL - BN;  // start column of buffer 1
     static constexpr int NCHUNK = BN / 64;
+    static constexpr int STG_BYTES = 4 * 2 * 32 * 32 * 4;  // per epilogue warp: two 32 x 32 f32 sub-tiles
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + BAR_BYTES + 1024;
+    static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + STG_BYTES + BAR_BYTES + 1024;
     static constexpr uint32_t IDESC = idesc_nvf4(BM, BN);
 };
 
-__device__ __forceinline__ void st_global_v4(float* p, float a, float b, float c, float d) {
-    asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+// Write 32 consecutive f32 values of row `lane` into a 32 x 32 sub-tile laid out
+// with the 128-byte swizzle the C tensor map expects (16-byte chunk c of row r
+// at chunk position c ^ (r % 8)); scaled by alpha.
+__device__ __forceinline__ void stage_row(float* tile, int lane, const uint32_t (&v)[32], float alpha) {
+    char* row = reinterpret_cast<char*>(tile) + lane * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        float4 f = make_float4(alpha * __uint_as_float(v[4 * c]), alpha * __uint_as_float(v[4 * c + 1]),
+                               alpha * __uint_as_float(v[4 * c + 2]), alpha * __uint_as_float(v[4 * c + 3]));
+        *reinterpret_cast<float4*>(row + ((c ^ (lane & 7)) << 4)) = f;
+    }
 }
 
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const uint8_t* __restrict__ sfA, const uint8_t* __restrict__ sfB,
-                     const float* __restrict__ scaleA, const float* __restrict__ scaleB, float* __restrict__ C,
-                     int64_t ldc, int M, int N, int K, unsigned int* __restrict__ err) {
+                     const __grid_constant__ CUtensorMap tmC, const uint8_t* __restrict__ sfA,
+                     const uint8_t* __restrict__ sfB, const float* __restrict__ scaleA,
+                     const float* __restrict__ scaleB, int M, int N, int K, unsigned int* __restrict__ err) {
     using G = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -65,7 +77,8 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* sB = sA + G::STAGES * G::A_BYTES;
     uint8_t* sSFA = sB + G::STAGES * G::B_BYTES;
     uint8_t* sSFB = sSFA + G::STAGES * G::SFA_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + G::STAGES * G::SFB_BYTES);
+    float* sStage = reinterpret_cast<float*>(sSFB + G::STAGES * G::SFB_BYTES);  // 1024-byte aligned
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sStage) + G::STG_BYTES);
     uint64_t* empty = full + G::STAGES;
     uint64_t* acc_full = empty + G::STAGES;
     uint64_t* tmem_free = acc_full + 1;
@@ -94,6 +107,7 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        prefetch_tmap(&tmC);
     }
     tc_fence_before();
     __syncthreads();
@@ -182,14 +196,14 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------------------------------------------------- epilogue --
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const float alpha = __fmul_rn(*scaleA, *scaleB);
+        float* stg = sStage + (warp - 2) * 2 * 32 * 32;
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             const int m_idx = tile % num_m, n_idx = tile / num_m;
             const int buf = local & 1;
             if (!mbar_wait(acc_full, local & 1, err, kErrTimeoutEpi)) break;
             tc_fence_after();
-            const int row = m_idx * BM + q * 32 + lane;
-            float* crow = C + (int64_t)row * ldc;
+            const int row0 = m_idx * BM + q * 32;
 #pragma unroll 1
             for (int ci = 0; ci < G::NCHUNK; ++ci) {
                 // buffer 0 of the overlapping pair drains its shared (last) chunk first
@@ -204,27 +218,22 @@ __global__ void __launch_bounds__(192, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(tmem_free);
                 }
-                if (row < M) {
-                    const int col0 = n_idx * BN + c * 64;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int col = col0 + 4 * i;
-                        if (col < N)
-                            st_global_v4(crow + col, alpha * __uint_as_float(v0[4 * i]),
-                                         alpha * __uint_as_float(v0[4 * i + 1]), alpha * __uint_as_float(v0[4 * i + 2]),
-                                         alpha * __uint_as_float(v0[4 * i + 3]));
-                    }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int col = col0 + 32 + 4 * i;
-                        if (col < N)
-                            st_global_v4(crow + col, alpha * __uint_as_float(v1[4 * i]),
-                                         alpha * __uint_as_float(v1[4 * i + 1]), alpha * __uint_as_float(v1[4 * i + 2]),
-                                         alpha * __uint_as_float(v1[4 * i + 3]));
-                    }
+                // the staging tiles are free once the previous chunk's stores have read them
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+                stage_row(stg, lane, v0, alpha);
+                stage_row(stg + 32 * 32, lane, v1, alpha);
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int col0 = n_idx * BN + c * 64;
+                if (lane == 0 && row0 < M) {
+                    tma_store_2d(&tmC, stg, col0, row0);
+                    if (col0 + 32 < N) tma_store_2d(&tmC, stg + 32 * 32, col0 + 32, row0);
+                    bulk_commit();
                 }
             }
         }
+        if (lane == 0) bulk_wait<0>();
     }
 
     tc_fence_before();
@@ -239,10 +248,12 @@ template <int BN>
 nvfp4_status launch_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C, int64_t ldc, cudaStream_t st) {
     using G = Cfg<BN>;
     const int M = static_cast<int>(A.rows), N = static_cast<int>(B.rows), K = static_cast<int>(A.cols);
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     nvfp4_status s = make_tmap_u8_sw128(&ta, A.codes, A.rows, A.cols / 2, BM, K_TILE_BYTES);
     if (s != NVFP4_OK) return s;
     s = make_tmap_u8_sw128(&tb, B.codes, B.rows, B.cols / 2, BN, K_TILE_BYTES);
+    if (s != NVFP4_OK) return s;
+    s = make_tmap_f32_sw128(&tc, C, A.rows, B.rows, ldc, 32, 32);
     if (s != NVFP4_OK) return s;
     static bool attr_done[64] = {false};
     int dev = 0;
@@ -257,8 +268,8 @@ nvfp4_status launch_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C,
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_kernel<BN><<<grid, 192, G::SMEM, st>>>(ta, tb, A.sf, B.sf, A.global_scale, B.global_scale, C, ldc, M, N,
-                                                     K, err);
+    w4a4_gemm_kernel<BN><<<grid, 192, G::SMEM, st>>>(ta, tb, tc, A.sf, B.sf, A.global_scale, B.global_scale, M, N, K,
+                                                     err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm launch");
     return NVFP4_OK;

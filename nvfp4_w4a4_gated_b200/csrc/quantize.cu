@@ -84,21 +84,41 @@ __device__ __forceinline__ void unpack16B(const uint4& u, float* out, const floa
 }
 
 // Pass 1: amax over the matrix into *amax_bits (float bits of a non-negative
-// value, so unsigned order is float order).
+// value, so unsigned order is float order).  Each thread keeps four 16-byte
+// loads in flight per iteration.
 template <typename T>
 __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                                                    unsigned int* __restrict__ amax_bits) {
     constexpr int P = Vec<T>::kPer16B;
+    constexpr int U = 4;
     const int64_t vec_per_row = cols / P;
     const int64_t nvec = rows * vec_per_row;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     float m = 0.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (; i + (U - 1) * stride < nvec; i += U * stride) {
+        uint4 u[U];
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const int64_t ii = i + j * stride;
+            const int64_t r = ii / vec_per_row, c = (ii - r * vec_per_row) * P;
+            u[j] = __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
+        }
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            float f[8];
+            unpack16B(u[j], f, x);
+#pragma unroll
+            for (int e = 0; e < P; ++e) m = fmaxf(m, fabsf(f[e]));
+        }
+    }
+    for (; i < nvec; i += stride) {
         const int64_t r = i / vec_per_row, c = (i - r * vec_per_row) * P;
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
         float f[8];
         unpack16B(u, f, x);
 #pragma unroll
-        for (int j = 0; j < P; ++j) m = fmaxf(m, fabsf(f[j]));
+        for (int e = 0; e < P; ++e) m = fmaxf(m, fabsf(f[e]));
     }
     unsigned int b = __float_as_uint(m);
     b = __reduce_max_sync(0xffffffffu, b);
@@ -175,7 +195,7 @@ nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(amax)");
         const int64_t elems_per_vec = x_dtype == NVFP4_DTYPE_BF16 ? 8 : 4;
         const int64_t nvec = rows * (cols / elems_per_vec);
-        int64_t blocks = (nvec + 255) / 256;
+        int64_t blocks = (nvec + 1023) / 1024;
         const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
         if (blocks > cap) blocks = cap;
         if (x_dtype == NVFP4_DTYPE_BF16)

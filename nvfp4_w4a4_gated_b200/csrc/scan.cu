@@ -127,11 +127,12 @@ __device__ __forceinline__ void mma_f32(float (&d)[4], const float (&a)[4], cons
 // One CTA (256 threads) per (sequence, chunk, value head).
 template <int K, int V>
 struct PrepSmem {
-    static constexpr int KS = K + 4;  // row stride of K/Q tiles (== 4 mod 32)
+    // row stride of the K and Q tiles (== 4 mod 32); the Q tile later holds beta*V rows
+    static constexpr int KS = (K > V ? K : V) + 4;
     float ks[CH * KS];
     float qs[CH * KS];
     float L[CH * CH];
-    float gin[CH], gd[CH], bet[CH], graw[CH];
+    float gin[CH], gd[CH], bet[CH], graw[CH], df[CH];
 };
 
 template <int K, int V>
@@ -218,37 +219,61 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 if (warp < 4) {
                     sm.L[t * CH + i] = (i < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
                 } else {
-                    Mt[mbase + t * CH + i] = (i <= t) ? expf(sm.gin[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
+                    // stored already rounded to TF32: it is only ever a tensor-core operand
+                    const float mv = (i <= t) ? expf(sm.gin[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
+                    Mt[mbase + t * CH + i] = __uint_as_float(to_tf32(mv));
                 }
             }
         }
     }
-    if (tid < CH) Gt[((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH + tid] = sm.gin[tid];
+    if (tid < CH) {
+        Gt[((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH + tid] = sm.gin[tid];
+        sm.df[tid] = sm.bet[tid] * expf(sm.gd[tid]);
+    }
+    __syncthreads();
+    // Q is no longer needed: its tile now holds beta_t v_t, the U~ right-hand sides
+    constexpr int VV4 = V / 4;
+    for (int idx = tid; idx < CH * VV4; idx += 256) {
+        const int r = idx / VV4, c4 = idx - r * VV4;
+        float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < n) {
+            vv = *reinterpret_cast<const float4*>(v + (static_cast<int64_t>(b) * T + t0 + r) * ld_v +
+                                                  static_cast<int64_t>(h) * V + c4 * 4);
+            const float bt = sm.bet[r];
+            vv.x *= bt; vv.y *= bt; vv.z *= bt; vv.w *= bt;
+        }
+        *reinterpret_cast<float4*>(&sm.qs[r * KS + c4 * 4]) = vv;
+    }
     __syncthreads();
 
-    // forward substitution, one right-hand-side column per thread:
-    // columns [0, K) give W~ (rhs b_t e^{Gd_t} k_t), columns [K, K+V) give U~ (rhs beta_t v_t)
+    // forward substitution (I + L) X = RHS, one right-hand-side column per thread:
+    // columns [0, K) give W~ (rhs b_t e^{Gd_t} k_t), columns [K, K+V) give U~ (rhs beta_t v_t).
+    // L rows are read four at a time (broadcast) into four independent partial sums.
     if (tid < K + V) {
         const bool isW = tid < K;
         const int col = isW ? tid : tid - K;
         float x[CH];
 #pragma unroll
-        for (int t = 0; t < CH; ++t) {
-            float r;
-            if (isW) {
-                r = sm.bet[t] * expf(sm.gd[t]) * sm.ks[t * KS + col];
-            } else {
-                r = t < n ? sm.bet[t] * v[(static_cast<int64_t>(b) * T + t0 + t) * ld_v + static_cast<int64_t>(h) * V + col]
-                          : 0.0f;
-            }
+        for (int t = 0; t < CH; ++t) x[t] = 0.0f;
 #pragma unroll
-            for (int i = 0; i < t; ++i) r = fmaf(-sm.L[t * CH + i], x[i], r);
-            x[t] = r;
+        for (int t = 0; t < CH; ++t) {
+            float r0 = isW ? sm.df[t] * sm.ks[t * KS + col] : sm.qs[t * KS + col];
+            float r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll
+            for (int i4 = 0; i4 < (t + 3) / 4; ++i4) {
+                const float4 l = *reinterpret_cast<const float4*>(&sm.L[t * CH + 4 * i4]);
+                r0 = fmaf(-l.x, x[4 * i4], r0);
+                r1 = fmaf(-l.y, x[4 * i4 + 1], r1);
+                r2 = fmaf(-l.z, x[4 * i4 + 2], r2);
+                r3 = fmaf(-l.w, x[4 * i4 + 3], r3);
+            }
+            x[t] = (r0 + r1) + (r2 + r3);
         }
         const int64_t cb = (static_cast<int64_t>(b) * Hv + h) * NC + c;
         if (isW) {
+            // W~ is only a tensor-core operand downstream: store it rounded to TF32
 #pragma unroll
-            for (int t = 0; t < CH; ++t) Wt[(cb * CH + t) * K + col] = x[t];
+            for (int t = 0; t < CH; ++t) Wt[(cb * CH + t) * K + col] = __uint_as_float(to_tf32(x[t]));
         } else {
 #pragma unroll
             for (int t = 0; t < CH; ++t) Ut[(cb * CH + t) * V + col] = x[t];
@@ -263,13 +288,13 @@ struct SeqSmem {
     static constexpr int KS = K + 8;   // K tile row stride (== 8 mod 32, transposed reads)
     static constexpr int MS = CH + 4;  // masked Q K^T row stride
     static constexpr int SS = 40;      // state / U row stride (== 8 mod 32)
-    float x1[2 * CH * XS];
-    float kc[CH * KS];
-    float mc[CH * MS];
-    float s[K * SS];
-    float u[CH * SS];
-    float ud[CH * SS];
-    float gin[CH];
+    float x1[2 * CH * XS];             // rows 0..63: W~ (TF32-rounded), rows 64..127: Q
+    float kc[2][CH * KS];              // K of this chunk and the next one
+    float mc[2][CH * MS];              // masked decayed Q K^T (TF32-rounded), double-buffered
+    float s[K * SS];                   // float32 state slice [K x 32]
+    float u[CH * SS];                  // U (TF32-rounded)
+    float ud[CH * SS];                 // U scaled by e^{G_C - G_i} (TF32-rounded)
+    float gin[2][CH];
 };
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
@@ -283,7 +308,12 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // One CTA (256 threads) per (sequence, value head, 32-column slice of V).
-template <int K, bool PREC3>
+// Per chunk: P1 = [W~; Q] S on all 8 warps (warps 0-3: W~ S, warps 4-7: Q S);
+// warps 0-3 form U = U~ - W~ S; warps 4-7 then form o = scale (e^G Q S + M U)
+// while every warp advances its 16 state rows S <- e^{G_C} S + K^T (decayed U).
+// K, M and G of chunk c+1 are prefetched at the start of chunk c, W~ and Q of
+// chunk c+1 as soon as P1 of chunk c has consumed them.
+template <int K>
 __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict__ q, const float* __restrict__ k,
                                                         int64_t T, int Hk, int Hv, int V, float scale, int NC,
                                                         const float* __restrict__ Wt, const float* __restrict__ Ut,
@@ -320,30 +350,48 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
             cp_async16(&sm.x1[(CH + r) * XS + c4 * 4], q + qoff, valid);
         }
     };
-    auto load_km = [&](int c) {
+    auto load_km = [&](int c, int buf) {
         const int64_t t0 = static_cast<int64_t>(c) * CH;
         constexpr int V4 = K / 4;
         for (int idx = tid; idx < CH * V4; idx += 256) {
             const int r = idx / V4, c4 = idx - r * V4;
             const bool valid = t0 + r < T;
             const int64_t koff = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
-            cp_async16(&sm.kc[r * KS + c4 * 4], k + koff, valid);
+            cp_async16(&sm.kc[buf][r * KS + c4 * 4], k + koff, valid);
         }
         for (int idx = tid; idx < CH * CH / 4; idx += 256) {
             const int r = idx >> 4, c4 = idx & 15;
-            cp_async16(&sm.mc[r * MS + c4 * 4], Mt + ((hc + c) * CH + r) * CH + c4 * 4, true);
+            cp_async16(&sm.mc[buf][r * MS + c4 * 4], Mt + ((hc + c) * CH + r) * CH + c4 * 4, true);
         }
-        if (tid < CH / 4) cp_async16(&sm.gin[tid * 4], Gt + (hc + c) * CH + tid * 4, true);
+        if (tid < CH / 4) cp_async16(&sm.gin[buf][tid * 4], Gt + (hc + c) * CH + tid * 4, true);
     };
 
     load_wq(0);
-    load_km(0);
+    load_km(0, 0);
     cp_async_commit();
 
     for (int c = 0; c < NC; ++c) {
         const int64_t t0 = static_cast<int64_t>(c) * CH;
+        const int buf = c & 1;
         cp_async_wait<0>();
         __syncthreads();
+        if (c + 1 < NC) {
+            load_km(c + 1, buf ^ 1);
+            cp_async_commit();
+        }
+        // U~ for this warp's rows, fetched now so the latency hides behind P1
+        float ut[4][4];
+        if (warp < 4) {
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i = warp * 16 + grp + hh * 8;
+                    const float2 v2 = *reinterpret_cast<const float2*>(Ut + ((hc + c) * CH + i) * V + vs0 + nt * 8 + 2 * tig);
+                    ut[nt][2 * hh] = v2.x;
+                    ut[nt][2 * hh + 1] = v2.y;
+                }
+        }
 
         // P1: [W~; Q] (128 x K) times S (K x 32); warp w owns rows 16w..16w+15
         float acc[4][4];
@@ -351,30 +399,39 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
         for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         {
             const int r0 = warp * 16;
+            const bool a_rounded = warp < 4;  // W~ rows arrive rounded to TF32
 #pragma unroll 4
             for (int k0 = 0; k0 < K; k0 += 8) {
-                const float a[4] = {sm.x1[(r0 + grp) * XS + k0 + tig], sm.x1[(r0 + grp + 8) * XS + k0 + tig],
-                                    sm.x1[(r0 + grp) * XS + k0 + tig + 4], sm.x1[(r0 + grp + 8) * XS + k0 + tig + 4]};
+                const float af[4] = {sm.x1[(r0 + grp) * XS + k0 + tig], sm.x1[(r0 + grp + 8) * XS + k0 + tig],
+                                     sm.x1[(r0 + grp) * XS + k0 + tig + 4], sm.x1[(r0 + grp + 8) * XS + k0 + tig + 4]};
+                uint32_t a[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] = a_rounded ? __float_as_uint(af[i]) : to_tf32(af[i]);
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    const float bb[2] = {sm.s[(k0 + tig) * SS + nt * 8 + grp], sm.s[(k0 + tig + 4) * SS + nt * 8 + grp]};
-                    mma_f32<PREC3>(acc[nt], a, bb);
+                    const uint32_t bb[2] = {to_tf32(sm.s[(k0 + tig) * SS + nt * 8 + grp]),
+                                            to_tf32(sm.s[(k0 + tig + 4) * SS + nt * 8 + grp])};
+                    mma_tf32(acc[nt], a, bb);
                 }
             }
         }
-        const float glast = sm.gin[CH - 1];
+        const float glast = sm.gin[buf][CH - 1];
         if (warp < 4) {
-            // U = U~ - W~ S0; also U scaled by e^{G_C - G_i} for the state update
+            // U = U~ - W~ S0, and U decayed by e^{G_C - G_i} for the state update
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = warp * 16 + grp + hh * 8;
+                const float dec = expf(glast - sm.gin[buf][i]);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = warp * 16 + grp + (e >> 1) * 8;
-                    const int col = nt * 8 + 2 * tig + (e & 1);
-                    const float ut = Ut[((hc + c) * CH + i) * V + vs0 + col];
-                    const float uval = ut - acc[nt][e];
-                    sm.u[i * SS + col] = uval;
-                    sm.ud[i * SS + col] = expf(glast - sm.gin[i]) * uval;
+                for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                    for (int e1 = 0; e1 < 2; ++e1) {
+                        const int e = 2 * hh + e1;
+                        const int col = nt * 8 + 2 * tig + e1;
+                        const float uval = ut[nt][e] - acc[nt][e];
+                        sm.u[i * SS + col] = __uint_as_float(to_tf32(uval));
+                        sm.ud[i * SS + col] = __uint_as_float(to_tf32(dec * uval));
+                    }
                 }
             }
         }
@@ -388,31 +445,35 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
         if (warp >= 4) {
             // o = scale * (e^{G_t} Q S0 + Mqk U); rows t = 16(w-4)..
             const int r0 = (warp - 4) * 16;
+            const float* mc = sm.mc[buf];
             float mu[4][4];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) mu[nt][0] = mu[nt][1] = mu[nt][2] = mu[nt][3] = 0.f;
 #pragma unroll
             for (int k0 = 0; k0 < CH; k0 += 8) {
-                const float a[4] = {sm.mc[(r0 + grp) * MS + k0 + tig], sm.mc[(r0 + grp + 8) * MS + k0 + tig],
-                                    sm.mc[(r0 + grp) * MS + k0 + tig + 4], sm.mc[(r0 + grp + 8) * MS + k0 + tig + 4]};
+                const uint32_t a[4] = {__float_as_uint(mc[(r0 + grp) * MS + k0 + tig]),
+                                       __float_as_uint(mc[(r0 + grp + 8) * MS + k0 + tig]),
+                                       __float_as_uint(mc[(r0 + grp) * MS + k0 + tig + 4]),
+                                       __float_as_uint(mc[(r0 + grp + 8) * MS + k0 + tig + 4])};
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    const float bb[2] = {sm.u[(k0 + tig) * SS + nt * 8 + grp], sm.u[(k0 + tig + 4) * SS + nt * 8 + grp]};
-                    mma_f32<false>(mu[nt], a, bb);
+                    const uint32_t bb[2] = {__float_as_uint(sm.u[(k0 + tig) * SS + nt * 8 + grp]),
+                                            __float_as_uint(sm.u[(k0 + tig + 4) * SS + nt * 8 + grp])};
+                    mma_tf32(mu[nt], a, bb);
                 }
             }
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+            for (int hh = 0; hh < 2; ++hh) {
+                const int t = r0 + grp + hh * 8;
+                if (t0 + t < T) {
+                    const float eg = expf(sm.gin[buf][t]);
+                    float* orow = o + ((static_cast<int64_t>(b) * T + t0 + t) * Hv + h) * V + vs0;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int t = r0 + grp + hh * 8;
-                    if (t0 + t < T) {
-                        const float eg = expf(sm.gin[t]);
+                    for (int nt = 0; nt < 4; ++nt) {
                         const int col = nt * 8 + 2 * tig;
-                        const float o0 = scale * fmaf(eg, acc[nt][2 * hh], mu[nt][2 * hh]);
-                        const float o1 = scale * fmaf(eg, acc[nt][2 * hh + 1], mu[nt][2 * hh + 1]);
-                        *reinterpret_cast<float2*>(o + ((static_cast<int64_t>(b) * T + t0 + t) * Hv + h) * V + vs0 + col) =
-                            make_float2(o0, o1);
+                        *reinterpret_cast<float2*>(orow + col) =
+                            make_float2(scale * fmaf(eg, acc[nt][2 * hh], mu[nt][2 * hh]),
+                                        scale * fmaf(eg, acc[nt][2 * hh + 1], mu[nt][2 * hh + 1]));
                     }
                 }
             }
@@ -422,6 +483,7 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
         if (warp * 16 < K) {
             const int d0 = warp * 16;
             const float eg = expf(glast);
+            const float* kc = sm.kc[buf];
             float st[4][4];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
@@ -433,12 +495,14 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
             }
 #pragma unroll
             for (int k0 = 0; k0 < CH; k0 += 8) {
-                const float a[4] = {sm.kc[(k0 + tig) * KS + d0 + grp], sm.kc[(k0 + tig) * KS + d0 + grp + 8],
-                                    sm.kc[(k0 + tig + 4) * KS + d0 + grp], sm.kc[(k0 + tig + 4) * KS + d0 + grp + 8]};
+                const uint32_t a[4] = {to_tf32(kc[(k0 + tig) * KS + d0 + grp]), to_tf32(kc[(k0 + tig) * KS + d0 + grp + 8]),
+                                       to_tf32(kc[(k0 + tig + 4) * KS + d0 + grp]),
+                                       to_tf32(kc[(k0 + tig + 4) * KS + d0 + grp + 8])};
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt) {
-                    const float bb[2] = {sm.ud[(k0 + tig) * SS + nt * 8 + grp], sm.ud[(k0 + tig + 4) * SS + nt * 8 + grp]};
-                    mma_f32<PREC3>(st[nt], a, bb);
+                    const uint32_t bb[2] = {__float_as_uint(sm.ud[(k0 + tig) * SS + nt * 8 + grp]),
+                                            __float_as_uint(sm.ud[(k0 + tig + 4) * SS + nt * 8 + grp])};
+                    mma_tf32(st[nt], a, bb);
                 }
             }
 #pragma unroll
@@ -451,10 +515,6 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
             }
         }
         __syncthreads();
-        if (c + 1 < NC) {
-            load_km(c + 1);
-            cp_async_commit();
-        }
     }
     cp_async_wait<0>();
     __syncthreads();
@@ -500,7 +560,7 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
         cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prep)");
-        e = cudaFuncSetAttribute(chunk_seq_kernel<K, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
+        e = cudaFuncSetAttribute(chunk_seq_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq)");
         attr_done[dev] = true;
     }
@@ -508,7 +568,7 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, ws.Wt,
                                                                  ws.Ut, ws.Mt, ws.Gt);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    chunk_seq_kernel<K, false><<<seq_blocks, 256, seq_smem, st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt, ws.Ut,
+    chunk_seq_kernel<K><<<seq_blocks, 256, seq_smem, st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt, ws.Ut,
                                                                   ws.Mt, ws.Gt, s_in, s_out, o);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");

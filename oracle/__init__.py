@@ -241,13 +241,19 @@ def split_projection(P: np.ndarray, Hk: int, Hv: int, K: int, V: int):
 
 
 def layer_forward(x: np.ndarray, W_in_q, W_out_q, A_log, dt_bias, B: int, T: int, Hk: int, Hv: int,
-                  K: int, V: int, form=FORM_PAGES, S0=None, stages: bool = False):
+                  K: int, V: int, form=FORM_PAGES, S0=None, stages: bool = False, W_in_deq=None,
+                  W_out_deq=None):
     """The four steps composed.  x: float32 [B*T, H] (bf16 values);
     W_in_q, W_out_q: (codes, sf_linear, S) of the fused in_proj [N_in, H] and
-    out_proj [H, Hv*V].  Returns y [B*T, H] float64 and the final state (and
-    every intermediate when ``stages``)."""
+    out_proj [H, Hv*V] (or their dequantised float64 matrices in W_in_deq /
+    W_out_deq, to skip re-dequantising fixed weights).  Returns y [B*T, H]
+    float64 and the final state (and every intermediate when ``stages``)."""
     xq = quantize(x)                                            # step 1
-    P = w4a4_gemm(xq, W_in_q)                                   # step 2
+    if W_in_deq is None:
+        W_in_deq = dequantize(*W_in_q)
+    if W_out_deq is None:
+        W_out_deq = dequantize(*W_out_q)
+    P = gemm_nt(dequantize(*xq), W_in_deq)                      # step 2
     q, k, v, _z, a, b = split_projection(P, Hk, Hv, K, V)
     g, beta = gates(a, b, A_log, dt_bias)                       # step 3
     qh = l2norm(q.reshape(B, T, Hk, K))
@@ -256,7 +262,7 @@ def layer_forward(x: np.ndarray, W_in_q, W_out_q, A_log, dt_bias, B: int, T: int
                 form=form, S0=S0)                               # step 4
     o2 = o.reshape(B * T, Hv * V).astype(np.float32)            # the out_proj reads fp32 o
     oq = quantize(o2)
-    y = w4a4_gemm(oq, W_out_q)
+    y = gemm_nt(dequantize(*oq), W_out_deq)
     if stages:
         return dict(xq=xq, P=P, g=g, beta=beta, q_hat=qh, k_hat=kh, o=o, S=S, oq=oq, y=y)
     return y, S
