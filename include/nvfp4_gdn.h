@@ -171,6 +171,34 @@ NVFP4_API nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const fl
                       float* state_out, float* o, void* workspace, size_t workspace_bytes,
                       nvfp4_stream_t stream);
 
+/* No counterpart in the paper: an allocation-free variant of gdn_scan for
+ * callers that cannot allocate device memory themselves -- for example a
+ * plugin inside a host framework that owns every allocation, or code running
+ * while a stream is captured into a CUDA graph, where a cudaMalloc would break
+ * the capture.  It runs the chunked algorithm (GDN_SCAN_CHUNKED) exactly as
+ * gdn_scan does, with every argument meaning the same, but keeps the scratch in
+ * a fixed array inside the library instead of a caller-provided workspace.
+ * The array holds GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES bytes on each GPU that
+ * uses it and is kept until the process exits.  It calls no cudaMalloc /
+ * cudaFree and no allocating library routine.
+ *   - Size limit: a problem whose scratch, gdn_scan_workspace_size(B, T, dims,
+ *     GDN_SCAN_CHUNKED), exceeds the array is rejected with
+ *     NVFP4_ERR_WORKSPACE before anything is launched (64 MiB covers, e.g.,
+ *     B = 1, 32 value heads of 128 x 128, T <= 1600).
+ *   - First use: the first call on a device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture begins.
+ *   - Sharing: every call on a device uses the same array and leaves its
+ *     contents behind (the chunk preparation overwrites all of it, nothing has
+ *     to start at zero).  Calls whose executions overlap on the GPU -- on
+ *     different streams, or from different host threads -- race on the array
+ *     and give wrong results; serialise them. */
+#define GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES ((size_t)64 << 20) /* 64 MiB */
+NVFP4_API nvfp4_status gdn_scan_noalloc(const float* q_hat, const float* k_hat, const float* v, int64_t ld_v,
+                                        const float* g, const float* beta, int32_t B, int64_t T,
+                                        const gdn_dims* dims, float scale, int32_t form, const float* state_in,
+                                        float* state_out, float* o, nvfp4_stream_t stream);
+
 /* ---------------------------------------------------------------- layer -- */
 typedef struct {
     nvfp4_tensor w_in;    /* [N_in x hidden], N_in = 2*Hk*K + 2*Hv*V + 2*Hv, one global scale */

@@ -19,7 +19,7 @@ from . import build as _build
 
 __all__ = [
     "NVFP4Error", "NVFP4Matrix", "GdnDims", "LayerWeights", "lib", "nvfp4_quantize", "w4a4_gemm", "gdn_gates",
-    "gdn_scan", "gdn_layer_forward", "layer_workspace_layout", "check_device_error", "FORM_PAGES",
+    "gdn_scan", "gdn_scan_noalloc", "gdn_layer_forward", "layer_workspace_layout", "check_device_error", "FORM_PAGES",
     "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
 ]
 
@@ -33,8 +33,11 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4:
 EXPORTED_SYMBOLS = [
     "nvfp4_last_error", "nvfp4_check_device_error", "nvfp4_version", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_size", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan_workspace_size",
-    "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward",
+    "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc",
 ]
+
+# Size of the fixed scratch array gdn_scan_noalloc uses (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
+NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
 
 
 class NVFP4Error(RuntimeError):
@@ -91,10 +94,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_scan_workspace_size.argtypes = [i32, i64, DP, i32]
         L.gdn_scan_workspace_size.restype = sz
         L.gdn_scan.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, i32, P, P, P, P, sz, P]
+        L.gdn_scan_noalloc.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, P, P, P, P]
         L.gdn_layer_workspace_layout.argtypes = [ctypes.POINTER(_LayerWeights), i32, i64, ctypes.POINTER(_Layout)]
         L.gdn_layer_forward.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, i32, P, sz, P]
         for f in ("nvfp4_check_device_error", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
-                  "gdn_layer_workspace_layout", "gdn_layer_forward"):
+                  "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -243,6 +247,22 @@ def gdn_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: flo
     _check(lib().gdn_scan(_ptr(q_hat), _ptr(k_hat), _ptr(v), ld_v, _ptr(g), _ptr(beta), B, T, ctypes.byref(d),
                           float(scale), form, algo, _ptr(state_in), _ptr(state_out), _ptr(o), _ptr(workspace),
                           0 if workspace is None else workspace.numel(), _stream(stream)))
+    return o, state_out
+
+
+def gdn_scan_noalloc(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
+                     form: int = FORM_PAGES, state_in=None, state_out=None, o=None, stream=None):
+    """Chunked scan with the library's own fixed scratch array (no workspace
+    argument, nothing allocated by the library)."""
+    dev = q_hat.device
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.K)
+    if o is None:
+        o = torch.empty((B * T, dims.Hv, dims.V), dtype=torch.float32, device=dev)
+    d = dims.c()
+    _check(lib().gdn_scan_noalloc(_ptr(q_hat), _ptr(k_hat), _ptr(v), v.stride(0), _ptr(g), _ptr(beta), B, T,
+                                  ctypes.byref(d), float(scale), form, _ptr(state_in), _ptr(state_out), _ptr(o),
+                                  _stream(stream)))
     return o, state_out
 
 
