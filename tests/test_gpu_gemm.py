@@ -15,6 +15,17 @@ pytestmark = pytest.mark.gpu
 TOL = 1e-3
 
 
+@pytest.fixture(params=["auto", "pair", "single", "narrow"])
+def variant(request, monkeypatch):
+    """Kernel variant: CTA-pair 256x256, single-CTA 128x256, single-CTA 128x128,
+    or the library's own choice by shape."""
+    if request.param != "auto":
+        monkeypatch.setenv("NVFP4_GEMM_VARIANT", request.param)
+    else:
+        monkeypatch.delenv("NVFP4_GEMM_VARIANT", raising=False)
+    return request.param
+
+
 def _operands(seed, M, N, K, slices=None, gains=None):
     _, x = gdn_synth.activations(seed, M, K, hot="percent")
     W = gdn_synth.weights(seed + 1, N, K, slice_rows=slices, slice_gain=gains)
@@ -44,7 +55,7 @@ def _run(Aq, Bq, M, N, K, ldc=None):
     (1, 64, 64),          # smallest legal problem
     (1000, 1536, 640),    # many tiles per CTA
 ])
-def test_gemm_matches_oracle(cuda_dev, M, N, K):
+def test_gemm_matches_oracle(cuda_dev, variant, M, N, K):
     Aq, Bq = _operands(M + N + K, M, N, K)
     got = _run(Aq, Bq, M, N, K)
     ref = oracle.w4a4_gemm(Aq, Bq)
@@ -52,7 +63,7 @@ def test_gemm_matches_oracle(cuda_dev, M, N, K):
     assert np.max(np.abs(got - ref)) <= TOL * np.max(np.abs(ref))
 
 
-def test_gemm_writes_only_its_columns(cuda_dev):
+def test_gemm_writes_only_its_columns(cuda_dev, variant):
     M, N, K = 130, 260, 256
     Aq, Bq = _operands(3, M, N, K)
     got = _run(Aq, Bq, M, N, K, ldc=300)
@@ -86,7 +97,7 @@ def test_gemm_harmonised_fused_slices(cuda_dev):
     assert rel_fro(bad, good) > 0.5
 
 
-def test_gemm_full_size_sampled_rows(cuda_dev):
+def test_gemm_full_size_sampled_rows(cuda_dev, variant):
     """The standalone workload M=8192, N=12288 (q|k|v|z slices 2048|2048|4096|4096,
     module amax 4x apart), K=5120, in the launch configuration the benchmark
     times; 48 sampled rows checked against the float64 oracle."""
