@@ -21,6 +21,9 @@
 //    Q K^T and G; kernel 2 (one CTA per head x 32-column V slice) walks the
 //    chunks in order.  Products run on the tensor cores in TF32 with float32
 //    accumulation (mma.sync m16n8k8).
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 
 namespace nvg {
@@ -123,17 +126,75 @@ __device__ __forceinline__ void mma_f32(float (&d)[4], const float (&a)[4], cons
     }
 }
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------ chunk preparation --
 // One CTA (256 threads) per (sequence, chunk, value head).
 template <int K, int V>
 struct PrepSmem {
-    // row stride of the K and Q tiles (== 4 mod 32); the Q tile later holds beta*V rows
+    // row stride of the K and Q tiles (== 4 mod 32); the Q tile later holds the V rows
     static constexpr int KS = (K > V ? K : V) + 4;
+    static constexpr int TS = CH + 4;  // row stride of T (== 4 mod 32)
     float ks[CH * KS];
     float qs[CH * KS];
-    float L[CH * CH];
+    float L[CH * CH];                  // strictly lower, scaled: b_t e^{Gd_t - G_i} k_t.k_i
+    float T[CH * TS];                  // (I + L)^-1
+    float P[3 * 256];                  // 16 x 16 block products
     float gin[CH], gd[CH], bet[CH], graw[CH], df[CH];
 };
+
+// Output tile X [64 x 8*NT] = (T diag(s)) B with B [64 x 8*NT] (row stride KS) in
+// shared memory; warp rows r0..r0+15; 3xTF32 (hi/lo split) so the product is
+// float32-accurate.  X is written to global rows of `out` (row stride 8*NT),
+// rounded to TF32 when `round_out`.
+template <int NT, int KS, int TS>
+__device__ __forceinline__ void tri_apply(const float* __restrict__ Tm, const float* __restrict__ s,
+                                          const float* __restrict__ Bm, int r0, int lane, float* __restrict__ out,
+                                          bool round_out) {
+    const int grp = lane >> 2, tig = lane & 3;
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+    for (int k0 = 0; k0 < CH; k0 += 8) {
+        const float s0 = s[k0 + tig], s1 = s[k0 + tig + 4];
+        const float af[4] = {Tm[(r0 + grp) * TS + k0 + tig] * s0, Tm[(r0 + grp + 8) * TS + k0 + tig] * s0,
+                             Tm[(r0 + grp) * TS + k0 + tig + 4] * s1, Tm[(r0 + grp + 8) * TS + k0 + tig + 4] * s1};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_tf32(af[i], ah[i], al[i]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            uint32_t bh[2], bl[2];
+            split_tf32(Bm[(k0 + tig) * KS + nt * 8 + grp], bh[0], bl[0]);
+            split_tf32(Bm[(k0 + tig + 4) * KS + nt * 8 + grp], bh[1], bl[1]);
+            mma_tf32(acc[nt], al, bh);
+            mma_tf32(acc[nt], ah, bl);
+            mma_tf32(acc[nt], ah, bh);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int t = r0 + grp + hh * 8;
+            float x0 = acc[nt][2 * hh], x1 = acc[nt][2 * hh + 1];
+            if (round_out) {
+                x0 = __uint_as_float(to_tf32(x0));
+                x1 = __uint_as_float(to_tf32(x1));
+            }
+            *reinterpret_cast<float2*>(out + t * (8 * NT) + nt * 8 + 2 * tig) = make_float2(x0, x1);
+        }
+    }
+}
 
 template <int K, int V>
 __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict__ q, const float* __restrict__ k,
@@ -154,24 +215,22 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     const int n = static_cast<int>((T - t0) < CH ? (T - t0) : CH);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // load K, Q rows (zero past the end of the sequence), g and beta
+    // K, Q rows (zero past the end of the sequence) by asynchronous copies, g and beta
     constexpr int V4 = K / 4;
     for (int idx = tid; idx < CH * V4; idx += 256) {
         const int r = idx / V4, c4 = idx - r * V4;
-        float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv;
-        if (r < n) {
-            const int64_t off = ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4;
-            kv = *reinterpret_cast<const float4*>(k + off);
-            qv = *reinterpret_cast<const float4*>(q + off);
-        }
-        *reinterpret_cast<float4*>(&sm.ks[r * KS + c4 * 4]) = kv;
-        *reinterpret_cast<float4*>(&sm.qs[r * KS + c4 * 4]) = qv;
+        const bool valid = r < n;
+        const int64_t off = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
+        cp_async16(&sm.ks[r * KS + c4 * 4], k + off, valid);
+        cp_async16(&sm.qs[r * KS + c4 * 4], q + off, valid);
     }
+    cp_async_commit();
     if (tid < CH) {
         const int64_t gi = (static_cast<int64_t>(b) * T + t0 + tid) * Hv + h;
         sm.graw[tid] = tid < n ? g[gi] : 0.0f;
         sm.bet[tid] = tid < n ? beta[gi] : 0.0f;
     }
+    cp_async_wait<0>();
     __syncthreads();
     if (warp == 0) {
         // inclusive prefix sum of g over the chunk (2 values per lane)
@@ -230,55 +289,65 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         Gt[((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH + tid] = sm.gin[tid];
         sm.df[tid] = sm.bet[tid] * expf(sm.gd[tid]);
     }
+    constexpr int TS = SM::TS;
+    for (int idx = tid; idx < CH * TS; idx += 256) sm.T[idx] = 0.0f;
     __syncthreads();
-    // Q is no longer needed: its tile now holds beta_t v_t, the U~ right-hand sides
+    // Q is no longer needed: its tile now receives the V rows (zero past the sequence
+    // end); the copies land while the triangular inverse is formed
     constexpr int VV4 = V / 4;
     for (int idx = tid; idx < CH * VV4; idx += 256) {
         const int r = idx / VV4, c4 = idx - r * VV4;
-        float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < n) {
-            vv = *reinterpret_cast<const float4*>(v + (static_cast<int64_t>(b) * T + t0 + r) * ld_v +
-                                                  static_cast<int64_t>(h) * V + c4 * 4);
-            const float bt = sm.bet[r];
-            vv.x *= bt; vv.y *= bt; vv.z *= bt; vv.w *= bt;
+        const bool valid = r < n;
+        const int64_t off = valid ? (static_cast<int64_t>(b) * T + t0 + r) * ld_v + static_cast<int64_t>(h) * V + c4 * 4 : 0;
+        cp_async16(&sm.qs[r * KS + c4 * 4], v + off, valid);
+    }
+    cp_async_commit();
+
+    // T = (I + L)^-1, blockwise.  Diagonal 16 x 16 blocks by substitution
+    // (warp w < 4 takes block w, lane c < 16 column c); then block rows
+    // i = 1..3: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj.
+    if (warp < 4 && lane < 16) {
+        const int o = warp * 16;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == lane) ? 1.0f : 0.0f;
+#pragma unroll
+            for (int i = 0; i < r; ++i) acc = fmaf(-sm.L[(o + r) * CH + o + i], x[i], acc);
+            x[r] = acc;
         }
-        *reinterpret_cast<float4*>(&sm.qs[r * KS + c4 * 4]) = vv;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sm.T[(o + r) * TS + o + lane] = x[r];
     }
     __syncthreads();
-
-    // forward substitution (I + L) X = RHS, one right-hand-side column per thread:
-    // columns [0, K) give W~ (rhs b_t e^{Gd_t} k_t), columns [K, K+V) give U~ (rhs beta_t v_t).
-    // L rows are read four at a time (broadcast) into four independent partial sums.
-    if (tid < K + V) {
-        const bool isW = tid < K;
-        const int col = isW ? tid : tid - K;
-        float x[CH];
-#pragma unroll
-        for (int t = 0; t < CH; ++t) x[t] = 0.0f;
-#pragma unroll
-        for (int t = 0; t < CH; ++t) {
-            float r0 = isW ? sm.df[t] * sm.ks[t * KS + col] : sm.qs[t * KS + col];
-            float r1 = 0.f, r2 = 0.f, r3 = 0.f;
-#pragma unroll
-            for (int i4 = 0; i4 < (t + 3) / 4; ++i4) {
-                const float4 l = *reinterpret_cast<const float4*>(&sm.L[t * CH + 4 * i4]);
-                r0 = fmaf(-l.x, x[4 * i4], r0);
-                r1 = fmaf(-l.y, x[4 * i4 + 1], r1);
-                r2 = fmaf(-l.z, x[4 * i4 + 2], r2);
-                r3 = fmaf(-l.w, x[4 * i4 + 3], r3);
-            }
-            x[t] = (r0 + r1) + (r2 + r3);
+    for (int bi = 1; bi < 4; ++bi) {
+        for (int e = tid; e < bi * 256; e += 256) {
+            const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+            float acc = 0.0f;
+            for (int kk = 16 * j; kk < 16 * bi; ++kk)
+                acc = fmaf(sm.L[(16 * bi + r) * CH + kk], sm.T[kk * TS + 16 * j + cc], acc);
+            sm.P[e] = acc;
         }
-        const int64_t cb = (static_cast<int64_t>(b) * Hv + h) * NC + c;
-        if (isW) {
-            // W~ is only a tensor-core operand downstream: store it rounded to TF32
+        __syncthreads();
+        for (int e = tid; e < bi * 256; e += 256) {
+            const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+            float acc = 0.0f;
 #pragma unroll
-            for (int t = 0; t < CH; ++t) Wt[(cb * CH + t) * K + col] = __uint_as_float(to_tf32(x[t]));
-        } else {
-#pragma unroll
-            for (int t = 0; t < CH; ++t) Ut[(cb * CH + t) * V + col] = x[t];
+            for (int m = 0; m < 16; ++m) acc = fmaf(sm.T[(16 * bi + r) * TS + 16 * bi + m], sm.P[j * 256 + m * 16 + cc], acc);
+            sm.T[(16 * bi + r) * TS + 16 * j + cc] = -acc;
         }
+        __syncthreads();
     }
+
+    cp_async_wait<0>();
+    __syncthreads();
+    // W~ = T diag(b e^{Gd}) K (warps 0-3, stored TF32-rounded: a tensor-core operand downstream)
+    // U~ = T diag(beta) V   (warps 4-7)
+    const int64_t cb = (static_cast<int64_t>(b) * Hv + h) * NC + c;
+    if (warp < 4)
+        tri_apply<K / 8, KS, TS>(sm.T, sm.df, sm.ks, warp * 16, lane, Wt + cb * CH * K, true);
+    else
+        tri_apply<V / 8, KS, TS>(sm.T, sm.bet, sm.qs, (warp - 4) * 16, lane, Ut + cb * CH * V, false);
 }
 
 // ------------------------------------------------------ sequential chunks --
@@ -297,15 +366,6 @@ struct SeqSmem {
     float gin[2][CH];
 };
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // One CTA (256 threads) per (sequence, value head, 32-column slice of V).
 // Per chunk: P1 = [W~; Q] S on all 8 warps (warps 0-3: W~ S, warps 4-7: Q S);
@@ -526,6 +586,259 @@ __global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict_
     }
 }
 
+// ------------------------------------------- sequential chunks, tcgen05 --
+// Same per-chunk algebra as chunk_seq_kernel, on the sm_100 tensor cores: every
+// product reads its operands from shared memory (no-swizzle K-major canonical
+// tiles: 8-row x 16-byte core matrices) and accumulates in TMEM, so the warps
+// only move data between the two MMA rounds of a chunk:
+//   round 1:  D1 = [Q~; W~] S0            (M=128: rows 0..63 Q~ S0, 64..127 W~ S0)
+//   warps 2-3: U = U~ - W~ S0, Ud = diag(e^{G_C - G}) U  -> shared memory
+//   round 2:  D1 += [Mqk; *] U           (rows 0..63 become Q~ S0 + Mqk U;
+//                                          the W~ S0 rows receive garbage, unused)
+//             D2  = K^T Ud               (M=128 state rows)
+//   warps 0-1: o = scale * D1[0:64];  all: S <- e^{G_C} S + D2 (float32 registers)
+// Q~ = diag(e^{G}) Q is formed while rounding Q to TF32 in shared memory; K^T is
+// built from the staged K tile in the same pass.
+template <int K>
+struct SeqTcSmem {
+    static constexpr int A1_SBO = (K / 4) * 128;   // [Q~; W~] over the state dim: 8-row group stride
+    static constexpr int T_SBO = 16 * 128;         // tiles whose K extent is the 64 tokens
+    static constexpr int B1_SBO = (K / 4) * 128;   // S^T [32 x K]
+    float a1[128 * K];
+    float a2[2][64 * 64];                          // Mqk; a2[1] doubles as a2[0]'s unused upper rows
+    float kst[2][64 * K];                          // staged K rows [t][d]; kst[0] follows a2[1]
+    float a3[128 * 64];                            // K^T [d][t] (K = 64: upper half unused)
+    float b1[32 * K];                              // S^T [v][d]
+    float b2[32 * 64];                             // U^T [v][t]
+    float b3[32 * 64];                             // Ud^T
+    float gin[2][CH];
+    uint64_t bar[2];
+    uint32_t tmem_holder;
+};
+
+template <int K>
+__global__ void __launch_bounds__(128) chunk_seq_tc_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                                                           int64_t T, int Hk, int Hv, int V, float scale, int NC,
+                                                           const float* __restrict__ Wt, const float* __restrict__ Ut,
+                                                           const float* __restrict__ Mt, const float* __restrict__ Gt,
+                                                           const float* state_in, float* state_out,
+                                                           float* __restrict__ o, unsigned int* __restrict__ err) {
+    using SM = SeqTcSmem<K>;
+    extern __shared__ float4 smem_f4[];
+    SM& sm = *reinterpret_cast<SM*>(smem_f4);
+    const int nslice = V / 32;
+    const int slice = blockIdx.x % nslice;
+    const int h = (blockIdx.x / nslice) % Hv;
+    const int b = blockIdx.x / (nslice * Hv);
+    const int hk = static_cast<int>((static_cast<int64_t>(h) * Hk) / Hv);
+    const int vs0 = slice * 32;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
+    const int64_t hc = (static_cast<int64_t>(b) * Hv + h) * NC;
+    constexpr uint32_t IDESC = idesc_tf32(128, 32, false, false);
+
+    if (tid == 0) {
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_holder, 64);
+        tmem_relinquish();
+    }
+
+    // float offsets inside K-major canonical tiles: row r, column c, `cw` columns per row
+    auto kmaj = [](int r, int c, int cw) { return ((r >> 3) * (cw >> 2) + (c >> 2)) * 32 + (r & 7) * 4 + (c & 3); };
+
+    // state rows in registers: thread d < K holds S[d][vs0 .. vs0+31]
+    float S[32];
+    const bool has_row = tid < K;
+    if (has_row) {
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (state_in) x = *reinterpret_cast<const float4*>(state_in + sbase + static_cast<int64_t>(tid) * V + vs0 + 4 * v4);
+            S[4 * v4] = x.x; S[4 * v4 + 1] = x.y; S[4 * v4 + 2] = x.z; S[4 * v4 + 3] = x.w;
+        }
+#pragma unroll
+        for (int v = 0; v < 32; ++v) sm.b1[kmaj(v, tid, K)] = __uint_as_float(to_tf32(S[v]));
+    }
+
+    auto load_wq = [&](int c) {
+        const int64_t t0 = static_cast<int64_t>(c) * CH;
+        for (int idx = tid; idx < CH * (K / 4); idx += 128) {
+            const int t = idx / (K / 4), d4 = idx % (K / 4);
+            cp_async16(&sm.a1[kmaj(CH + t, 4 * d4, K)], Wt + ((hc + c) * CH + t) * K + 4 * d4, true);
+            const bool valid = t0 + t < T;
+            const int64_t qoff = valid ? ((static_cast<int64_t>(b) * T + t0 + t) * Hk + hk) * K + 4 * d4 : 0;
+            cp_async16(&sm.a1[kmaj(t, 4 * d4, K)], q + qoff, valid);
+        }
+    };
+    auto load_kmg = [&](int c, int buf) {
+        const int64_t t0 = static_cast<int64_t>(c) * CH;
+        for (int idx = tid; idx < CH * (K / 4); idx += 128) {
+            const int t = idx / (K / 4), d4 = idx % (K / 4);
+            const bool valid = t0 + t < T;
+            const int64_t koff = valid ? ((static_cast<int64_t>(b) * T + t0 + t) * Hk + hk) * K + 4 * d4 : 0;
+            cp_async16(&sm.kst[buf][t * K + 4 * d4], k + koff, valid);
+        }
+        for (int idx = tid; idx < CH * 16; idx += 128) {
+            const int t = idx >> 4, i4 = idx & 15;
+            cp_async16(&sm.a2[buf][kmaj(t, 4 * i4, CH)], Mt + ((hc + c) * CH + t) * CH + 4 * i4, true);
+        }
+        if (tid < CH / 4) cp_async16(&sm.gin[buf][4 * tid], Gt + (hc + c) * CH + 4 * tid, true);
+    };
+    float ut[32];
+    auto load_ut = [&](int c) {
+        if (warp >= 2) {
+            const float* src = Ut + ((hc + c) * CH + (tid - 64)) * V + vs0;
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4) {
+                const float4 x = *reinterpret_cast<const float4*>(src + 4 * v4);
+                ut[4 * v4] = x.x; ut[4 * v4 + 1] = x.y; ut[4 * v4 + 2] = x.z; ut[4 * v4 + 3] = x.w;
+            }
+        }
+    };
+
+    load_wq(0);
+    load_kmg(0, 0);
+    cp_async_commit();
+    load_ut(0);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_holder;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t D1 = tmem, D2 = tmem + 32;
+    bool ok = true;
+
+    for (int c = 0; c < NC && ok; ++c) {
+        const int buf = c & 1;
+        const int64_t t0 = static_cast<int64_t>(c) * CH;
+        cp_async_wait<0>();
+        __syncthreads();
+        // Q~ = e^{G_t} Q rounded to TF32 in place; K^T [d][t] built from the staged rows, rounded
+        for (int idx = tid; idx < CH * (K / 4); idx += 128) {
+            const int t = idx / (K / 4), d4 = idx % (K / 4);
+            float4* qp = reinterpret_cast<float4*>(&sm.a1[kmaj(t, 4 * d4, K)]);
+            const float eg = expf(sm.gin[buf][t]);
+            const float4 xq = *qp;
+            *qp = make_float4(__uint_as_float(to_tf32(eg * xq.x)), __uint_as_float(to_tf32(eg * xq.y)),
+                              __uint_as_float(to_tf32(eg * xq.z)), __uint_as_float(to_tf32(eg * xq.w)));
+            const float4 xk = *reinterpret_cast<const float4*>(&sm.kst[buf][t * K + 4 * d4]);
+            sm.a3[kmaj(4 * d4 + 0, t, CH)] = __uint_as_float(to_tf32(xk.x));
+            sm.a3[kmaj(4 * d4 + 1, t, CH)] = __uint_as_float(to_tf32(xk.y));
+            sm.a3[kmaj(4 * d4 + 2, t, CH)] = __uint_as_float(to_tf32(xk.z));
+            sm.a3[kmaj(4 * d4 + 3, t, CH)] = __uint_as_float(to_tf32(xk.w));
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (c + 1 < NC) {
+            load_kmg(c + 1, buf ^ 1);
+            cp_async_commit();
+        }
+        const float glast = sm.gin[buf][CH - 1];
+
+        // ---- round 1: D1 = [Q~; W~] S0
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t a1 = smem_u32(sm.a1), b1 = smem_u32(sm.b1);
+#pragma unroll
+            for (int j = 0; j < K / 8; ++j)
+                mma_tf32_ss(D1, sdesc_noswz(a1 + j * 256, 128, SM::A1_SBO), sdesc_noswz(b1 + j * 256, 128, SM::B1_SBO),
+                            IDESC, j > 0 ? 1u : 0u);
+            mma_commit(&sm.bar[0]);
+        }
+        // every thread waits; the outcome is made block-uniform before warp-collective TMEM loads
+        ok = __syncthreads_and(mbar_wait(&sm.bar[0], c & 1, err, kErrTimeoutMma) ? 1 : 0) != 0;
+        tc_fence_after();
+        if (warp >= 2 && ok) {
+            // U = U~ - W~ S0 for token i (TMEM lanes 64..127), and the decayed copy
+            const int i = tid - 64;
+            uint32_t x[32];
+            tmem_ld_32x32b_x32(D1 + lane_base, x);
+            tmem_wait_ld();
+            const float dec = expf(glast - sm.gin[buf][i]);
+#pragma unroll
+            for (int v = 0; v < 32; ++v) {
+                const float u = ut[v] - __uint_as_float(x[v]);
+                sm.b2[kmaj(v, i, CH)] = __uint_as_float(to_tf32(u));
+                sm.b3[kmaj(v, i, CH)] = __uint_as_float(to_tf32(dec * u));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // the [Q~; W~] tile is consumed: fetch the next chunk's
+        if (c + 1 < NC) {
+            load_wq(c + 1);
+            cp_async_commit();
+        }
+
+        // ---- round 2: D1[0:64] += Mqk U ; D2 = K^T Ud
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t a2 = smem_u32(sm.a2[buf]), a3 = smem_u32(sm.a3);
+            const uint32_t b2 = smem_u32(sm.b2), b3 = smem_u32(sm.b3);
+#pragma unroll
+            for (int j = 0; j < CH / 8; ++j)
+                mma_tf32_ss(D1, sdesc_noswz(a2 + j * 256, 128, SM::T_SBO), sdesc_noswz(b2 + j * 256, 128, SM::T_SBO),
+                            IDESC, 1u);
+#pragma unroll
+            for (int j = 0; j < CH / 8; ++j)
+                mma_tf32_ss(D2, sdesc_noswz(a3 + j * 256, 128, SM::T_SBO), sdesc_noswz(b3 + j * 256, 128, SM::T_SBO),
+                            IDESC, j > 0 ? 1u : 0u);
+            mma_commit(&sm.bar[1]);
+        }
+        ok = __syncthreads_and(mbar_wait(&sm.bar[1], c & 1, err, kErrTimeoutMma) ? 1 : 0) != 0;
+        tc_fence_after();
+        if (ok) {
+            if (warp < 2) {
+                const int t = tid;
+                uint32_t x[32];
+                tmem_ld_32x32b_x32(D1 + lane_base, x);
+                tmem_wait_ld();
+                if (t0 + t < T) {
+                    float* orow = o + ((static_cast<int64_t>(b) * T + t0 + t) * Hv + h) * V + vs0;
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4)
+                        *reinterpret_cast<float4*>(orow + 4 * v4) =
+                            make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
+                                        scale * __uint_as_float(x[4 * v4 + 2]), scale * __uint_as_float(x[4 * v4 + 3]));
+                }
+            }
+            uint32_t x[32];
+            tmem_ld_32x32b_x32(D2 + lane_base, x);
+            tmem_wait_ld();
+            if (has_row) {
+                const float eg = expf(glast);
+#pragma unroll
+                for (int v = 0; v < 32; ++v) {
+                    S[v] = fmaf(eg, S[v], __uint_as_float(x[v]));
+                    sm.b1[kmaj(v, tid, K)] = __uint_as_float(to_tf32(S[v]));
+                }
+            }
+            if (c + 1 < NC) load_ut(c + 1);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    if (state_out && has_row) {
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4)
+            *reinterpret_cast<float4*>(state_out + sbase + static_cast<int64_t>(tid) * V + vs0 + 4 * v4) =
+                make_float4(S[4 * v4], S[4 * v4 + 1], S[4 * v4 + 2], S[4 * v4 + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+}
+
 struct ChunkWs {
     float *Wt, *Ut, *Mt, *Gt;
     size_t bytes;
@@ -562,14 +875,25 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prep)");
         e = cudaFuncSetAttribute(chunk_seq_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq)");
+        e = cudaFuncSetAttribute(chunk_seq_tc_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(SeqTcSmem<K>)));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq tc)");
         attr_done[dev] = true;
     }
     const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
     chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, ws.Wt,
                                                                  ws.Ut, ws.Mt, ws.Gt);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    chunk_seq_kernel<K><<<seq_blocks, 256, seq_smem, st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt, ws.Ut,
-                                                                  ws.Mt, ws.Gt, s_in, s_out, o);
+    const char* var = getenv("NVFP4_SCAN_SEQ_VARIANT");
+    if (!var || strcmp(var, "tc") != 0) {
+        chunk_seq_kernel<K><<<seq_blocks, 256, seq_smem, st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt, ws.Ut, ws.Mt,
+                                                               ws.Gt, s_in, s_out, o);
+    } else {
+        unsigned int* err = device_error_word();
+        if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
+        chunk_seq_tc_kernel<K><<<seq_blocks, 128, sizeof(SeqTcSmem<K>), st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt,
+                                                                              ws.Ut, ws.Mt, ws.Gt, s_in, s_out, o, err);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     return NVFP4_OK;
