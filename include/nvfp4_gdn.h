@@ -184,7 +184,7 @@ NVFP4_API nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const fl
  *   - Size limit: a problem whose scratch, gdn_scan_workspace_size(B, T, dims,
  *     GDN_SCAN_CHUNKED), exceeds the array is rejected with
  *     NVFP4_ERR_WORKSPACE before anything is launched (64 MiB covers, e.g.,
- *     B = 1, 32 value heads of 128 x 128, T <= 1600).
+ *     B = 1, 32 value heads of 128 x 128, T <= 896).
  *   - First use: the first call on a device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that first
  *     call before any stream capture begins.

@@ -37,6 +37,7 @@ nvfp4_status make_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t ro
 constexpr unsigned int kErrTimeoutTma = 1u;
 constexpr unsigned int kErrTimeoutMma = 2u;
 constexpr unsigned int kErrTimeoutEpi = 4u;
+constexpr unsigned int kErrTimeoutSeq = 8u;
 
 // ---------------------------------------------------------------- device ---
 // Bounded waits give up after this many SM clocks (about half a second);

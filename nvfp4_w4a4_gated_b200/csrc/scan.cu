@@ -21,9 +21,6 @@
 //    Q K^T and G; kernel 2 (one CTA per head x 32-column V slice) walks the
 //    chunks in order.  Products run on the tensor cores in TF32 with float32
 //    accumulation (mma.sync m16n8k8).
-#include <cstdlib>
-#include <cstring>
-
 #include "common.cuh"
 
 namespace nvg {
@@ -31,6 +28,38 @@ namespace nvg {
 namespace {
 
 constexpr int CH = 64;  // chunk length
+
+// Byte offset of element (r, col) in a K-major tcgen05 operand image with the
+// 128-byte swizzle: the columns are split into 32-float atom columns, each
+// holding `rows` rows of 128 bytes; inside an 8-row group the 16-byte chunk
+// index is XORed with the row index (r mod 8).  Atom columns start on 1024-byte
+// boundaries.
+__host__ __device__ constexpr uint32_t sw128_off(int r, int col, int rows) {
+    return static_cast<uint32_t>((col >> 5) * rows * 128 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) +
+                                 ((col & 3) << 2));
+}
+
+// Per (sequence, value head, chunk) record written by the preparation kernel
+// and copied, section by section, into the sequential kernel's shared memory:
+//   A1  [Q~; W~]  128 x K   Q~ = diag(e^{G}) Q (rows 0..63), W~ (rows 64..127)
+//   A2  Mqk       64 x 64   masked decayed Q K^T, M_ti = e^{G_t - G_i} q_t.k_i (i <= t)
+//   A3  K^ ^T     K x 64    K^_t = e^{G_C - G_t} k_t (atom columns of 128 rows)
+//   UT  U~        64 x V    one 8 KB swizzled 64 x 32 tile per 32-column slice
+//   GC  G_C       the chunk's total log-decay
+// A1..A3 hold TF32-rounded values in the swizzled layout above; U~ is float32.
+template <int K, int V>
+struct ChunkRec {
+    static constexpr uint32_t A1 = 0;
+    static constexpr uint32_t A1_BYTES = 128 * K * 4;
+    static constexpr uint32_t A2 = A1 + A1_BYTES;
+    static constexpr uint32_t A2_BYTES = CH * CH * 4;
+    static constexpr uint32_t A3 = A2 + A2_BYTES;
+    static constexpr uint32_t A3_BYTES = 2 * 128 * 128;
+    static constexpr uint32_t UT = A3 + A3_BYTES;
+    static constexpr uint32_t UT_SLICE = CH * 32 * 4;
+    static constexpr uint32_t GC = UT + (V / 32) * UT_SLICE;
+    static constexpr uint32_t BYTES = GC + 1024;
+};
 
 // --------------------------------------------------------------- recurrent --
 template <int K>
@@ -153,12 +182,11 @@ struct PrepSmem {
 
 // Output tile X [64 x 8*NT] = (T diag(s)) B with B [64 x 8*NT] (row stride KS) in
 // shared memory; warp rows r0..r0+15; 3xTF32 (hi/lo split) so the product is
-// float32-accurate.  X is written to global rows of `out` (row stride 8*NT),
-// rounded to TF32 when `round_out`.
-template <int NT, int KS, int TS>
+// float32-accurate.  Each pair of adjacent outputs (t, col), (t, col+1), col even,
+// goes to store(t, col, x0, x1).
+template <int NT, int KS, int TS, typename Store>
 __device__ __forceinline__ void tri_apply(const float* __restrict__ Tm, const float* __restrict__ s,
-                                          const float* __restrict__ Bm, int r0, int lane, float* __restrict__ out,
-                                          bool round_out) {
+                                          const float* __restrict__ Bm, int r0, int lane, Store store) {
     const int grp = lane >> 2, tig = lane & 3;
     float acc[NT][4];
 #pragma unroll
@@ -184,15 +212,7 @@ __device__ __forceinline__ void tri_apply(const float* __restrict__ Tm, const fl
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int t = r0 + grp + hh * 8;
-            float x0 = acc[nt][2 * hh], x1 = acc[nt][2 * hh + 1];
-            if (round_out) {
-                x0 = __uint_as_float(to_tf32(x0));
-                x1 = __uint_as_float(to_tf32(x1));
-            }
-            *reinterpret_cast<float2*>(out + t * (8 * NT) + nt * 8 + 2 * tig) = make_float2(x0, x1);
-        }
+        for (int hh = 0; hh < 2; ++hh) store(r0 + grp + hh * 8, nt * 8 + 2 * tig, acc[nt][2 * hh], acc[nt][2 * hh + 1]);
     }
 }
 
@@ -201,9 +221,9 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                                                          const float* __restrict__ v, int64_t ld_v,
                                                          const float* __restrict__ g, const float* __restrict__ beta,
                                                          int64_t T, int Hk, int Hv, int form, int NC,
-                                                         float* __restrict__ Wt, float* __restrict__ Ut,
-                                                         float* __restrict__ Mt, float* __restrict__ Gt) {
+                                                         uint8_t* __restrict__ recs) {
     using SM = PrepSmem<K, V>;
+    using RC = ChunkRec<K, V>;
     constexpr int KS = SM::KS;
     extern __shared__ float4 smem_f4[];
     SM& sm = *reinterpret_cast<SM*>(smem_f4);
@@ -214,6 +234,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     const int64_t t0 = static_cast<int64_t>(c) * CH;
     const int n = static_cast<int>((T - t0) < CH ? (T - t0) : CH);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* rec = recs + ((static_cast<int64_t>(b) * Hv + h) * NC + c) * RC::BYTES;
 
     // K, Q rows (zero past the end of the sequence) by asynchronous copies, g and beta
     constexpr int V4 = K / 4;
@@ -268,26 +289,44 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 mma_f32<false>(acc[nt], a, bb);
             }
         }
-        const int64_t mbase = ((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH * CH;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = r0 + grp + (e >> 1) * 8;
-                const int i = nt * 8 + 2 * tig + (e & 1);
+            for (int hh = 0; hh < 2; ++hh) {
+                const int t = r0 + grp + hh * 8;
+                const int i = nt * 8 + 2 * tig;
                 if (warp < 4) {
-                    sm.L[t * CH + i] = (i < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
+                    sm.L[t * CH + i] = (i < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
+                    sm.L[t * CH + i + 1] =
+                        (i + 1 < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
                 } else {
-                    // stored already rounded to TF32: it is only ever a tensor-core operand
-                    const float mv = (i <= t) ? expf(sm.gin[t] - sm.gin[i]) * acc[nt][e] : 0.0f;
-                    Mt[mbase + t * CH + i] = __uint_as_float(to_tf32(mv));
+                    // rounded to TF32 here: it is only ever a tensor-core operand
+                    const float m0 = (i <= t) ? expf(sm.gin[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
+                    const float m1 = (i + 1 <= t) ? expf(sm.gin[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
+                    *reinterpret_cast<float2*>(rec + RC::A2 + sw128_off(t, i, CH)) =
+                        make_float2(__uint_as_float(to_tf32(m0)), __uint_as_float(to_tf32(m1)));
                 }
             }
         }
     }
-    if (tid < CH) {
-        Gt[((static_cast<int64_t>(b) * Hv + h) * NC + c) * CH + tid] = sm.gin[tid];
-        sm.df[tid] = sm.bet[tid] * expf(sm.gd[tid]);
+    if (tid < CH) sm.df[tid] = sm.bet[tid] * expf(sm.gd[tid]);
+    if (tid == 0) *reinterpret_cast<float*>(rec + RC::GC) = sm.gin[CH - 1];
+    // Q~ = e^{G_t} q_t (rows 0..63 of A1) and K^ ^T, K^_t = e^{G_C - G_t} k_t (A3), TF32-rounded
+    for (int idx = tid; idx < CH * (K / 4); idx += 256) {
+        const int t = idx / (K / 4), c4 = idx - t * (K / 4);
+        const float eg = expf(sm.gin[t]);
+        const float4 x = *reinterpret_cast<const float4*>(&sm.qs[t * KS + 4 * c4]);
+        *reinterpret_cast<float4*>(rec + RC::A1 + sw128_off(t, 4 * c4, 128)) =
+            make_float4(__uint_as_float(to_tf32(eg * x.x)), __uint_as_float(to_tf32(eg * x.y)),
+                        __uint_as_float(to_tf32(eg * x.z)), __uint_as_float(to_tf32(eg * x.w)));
+    }
+    for (int idx = tid; idx < K * (CH / 4); idx += 256) {
+        const int dd = idx % K, t4 = idx / K;
+        const float gc = sm.gin[CH - 1];
+        float x[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(to_tf32(expf(gc - sm.gin[4 * t4 + w]) * sm.ks[(4 * t4 + w) * KS + dd]));
+        *reinterpret_cast<float4*>(rec + RC::A3 + sw128_off(dd, 4 * t4, 128)) = make_float4(x[0], x[1], x[2], x[3]);
     }
     constexpr int TS = SM::TS;
     for (int idx = tid; idx < CH * TS; idx += 256) sm.T[idx] = 0.0f;
@@ -343,560 +382,309 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     __syncthreads();
     // W~ = T diag(b e^{Gd}) K (warps 0-3, stored TF32-rounded: a tensor-core operand downstream)
     // U~ = T diag(beta) V   (warps 4-7)
-    const int64_t cb = (static_cast<int64_t>(b) * Hv + h) * NC + c;
-    if (warp < 4)
-        tri_apply<K / 8, KS, TS>(sm.T, sm.df, sm.ks, warp * 16, lane, Wt + cb * CH * K, true);
-    else
-        tri_apply<V / 8, KS, TS>(sm.T, sm.bet, sm.qs, (warp - 4) * 16, lane, Ut + cb * CH * V, false);
+    if (warp < 4) {
+        tri_apply<K / 8, KS, TS>(sm.T, sm.df, sm.ks, warp * 16, lane, [&](int t, int col, float x0, float x1) {
+            *reinterpret_cast<float2*>(rec + RC::A1 + sw128_off(CH + t, col, 128)) =
+                make_float2(__uint_as_float(to_tf32(x0)), __uint_as_float(to_tf32(x1)));
+        });
+    } else {
+        tri_apply<V / 8, KS, TS>(sm.T, sm.bet, sm.qs, (warp - 4) * 16, lane, [&](int t, int col, float x0, float x1) {
+            *reinterpret_cast<float2*>(rec + RC::UT + (col >> 5) * RC::UT_SLICE + sw128_off(t, col & 31, CH)) =
+                make_float2(x0, x1);
+        });
+    }
 }
 
 // ------------------------------------------------------ sequential chunks --
+// One CTA per (sequence, value head, 32-column slice of V) walks the chunks in
+// order, on the tcgen05 tensor cores (kind::tf32, float32 accumulation in TMEM,
+// M = 128, N = 32).  Per chunk:
+//   round 1:  D1 = [Q~; W~] S0        rows 0..63: Q~ S0, rows 64..127: W~ S0
+//   U = U~ - W~ S0 (TF32)  ->  U^T in shared memory
+//   round 2:  D1 += [Mqk; *] U         rows 0..63: o / scale (rows 64..127 unused)
+//             D2  = K^ ^T U             K^_t = e^{G_C - G_t} k_t
+//   S <- e^{G_C} S + D2 (float32, registers)  ->  S^T (TF32) in shared memory
+// Warp roles: warp 0 copies the chunk records into shared memory (bulk copies,
+// [Q~; W~] and U~ double-buffered), warp 1 issues the MMAs, warps 2..5 (one per
+// TMEM lane quarter) form U, the state and the output.  D1 alternates between two
+// TMEM buffers so the output of chunk c drains while round 1 of chunk c+1 runs.
 template <int K>
-struct SeqSmem {
-    static constexpr int XS = K + 4;   // [W~; Q] tile row stride (== 4 mod 32)
-    static constexpr int KS = K + 8;   // K tile row stride (== 8 mod 32, transposed reads)
-    static constexpr int MS = CH + 4;  // masked Q K^T row stride
-    static constexpr int SS = 40;      // state / U row stride (== 8 mod 32)
-    float x1[2 * CH * XS];             // rows 0..63: W~ (TF32-rounded), rows 64..127: Q
-    float kc[2][CH * KS];              // K of this chunk and the next one
-    float mc[2][CH * MS];              // masked decayed Q K^T (TF32-rounded), double-buffered
-    float s[K * SS];                   // float32 state slice [K x 32]
-    float u[CH * SS];                  // U (TF32-rounded)
-    float ud[CH * SS];                 // U scaled by e^{G_C - G_i} (TF32-rounded)
-    float gin[2][CH];
+struct SeqLayout {
+    static constexpr uint32_t A1_BYTES = 128 * K * 4;
+    static constexpr uint32_t A1 = 0;                         // two stages
+    static constexpr uint32_t A23 = 2 * A1_BYTES;             // Mqk (16 KB) then K^ ^T (32 KB)
+    static constexpr uint32_t A23_BYTES = CH * CH * 4 + 2 * 128 * 128;
+    static constexpr uint32_t UT = A23 + A23_BYTES;           // two stages of a 64 x 32 U~ slice
+    static constexpr uint32_t UT_BYTES = CH * 32 * 4;
+    static constexpr uint32_t B1 = UT + 2 * UT_BYTES;         // S^T: K/32 atom columns of 32 rows
+    static constexpr uint32_t B2 = B1 + K * 128;              // U^T: 2 atom columns of 32 rows
+    static constexpr uint32_t BAR = B2 + CH * 128;
+    static constexpr uint32_t BYTES = BAR + 256 + 1024;       // + alignment slack
 };
 
-
-// One CTA (256 threads) per (sequence, value head, 32-column slice of V).
-// Per chunk: P1 = [W~; Q] S on all 8 warps (warps 0-3: W~ S, warps 4-7: Q S);
-// warps 0-3 form U = U~ - W~ S; warps 4-7 then form o = scale (e^G Q S + M U)
-// while every warp advances its 16 state rows S <- e^{G_C} S + K^T (decayed U).
-// K, M and G of chunk c+1 are prefetched at the start of chunk c, W~ and Q of
-// chunk c+1 as soon as P1 of chunk c has consumed them.
-template <int K>
-__global__ void __launch_bounds__(256) chunk_seq_kernel(const float* __restrict__ q, const float* __restrict__ k,
-                                                        int64_t T, int Hk, int Hv, int V, float scale, int NC,
-                                                        const float* __restrict__ Wt, const float* __restrict__ Ut,
-                                                        const float* __restrict__ Mt, const float* __restrict__ Gt,
-                                                        const float* state_in, float* state_out, float* __restrict__ o) {
-    using SM = SeqSmem<K>;
-    constexpr int XS = SM::XS, KS = SM::KS, MS = SM::MS, SS = SM::SS;
-    extern __shared__ float4 smem_f4[];
-    SM& sm = *reinterpret_cast<SM*>(smem_f4);
-    const int nslice = V / 32;
-    const int slice = blockIdx.x % nslice;
-    const int h = (blockIdx.x / nslice) % Hv;
-    const int b = blockIdx.x / (nslice * Hv);
-    const int hk = static_cast<int>((static_cast<int64_t>(h) * Hk) / Hv);
-    const int vs0 = slice * 32;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int grp = lane >> 2, tig = lane & 3;
-    const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
-    const int64_t hc = (static_cast<int64_t>(b) * Hv + h) * NC;
-
-    for (int idx = tid; idx < K * 32; idx += 256) {
-        const int r = idx >> 5, cc = idx & 31;
-        sm.s[r * SS + cc] = state_in ? state_in[sbase + static_cast<int64_t>(r) * V + vs0 + cc] : 0.0f;
-    }
-
-    auto load_wq = [&](int c) {
-        const int64_t t0 = static_cast<int64_t>(c) * CH;
-        constexpr int V4 = K / 4;
-        for (int idx = tid; idx < CH * V4; idx += 256) {
-            const int r = idx / V4, c4 = idx - r * V4;
-            cp_async16(&sm.x1[r * XS + c4 * 4], Wt + ((hc + c) * CH + r) * K + c4 * 4, true);
-            const bool valid = t0 + r < T;
-            const int64_t qoff = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
-            cp_async16(&sm.x1[(CH + r) * XS + c4 * 4], q + qoff, valid);
-        }
-    };
-    auto load_km = [&](int c, int buf) {
-        const int64_t t0 = static_cast<int64_t>(c) * CH;
-        constexpr int V4 = K / 4;
-        for (int idx = tid; idx < CH * V4; idx += 256) {
-            const int r = idx / V4, c4 = idx - r * V4;
-            const bool valid = t0 + r < T;
-            const int64_t koff = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
-            cp_async16(&sm.kc[buf][r * KS + c4 * 4], k + koff, valid);
-        }
-        for (int idx = tid; idx < CH * CH / 4; idx += 256) {
-            const int r = idx >> 4, c4 = idx & 15;
-            cp_async16(&sm.mc[buf][r * MS + c4 * 4], Mt + ((hc + c) * CH + r) * CH + c4 * 4, true);
-        }
-        if (tid < CH / 4) cp_async16(&sm.gin[buf][tid * 4], Gt + (hc + c) * CH + tid * 4, true);
-    };
-
-    load_wq(0);
-    load_km(0, 0);
-    cp_async_commit();
-
-    for (int c = 0; c < NC; ++c) {
-        const int64_t t0 = static_cast<int64_t>(c) * CH;
-        const int buf = c & 1;
-        cp_async_wait<0>();
-        __syncthreads();
-        if (c + 1 < NC) {
-            load_km(c + 1, buf ^ 1);
-            cp_async_commit();
-        }
-        // U~ for this warp's rows, fetched now so the latency hides behind P1
-        float ut[4][4];
-        if (warp < 4) {
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int i = warp * 16 + grp + hh * 8;
-                    const float2 v2 = *reinterpret_cast<const float2*>(Ut + ((hc + c) * CH + i) * V + vs0 + nt * 8 + 2 * tig);
-                    ut[nt][2 * hh] = v2.x;
-                    ut[nt][2 * hh + 1] = v2.y;
-                }
-        }
-
-        // P1: [W~; Q] (128 x K) times S (K x 32); warp w owns rows 16w..16w+15
-        float acc[4][4];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        {
-            const int r0 = warp * 16;
-            const bool a_rounded = warp < 4;  // W~ rows arrive rounded to TF32
-#pragma unroll 4
-            for (int k0 = 0; k0 < K; k0 += 8) {
-                const float af[4] = {sm.x1[(r0 + grp) * XS + k0 + tig], sm.x1[(r0 + grp + 8) * XS + k0 + tig],
-                                     sm.x1[(r0 + grp) * XS + k0 + tig + 4], sm.x1[(r0 + grp + 8) * XS + k0 + tig + 4]};
-                uint32_t a[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) a[i] = a_rounded ? __float_as_uint(af[i]) : to_tf32(af[i]);
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const uint32_t bb[2] = {to_tf32(sm.s[(k0 + tig) * SS + nt * 8 + grp]),
-                                            to_tf32(sm.s[(k0 + tig + 4) * SS + nt * 8 + grp])};
-                    mma_tf32(acc[nt], a, bb);
-                }
-            }
-        }
-        const float glast = sm.gin[buf][CH - 1];
-        if (warp < 4) {
-            // U = U~ - W~ S0, and U decayed by e^{G_C - G_i} for the state update
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int i = warp * 16 + grp + hh * 8;
-                const float dec = expf(glast - sm.gin[buf][i]);
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-                    for (int e1 = 0; e1 < 2; ++e1) {
-                        const int e = 2 * hh + e1;
-                        const int col = nt * 8 + 2 * tig + e1;
-                        const float uval = ut[nt][e] - acc[nt][e];
-                        sm.u[i * SS + col] = __uint_as_float(to_tf32(uval));
-                        sm.ud[i * SS + col] = __uint_as_float(to_tf32(dec * uval));
-                    }
-                }
-            }
-        }
-        __syncthreads();
-        // X1 is free: prefetch the next chunk's W~ and Q while this chunk finishes
-        if (c + 1 < NC) {
-            load_wq(c + 1);
-            cp_async_commit();
-        }
-
-        if (warp >= 4) {
-            // o = scale * (e^{G_t} Q S0 + Mqk U); rows t = 16(w-4)..
-            const int r0 = (warp - 4) * 16;
-            const float* mc = sm.mc[buf];
-            float mu[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) mu[nt][0] = mu[nt][1] = mu[nt][2] = mu[nt][3] = 0.f;
-#pragma unroll
-            for (int k0 = 0; k0 < CH; k0 += 8) {
-                const uint32_t a[4] = {__float_as_uint(mc[(r0 + grp) * MS + k0 + tig]),
-                                       __float_as_uint(mc[(r0 + grp + 8) * MS + k0 + tig]),
-                                       __float_as_uint(mc[(r0 + grp) * MS + k0 + tig + 4]),
-                                       __float_as_uint(mc[(r0 + grp + 8) * MS + k0 + tig + 4])};
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const uint32_t bb[2] = {__float_as_uint(sm.u[(k0 + tig) * SS + nt * 8 + grp]),
-                                            __float_as_uint(sm.u[(k0 + tig + 4) * SS + nt * 8 + grp])};
-                    mma_tf32(mu[nt], a, bb);
-                }
-            }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int t = r0 + grp + hh * 8;
-                if (t0 + t < T) {
-                    const float eg = expf(sm.gin[buf][t]);
-                    float* orow = o + ((static_cast<int64_t>(b) * T + t0 + t) * Hv + h) * V + vs0;
-#pragma unroll
-                    for (int nt = 0; nt < 4; ++nt) {
-                        const int col = nt * 8 + 2 * tig;
-                        *reinterpret_cast<float2*>(orow + col) =
-                            make_float2(scale * fmaf(eg, acc[nt][2 * hh], mu[nt][2 * hh]),
-                                        scale * fmaf(eg, acc[nt][2 * hh + 1], mu[nt][2 * hh + 1]));
-                    }
-                }
-            }
-        }
-
-        // S <- e^{G_C} S + K^T (diag(e^{G_C - G}) U); warp w owns state rows 16w..16w+15
-        if (warp * 16 < K) {
-            const int d0 = warp * 16;
-            const float eg = expf(glast);
-            const float* kc = sm.kc[buf];
-            float st[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int col = nt * 8 + 2 * tig;
-                st[nt][0] = eg * sm.s[(d0 + grp) * SS + col];
-                st[nt][1] = eg * sm.s[(d0 + grp) * SS + col + 1];
-                st[nt][2] = eg * sm.s[(d0 + grp + 8) * SS + col];
-                st[nt][3] = eg * sm.s[(d0 + grp + 8) * SS + col + 1];
-            }
-#pragma unroll
-            for (int k0 = 0; k0 < CH; k0 += 8) {
-                const uint32_t a[4] = {to_tf32(kc[(k0 + tig) * KS + d0 + grp]), to_tf32(kc[(k0 + tig) * KS + d0 + grp + 8]),
-                                       to_tf32(kc[(k0 + tig + 4) * KS + d0 + grp]),
-                                       to_tf32(kc[(k0 + tig + 4) * KS + d0 + grp + 8])};
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const uint32_t bb[2] = {__float_as_uint(sm.ud[(k0 + tig) * SS + nt * 8 + grp]),
-                                            __float_as_uint(sm.ud[(k0 + tig + 4) * SS + nt * 8 + grp])};
-                    mma_tf32(st[nt], a, bb);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int col = nt * 8 + 2 * tig;
-                sm.s[(d0 + grp) * SS + col] = st[nt][0];
-                sm.s[(d0 + grp) * SS + col + 1] = st[nt][1];
-                sm.s[(d0 + grp + 8) * SS + col] = st[nt][2];
-                sm.s[(d0 + grp + 8) * SS + col + 1] = st[nt][3];
-            }
-        }
-        __syncthreads();
-    }
-    cp_async_wait<0>();
-    __syncthreads();
-    if (state_out) {
-        for (int idx = tid; idx < K * 32; idx += 256) {
-            const int r = idx >> 5, cc = idx & 31;
-            state_out[sbase + static_cast<int64_t>(r) * V + vs0 + cc] = sm.s[r * SS + cc];
-        }
-    }
-}
-
-// ------------------------------------------- sequential chunks, tcgen05 --
-// Same per-chunk algebra as chunk_seq_kernel, on the sm_100 tensor cores: every
-// product reads its operands from shared memory (no-swizzle K-major canonical
-// tiles: 8-row x 16-byte core matrices) and accumulates in TMEM, so the warps
-// only move data between the two MMA rounds of a chunk:
-//   round 1:  D1 = [Q~; W~] S0            (M=128: rows 0..63 Q~ S0, 64..127 W~ S0)
-//   warps 2-3: U = U~ - W~ S0, Ud = diag(e^{G_C - G}) U  -> shared memory
-//   round 2:  D1 += [Mqk; *] U           (rows 0..63 become Q~ S0 + Mqk U;
-//                                          the W~ S0 rows receive garbage, unused)
-//             D2  = K^T Ud               (M=128 state rows)
-//   warps 0-1: o = scale * D1[0:64];  all: S <- e^{G_C} S + D2 (float32 registers)
-// Q~ = diag(e^{G}) Q is formed while rounding Q to TF32 in shared memory; K^T is
-// built from the staged K tile in the same pass.
-template <int K>
-struct SeqTcSmem {
-    static constexpr int A1_SBO = (K / 4) * 128;   // [Q~; W~] over the state dim: 8-row group stride
-    static constexpr int T_SBO = 16 * 128;         // tiles whose K extent is the 64 tokens
-    static constexpr int B1_SBO = (K / 4) * 128;   // S^T [32 x K]
-    float a1[128 * K];
-    float a2[2][64 * 64];                          // Mqk; a2[1] doubles as a2[0]'s unused upper rows
-    float kst[2][64 * K];                          // staged K rows [t][d]; kst[0] follows a2[1]
-    float a3[128 * 64];                            // K^T [d][t] (K = 64: upper half unused)
-    float b1[32 * K];                              // S^T [v][d]
-    float b2[32 * 64];                             // U^T [v][t]
-    float b3[32 * 64];                             // Ud^T
-    float gin[2][CH];
-    uint64_t bar[2];
-    uint32_t tmem_holder;
+enum SeqBar : int {
+    kA1Full = 0,   // [2]
+    kA1Empty = 2,  // [2]
+    kA23Full = 4,
+    kA23Empty = 5,
+    kUtFull = 6,   // [2]
+    kUtEmpty = 8,  // [2]
+    kR1Done = 10,
+    kR2Done = 11,
+    kUReady = 12,
+    kSReady = 13,
+    kFin = 14,
+    kNumSeqBars = 15
 };
 
-template <int K>
-__global__ void __launch_bounds__(128) chunk_seq_tc_kernel(const float* __restrict__ q, const float* __restrict__ k,
-                                                           int64_t T, int Hk, int Hv, int V, float scale, int NC,
-                                                           const float* __restrict__ Wt, const float* __restrict__ Ut,
-                                                           const float* __restrict__ Mt, const float* __restrict__ Gt,
-                                                           const float* state_in, float* state_out,
-                                                           float* __restrict__ o, unsigned int* __restrict__ err) {
-    using SM = SeqTcSmem<K>;
-    extern __shared__ float4 smem_f4[];
-    SM& sm = *reinterpret_cast<SM*>(smem_f4);
-    const int nslice = V / 32;
-    const int slice = blockIdx.x % nslice;
-    const int h = (blockIdx.x / nslice) % Hv;
-    const int b = blockIdx.x / (nslice * Hv);
-    const int hk = static_cast<int>((static_cast<int64_t>(h) * Hk) / Hv);
+template <int K, int V>
+__global__ void __launch_bounds__(192, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
+                                                           float scale, int NC, const float* state_in,
+                                                           float* state_out, float* __restrict__ o,
+                                                           unsigned int* __restrict__ err) {
+    using L = SeqLayout<K>;
+    using RC = ChunkRec<K, V>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + kNumSeqBars);
+    constexpr int NSL = V / 32;
+    const int slice = blockIdx.x % NSL;
+    const int h = (blockIdx.x / NSL) % Hv;
+    const int b = blockIdx.x / (NSL * Hv);
     const int vs0 = slice * 32;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
-    const int64_t hc = (static_cast<int64_t>(b) * Hv + h) * NC;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint8_t* rec0 = recs + (static_cast<int64_t>(b) * Hv + h) * NC * RC::BYTES;
     constexpr uint32_t IDESC = idesc_tf32(128, 32, false, false);
 
-    if (tid == 0) {
-        mbar_init(&sm.bar[0], 1);
-        mbar_init(&sm.bar[1], 1);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumSeqBars; ++i) {
+            const bool many = i == kUtEmpty || i == kUtEmpty + 1 || i == kUReady;
+            mbar_init(&bar[i], i == kSReady ? 128 : (many ? 64 : 1));
+        }
         fence_mbar_init();
     }
-    if (warp == 0) {
-        tmem_alloc(&sm.tmem_holder, 64);
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 128);
         tmem_relinquish();
     }
-
-    // float offsets inside K-major canonical tiles: row r, column c, `cw` columns per row
-    auto kmaj = [](int r, int c, int cw) { return ((r >> 3) * (cw >> 2) + (c >> 2)) * 32 + (r & 7) * 4 + (c & 3); };
-
-    // state rows in registers: thread d < K holds S[d][vs0 .. vs0+31]
-    float S[32];
-    const bool has_row = tid < K;
-    if (has_row) {
-#pragma unroll
-        for (int v4 = 0; v4 < 8; ++v4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (state_in) x = *reinterpret_cast<const float4*>(state_in + sbase + static_cast<int64_t>(tid) * V + vs0 + 4 * v4);
-            S[4 * v4] = x.x; S[4 * v4 + 1] = x.y; S[4 * v4 + 2] = x.z; S[4 * v4 + 3] = x.w;
-        }
-#pragma unroll
-        for (int v = 0; v < 32; ++v) sm.b1[kmaj(v, tid, K)] = __uint_as_float(to_tf32(S[v]));
-    }
-
-    auto load_wq = [&](int c) {
-        const int64_t t0 = static_cast<int64_t>(c) * CH;
-        for (int idx = tid; idx < CH * (K / 4); idx += 128) {
-            const int t = idx / (K / 4), d4 = idx % (K / 4);
-            cp_async16(&sm.a1[kmaj(CH + t, 4 * d4, K)], Wt + ((hc + c) * CH + t) * K + 4 * d4, true);
-            const bool valid = t0 + t < T;
-            const int64_t qoff = valid ? ((static_cast<int64_t>(b) * T + t0 + t) * Hk + hk) * K + 4 * d4 : 0;
-            cp_async16(&sm.a1[kmaj(t, 4 * d4, K)], q + qoff, valid);
-        }
-    };
-    auto load_kmg = [&](int c, int buf) {
-        const int64_t t0 = static_cast<int64_t>(c) * CH;
-        for (int idx = tid; idx < CH * (K / 4); idx += 128) {
-            const int t = idx / (K / 4), d4 = idx % (K / 4);
-            const bool valid = t0 + t < T;
-            const int64_t koff = valid ? ((static_cast<int64_t>(b) * T + t0 + t) * Hk + hk) * K + 4 * d4 : 0;
-            cp_async16(&sm.kst[buf][t * K + 4 * d4], k + koff, valid);
-        }
-        for (int idx = tid; idx < CH * 16; idx += 128) {
-            const int t = idx >> 4, i4 = idx & 15;
-            cp_async16(&sm.a2[buf][kmaj(t, 4 * i4, CH)], Mt + ((hc + c) * CH + t) * CH + 4 * i4, true);
-        }
-        if (tid < CH / 4) cp_async16(&sm.gin[buf][4 * tid], Gt + (hc + c) * CH + 4 * tid, true);
-    };
-    float ut[32];
-    auto load_ut = [&](int c) {
-        if (warp >= 2) {
-            const float* src = Ut + ((hc + c) * CH + (tid - 64)) * V + vs0;
-#pragma unroll
-            for (int v4 = 0; v4 < 8; ++v4) {
-                const float4 x = *reinterpret_cast<const float4*>(src + 4 * v4);
-                ut[4 * v4] = x.x; ut[4 * v4 + 1] = x.y; ut[4 * v4 + 2] = x.z; ut[4 * v4 + 3] = x.w;
-            }
-        }
-    };
-
-    load_wq(0);
-    load_kmg(0, 0);
-    cp_async_commit();
-    load_ut(0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sm.tmem_holder;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t D1 = tmem, D2 = tmem + 32;
-    bool ok = true;
+    const uint32_t tmem = *tmem_holder;
 
-    for (int c = 0; c < NC && ok; ++c) {
-        const int buf = c & 1;
-        const int64_t t0 = static_cast<int64_t>(c) * CH;
-        cp_async_wait<0>();
-        __syncthreads();
-        // Q~ = e^{G_t} Q rounded to TF32 in place; K^T [d][t] built from the staged rows, rounded
-        for (int idx = tid; idx < CH * (K / 4); idx += 128) {
-            const int t = idx / (K / 4), d4 = idx % (K / 4);
-            float4* qp = reinterpret_cast<float4*>(&sm.a1[kmaj(t, 4 * d4, K)]);
-            const float eg = expf(sm.gin[buf][t]);
-            const float4 xq = *qp;
-            *qp = make_float4(__uint_as_float(to_tf32(eg * xq.x)), __uint_as_float(to_tf32(eg * xq.y)),
-                              __uint_as_float(to_tf32(eg * xq.z)), __uint_as_float(to_tf32(eg * xq.w)));
-            const float4 xk = *reinterpret_cast<const float4*>(&sm.kst[buf][t * K + 4 * d4]);
-            sm.a3[kmaj(4 * d4 + 0, t, CH)] = __uint_as_float(to_tf32(xk.x));
-            sm.a3[kmaj(4 * d4 + 1, t, CH)] = __uint_as_float(to_tf32(xk.y));
-            sm.a3[kmaj(4 * d4 + 2, t, CH)] = __uint_as_float(to_tf32(xk.z));
-            sm.a3[kmaj(4 * d4 + 3, t, CH)] = __uint_as_float(to_tf32(xk.w));
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (c + 1 < NC) {
-            load_kmg(c + 1, buf ^ 1);
-            cp_async_commit();
-        }
-        const float glast = sm.gin[buf][CH - 1];
-
-        // ---- round 1: D1 = [Q~; W~] S0
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t a1 = smem_u32(sm.a1), b1 = smem_u32(sm.b1);
-#pragma unroll
-            for (int j = 0; j < K / 8; ++j)
-                mma_tf32_ss(D1, sdesc_noswz(a1 + j * 256, 128, SM::A1_SBO), sdesc_noswz(b1 + j * 256, 128, SM::B1_SBO),
-                            IDESC, j > 0 ? 1u : 0u);
-            mma_commit(&sm.bar[0]);
-        }
-        // every thread waits; the outcome is made block-uniform before warp-collective TMEM loads
-        ok = __syncthreads_and(mbar_wait(&sm.bar[0], c & 1, err, kErrTimeoutMma) ? 1 : 0) != 0;
-        tc_fence_after();
-        if (warp >= 2 && ok) {
-            // U = U~ - W~ S0 for token i (TMEM lanes 64..127), and the decayed copy
-            const int i = tid - 64;
-            uint32_t x[32];
-            tmem_ld_32x32b_x32(D1 + lane_base, x);
-            tmem_wait_ld();
-            const float dec = expf(glast - sm.gin[buf][i]);
-#pragma unroll
-            for (int v = 0; v < 32; ++v) {
-                const float u = ut[v] - __uint_as_float(x[v]);
-                sm.b2[kmaj(v, i, CH)] = __uint_as_float(to_tf32(u));
-                sm.b3[kmaj(v, i, CH)] = __uint_as_float(to_tf32(dec * u));
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- producer: chunk records -> shared memory
+            int last_c = -1;  // last chunk whose three sections were all issued
+            int last_a1 = -1, last_ut = -1;
+            for (int c = 0; c < NC; ++c) {
+                const uint8_t* rc = rec0 + static_cast<int64_t>(c) * RC::BYTES;
+                const int s = c & 1;
+                if (c >= 2 && !mbar_wait(&bar[kA1Empty + s], ((c >> 1) - 1) & 1, err, kErrTimeoutSeq)) break;
+                mbar_arrive_expect_tx(&bar[kA1Full + s], L::A1_BYTES);
+                for (uint32_t p = 0; p < L::A1_BYTES; p += 16384)
+                    bulk_load(sm + L::A1 + s * L::A1_BYTES + p, rc + RC::A1 + p, 16384, &bar[kA1Full + s]);
+                last_a1 = c;
+                if (c >= 2 && !mbar_wait(&bar[kUtEmpty + s], ((c >> 1) - 1) & 1, err, kErrTimeoutSeq)) break;
+                mbar_arrive_expect_tx(&bar[kUtFull + s], L::UT_BYTES);
+                bulk_load(sm + L::UT + s * L::UT_BYTES, rc + RC::UT + slice * RC::UT_SLICE, L::UT_BYTES,
+                          &bar[kUtFull + s]);
+                last_ut = c;
+                if (c >= 1 && !mbar_wait(&bar[kA23Empty], (c - 1) & 1, err, kErrTimeoutSeq)) break;
+                mbar_arrive_expect_tx(&bar[kA23Full], L::A23_BYTES);
+                for (uint32_t p = 0; p < L::A23_BYTES; p += 16384)
+                    bulk_load(sm + L::A23 + p, rc + RC::A2 + p, 16384, &bar[kA23Full]);
+                last_c = c;
             }
+            // every copy issued has landed before the CTA may exit
+            // (stage s last received chunk last - (last - s) % 2, for the last chunk issued to it)
+            for (int s = 0; s < 2; ++s) {
+                const int ca = last_a1 - ((last_a1 - s) & 1), cu = last_ut - ((last_ut - s) & 1);
+                if (ca >= 0) mbar_wait(&bar[kA1Full + s], (ca >> 1) & 1, err, kErrTimeoutSeq);
+                if (cu >= 0) mbar_wait(&bar[kUtFull + s], (cu >> 1) & 1, err, kErrTimeoutSeq);
+            }
+            if (last_c >= 0) mbar_wait(&bar[kA23Full], last_c & 1, err, kErrTimeoutSeq);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer
+            const uint32_t b1 = smem_u32(sm + L::B1), b2 = smem_u32(sm + L::B2);
+            const uint32_t a2 = smem_u32(sm + L::A23), a3 = a2 + CH * CH * 4;
+            const uint32_t D2 = tmem + 64;
+            for (int c = 0; c < NC; ++c) {
+                const int s = c & 1;
+                const uint32_t D1 = tmem + 32 * s;
+                if (!mbar_wait(&bar[kSReady], c & 1, err, kErrTimeoutSeq)) break;
+                if (!mbar_wait(&bar[kA1Full + s], (c >> 1) & 1, err, kErrTimeoutSeq)) break;
+                tc_fence_after();
+                const uint32_t a1 = smem_u32(sm + L::A1 + s * L::A1_BYTES);
+#pragma unroll
+                for (int j = 0; j < K / 8; ++j)
+                    mma_tf32_ss(D1, sdesc_kmajor_sw128(a1 + (j >> 2) * 128 * 128 + (j & 3) * 32),
+                                sdesc_kmajor_sw128(b1 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
+                mma_commit(&bar[kA1Empty + s]);
+                mma_commit(&bar[kR1Done]);
+                if (!mbar_wait(&bar[kUReady], c & 1, err, kErrTimeoutSeq)) break;
+                if (!mbar_wait(&bar[kA23Full], c & 1, err, kErrTimeoutSeq)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < CH / 8; ++j)
+                    mma_tf32_ss(D1, sdesc_kmajor_sw128(a2 + (j >> 2) * CH * 128 + (j & 3) * 32),
+                                sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, 1u);
+#pragma unroll
+                for (int j = 0; j < CH / 8; ++j)
+                    mma_tf32_ss(D2, sdesc_kmajor_sw128(a3 + (j >> 2) * 128 * 128 + (j & 3) * 32),
+                                sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
+                mma_commit(&bar[kA23Empty]);
+                mma_commit(&bar[kR2Done]);
+            }
+            // all MMAs issued have completed before TMEM is released
+            mma_commit(&bar[kFin]);
+            mbar_wait(&bar[kFin], 0, err, kErrTimeoutSeq);
+        }
+    } else {
+        // ---- warps 2..5: TMEM lane quarter q = warp % 4
+        const int q = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int d = q * 32 + lane;             // state row
+        const bool has_row = d < K;
+        const bool u_role = q >= 2;              // tokens 0..63 of W~ S0 live in lanes 64..127
+        const int tu = d - 64;
+        const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
+        uint8_t* b1p = sm + L::B1;
+        uint8_t* b2p = sm + L::B2;
+        float S[32];
+#pragma unroll
+        for (int v4 = 0; v4 < 8; ++v4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (state_in && has_row)
+                x = *reinterpret_cast<const float4*>(state_in + sbase + static_cast<int64_t>(d) * V + vs0 + 4 * v4);
+            S[4 * v4] = x.x; S[4 * v4 + 1] = x.y; S[4 * v4 + 2] = x.z; S[4 * v4 + 3] = x.w;
+        }
+        if (has_row) {
+#pragma unroll
+            for (int v = 0; v < 32; ++v)
+                *reinterpret_cast<float*>(b1p + sw128_off(v, d, 32)) = __uint_as_float(to_tf32(S[v]));
         }
         fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // the [Q~; W~] tile is consumed: fetch the next chunk's
-        if (c + 1 < NC) {
-            load_wq(c + 1);
-            cp_async_commit();
-        }
-
-        // ---- round 2: D1[0:64] += Mqk U ; D2 = K^T Ud
-        if (tid == 0) {
+        mbar_arrive(&bar[kSReady]);
+        bool ok = true;
+        for (int c = 0; c < NC && ok; ++c) {
+            const int s = c & 1;
+            const int64_t t0 = static_cast<int64_t>(c) * CH;
+            const float gc = *reinterpret_cast<const float*>(rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::GC);
+            float ut[32];
+            if (u_role) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar[kUtFull + s], (c >> 1) & 1, err, kErrTimeoutSeq));
+                if (!ok) break;
+                const uint8_t* up = sm + L::UT + s * L::UT_BYTES + tu * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 x = *reinterpret_cast<const float4*>(up + ((j ^ (tu & 7)) << 4));
+                    ut[4 * j] = x.x; ut[4 * j + 1] = x.y; ut[4 * j + 2] = x.z; ut[4 * j + 3] = x.w;
+                }
+                mbar_arrive(&bar[kUtEmpty + s]);
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR1Done], c & 1, err, kErrTimeoutSeq));
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t a2 = smem_u32(sm.a2[buf]), a3 = smem_u32(sm.a3);
-            const uint32_t b2 = smem_u32(sm.b2), b3 = smem_u32(sm.b3);
-#pragma unroll
-            for (int j = 0; j < CH / 8; ++j)
-                mma_tf32_ss(D1, sdesc_noswz(a2 + j * 256, 128, SM::T_SBO), sdesc_noswz(b2 + j * 256, 128, SM::T_SBO),
-                            IDESC, 1u);
-#pragma unroll
-            for (int j = 0; j < CH / 8; ++j)
-                mma_tf32_ss(D2, sdesc_noswz(a3 + j * 256, 128, SM::T_SBO), sdesc_noswz(b3 + j * 256, 128, SM::T_SBO),
-                            IDESC, j > 0 ? 1u : 0u);
-            mma_commit(&sm.bar[1]);
-        }
-        ok = __syncthreads_and(mbar_wait(&sm.bar[1], c & 1, err, kErrTimeoutMma) ? 1 : 0) != 0;
-        tc_fence_after();
-        if (ok) {
-            if (warp < 2) {
-                const int t = tid;
+            if (u_role) {
                 uint32_t x[32];
-                tmem_ld_32x32b_x32(D1 + lane_base, x);
+                tmem_ld_32x32b_x32(tmem + 32 * s + lane_base, x);
                 tmem_wait_ld();
-                if (t0 + t < T) {
-                    float* orow = o + ((static_cast<int64_t>(b) * T + t0 + t) * Hv + h) * V + vs0;
+#pragma unroll
+                for (int v = 0; v < 32; ++v)
+                    *reinterpret_cast<float*>(b2p + sw128_off(v, tu, 32)) =
+                        __uint_as_float(to_tf32(ut[v] - __uint_as_float(x[v])));
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar[kUReady]);
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR2Done], c & 1, err, kErrTimeoutSeq));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                uint32_t x[32];
+                tmem_ld_32x32b_x32(tmem + 64 + lane_base, x);
+                tmem_wait_ld();
+                if (has_row) {
+                    const float eg = expf(gc);
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) {
+                        S[v] = fmaf(eg, S[v], __uint_as_float(x[v]));
+                        *reinterpret_cast<float*>(b1p + sw128_off(v, d, 32)) = __uint_as_float(to_tf32(S[v]));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar[kSReady]);
+            if (!u_role) {
+                // output rows t = d (lanes 0..63 of D1)
+                uint32_t x[32];
+                tmem_ld_32x32b_x32(tmem + 32 * s + lane_base, x);
+                tmem_wait_ld();
+                if (t0 + d < T) {
+                    float* orow = o + ((static_cast<int64_t>(b) * T + t0 + d) * Hv + h) * V + vs0;
 #pragma unroll
                     for (int v4 = 0; v4 < 8; ++v4)
                         *reinterpret_cast<float4*>(orow + 4 * v4) =
                             make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
                                         scale * __uint_as_float(x[4 * v4 + 2]), scale * __uint_as_float(x[4 * v4 + 3]));
                 }
+                tc_fence_before();
             }
-            uint32_t x[32];
-            tmem_ld_32x32b_x32(D2 + lane_base, x);
-            tmem_wait_ld();
-            if (has_row) {
-                const float eg = expf(glast);
-#pragma unroll
-                for (int v = 0; v < 32; ++v) {
-                    S[v] = fmaf(eg, S[v], __uint_as_float(x[v]));
-                    sm.b1[kmaj(v, tid, K)] = __uint_as_float(to_tf32(S[v]));
-                }
-            }
-            if (c + 1 < NC) load_ut(c + 1);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-    }
-    cp_async_wait<0>();
-    if (state_out && has_row) {
+        if (ok && state_out && has_row) {
 #pragma unroll
-        for (int v4 = 0; v4 < 8; ++v4)
-            *reinterpret_cast<float4*>(state_out + sbase + static_cast<int64_t>(tid) * V + vs0 + 4 * v4) =
-                make_float4(S[4 * v4], S[4 * v4 + 1], S[4 * v4 + 2], S[4 * v4 + 3]);
+            for (int v4 = 0; v4 < 8; ++v4)
+                *reinterpret_cast<float4*>(state_out + sbase + static_cast<int64_t>(d) * V + vs0 + 4 * v4) =
+                    make_float4(S[4 * v4], S[4 * v4 + 1], S[4 * v4 + 2], S[4 * v4 + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, 128);
     }
-}
-
-struct ChunkWs {
-    float *Wt, *Ut, *Mt, *Gt;
-    size_t bytes;
-};
-
-ChunkWs chunk_ws(void* base, int B, int64_t T, const gdn_dims& d) {
-    const int64_t NC = (T + CH - 1) / CH;
-    const int64_t units = static_cast<int64_t>(B) * d.Hv * NC;
-    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t w = al(units * CH * d.K * 4), u = al(units * CH * d.V * 4), m = al(units * CH * CH * 4),
-                 gg = al(units * CH * 4);
-    ChunkWs ws;
-    char* p = static_cast<char*>(base);
-    ws.Wt = reinterpret_cast<float*>(p);
-    ws.Ut = reinterpret_cast<float*>(p + w);
-    ws.Mt = reinterpret_cast<float*>(p + w + u);
-    ws.Gt = reinterpret_cast<float*>(p + w + u + m);
-    ws.bytes = w + u + m + gg;
-    return ws;
 }
 
 template <int K, int V>
 nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                                const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form,
-                               const float* s_in, float* s_out, float* o, const ChunkWs& ws, cudaStream_t st) {
+                               const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st) {
     const int NC = static_cast<int>((T + CH - 1) / CH);
     const int prep_smem = sizeof(PrepSmem<K, V>);
-    const int seq_smem = sizeof(SeqSmem<K>);
+    const int seq_smem = SeqLayout<K>::BYTES;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_done[dev]) {
         cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prep)");
-        e = cudaFuncSetAttribute(chunk_seq_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
+        e = cudaFuncSetAttribute(chunk_seq_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq)");
-        e = cudaFuncSetAttribute(chunk_seq_tc_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(SeqTcSmem<K>)));
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq tc)");
         attr_done[dev] = true;
     }
+    unsigned int* err = device_error_word();
+    if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
+    uint8_t* recs = static_cast<uint8_t*>(ws);
     const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
-    chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, ws.Wt,
-                                                                 ws.Ut, ws.Mt, ws.Gt);
+    chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, recs);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    const char* var = getenv("NVFP4_SCAN_SEQ_VARIANT");
-    if (!var || strcmp(var, "tc") != 0) {
-        chunk_seq_kernel<K><<<seq_blocks, 256, seq_smem, st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt, ws.Ut, ws.Mt,
-                                                               ws.Gt, s_in, s_out, o);
-    } else {
-        unsigned int* err = device_error_word();
-        if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
-        chunk_seq_tc_kernel<K><<<seq_blocks, 128, sizeof(SeqTcSmem<K>), st>>>(q, k, T, d.Hk, d.Hv, V, scale, NC, ws.Wt,
-                                                                              ws.Ut, ws.Mt, ws.Gt, s_in, s_out, o, err);
-    }
+    chunk_seq_kernel<K, V><<<seq_blocks, 192, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     return NVFP4_OK;
+}
+
+size_t chunk_rec_bytes(const gdn_dims& d) {
+    if (d.K == 128 && d.V == 128) return ChunkRec<128, 128>::BYTES;
+    if (d.K == 128 && d.V == 64) return ChunkRec<128, 64>::BYTES;
+    if (d.K == 64 && d.V == 128) return ChunkRec<64, 128>::BYTES;
+    return ChunkRec<64, 64>::BYTES;
 }
 
 }  // namespace
@@ -906,7 +694,8 @@ nvfp4_status validate_dims(const gdn_dims* d);
 size_t scan_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo) {
     const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
     if (!chunked) return 0;
-    return chunk_ws(nullptr, B, T, d).bytes;
+    const int64_t NC = (T + CH - 1) / CH;
+    return static_cast<size_t>(B) * d.Hv * NC * chunk_rec_bytes(d);
 }
 
 nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
@@ -925,14 +714,13 @@ nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t
         if (e != cudaSuccess) return cuda_fail(e, "recurrent scan launch");
         return NVFP4_OK;
     }
-    const ChunkWs cws = chunk_ws(ws, B, T, d);
     if (d.K == 128 && d.V == 128)
-        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
     if (d.K == 128 && d.V == 64)
-        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
     if (d.K == 64 && d.V == 128)
-        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
-    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, cws, st);
+        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
+    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
 }
 
 }  // namespace nvg

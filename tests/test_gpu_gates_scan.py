@@ -17,16 +17,6 @@ pytestmark = pytest.mark.gpu
 SCAN_TOL = 2e-3
 
 
-@pytest.fixture(params=["tc", "mmasync"])
-def seq_variant(request, monkeypatch):
-    """Sequential chunk kernel: the mma.sync one (default) or tcgen05."""
-    if request.param == "tc":
-        monkeypatch.setenv("NVFP4_SCAN_SEQ_VARIANT", "tc")
-    else:
-        monkeypatch.delenv("NVFP4_SCAN_SEQ_VARIANT", raising=False)
-    return request.param
-
-
 @pytest.mark.parametrize("n,Hk,Hv,K,V", [(64, 2, 2, 64, 64), (300, 16, 32, 128, 128), (5, 1, 4, 128, 64)])
 def test_gates_match_oracle(cuda_dev, n, Hk, Hv, K, V):
     dims = nv.GdnDims(Hk, Hv, K, V)
@@ -66,14 +56,14 @@ def _scan_case(B, T, Hk, Hv, K, V, seed, form, algo, state=True, alpha=(0.9, 0.9
     (1, 1, 1, 2, 128, 64),       # one token (decode)
     (1, 130, 2, 2, 64, 128),     # K != V
 ])
-def test_scan_matches_oracle(cuda_dev, seq_variant, algo, form, B, T, Hk, Hv, K, V):
+def test_scan_matches_oracle(cuda_dev, algo, form, B, T, Hk, Hv, K, V):
     o, S, o_ref, S_ref = _scan_case(B, T, Hk, Hv, K, V, 11 + T, form, algo)
     assert rel_fro(o, o_ref) <= SCAN_TOL
     assert rel_fro(S, S_ref) <= SCAN_TOL
 
 
 @pytest.mark.parametrize("algo", [nv.SCAN_RECURRENT, nv.SCAN_CHUNKED])
-def test_scan_long_memory(cuda_dev, seq_variant, algo):
+def test_scan_long_memory(cuda_dev, algo):
     """alpha in (0.99, 0.9999): the state carries over all 16 chunks."""
     o, S, o_ref, S_ref = _scan_case(1, 1000, 1, 2, 128, 128, 5, nv.FORM_PAGES, algo, alpha=(0.99, 0.9999))
     assert rel_fro(o, o_ref) <= SCAN_TOL
@@ -103,7 +93,7 @@ def test_scan_chaining_on_gpu(cuda_dev, t, tol):
     assert rel_fro(end.cpu().numpy(), full_s.cpu().numpy()) <= tol
 
 
-def test_scan_full_size_subset_of_heads(cuda_dev, seq_variant):
+def test_scan_full_size_subset_of_heads(cuda_dev):
     """T = 4096, 16 key / 32 value heads, K = V = 128 (the layer-prefill scan
     launch); the oracle recomputes value heads 0, 1 and 31."""
     B, T, Hk, Hv, K, V = 1, 4096, 16, 32, 128, 128

@@ -31,7 +31,7 @@ def _inputs(seed, B, T, Hk, Hv, K, V):
 
 @pytest.mark.parametrize("form", [nv.FORM_PAGES, nv.FORM_STANDARD])
 def test_noalloc_scan_matches_workspace_scan_twice(cuda_dev, form):
-    cases = [(1, 1000, 16, 32, 128, 128, 3), (2, 130, 2, 4, 64, 128, 4)]   # two calls, different shapes
+    cases = [(1, 800, 16, 32, 128, 128, 3), (2, 130, 2, 4, 64, 128, 4)]   # two calls, different shapes
     for B, T, Hk, Hv, K, V, seed in cases:
         dims = nv.GdnDims(Hk, Hv, K, V)
         q, k, v, g, beta, S0 = _inputs(seed, B, T, Hk, Hv, K, V)
@@ -48,14 +48,14 @@ def test_noalloc_scan_matches_workspace_scan_twice(cuda_dev, form):
 
 
 def test_noalloc_scan_refuses_oversize(cuda_dev):
-    # B = 1, 32 value heads of 128 x 128: 1600 tokens fit in the 64 MiB array, 1664 do not
+    # B = 1, 32 value heads of 128 x 128: 896 tokens fit in the 64 MiB array, 960 do not
     B, Hk, Hv, K, V = 1, 16, 32, 128, 128
     dims = nv.GdnDims(Hk, Hv, K, V)
-    q, k, v, g, beta, S0 = _inputs(5, B, 1664, Hk, Hv, K, V)
+    q, k, v, g, beta, S0 = _inputs(5, B, 960, Hk, Hv, K, V)
     with pytest.raises(nv.NVFP4Error) as ei:
-        nv.gdn_scan_noalloc(q, k, v, g, beta, B, 1664, dims)
+        nv.gdn_scan_noalloc(q, k, v, g, beta, B, 960, dims)
     assert ei.value.status == 6 and "scratch" in str(ei.value)
-    o, _ = nv.gdn_scan_noalloc(q[:1600], k[:1600], v[:1600], g[:1600], beta[:1600], B, 1600, dims)
+    o, _ = nv.gdn_scan_noalloc(q[:896], k[:896], v[:896], g[:896], beta[:896], B, 896, dims)
     torch.cuda.synchronize()
     assert torch.isfinite(o).all()
     assert nv.NOALLOC_MAX_SCRATCH_BYTES == 64 << 20
