@@ -131,30 +131,6 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// 3xTF32: a*b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi (float32-level accuracy).
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-    hi = to_tf32(x);
-    lo = to_tf32(x - __uint_as_float(hi));
-}
-
-template <bool PREC3>
-__device__ __forceinline__ void mma_f32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
-    if constexpr (PREC3) {
-        uint32_t ah[4], al[4], bh[2], bl[2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], al[i]);
-        split_tf32(b[0], bh[0], bl[0]);
-        split_tf32(b[1], bh[1], bl[1]);
-        mma_tf32(d, al, bh);
-        mma_tf32(d, ah, bl);
-        mma_tf32(d, ah, bh);
-    } else {
-        const uint32_t ai[4] = {to_tf32(a[0]), to_tf32(a[1]), to_tf32(a[2]), to_tf32(a[3])};
-        const uint32_t bi[2] = {to_tf32(b[0]), to_tf32(b[1])};
-        mma_tf32(d, ai, bi);
-    }
-}
-
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
@@ -180,40 +156,49 @@ struct PrepSmem {
     float gin[CH], gd[CH], bet[CH], graw[CH], df[CH];
 };
 
-// Output tile X [64 x 8*NT] = (T diag(s)) B with B [64 x 8*NT] (row stride KS) in
-// shared memory; warp rows r0..r0+15; 3xTF32 (hi/lo split) so the product is
-// float32-accurate.  Each pair of adjacent outputs (t, col), (t, col+1), col even,
-// goes to store(t, col, x0, x1).
-template <int NT, int KS, int TS, typename Store>
+// X = (T diag(s)) B for a 32-column strip of X: T [64 x 64] unit lower triangular
+// (row stride TS), B [64 x N] (row stride KS), columns c0..c0+31, all 64 rows; one
+// warp.  TF32 tensor cores (operands rounded to nearest), float32 accumulation; the
+// k-steps above the diagonal of each 16-row tile are skipped (T is zero there).
+// Each pair of adjacent outputs (t, col), (t, col+1), col even, goes to
+// store(t, col, x0, x1).
+template <int KS, int TS, typename Store>
 __device__ __forceinline__ void tri_apply(const float* __restrict__ Tm, const float* __restrict__ s,
-                                          const float* __restrict__ Bm, int r0, int lane, Store store) {
+                                          const float* __restrict__ Bm, int c0, int lane, Store store) {
     const int grp = lane >> 2, tig = lane & 3;
-    float acc[NT][4];
+    float acc[4][4][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 2
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) acc[m][nt][0] = acc[m][nt][1] = acc[m][nt][2] = acc[m][nt][3] = 0.f;
+#pragma unroll
     for (int k0 = 0; k0 < CH; k0 += 8) {
+        uint32_t bf[4][2];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            bf[nt][0] = to_tf32(Bm[(k0 + tig) * KS + c0 + nt * 8 + grp]);
+            bf[nt][1] = to_tf32(Bm[(k0 + tig + 4) * KS + c0 + nt * 8 + grp]);
+        }
         const float s0 = s[k0 + tig], s1 = s[k0 + tig + 4];
-        const float af[4] = {Tm[(r0 + grp) * TS + k0 + tig] * s0, Tm[(r0 + grp + 8) * TS + k0 + tig] * s0,
-                             Tm[(r0 + grp) * TS + k0 + tig + 4] * s1, Tm[(r0 + grp + 8) * TS + k0 + tig + 4] * s1};
-        uint32_t ah[4], al[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) split_tf32(af[i], ah[i], al[i]);
+        for (int m = 0; m < 4; ++m) {
+            if (k0 >= 16 * (m + 1)) continue;
+            const int r0 = 16 * m;
+            const uint32_t a[4] = {to_tf32(Tm[(r0 + grp) * TS + k0 + tig] * s0),
+                                   to_tf32(Tm[(r0 + grp + 8) * TS + k0 + tig] * s0),
+                                   to_tf32(Tm[(r0 + grp) * TS + k0 + tig + 4] * s1),
+                                   to_tf32(Tm[(r0 + grp + 8) * TS + k0 + tig + 4] * s1)};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            uint32_t bh[2], bl[2];
-            split_tf32(Bm[(k0 + tig) * KS + nt * 8 + grp], bh[0], bl[0]);
-            split_tf32(Bm[(k0 + tig + 4) * KS + nt * 8 + grp], bh[1], bl[1]);
-            mma_tf32(acc[nt], al, bh);
-            mma_tf32(acc[nt], ah, bl);
-            mma_tf32(acc[nt], ah, bh);
+            for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[m][nt], a, bf[nt]);
         }
     }
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) store(r0 + grp + hh * 8, nt * 8 + 2 * tig, acc[nt][2 * hh], acc[nt][2 * hh + 1]);
-    }
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                store(16 * m + grp + hh * 8, c0 + nt * 8 + 2 * tig, acc[m][nt][2 * hh], acc[m][nt][2 * hh + 1]);
 }
 
 template <int K, int V>
@@ -283,10 +268,14 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         for (int k0 = 0; k0 < K; k0 += 8) {
             const float a[4] = {A[(r0 + grp) * KS + k0 + tig], A[(r0 + grp + 8) * KS + k0 + tig],
                                 A[(r0 + grp) * KS + k0 + tig + 4], A[(r0 + grp + 8) * KS + k0 + tig + 4]};
+            const uint32_t ai[4] = {to_tf32(a[0]), to_tf32(a[1]), to_tf32(a[2]), to_tf32(a[3])};
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
-                const float bb[2] = {sm.ks[(nt * 8 + grp) * KS + k0 + tig], sm.ks[(nt * 8 + grp) * KS + k0 + tig + 4]};
-                mma_f32<false>(acc[nt], a, bb);
+                // tiles right of this warp's diagonal block are masked out afterwards
+                if (nt * 8 > r0 + 15) continue;
+                const uint32_t bb[2] = {to_tf32(sm.ks[(nt * 8 + grp) * KS + k0 + tig]),
+                                        to_tf32(sm.ks[(nt * 8 + grp) * KS + k0 + tig + 4])};
+                mma_tf32(acc[nt], ai, bb);
             }
         }
 #pragma unroll
@@ -382,16 +371,20 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     __syncthreads();
     // W~ = T diag(b e^{Gd}) K (warps 0-3, stored TF32-rounded: a tensor-core operand downstream)
     // U~ = T diag(beta) V   (warps 4-7)
-    if (warp < 4) {
-        tri_apply<K / 8, KS, TS>(sm.T, sm.df, sm.ks, warp * 16, lane, [&](int t, int col, float x0, float x1) {
-            *reinterpret_cast<float2*>(rec + RC::A1 + sw128_off(CH + t, col, 128)) =
-                make_float2(__uint_as_float(to_tf32(x0)), __uint_as_float(to_tf32(x1)));
-        });
-    } else {
-        tri_apply<V / 8, KS, TS>(sm.T, sm.bet, sm.qs, (warp - 4) * 16, lane, [&](int t, int col, float x0, float x1) {
-            *reinterpret_cast<float2*>(rec + RC::UT + (col >> 5) * RC::UT_SLICE + sw128_off(t, col & 31, CH)) =
-                make_float2(x0, x1);
-        });
+    // 32-column strips: W~ strips first (K/32 of them), then U~ strips (V/32), over the 8 warps
+    for (int strip = warp; strip < K / 32 + V / 32; strip += 8) {
+        if (strip < K / 32) {
+            tri_apply<KS, TS>(sm.T, sm.df, sm.ks, 32 * strip, lane, [&](int t, int col, float x0, float x1) {
+                *reinterpret_cast<float2*>(rec + RC::A1 + sw128_off(CH + t, col, 128)) =
+                    make_float2(__uint_as_float(to_tf32(x0)), __uint_as_float(to_tf32(x1)));
+            });
+        } else {
+            const int vs = strip - K / 32;
+            tri_apply<KS, TS>(sm.T, sm.bet, sm.qs, 32 * vs, lane, [&](int t, int col, float x0, float x1) {
+                *reinterpret_cast<float2*>(rec + RC::UT + vs * RC::UT_SLICE + sw128_off(t, col - 32 * vs, CH)) =
+                    make_float2(x0, x1);
+            });
+        }
     }
 }
 
