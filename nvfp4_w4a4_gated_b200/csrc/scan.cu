@@ -154,6 +154,7 @@ struct PrepSmem {
     float T[CH * TS];                  // (I + L)^-1
     float P[3 * 256];                  // 16 x 16 block products
     float gin[CH], gd[CH], bet[CH], graw[CH], df[CH];
+    float eG[CH], eKh[CH];             // e^{G_t}, e^{G_C - G_t}
 };
 
 // X = (T diag(s)) B for a 32-column strip of X: T [64 x 64] unit lower triangular
@@ -251,8 +252,17 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         const float g0 = excl + a0, g1 = s;
         sm.gin[2 * lane] = g0;
         sm.gin[2 * lane + 1] = g1;
-        sm.gd[2 * lane] = form == GDN_FORM_STANDARD ? g0 : excl;
-        sm.gd[2 * lane + 1] = form == GDN_FORM_STANDARD ? g1 : g0;
+        const float d0 = form == GDN_FORM_STANDARD ? g0 : excl;
+        const float d1 = form == GDN_FORM_STANDARD ? g1 : g0;
+        sm.gd[2 * lane] = d0;
+        sm.gd[2 * lane + 1] = d1;
+        const float gc = __shfl_sync(0xffffffffu, g1, 31);
+        sm.eG[2 * lane] = expf(g0);
+        sm.eG[2 * lane + 1] = expf(g1);
+        sm.eKh[2 * lane] = expf(gc - g0);
+        sm.eKh[2 * lane + 1] = expf(gc - g1);
+        sm.df[2 * lane] = sm.bet[2 * lane] * expf(d0);
+        sm.df[2 * lane + 1] = sm.bet[2 * lane + 1] * expf(d1);
     }
     __syncthreads();
 
@@ -285,25 +295,24 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 const int t = r0 + grp + hh * 8;
                 const int i = nt * 8 + 2 * tig;
                 if (warp < 4) {
-                    sm.L[t * CH + i] = (i < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
+                    sm.L[t * CH + i] = (i < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
                     sm.L[t * CH + i + 1] =
-                        (i + 1 < t) ? sm.bet[t] * expf(sm.gd[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
+                        (i + 1 < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
                 } else {
                     // rounded to TF32 here: it is only ever a tensor-core operand
-                    const float m0 = (i <= t) ? expf(sm.gin[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
-                    const float m1 = (i + 1 <= t) ? expf(sm.gin[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
+                    const float m0 = (i <= t) ? __expf(sm.gin[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
+                    const float m1 = (i + 1 <= t) ? __expf(sm.gin[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
                     *reinterpret_cast<float2*>(rec + RC::A2 + sw128_off(t, i, CH)) =
                         make_float2(__uint_as_float(to_tf32(m0)), __uint_as_float(to_tf32(m1)));
                 }
             }
         }
     }
-    if (tid < CH) sm.df[tid] = sm.bet[tid] * expf(sm.gd[tid]);
     if (tid == 0) *reinterpret_cast<float*>(rec + RC::GC) = sm.gin[CH - 1];
     // Q~ = e^{G_t} q_t (rows 0..63 of A1) and K^ ^T, K^_t = e^{G_C - G_t} k_t (A3), TF32-rounded
     for (int idx = tid; idx < CH * (K / 4); idx += 256) {
         const int t = idx / (K / 4), c4 = idx - t * (K / 4);
-        const float eg = expf(sm.gin[t]);
+        const float eg = sm.eG[t];
         const float4 x = *reinterpret_cast<const float4*>(&sm.qs[t * KS + 4 * c4]);
         *reinterpret_cast<float4*>(rec + RC::A1 + sw128_off(t, 4 * c4, 128)) =
             make_float4(__uint_as_float(to_tf32(eg * x.x)), __uint_as_float(to_tf32(eg * x.y)),
@@ -311,10 +320,9 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     }
     for (int idx = tid; idx < K * (CH / 4); idx += 256) {
         const int dd = idx % K, t4 = idx / K;
-        const float gc = sm.gin[CH - 1];
         float x[4];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(to_tf32(expf(gc - sm.gin[4 * t4 + w]) * sm.ks[(4 * t4 + w) * KS + dd]));
+        for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(to_tf32(sm.eKh[4 * t4 + w] * sm.ks[(4 * t4 + w) * KS + dd]));
         *reinterpret_cast<float4*>(rec + RC::A3 + sw128_off(dd, 4 * t4, 128)) = make_float4(x[0], x[1], x[2], x[3]);
     }
     constexpr int TS = SM::TS;
@@ -392,15 +400,17 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
 // One CTA per (sequence, value head, 32-column slice of V) walks the chunks in
 // order, on the tcgen05 tensor cores (kind::tf32, float32 accumulation in TMEM,
 // M = 128, N = 32).  Per chunk:
-//   round 1:  D1 = [Q~; W~] S0        rows 0..63: Q~ S0, rows 64..127: W~ S0
+//   R1:   D1 = [Q~; W~] S0          rows 0..63: Q~ S0, rows 64..127: W~ S0
 //   U = U~ - W~ S0 (TF32)  ->  U^T in shared memory
-//   round 2:  D1 += [Mqk; *] U         rows 0..63: o / scale (rows 64..127 unused)
-//             D2  = K^ ^T U             K^_t = e^{G_C - G_t} k_t
+//   R2a:  D2  = K^ ^T U              K^_t = e^{G_C - G_t} k_t
+//   R2b:  D1 += [Mqk; *] U           rows 0..63: o / scale (rows 64..127 unused)
 //   S <- e^{G_C} S + D2 (float32, registers)  ->  S^T (TF32) in shared memory
-// Warp roles: warp 0 copies the chunk records into shared memory (bulk copies,
-// [Q~; W~] and U~ double-buffered), warp 1 issues the MMAs, warps 2..5 (one per
-// TMEM lane quarter) form U, the state and the output.  D1 alternates between two
-// TMEM buffers so the output of chunk c drains while round 1 of chunk c+1 runs.
+// The recurrence runs through R1 -> U -> R2a -> S only; R2b and the output rows
+// drain while the next chunk's R1 and U run (D1 alternates between two TMEM
+// buffers).  Warp 0 copies the chunk records into shared memory (bulk copies,
+// [Q~; W~] and U~ double-buffered); warps 1..4 (one per TMEM lane quarter) form
+// U, the state and the output, and one lane of warp 2 issues the MMAs right
+// after the named barrier that publishes their operands.
 template <int K>
 struct SeqLayout {
     static constexpr uint32_t A1_BYTES = 128 * K * 4;
@@ -416,22 +426,26 @@ struct SeqLayout {
 };
 
 enum SeqBar : int {
-    kA1Full = 0,   // [2]
-    kA1Empty = 2,  // [2]
-    kA23Full = 4,
-    kA23Empty = 5,
-    kUtFull = 6,   // [2]
-    kUtEmpty = 8,  // [2]
+    kA1Full = 0,   // [2] [Q~; W~] stage landed
+    kA1Empty = 2,  // [2] R1 has read the stage
+    kA2Full = 4,   // Mqk landed
+    kA3Full = 5,   // K^ ^T landed
+    kUtFull = 6,   // [2] U~ slice stage landed
+    kUtEmpty = 8,  // [2] U~ slice read (one arrival per U warp)
     kR1Done = 10,
-    kR2Done = 11,
-    kUReady = 12,
-    kSReady = 13,
-    kFin = 14,
-    kNumSeqBars = 15
+    kR2Done = 11,  // R2a complete: the state update may start, K^ ^T is free
+    kODone = 12,   // R2b complete: output rows of D1 final, U^T and Mqk free
+    kOFree = 13,   // the output warps have drained D1 of the previous chunk
+    kUReady = 14,  // R2a issued (the producer then issues R2b)
+    kFin = 15,     // completion of the MMA warp's MMAs
+    kFinP = 16,    // completion of the producer's MMAs
+    kSReady = 17,  // S^T published (one arrival per compute warp)
+    kUPub = 18,    // U^T published (one arrival per U warp)
+    kNumSeqBars = 19
 };
 
 template <int K, int V>
-__global__ void __launch_bounds__(192, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
+__global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
                                                            float scale, int NC, const float* state_in,
                                                            float* state_out, float* __restrict__ o,
                                                            unsigned int* __restrict__ err) {
@@ -451,10 +465,8 @@ __global__ void __launch_bounds__(192, 1) chunk_seq_kernel(const uint8_t* __rest
     constexpr uint32_t IDESC = idesc_tf32(128, 32, false, false);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNumSeqBars; ++i) {
-            const bool many = i == kUtEmpty || i == kUtEmpty + 1 || i == kUReady;
-            mbar_init(&bar[i], i == kSReady ? 128 : (many ? 64 : 1));
-        }
+        for (int i = 0; i < kNumSeqBars; ++i)
+            mbar_init(&bar[i], i == kSReady ? 8 : (i == kUtEmpty || i == kUtEmpty + 1 || i == kOFree || i == kUPub) ? 4 : 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -468,171 +480,260 @@ __global__ void __launch_bounds__(192, 1) chunk_seq_kernel(const uint8_t* __rest
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---- producer: chunk records -> shared memory
-            int last_c = -1;  // last chunk whose three sections were all issued
-            int last_a1 = -1, last_ut = -1;
-            for (int c = 0; c < NC; ++c) {
-                const uint8_t* rc = rec0 + static_cast<int64_t>(c) * RC::BYTES;
+            // ---- producer: chunk records -> shared memory, and R2b (off the recurrence)
+            auto load_a1 = [&](int c) {
                 const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&bar[kA1Empty + s], ((c >> 1) - 1) & 1, err, kErrTimeoutSeq)) break;
                 mbar_arrive_expect_tx(&bar[kA1Full + s], L::A1_BYTES);
                 for (uint32_t p = 0; p < L::A1_BYTES; p += 16384)
-                    bulk_load(sm + L::A1 + s * L::A1_BYTES + p, rc + RC::A1 + p, 16384, &bar[kA1Full + s]);
-                last_a1 = c;
-                if (c >= 2 && !mbar_wait(&bar[kUtEmpty + s], ((c >> 1) - 1) & 1, err, kErrTimeoutSeq)) break;
+                    bulk_load(sm + L::A1 + s * L::A1_BYTES + p, rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::A1 + p,
+                              16384, &bar[kA1Full + s]);
+            };
+            auto load_ut = [&](int c) {
+                const int s = c & 1;
                 mbar_arrive_expect_tx(&bar[kUtFull + s], L::UT_BYTES);
-                bulk_load(sm + L::UT + s * L::UT_BYTES, rc + RC::UT + slice * RC::UT_SLICE, L::UT_BYTES,
+                bulk_load(sm + L::UT + s * L::UT_BYTES,
+                          rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::UT + slice * RC::UT_SLICE, L::UT_BYTES,
                           &bar[kUtFull + s]);
-                last_ut = c;
-                if (c >= 1 && !mbar_wait(&bar[kA23Empty], (c - 1) & 1, err, kErrTimeoutSeq)) break;
-                mbar_arrive_expect_tx(&bar[kA23Full], L::A23_BYTES);
-                for (uint32_t p = 0; p < L::A23_BYTES; p += 16384)
-                    bulk_load(sm + L::A23 + p, rc + RC::A2 + p, 16384, &bar[kA23Full]);
-                last_c = c;
+            };
+            auto load_m = [&](int c) {
+                mbar_arrive_expect_tx(&bar[kA2Full], CH * CH * 4);
+                bulk_load(sm + L::A23, rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::A2, CH * CH * 4, &bar[kA2Full]);
+            };
+            auto load_kh = [&](int c) {
+                mbar_arrive_expect_tx(&bar[kA3Full], RC::A3_BYTES);
+                for (uint32_t p = 0; p < RC::A3_BYTES; p += 16384)
+                    bulk_load(sm + L::A23 + CH * CH * 4 + p, rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::A3 + p,
+                              16384, &bar[kA3Full]);
+            };
+            // the sections of chunk c this CTA reads, pulled into L2 ahead of their copies
+            auto prefetch = [&](int c) {
+                const uint8_t* rc = rec0 + static_cast<int64_t>(c) * RC::BYTES;
+                for (uint32_t p = 0; p < RC::UT; p += 16384) bulk_prefetch_l2(rc + p, 16384);
+                bulk_prefetch_l2(rc + RC::UT + slice * RC::UT_SLICE, RC::UT_SLICE);
+            };
+            const uint32_t a2 = smem_u32(sm + L::A23), b2 = smem_u32(sm + L::B2);
+            int last_a1 = 0, last_ut = 0, last_m = 0, last_kh = 0;   // last chunk issued to each buffer
+            bool mma_issued = false;
+            load_a1(0);
+            load_ut(0);
+            load_m(0);
+            load_kh(0);
+            if (NC > 1) {
+                load_a1(1);
+                load_ut(1);
+                last_a1 = last_ut = 1;
             }
-            // every copy issued has landed before the CTA may exit
+            for (int c = 1; c < 3 && c < NC; ++c) prefetch(c);
+            for (int c = 0; c < NC; ++c) {
+                const int s = c & 1;
+                // R2b(c): D1[s] += Mqk U once U^T is published and R2a(c) has left the tensor
+                // pipe (so R2b runs during the state update instead of ahead of it), with D1[s]
+                // of chunk c-2 drained
+                if (c + 3 < NC) prefetch(c + 3);
+                bool w = mbar_wait(&bar[kUReady], c & 1, err, kErrTimeoutSeq) &&
+                         mbar_wait(&bar[kR2Done], c & 1, err, kErrTimeoutSeq);
+                if (!w) break;
+                // R2a(c) has read K^ ^T: bring in the next chunk's
+                if (c + 1 < NC) {
+                    load_kh(c + 1);
+                    last_kh = c + 1;
+                }
+                w = mbar_wait(&bar[kA2Full], c & 1, err, kErrTimeoutSeq) &&
+                    (c == 0 || mbar_wait(&bar[kOFree], (c - 1) & 1, err, kErrTimeoutSeq));
+                if (!w) break;
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < CH / 8; ++j)
+                    mma_tf32_ss(tmem + 32 * s, sdesc_kmajor_sw128(a2 + (j >> 2) * CH * 128 + (j & 3) * 32),
+                                sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, 1u);
+                mma_commit(&bar[kODone]);
+                mma_issued = true;
+                // Mqk of chunk c+1 once R2b(c) has read this chunk's
+                if (c + 1 < NC) {
+                    if (!mbar_wait(&bar[kODone], c & 1, err, kErrTimeoutSeq)) break;
+                    load_m(c + 1);
+                    last_m = c + 1;
+                }
+                // [Q~; W~] and U~ of chunk c+2 into the stage chunk c used
+                if (c + 2 < NC) {
+                    if (!mbar_wait(&bar[kA1Empty + s], (c >> 1) & 1, err, kErrTimeoutSeq)) break;
+                    load_a1(c + 2);
+                    last_a1 = c + 2;
+                    if (!mbar_wait(&bar[kUtEmpty + s], (c >> 1) & 1, err, kErrTimeoutSeq)) break;
+                    load_ut(c + 2);
+                    last_ut = c + 2;
+                }
+            }
+            // every copy issued has landed, and every MMA issued here has completed, before exit
             // (stage s last received chunk last - (last - s) % 2, for the last chunk issued to it)
             for (int s = 0; s < 2; ++s) {
                 const int ca = last_a1 - ((last_a1 - s) & 1), cu = last_ut - ((last_ut - s) & 1);
                 if (ca >= 0) mbar_wait(&bar[kA1Full + s], (ca >> 1) & 1, err, kErrTimeoutSeq);
                 if (cu >= 0) mbar_wait(&bar[kUtFull + s], (cu >> 1) & 1, err, kErrTimeoutSeq);
             }
-            if (last_c >= 0) mbar_wait(&bar[kA23Full], last_c & 1, err, kErrTimeoutSeq);
+            mbar_wait(&bar[kA2Full], last_m & 1, err, kErrTimeoutSeq);
+            mbar_wait(&bar[kA3Full], last_kh & 1, err, kErrTimeoutSeq);
+            if (mma_issued) {
+                mma_commit(&bar[kFinP]);
+                mbar_wait(&bar[kFinP], 0, err, kErrTimeoutSeq);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ---- MMA issuer
+            // ---- MMA warp: R1 and R2a, the two products on the recurrence
             const uint32_t b1 = smem_u32(sm + L::B1), b2 = smem_u32(sm + L::B2);
-            const uint32_t a2 = smem_u32(sm + L::A23), a3 = a2 + CH * CH * 4;
-            const uint32_t D2 = tmem + 64;
+            const uint32_t a3 = smem_u32(sm + L::A23) + CH * CH * 4;
             for (int c = 0; c < NC; ++c) {
                 const int s = c & 1;
-                const uint32_t D1 = tmem + 32 * s;
-                if (!mbar_wait(&bar[kSReady], c & 1, err, kErrTimeoutSeq)) break;
-                if (!mbar_wait(&bar[kA1Full + s], (c >> 1) & 1, err, kErrTimeoutSeq)) break;
+                if (!mbar_wait(&bar[kSReady], c & 1, err, kErrTimeoutSeq) ||
+                    !mbar_wait(&bar[kA1Full + s], (c >> 1) & 1, err, kErrTimeoutSeq))
+                    break;
                 tc_fence_after();
                 const uint32_t a1 = smem_u32(sm + L::A1 + s * L::A1_BYTES);
 #pragma unroll
                 for (int j = 0; j < K / 8; ++j)
-                    mma_tf32_ss(D1, sdesc_kmajor_sw128(a1 + (j >> 2) * 128 * 128 + (j & 3) * 32),
+                    mma_tf32_ss(tmem + 32 * s, sdesc_kmajor_sw128(a1 + (j >> 2) * 128 * 128 + (j & 3) * 32),
                                 sdesc_kmajor_sw128(b1 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
                 mma_commit(&bar[kA1Empty + s]);
                 mma_commit(&bar[kR1Done]);
-                if (!mbar_wait(&bar[kUReady], c & 1, err, kErrTimeoutSeq)) break;
-                if (!mbar_wait(&bar[kA23Full], c & 1, err, kErrTimeoutSeq)) break;
+                if (!mbar_wait(&bar[kUPub], c & 1, err, kErrTimeoutSeq) ||
+                    !mbar_wait(&bar[kA3Full], c & 1, err, kErrTimeoutSeq))
+                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int j = 0; j < CH / 8; ++j)
-                    mma_tf32_ss(D1, sdesc_kmajor_sw128(a2 + (j >> 2) * CH * 128 + (j & 3) * 32),
-                                sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, 1u);
-#pragma unroll
-                for (int j = 0; j < CH / 8; ++j)
-                    mma_tf32_ss(D2, sdesc_kmajor_sw128(a3 + (j >> 2) * 128 * 128 + (j & 3) * 32),
+                    mma_tf32_ss(tmem + 64, sdesc_kmajor_sw128(a3 + (j >> 2) * 128 * 128 + (j & 3) * 32),
                                 sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
-                mma_commit(&bar[kA23Empty]);
                 mma_commit(&bar[kR2Done]);
+                mbar_arrive(&bar[kUReady]);
             }
-            // all MMAs issued have completed before TMEM is released
+            // all MMAs issued here have completed before TMEM is released
             mma_commit(&bar[kFin]);
             mbar_wait(&bar[kFin], 0, err, kErrTimeoutSeq);
         }
     } else {
-        // ---- warps 2..5: TMEM lane quarter q = warp % 4
+        // ---- warps 2..9: TMEM lane quarter q = warp % 4, columns c0..c0+15 of the slice
         const int q = warp & 3;
+        const int c0 = 16 * ((warp - 2) >> 2);
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int d = q * 32 + lane;             // state row
         const bool has_row = d < K;
-        const bool u_role = q >= 2;              // tokens 0..63 of W~ S0 live in lanes 64..127
+        const bool u_role = q >= 2;              // W~ S0 of tokens 0..63 lands in lanes 64..127
         const int tu = d - 64;
         const int64_t sbase = (static_cast<int64_t>(b) * Hv + h) * K * V;
+        // Byte offsets of (row c0 + i, column col) in a 32-row K-major swizzled image:
+        // base + (i / 8) * 1024 + xo[i % 8] (only 8 swizzle patterns per column).
+        auto swz_cols = [&](int col, uint32_t& base, uint32_t (&xo)[8]) {
+            base = (col >> 5) * 32 * 128 + ((col & 3) << 2) + c0 * 128;
+#pragma unroll
+            for (int r = 0; r < 8; ++r) xo[r] = r * 128 + ((((col & 31) >> 2) ^ r) << 4);
+        };
         uint8_t* b1p = sm + L::B1;
         uint8_t* b2p = sm + L::B2;
-        float S[32];
+        uint32_t s_base = 0, s_xo[8];
+        swz_cols(has_row ? d : 0, s_base, s_xo);
+        uint32_t u_base = 0, u_xo[8];
+        swz_cols(u_role ? tu : 0, u_base, u_xo);
+
+        auto publish = [&](int bar_id) {
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[bar_id]);
+        };
+        // output rows t = d (lanes 0..63) of chunk c from D1
+        auto drain_o = [&](int c, bool ok) -> bool {
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar[kODone], c & 1, err, kErrTimeoutSeq));
+            if (!ok) return false;
+            tc_fence_after();
+            uint32_t x[16];
+            tmem_ld_32x32b_x16(tmem + 32 * (c & 1) + c0 + lane_base, x);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kOFree]);
+            const int64_t t = static_cast<int64_t>(c) * CH + d;
+            if (t < T) {
+                float* orow = o + ((static_cast<int64_t>(b) * T + t) * Hv + h) * V + vs0 + c0;
 #pragma unroll
-        for (int v4 = 0; v4 < 8; ++v4) {
+                for (int v4 = 0; v4 < 4; ++v4)
+                    *reinterpret_cast<float4*>(orow + 4 * v4) =
+                        make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
+                                    scale * __uint_as_float(x[4 * v4 + 2]), scale * __uint_as_float(x[4 * v4 + 3]));
+            }
+            return true;
+        };
+
+        float S[16];
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (state_in && has_row)
-                x = *reinterpret_cast<const float4*>(state_in + sbase + static_cast<int64_t>(d) * V + vs0 + 4 * v4);
+                x = *reinterpret_cast<const float4*>(state_in + sbase + static_cast<int64_t>(d) * V + vs0 + c0 + 4 * v4);
             S[4 * v4] = x.x; S[4 * v4 + 1] = x.y; S[4 * v4 + 2] = x.z; S[4 * v4 + 3] = x.w;
         }
         if (has_row) {
 #pragma unroll
-            for (int v = 0; v < 32; ++v)
-                *reinterpret_cast<float*>(b1p + sw128_off(v, d, 32)) = __uint_as_float(to_tf32(S[v]));
+            for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) = __uint_as_float(to_tf32(S[i]));
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&bar[kSReady]);
+        publish(kSReady);
         bool ok = true;
         for (int c = 0; c < NC && ok; ++c) {
             const int s = c & 1;
-            const int64_t t0 = static_cast<int64_t>(c) * CH;
             const float gc = *reinterpret_cast<const float*>(rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::GC);
-            float ut[32];
             if (u_role) {
+                float ut[16];
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar[kUtFull + s], (c >> 1) & 1, err, kErrTimeoutSeq));
                 if (!ok) break;
                 const uint8_t* up = sm + L::UT + s * L::UT_BYTES + tu * 128;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = (c0 >> 2) + jj;
                     const float4 x = *reinterpret_cast<const float4*>(up + ((j ^ (tu & 7)) << 4));
-                    ut[4 * j] = x.x; ut[4 * j + 1] = x.y; ut[4 * j + 2] = x.z; ut[4 * j + 3] = x.w;
+                    ut[4 * jj] = x.x; ut[4 * jj + 1] = x.y; ut[4 * jj + 2] = x.z; ut[4 * jj + 3] = x.w;
                 }
-                mbar_arrive(&bar[kUtEmpty + s]);
-            }
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR1Done], c & 1, err, kErrTimeoutSeq));
-            if (!ok) break;
-            tc_fence_after();
-            if (u_role) {
-                uint32_t x[32];
-                tmem_ld_32x32b_x32(tmem + 32 * s + lane_base, x);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kUtEmpty + s]);
+                // R1 done; R2b of the previous chunk has finished reading U^T
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR1Done], c & 1, err, kErrTimeoutSeq) &&
+                                                 (c == 0 || mbar_wait(&bar[kODone], (c - 1) & 1, err, kErrTimeoutSeq)));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t x[16];
+                tmem_ld_32x32b_x16(tmem + 32 * s + c0 + lane_base, x);
                 tmem_wait_ld();
 #pragma unroll
-                for (int v = 0; v < 32; ++v)
-                    *reinterpret_cast<float*>(b2p + sw128_off(v, tu, 32)) =
-                        __uint_as_float(to_tf32(ut[v] - __uint_as_float(x[v])));
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bar[kUReady]);
+                for (int i = 0; i < 16; ++i)
+                    *reinterpret_cast<float*>(b2p + u_base + (i >> 3) * 1024 + u_xo[i & 7]) =
+                        __uint_as_float(to_tf32(ut[i] - __uint_as_float(x[i])));
+                publish(kUPub);
+            } else if (c > 0) {
+                ok = drain_o(c - 1, ok);
+                if (!ok) break;
             }
             ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR2Done], c & 1, err, kErrTimeoutSeq));
             if (!ok) break;
             tc_fence_after();
-            {
-                uint32_t x[32];
-                tmem_ld_32x32b_x32(tmem + 64 + lane_base, x);
-                tmem_wait_ld();
-                if (has_row) {
-                    const float eg = expf(gc);
+            uint32_t x[16];
+            tmem_ld_32x32b_x16(tmem + 64 + c0 + lane_base, x);
+            tmem_wait_ld();
+            if (has_row) {
+                const float eg = expf(gc);
 #pragma unroll
-                    for (int v = 0; v < 32; ++v) {
-                        S[v] = fmaf(eg, S[v], __uint_as_float(x[v]));
-                        *reinterpret_cast<float*>(b1p + sw128_off(v, d, 32)) = __uint_as_float(to_tf32(S[v]));
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    S[i] = fmaf(eg, S[i], __uint_as_float(x[i]));
+                    *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) =
+                        __uint_as_float(to_tf32(S[i]));
                 }
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[kSReady]);
-            if (!u_role) {
-                // output rows t = d (lanes 0..63 of D1)
-                uint32_t x[32];
-                tmem_ld_32x32b_x32(tmem + 32 * s + lane_base, x);
-                tmem_wait_ld();
-                if (t0 + d < T) {
-                    float* orow = o + ((static_cast<int64_t>(b) * T + t0 + d) * Hv + h) * V + vs0;
-#pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        *reinterpret_cast<float4*>(orow + 4 * v4) =
-                            make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
-                                        scale * __uint_as_float(x[4 * v4 + 2]), scale * __uint_as_float(x[4 * v4 + 3]));
-                }
-                tc_fence_before();
-            }
+            publish(kSReady);
         }
+        if (ok && !u_role) ok = drain_o(NC - 1, ok);
         if (ok && state_out && has_row) {
 #pragma unroll
-            for (int v4 = 0; v4 < 8; ++v4)
-                *reinterpret_cast<float4*>(state_out + sbase + static_cast<int64_t>(d) * V + vs0 + 4 * v4) =
+            for (int v4 = 0; v4 < 4; ++v4)
+                *reinterpret_cast<float4*>(state_out + sbase + static_cast<int64_t>(d) * V + vs0 + c0 + 4 * v4) =
                     make_float4(S[4 * v4], S[4 * v4 + 1], S[4 * v4 + 2], S[4 * v4 + 3]);
         }
     }
@@ -667,7 +768,7 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
     chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, recs);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    chunk_seq_kernel<K, V><<<seq_blocks, 192, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, err);
+    chunk_seq_kernel<K, V><<<seq_blocks, 320, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     return NVFP4_OK;
