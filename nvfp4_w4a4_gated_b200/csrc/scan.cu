@@ -147,59 +147,89 @@ template <int K, int V>
 struct PrepSmem {
     // row stride of the K and Q tiles (== 4 mod 32); the Q tile later holds the V rows
     static constexpr int KS = (K > V ? K : V) + 4;
-    static constexpr int TS = CH + 4;  // row stride of T (== 4 mod 32)
+    static constexpr int LS = CH + 4;  // row stride of L (== 4 mod 32)
+    static constexpr int TBS = 20;     // row stride of the diagonal-block inverses
     float ks[CH * KS];
     float qs[CH * KS];
-    float L[CH * CH];                  // strictly lower, scaled: b_t e^{Gd_t - G_i} k_t.k_i
-    float T[CH * TS];                  // (I + L)^-1
-    float P[3 * 256];                  // 16 x 16 block products
+    float L[CH * LS];                  // strictly lower, scaled: b_t e^{Gd_t - G_i} k_t.k_i
+    float Tb[4 * 16 * TBS];            // (I + L_bb)^-1 for the four 16 x 16 diagonal blocks
     float gin[CH], gd[CH], bet[CH], graw[CH], df[CH];
     float eG[CH], eKh[CH];             // e^{G_t}, e^{G_C - G_t}
 };
 
-// X = (T diag(s)) B for a 32-column strip of X: T [64 x 64] unit lower triangular
-// (row stride TS), B [64 x N] (row stride KS), columns c0..c0+31, all 64 rows; one
-// warp.  TF32 tensor cores (operands rounded to nearest), float32 accumulation; the
-// k-steps above the diagonal of each 16-row tile are skipped (T is zero there).
-// Each pair of adjacent outputs (t, col), (t, col+1), col even, goes to
-// store(t, col, x0, x1).
-template <int KS, int TS, typename Store>
-__device__ __forceinline__ void tri_apply(const float* __restrict__ Tm, const float* __restrict__ s,
-                                          const float* __restrict__ Bm, int c0, int lane, Store store) {
+// W = (I + L)^-1 diag(s) X for the 32-column strip c0..c0+31 of X [64 x N] (row
+// stride KS) in shared memory, by block forward substitution over 16-row blocks:
+//   W_b = T_bb (diag(s_b) X_b - sum_{k<b} L_bk W_k),   T_bb = (I + L_bb)^-1.
+// The strip is overwritten by W (float32) and each pair of adjacent outputs (t, col),
+// (t, col+1), col even, also goes to store(t, col, x0, x1).  One warp, which alone
+// touches these columns.  TF32 tensor cores (operands rounded to nearest), float32
+// accumulation.
+template <int KS, int LS, int TBS, typename Store>
+__device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const float* __restrict__ Tb,
+                                            const float* __restrict__ s, float* __restrict__ X, int c0, int lane,
+                                            Store store) {
     const int grp = lane >> 2, tig = lane & 3;
-    float acc[4][4][4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) acc[m][nt][0] = acc[m][nt][1] = acc[m][nt][2] = acc[m][nt][3] = 0.f;
-#pragma unroll
-    for (int k0 = 0; k0 < CH; k0 += 8) {
-        uint32_t bf[4][2];
+    for (int b = 0; b < 4; ++b) {
+        const int r0 = 16 * b;
+        float acc[4][4];
+        const float s0 = s[r0 + grp], s1 = s[r0 + grp + 8];
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            bf[nt][0] = to_tf32(Bm[(k0 + tig) * KS + c0 + nt * 8 + grp]);
-            bf[nt][1] = to_tf32(Bm[(k0 + tig + 4) * KS + c0 + nt * 8 + grp]);
+            const int col = c0 + nt * 8 + 2 * tig;
+            const float2 x0 = *reinterpret_cast<const float2*>(&X[(r0 + grp) * KS + col]);
+            const float2 x1 = *reinterpret_cast<const float2*>(&X[(r0 + grp + 8) * KS + col]);
+            acc[nt][0] = s0 * x0.x;
+            acc[nt][1] = s0 * x0.y;
+            acc[nt][2] = s1 * x1.x;
+            acc[nt][3] = s1 * x1.y;
         }
-        const float s0 = s[k0 + tig], s1 = s[k0 + tig + 4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            if (k0 >= 16 * (m + 1)) continue;
-            const int r0 = 16 * m;
-            const uint32_t a[4] = {to_tf32(Tm[(r0 + grp) * TS + k0 + tig] * s0),
-                                   to_tf32(Tm[(r0 + grp + 8) * TS + k0 + tig] * s0),
-                                   to_tf32(Tm[(r0 + grp) * TS + k0 + tig + 4] * s1),
-                                   to_tf32(Tm[(r0 + grp + 8) * TS + k0 + tig + 4] * s1)};
+        for (int k0 = 0; k0 < r0; k0 += 8) {
+            const uint32_t a[4] = {to_tf32(-Lm[(r0 + grp) * LS + k0 + tig]), to_tf32(-Lm[(r0 + grp + 8) * LS + k0 + tig]),
+                                   to_tf32(-Lm[(r0 + grp) * LS + k0 + tig + 4]),
+                                   to_tf32(-Lm[(r0 + grp + 8) * LS + k0 + tig + 4])};
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) mma_tf32(acc[m][nt], a, bf[nt]);
+            for (int nt = 0; nt < 4; ++nt) {
+                const uint32_t bb[2] = {to_tf32(X[(k0 + tig) * KS + c0 + nt * 8 + grp]),
+                                        to_tf32(X[(k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
+                mma_tf32(acc[nt], a, bb);
+            }
         }
+        // Y_b over X_b: every lane rewrites exactly the positions it read
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = c0 + nt * 8 + 2 * tig;
+            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) = make_float2(acc[nt][0], acc[nt][1]);
+            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) = make_float2(acc[nt][2], acc[nt][3]);
+        }
+        __syncwarp();
+        float w[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) w[nt][0] = w[nt][1] = w[nt][2] = w[nt][3] = 0.f;
+        const float* Tbb = Tb + b * 16 * TBS;
+#pragma unroll
+        for (int k0 = 0; k0 < 16; k0 += 8) {
+            const uint32_t a[4] = {to_tf32(Tbb[grp * TBS + k0 + tig]), to_tf32(Tbb[(grp + 8) * TBS + k0 + tig]),
+                                   to_tf32(Tbb[grp * TBS + k0 + tig + 4]), to_tf32(Tbb[(grp + 8) * TBS + k0 + tig + 4])};
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const uint32_t bb[2] = {to_tf32(X[(r0 + k0 + tig) * KS + c0 + nt * 8 + grp]),
+                                        to_tf32(X[(r0 + k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
+                mma_tf32(w[nt], a, bb);
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int col = c0 + nt * 8 + 2 * tig;
+            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) = make_float2(w[nt][0], w[nt][1]);
+            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) = make_float2(w[nt][2], w[nt][3]);
+            store(r0 + grp, col, w[nt][0], w[nt][1]);
+            store(r0 + grp + 8, col, w[nt][2], w[nt][3]);
+        }
+        __syncwarp();
     }
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                store(16 * m + grp + hh * 8, c0 + nt * 8 + 2 * tig, acc[m][nt][2 * hh], acc[m][nt][2 * hh + 1]);
 }
 
 template <int K, int V>
@@ -295,8 +325,8 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 const int t = r0 + grp + hh * 8;
                 const int i = nt * 8 + 2 * tig;
                 if (warp < 4) {
-                    sm.L[t * CH + i] = (i < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
-                    sm.L[t * CH + i + 1] =
+                    sm.L[t * SM::LS + i] = (i < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
+                    sm.L[t * SM::LS + i + 1] =
                         (i + 1 < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
                 } else {
                     // rounded to TF32 here: it is only ever a tensor-core operand
@@ -325,11 +355,9 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(to_tf32(sm.eKh[4 * t4 + w] * sm.ks[(4 * t4 + w) * KS + dd]));
         *reinterpret_cast<float4*>(rec + RC::A3 + sw128_off(dd, 4 * t4, 128)) = make_float4(x[0], x[1], x[2], x[3]);
     }
-    constexpr int TS = SM::TS;
-    for (int idx = tid; idx < CH * TS; idx += 256) sm.T[idx] = 0.0f;
     __syncthreads();
     // Q is no longer needed: its tile now receives the V rows (zero past the sequence
-    // end); the copies land while the triangular inverse is formed
+    // end); the copies land while the diagonal blocks are inverted
     constexpr int VV4 = V / 4;
     for (int idx = tid; idx < CH * VV4; idx += 256) {
         const int r = idx / VV4, c4 = idx - r * VV4;
@@ -339,56 +367,44 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     }
     cp_async_commit();
 
-    // T = (I + L)^-1, blockwise.  Diagonal 16 x 16 blocks by substitution
-    // (warp w < 4 takes block w, lane c < 16 column c); then block rows
-    // i = 1..3: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj.
-    if (warp < 4 && lane < 16) {
-        const int o = warp * 16;
-        float x[16];
+    // T_bb = (I + L_bb)^-1 for the four 16 x 16 diagonal blocks, by forward substitution
+    // in registers: warp b takes block b, lane r (and r + 16) holds row r; once row i is
+    // final it is broadcast and every later row r subtracts L_ri times it.
+    constexpr int LS = SM::LS, TBS = SM::TBS;
+    if (warp < 4) {
+        const int o = 16 * warp, r = lane & 15;
+        float Lr[16], Tr[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = (r == lane) ? 1.0f : 0.0f;
-#pragma unroll
-            for (int i = 0; i < r; ++i) acc = fmaf(-sm.L[(o + r) * CH + o + i], x[i], acc);
-            x[r] = acc;
+        for (int i = 0; i < 16; ++i) {
+            Lr[i] = i < r ? sm.L[(o + r) * LS + o + i] : 0.0f;
+            Tr[i] = i == r ? 1.0f : 0.0f;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sm.T[(o + r) * TS + o + lane] = x[r];
+        for (int i = 0; i < 15; ++i) {
+#pragma unroll
+            for (int j = 0; j <= i; ++j) {
+                const float tij = __shfl_sync(0xffffffffu, Tr[j], i);
+                Tr[j] = fmaf(-Lr[i], tij, Tr[j]);
+            }
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) sm.Tb[warp * 16 * TBS + r * TBS + j] = Tr[j];
+        }
     }
-    __syncthreads();
-    for (int bi = 1; bi < 4; ++bi) {
-        for (int e = tid; e < bi * 256; e += 256) {
-            const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.0f;
-            for (int kk = 16 * j; kk < 16 * bi; ++kk)
-                acc = fmaf(sm.L[(16 * bi + r) * CH + kk], sm.T[kk * TS + 16 * j + cc], acc);
-            sm.P[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < bi * 256; e += 256) {
-            const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.0f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m) acc = fmaf(sm.T[(16 * bi + r) * TS + 16 * bi + m], sm.P[j * 256 + m * 16 + cc], acc);
-            sm.T[(16 * bi + r) * TS + 16 * j + cc] = -acc;
-        }
-        __syncthreads();
-    }
-
     cp_async_wait<0>();
     __syncthreads();
-    // W~ = T diag(b e^{Gd}) K (warps 0-3, stored TF32-rounded: a tensor-core operand downstream)
-    // U~ = T diag(beta) V   (warps 4-7)
-    // 32-column strips: W~ strips first (K/32 of them), then U~ strips (V/32), over the 8 warps
+    // W~ = (I + L)^-1 diag(b e^{Gd}) K (stored TF32-rounded: a tensor-core operand downstream),
+    // U~ = (I + L)^-1 diag(beta) V; 32-column strips, W~ strips first, one warp each
     for (int strip = warp; strip < K / 32 + V / 32; strip += 8) {
         if (strip < K / 32) {
-            tri_apply<KS, TS>(sm.T, sm.df, sm.ks, 32 * strip, lane, [&](int t, int col, float x0, float x1) {
+            block_subst<KS, LS, TBS>(sm.L, sm.Tb, sm.df, sm.ks, 32 * strip, lane, [&](int t, int col, float x0, float x1) {
                 *reinterpret_cast<float2*>(rec + RC::A1 + sw128_off(CH + t, col, 128)) =
                     make_float2(__uint_as_float(to_tf32(x0)), __uint_as_float(to_tf32(x1)));
             });
         } else {
             const int vs = strip - K / 32;
-            tri_apply<KS, TS>(sm.T, sm.bet, sm.qs, 32 * vs, lane, [&](int t, int col, float x0, float x1) {
+            block_subst<KS, LS, TBS>(sm.L, sm.Tb, sm.bet, sm.qs, 32 * vs, lane, [&](int t, int col, float x0, float x1) {
                 *reinterpret_cast<float2*>(rec + RC::UT + vs * RC::UT_SLICE + sw128_off(t, col - 32 * vs, CH)) =
                     make_float2(x0, x1);
             });
