@@ -33,6 +33,11 @@ nvfp4_status make_tmap_u8_sw128(CUtensorMap* map, const void* base, uint64_t row
 nvfp4_status make_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
                                  uint32_t box_rows, uint32_t box_cols);
 
+// Internal quantiser mode (not part of the C ABI): the workspace already holds the
+// amax of the input as float bits (for instance folded into the kernel that produced
+// the input), so only the quantisation pass runs.
+constexpr int32_t kQuantFromAmax = 0x100;
+
 // Error codes recorded in the device error word.
 constexpr unsigned int kErrTimeoutTma = 1u;
 constexpr unsigned int kErrTimeoutMma = 2u;

@@ -23,7 +23,8 @@ nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_di
 size_t scan_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo);
 nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                          const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form, int algo,
-                         const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st);
+                         const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st,
+                         unsigned int* o_amax);
 
 static int64_t n_in_of(const gdn_dims& d) { return 2ll * d.Hk * d.K + 2ll * d.Hv * d.V + 2ll * d.Hv; }
 static int64_t ld_proj_of(const gdn_dims& d) { return (n_in_of(d) + 3) / 4 * 4; }
@@ -119,11 +120,15 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
     if ((s = gemm_launch(xq, w->w_in, proj, ldp, st)) != NVFP4_OK) return s;
     if ((s = gates_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, q_hat, k_hat, g, beta, st)) != NVFP4_OK) return s;
     const float scale = 1.0f / sqrtf(static_cast<float>(d.K));
+    // the scan folds max|o| into the quantiser's amax word as it writes o, so the o
+    // quantiser runs its quantisation pass only
+    unsigned int* o_amax = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
+    cudaError_t e = cudaMemsetAsync(o_amax, 0, sizeof(unsigned int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(o amax)");
     if ((s = scan_launch(q_hat, k_hat, proj + 2ll * d.Hk * d.K, ldp, g, beta, B, T, d, scale, form, GDN_SCAN_AUTO,
-                         state_in, state_out, o, ws + L.scan_ws, st)) != NVFP4_OK)
+                         state_in, state_out, o, ws + L.scan_ws, st, o_amax)) != NVFP4_OK)
         return s;
-    if ((s = quantize_launch(o, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, NVFP4_QUANT_COMPUTE_SCALE, ws + L.quant_ws, st)) !=
-        NVFP4_OK)
+    if ((s = quantize_launch(o, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, ws + L.quant_ws, st)) != NVFP4_OK)
         return s;
     return gemm_launch(oq, w->w_out, y, H, st);
 }

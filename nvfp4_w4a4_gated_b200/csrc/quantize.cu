@@ -7,9 +7,9 @@
 // tensor itself at run time (the SoloQ summary page's dynamic NVFP4 variant).
 //
 // Two launches: (1) a grid-wide amax (128-bit loads, warp max, one atomicMax
-// per CTA); (2) one CTA per 512-byte scale atom (128 rows x 64 columns), one
-// thread per 16-element block.  Thread t of a CTA owns byte t of the atom, so
-// the scale store is one coalesced 512-byte write per CTA.
+// per CTA); (2) a grid-stride walk over the 512-byte scale atoms (128 rows x 64
+// columns), one thread per four 16-element blocks, the scale bytes of an atom
+// stored as four coalesced 128-byte rows.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -84,46 +84,45 @@ __device__ __forceinline__ void unpack16B(const uint4& u, float* out, const floa
 }
 
 // Pass 1: amax over the matrix into *amax_bits (float bits of a non-negative
-// value, so unsigned order is float order).  Each thread keeps four 16-byte
-// loads in flight per iteration.
+// value, so unsigned order is float order).  Each warp walks whole rows, its lanes
+// striding along the row with eight 16-byte loads in flight; warp max, then one
+// atomicMax per CTA.
 template <typename T>
 __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                                                    unsigned int* __restrict__ amax_bits) {
     constexpr int P = Vec<T>::kPer16B;
-    constexpr int U = 4;
-    const int64_t vec_per_row = cols / P;
-    const int64_t nvec = rows * vec_per_row;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    constexpr int U = 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t nvec = cols / P;   // 16-byte vectors per row
     float m = 0.0f;
-    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    for (; i + (U - 1) * stride < nvec; i += U * stride) {
-        uint4 u[U];
+    for (int64_t r = warp0; r < rows; r += nwarps) {
+        const uint4* row = reinterpret_cast<const uint4*>(x + r * ld);
+        int64_t c = lane;
+        for (; c + 32 * (U - 1) < nvec; c += 32 * U) {
+            uint4 u[U];
 #pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t ii = i + j * stride;
-            const int64_t r = ii / vec_per_row, c = (ii - r * vec_per_row) * P;
-            u[j] = __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
+            for (int j = 0; j < U; ++j) u[j] = __ldg(row + c + 32 * j);
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                float f[8];
+                unpack16B(u[j], f, x);
+#pragma unroll
+                for (int e = 0; e < P; ++e) m = fmaxf(m, fabsf(f[e]));
+            }
         }
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
+        for (; c < nvec; c += 32) {
             float f[8];
-            unpack16B(u[j], f, x);
+            unpack16B(__ldg(row + c), f, x);
 #pragma unroll
             for (int e = 0; e < P; ++e) m = fmaxf(m, fabsf(f[e]));
         }
     }
-    for (; i < nvec; i += stride) {
-        const int64_t r = i / vec_per_row, c = (i - r * vec_per_row) * P;
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
-        float f[8];
-        unpack16B(u, f, x);
-#pragma unroll
-        for (int e = 0; e < P; ++e) m = fmaxf(m, fabsf(f[e]));
-    }
     unsigned int b = __float_as_uint(m);
     b = __reduce_max_sync(0xffffffffu, b);
     __shared__ unsigned int warp_max[8];
-    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = b;
+    if (lane == 0) warp_max[threadIdx.x >> 5] = b;
     __syncthreads();
     if (threadIdx.x < 32) {
         unsigned int v = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0u;
@@ -132,56 +131,73 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     }
 }
 
-// Pass 2: one CTA of 512 threads per scale atom.
+// Pass 2: CTAs of 128 threads walk the scale atoms (128 rows x 64 columns, 512
+// blocks of 16) in a grid-stride loop.  Thread t owns atom bytes t, t+128, t+256,
+// t+384, i.e. the blocks (r, j) with r % 32 = (byte >> 4), r / 32 = (byte >> 2) & 3,
+// j = byte & 3; all four blocks' loads are issued before any is used, and each
+// group of 128 scale bytes is one coalesced store.
+constexpr int kQuantThreads = 128;
+constexpr int kQuantBPT = 512 / kQuantThreads;
+
 template <typename T>
-__global__ void __launch_bounds__(512) quant_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                                                    const unsigned int* __restrict__ amax_bits,
-                                                    float* __restrict__ global_scale, int given_scale,
-                                                    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+__global__ void __launch_bounds__(kQuantThreads) quant_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
+                                                              int64_t ld, const unsigned int* __restrict__ amax_bits,
+                                                              float* __restrict__ global_scale, int given_scale,
+                                                              uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
     constexpr int P = Vec<T>::kPer16B;
+    constexpr int NV = 16 / P;   // 16-byte loads per block
     const int64_t k_atoms = cols / 64;
-    const int64_t atom = blockIdx.x;
-    const int64_t rb = atom / k_atoms, ka = atom - rb * k_atoms;
+    const int64_t natoms = ((rows + 127) / 128) * k_atoms;
     const int t = threadIdx.x;
-    const int64_t r = rb * 128 + (t >> 4) + 32 * ((t >> 2) & 3);
-    const int64_t kb = ka * 4 + (t & 3);
 
     float S;
     if (given_scale) {
         S = *global_scale;
     } else {
         S = global_scale_from_amax(__uint_as_float(*amax_bits));
-        if (atom == 0 && t == 0) *global_scale = S;
+        if (blockIdx.x == 0 && t == 0) *global_scale = S;
     }
+    const float d6 = __fmul_rn(6.0f, S);
 
-    uint32_t sb = 0;
-    if (r < rows) {
-        float v[16];
-        const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + kb * 16);
+    for (int64_t atom = blockIdx.x; atom < natoms; atom += gridDim.x) {
+        const int64_t rb = atom / k_atoms, ka = atom - rb * k_atoms;
+        uint4 u[kQuantBPT][NV];
+        int64_t r[kQuantBPT], kb[kQuantBPT];
 #pragma unroll
-        for (int j = 0; j < 16 / P; ++j) unpack16B(__ldg(src + j), v + j * P, x);
-        float m = 0.0f;
+        for (int i = 0; i < kQuantBPT; ++i) {
+            const int byte = t + i * kQuantThreads;
+            r[i] = rb * 128 + (byte >> 4) + 32 * ((byte >> 2) & 3);
+            kb[i] = ka * 4 + (byte & 3);
+            const uint4* src = reinterpret_cast<const uint4*>(x + (r[i] < rows ? r[i] : 0) * ld + kb[i] * 16);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
-        const float d = __fmul_rn(6.0f, S);
-        const float s_f = __fdiv_rn(m, d);
-        sb = f32_to_e4m3(s_f);
-        const float dec = __fmul_rn(e4m3_to_f32(sb), S);
-        uint2 packed = make_uint2(0u, 0u);
-        if (dec != 0.0f) {
-            const float inv = __frcp_rn(dec);
-            float y0[8], y1[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                y0[j] = __fmul_rn(v[j], inv);
-                y1[j] = __fmul_rn(v[8 + j], inv);
-            }
-            packed.x = f32x8_to_e2m1(y0);
-            packed.y = f32x8_to_e2m1(y1);
+            for (int j = 0; j < NV; ++j) u[i][j] = r[i] < rows ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
         }
-        *reinterpret_cast<uint2*>(codes + r * (cols / 2) + kb * 8) = packed;
+#pragma unroll
+        for (int i = 0; i < kQuantBPT; ++i) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < NV; ++j) unpack16B(u[i][j], v + j * P, x);
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+            const uint32_t sb = f32_to_e4m3(__fdiv_rn(m, d6));
+            const float dec = __fmul_rn(e4m3_to_f32(sb), S);
+            uint2 packed = make_uint2(0u, 0u);
+            if (dec != 0.0f) {
+                const float inv = __frcp_rn(dec);
+                float y0[8], y1[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    y0[j] = __fmul_rn(v[j], inv);
+                    y1[j] = __fmul_rn(v[8 + j], inv);
+                }
+                packed.x = f32x8_to_e2m1(y0);
+                packed.y = f32x8_to_e2m1(y1);
+            }
+            if (r[i] < rows) *reinterpret_cast<uint2*>(codes + r[i] * (cols / 2) + kb[i] * 8) = packed;
+            sf[atom * 512 + t + i * kQuantThreads] = static_cast<uint8_t>(r[i] < rows ? sb : 0u);
+        }
     }
-    sf[atom * 512 + t] = static_cast<uint8_t>(sb);
 }
 
 }  // namespace
@@ -190,12 +206,11 @@ nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64
                              const nvfp4_tensor& out, int32_t flags, void* workspace, cudaStream_t st) {
     const bool given = flags == NVFP4_QUANT_GIVEN_SCALE;
     unsigned int* amax = static_cast<unsigned int*>(workspace);
-    if (!given) {
+    if (!given && flags != kQuantFromAmax) {
         cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(amax)");
-        const int64_t elems_per_vec = x_dtype == NVFP4_DTYPE_BF16 ? 8 : 4;
-        const int64_t nvec = rows * (cols / elems_per_vec);
-        int64_t blocks = (nvec + 1023) / 1024;
+        // one warp per row, up to 8 resident CTAs of 8 warps per SM
+        int64_t blocks = (rows + 7) / 8;
         const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
         if (blocks > cap) blocks = cap;
         if (x_dtype == NVFP4_DTYPE_BF16)
@@ -205,12 +220,14 @@ nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64
             amax_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(static_cast<const float*>(x), rows, cols, ld, amax);
     }
     const int64_t atoms = ((rows + 127) / 128) * (cols / 64);
+    int64_t qblocks = static_cast<int64_t>(num_sms()) * 12;
+    if (qblocks > atoms) qblocks = atoms;
     if (x_dtype == NVFP4_DTYPE_BF16)
-        quant_kernel<__nv_bfloat16><<<(unsigned)atoms, 512, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rows, cols,
+        quant_kernel<__nv_bfloat16><<<(unsigned)qblocks, kQuantThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rows, cols,
                                                                       ld, amax, out.global_scale, given ? 1 : 0,
                                                                       out.codes, out.sf);
     else
-        quant_kernel<float><<<(unsigned)atoms, 512, 0, st>>>(static_cast<const float*>(x), rows, cols, ld, amax,
+        quant_kernel<float><<<(unsigned)qblocks, kQuantThreads, 0, st>>>(static_cast<const float*>(x), rows, cols, ld, amax,
                                                               out.global_scale, given ? 1 : 0, out.codes, out.sf);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");

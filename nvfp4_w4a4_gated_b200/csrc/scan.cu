@@ -66,7 +66,7 @@ template <int K>
 __global__ void __launch_bounds__(128) scan_recurrent_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, int64_t ld_v,
     const float* __restrict__ g, const float* __restrict__ beta, int B, int64_t T, int Hk, int Hv, int V, float scale,
-    int form, const float* state_in, float* state_out, float* __restrict__ o) {
+    int form, const float* state_in, float* state_out, float* __restrict__ o, unsigned int* __restrict__ o_amax) {
     constexpr int RW = K / 4;
     const int nslice = V / 32;
     const int bh = blockIdx.x / nslice, slice = blockIdx.x - bh * nslice;
@@ -108,7 +108,14 @@ __global__ void __launch_bounds__(128) scan_recurrent_kernel(
         }
         red2[w][lane] = acc;
         __syncthreads();
-        if (w == 0) o[(tok * Hv + h) * V + j] = scale * ((red2[0][lane] + red2[1][lane]) + (red2[2][lane] + red2[3][lane]));
+        if (w == 0) {
+            const float ov = scale * ((red2[0][lane] + red2[1][lane]) + (red2[2][lane] + red2[3][lane]));
+            o[(tok * Hv + h) * V + j] = ov;
+            if (o_amax) {
+                const unsigned int mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(ov)));
+                if (lane == 0) atomicMax(o_amax, mb);
+            }
+        }
     }
     if (state_out) {
 #pragma unroll
@@ -464,6 +471,7 @@ template <int K, int V>
 __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
                                                            float scale, int NC, const float* state_in,
                                                            float* state_out, float* __restrict__ o,
+                                                           unsigned int* __restrict__ o_amax,
                                                            unsigned int* __restrict__ err) {
     using L = SeqLayout<K>;
     using RC = ChunkRec<K, V>;
@@ -669,13 +677,21 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[kOFree]);
             const int64_t t = static_cast<int64_t>(c) * CH + d;
+            float om = 0.0f;
             if (t < T) {
                 float* orow = o + ((static_cast<int64_t>(b) * T + t) * Hv + h) * V + vs0 + c0;
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4)
-                    *reinterpret_cast<float4*>(orow + 4 * v4) =
-                        make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
-                                    scale * __uint_as_float(x[4 * v4 + 2]), scale * __uint_as_float(x[4 * v4 + 3]));
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    const float4 ov = make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
+                                                  scale * __uint_as_float(x[4 * v4 + 2]),
+                                                  scale * __uint_as_float(x[4 * v4 + 3]));
+                    *reinterpret_cast<float4*>(orow + 4 * v4) = ov;
+                    om = fmaxf(om, fmaxf(fmaxf(fabsf(ov.x), fabsf(ov.y)), fmaxf(fabsf(ov.z), fabsf(ov.w))));
+                }
+            }
+            if (o_amax) {
+                const unsigned int mb = __reduce_max_sync(0xffffffffu, __float_as_uint(om));
+                if (lane == 0) atomicMax(o_amax, mb);
             }
             return true;
         };
@@ -764,7 +780,8 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
 template <int K, int V>
 nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                                const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form,
-                               const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st) {
+                               const float* s_in, float* s_out, float* o, void* ws, unsigned int* o_amax,
+                               cudaStream_t st) {
     const int NC = static_cast<int>((T + CH - 1) / CH);
     const int prep_smem = sizeof(PrepSmem<K, V>);
     const int seq_smem = SeqLayout<K>::BYTES;
@@ -784,7 +801,7 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
     chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, recs);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    chunk_seq_kernel<K, V><<<seq_blocks, 320, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, err);
+    chunk_seq_kernel<K, V><<<seq_blocks, 320, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, o_amax, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     return NVFP4_OK;
@@ -810,27 +827,28 @@ size_t scan_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo) {
 
 nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                          const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form, int algo,
-                         const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st) {
+                         const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st,
+                         unsigned int* o_amax) {
     const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
     if (!chunked) {
         const unsigned blocks = static_cast<unsigned>(B * d.Hv * (d.V / 32));
         if (d.K == 128)
             scan_recurrent_kernel<128><<<blocks, 128, 0, st>>>(q, k, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form,
-                                                               s_in, s_out, o);
+                                                               s_in, s_out, o, o_amax);
         else
             scan_recurrent_kernel<64><<<blocks, 128, 0, st>>>(q, k, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form,
-                                                              s_in, s_out, o);
+                                                              s_in, s_out, o, o_amax);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "recurrent scan launch");
         return NVFP4_OK;
     }
     if (d.K == 128 && d.V == 128)
-        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
+        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
     if (d.K == 128 && d.V == 64)
-        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
+        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
     if (d.K == 64 && d.V == 128)
-        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
-    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, st);
+        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
+    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
 }
 
 }  // namespace nvg
@@ -860,5 +878,5 @@ extern "C" nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const f
     if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)))
         return fail(NVFP4_ERR_WORKSPACE, "scan workspace missing, too small or not 256-byte aligned");
     return scan_launch(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, algo, state_in, state_out, o,
-                       workspace, as_stream(stream));
+                       workspace, as_stream(stream), nullptr);
 }
