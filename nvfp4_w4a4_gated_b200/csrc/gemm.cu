@@ -235,27 +235,44 @@ __global__ void __launch_bounds__(320, 1)
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kt = 0; kt < num_kt; ++kt) {
                 const int slot = static_cast<int>(kt_all & 1u);
-                if (!mbar_wait(&full[stage], phase, err, kErrTimeoutEpi) ||
-                    (kt_all >= 2 && !mbar_wait(&sf_free[slot], ((kt_all >> 1) - 1) & 1u, err, kErrTimeoutEpi))) {
+                if (!mbar_wait(&full[stage], phase, err, kErrTimeoutEpi)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const int nkb = min(4, kb_total - kt * 4);
                 // A: the MMA reads row m's word at lane m, column base + m/32 -> this
                 // quarter writes its own rows' words into column base + q.
                 // B: output rows of lane quarter q read B row n's word at lane
                 // 32q + n%32, column base + n/32 -> every quarter holds all four
                 // words of each 128-row atom (16 bytes per lane).
+                // The words are read into registers before the slot is free, so only
+                // the TMEM stores remain once it is.
                 const uint8_t* a = sSFA + stage * G::SFA_BYTES + lane * 16 + q * 4;
                 const uint8_t* b = sSFB + stage * G::SFB_BYTES + lane * 16;
-                for (int j = 0; j < nkb; ++j) {
-                    tmem_st_32x32b_x1(G::TP::sfa(tmem, slot, j) + lane_base + q,
-                                      *reinterpret_cast<const uint32_t*>(a + j * 512));
+                uint32_t wa[4];
+                uint4 wb[4][BN / 128];
 #pragma unroll
-                    for (int nb = 0; nb < BN / 128; ++nb)
-                        tmem_st_32x32b_x4(G::TP::sfb(tmem, slot, j) + nb * 4 + lane_base,
-                                          *reinterpret_cast<const uint4*>(b + nb * 2048 + j * 512));
+                for (int j = 0; j < 4; ++j) {
+                    if (j < nkb) {
+                        wa[j] = *reinterpret_cast<const uint32_t*>(a + j * 512);
+#pragma unroll
+                        for (int nb = 0; nb < BN / 128; ++nb)
+                            wb[j][nb] = *reinterpret_cast<const uint4*>(b + nb * 2048 + j * 512);
+                    }
+                }
+                if (kt_all >= 2 && !mbar_wait(&sf_free[slot], ((kt_all >> 1) - 1) & 1u, err, kErrTimeoutEpi)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j < nkb) {
+                        tmem_st_32x32b_x1(G::TP::sfa(tmem, slot, j) + lane_base + q, wa[j]);
+#pragma unroll
+                        for (int nb = 0; nb < BN / 128; ++nb)
+                            tmem_st_32x32b_x4(G::TP::sfb(tmem, slot, j) + nb * 4 + lane_base, wb[j][nb]);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -280,19 +297,12 @@ __global__ void __launch_bounds__(320, 1)
             if (!mbar_wait(acc_full, local & 1, err, kErrTimeoutEpi)) break;
             tc_fence_after();
             const int row0 = m_idx * BM + q * 32;
-#pragma unroll 1
-            for (int ci = 0; ci < G::TP::NCH; ++ci) {
-                // buffer 0 drains the columns it shares with buffer 1 first
-                const int c = buf == 0 ? (ci + G::TP::FIRST) % G::TP::NCH : ci;
-                const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * G::ACC_OFF + c * 32;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(taddr, v);
-                tmem_wait_ld();
-                if (ci == G::TP::RELEASE_AFTER - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tmem_free);
-                }
+            // buffer 0 drains the columns it shares with buffer 1 first
+            auto chunk_col = [&](int ci) { return buf == 0 ? (ci + G::TP::FIRST) % G::TP::NCH : ci; };
+            auto chunk_addr = [&](int ci) {
+                return tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * G::ACC_OFF + chunk_col(ci) * 32;
+            };
+            auto store_chunk = [&](int ci, const uint32_t (&v)[32]) {
                 // staging tile (ci & 1) is free once the store issued two chunks ago has read it
                 float* tile = stg + (ci & 1) * 32 * 32;
                 if (lane == 0) bulk_wait_read<1>();
@@ -300,9 +310,28 @@ __global__ void __launch_bounds__(320, 1)
                 stage_row(tile, lane, v, alpha);
                 fence_proxy_async_smem();
                 __syncwarp();
-                const int col0 = n_idx * BN + c * 32;
+                const int col0 = n_idx * BN + chunk_col(ci) * 32;
                 if (lane == 0 && row0 < M && col0 < N) tma_store_2d(&tmC, tile, col0, row0);
                 if (lane == 0) bulk_commit();
+            };
+            // the chunks the next tile's accumulator reuses go to registers first, so the
+            // MMA warp can start that tile before they are staged and stored
+            constexpr int RA = G::TP::RELEASE_AFTER;
+            uint32_t vr[RA][32];
+#pragma unroll
+            for (int ci = 0; ci < RA; ++ci) tmem_ld_32x32b_x32(chunk_addr(ci), vr[ci]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_free);
+#pragma unroll
+            for (int ci = 0; ci < RA; ++ci) store_chunk(ci, vr[ci]);
+#pragma unroll 1
+            for (int ci = RA; ci < G::TP::NCH; ++ci) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(chunk_addr(ci), v);
+                tmem_wait_ld();
+                store_chunk(ci, v);
             }
         }
         if (lane == 0) bulk_wait<0>();
@@ -319,8 +348,9 @@ __global__ void __launch_bounds__(320, 1)
 // ------------------------------------------------------------ CTA-pair kernel --
 // Cluster of 2 CTAs computes a 256 x 256 tile: CTA r holds A rows [128r, 128r+128)
 // of the tile and B rows [128r, 128r+128) of its N range, plus the scale atoms for
-// its A rows and for all 256 B rows.  The even CTA issues tcgen05.mma.cta_group::2
-// (M=256, N=256, K=64) and the scale copies for both; each CTA's TMEM receives its
+// its A rows and for all 256 B rows.  Each CTA's warps 6..9 write those scales into
+// its own TMEM (tcgen05.st) and report to the even CTA, which issues
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=64); each CTA's TMEM receives its
 // 128 rows of the accumulator.  Per stage a CTA loads 16 + 16 KB of codes instead of
 // 16 + 32 KB, so operand bytes per FLOP drop by a third.
 //   - The odd CTA's warp 1 relays "my stage is full" to the even CTA with a
@@ -343,7 +373,7 @@ struct CfgPair {
     static constexpr uint32_t IDESC = idesc_nvf4(256, 256);
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     w4a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const uint8_t* __restrict__ sfA,
                           const uint8_t* __restrict__ sfB, const float* __restrict__ scaleA,
@@ -361,7 +391,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     uint64_t* peer_full = empty + G::STAGES;   // even CTA only: the odd CTA's stage landed
     uint64_t* acc_full = peer_full + G::STAGES;
     uint64_t* tmem_free = acc_full + 1;        // even CTA only: 4 + 4 epilogue warps
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tmem_free + 1);
+    uint64_t* sf_full = tmem_free + 1;         // [2] even CTA only: 4 + 4 scale-writer warps
+    uint64_t* sf_free = sf_full + 2;           // [2] both CTAs: the MMAs of that slot completed
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_free + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -381,6 +413,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(tmem_free, 8);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sf_full[i], 8);
+            mbar_init(&sf_free[i], 1);
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -453,20 +489,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         ok = false;
                         break;
                     }
+                    const int slot = static_cast<int>(kt_all & 1u);
+                    // both CTAs' scale writers have filled this slot of their TMEM
+                    if (!mbar_wait_cluster(&sf_full[slot], (kt_all >> 1) & 1u, err, kErrTimeoutMma)) {
+                        ok = false;
+                        break;
+                    }
+                    ++kt_all;
                     tc_fence_after();
                     const int nkb = min(4, kb_total - kt * 4);
                     const uint32_t a_base = smem_u32(sA + stage * G::A_BYTES);
                     const uint32_t b_base = smem_u32(sB + stage * G::B_BYTES);
-                    const uint32_t sfa_base = smem_u32(sSFA + stage * G::SFA_BYTES);
-                    const uint32_t sfb_base = smem_u32(sSFB + stage * G::SFB_BYTES);
-                    const int slot = static_cast<int>(kt_all++ & 1u);
-                    for (int j = 0; j < nkb; ++j) {
-                        tmem_cp_sf_atom_pair(G::TP::sfa(tmem, slot, j), sdesc_sf_atom(sfa_base + j * 512));
-#pragma unroll
-                        for (int nb = 0; nb < 2; ++nb)
-                            tmem_cp_sf_atom_pair(G::TP::sfb(tmem, slot, j) + nb * 4,
-                                                 sdesc_sf_atom(sfb_base + nb * 2048 + j * 512));
-                    }
                     for (int j = 0; j < nkb; ++j) {
                         mma_nvf4_pair(acc, sdesc_kmajor_sw128(a_base + j * 32), sdesc_kmajor_sw128(b_base + j * 32),
                                       G::IDESC, G::TP::sfa(tmem, slot, j), G::TP::sfb(tmem, slot, j),
@@ -474,6 +507,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     }
                     mma_commit_pair(smem_u32(&empty[stage]));
                     mma_commit_pair(mapa_shared(smem_u32(&empty[stage]), 1));
+                    mma_commit_pair(smem_u32(&sf_free[slot]));
+                    mma_commit_pair(mapa_shared(smem_u32(&sf_free[slot]), 1));
                     if (++stage == G::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -500,6 +535,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     }
                 }
                 if (!ok) break;
+            }
+        }
+    } else if (warp >= 6) {
+        // ----------------------------------------------------- scale writers --
+        // Same TMEM layout as the single-CTA kernel, in each CTA's own TMEM: its A
+        // rows' words (x1, column base + q) and all 256 B rows' words (x4 per atom).
+        const int q = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        uint32_t stage = 0, phase = 0, kt_all = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+            for (int kt = 0; kt < num_kt; ++kt) {
+                const int slot = static_cast<int>(kt_all & 1u);
+                if (!mbar_wait(&full[stage], phase, err, kErrTimeoutEpi) ||
+                    (kt_all >= 2 && !mbar_wait(&sf_free[slot], ((kt_all >> 1) - 1) & 1u, err, kErrTimeoutEpi))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int nkb = min(4, kb_total - kt * 4);
+                const uint8_t* a = sSFA + stage * G::SFA_BYTES + lane * 16 + q * 4;
+                const uint8_t* b = sSFB + stage * G::SFB_BYTES + lane * 16;
+                for (int j = 0; j < nkb; ++j) {
+                    tmem_st_32x32b_x1(G::TP::sfa(tmem, slot, j) + lane_base + q,
+                                      *reinterpret_cast<const uint32_t*>(a + j * 512));
+#pragma unroll
+                    for (int nb = 0; nb < 2; ++nb)
+                        tmem_st_32x32b_x4(G::TP::sfb(tmem, slot, j) + nb * 4 + lane_base,
+                                          *reinterpret_cast<const uint4*>(b + nb * 2048 + j * 512));
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[slot]), 0));
+                ++kt_all;
+                if (++stage == G::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
     } else {
@@ -572,7 +646,7 @@ nvfp4_status launch_gemm_pair(const nvfp4_tensor& A, const nvfp4_tensor& B, floa
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
-    w4a4_gemm_pair_kernel<<<pairs * 2, 192, G::SMEM, st>>>(ta, tb, tc, A.sf, B.sf, A.global_scale, B.global_scale, M,
+    w4a4_gemm_pair_kernel<<<pairs * 2, 320, G::SMEM, st>>>(ta, tb, tc, A.sf, B.sf, A.global_scale, B.global_scale, M,
                                                           N, K, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm pair launch");
