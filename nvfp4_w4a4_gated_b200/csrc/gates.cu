@@ -76,6 +76,9 @@ nvfp4_status validate_dims(const gdn_dims* d) {
     return NVFP4_OK;
 }
 
+nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
+                              const float* dt_bias, float* g, float* beta, cudaStream_t st);
+
 nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
                           const float* dt_bias, float* q_hat, float* k_hat, float* g, float* beta, cudaStream_t st) {
     const int64_t warps = n * d.Hk * 2;
@@ -84,6 +87,12 @@ nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_di
         l2norm_kernel<128><<<blocks_n, 256, 0, st>>>(proj, ld, n, d.Hk, q_hat, k_hat);
     else
         l2norm_kernel<64><<<blocks_n, 256, 0, st>>>(proj, ld, n, d.Hk, q_hat, k_hat);
+    return gate_only_launch(proj, ld, n, d, A_log, dt_bias, g, beta, st);
+}
+
+// g and beta only (the chunked scan can normalise q, k itself while loading them).
+nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
+                              const float* dt_bias, float* g, float* beta, cudaStream_t st) {
     const int64_t col_a = 2ll * d.Hk * d.K + 2ll * d.Hv * d.V;
     const unsigned blocks_g = static_cast<unsigned>((n * d.Hv + 255) / 256);
     gate_kernel<<<blocks_g, 256, 0, st>>>(proj, ld, n, d.Hv, col_a, col_a + d.Hv, A_log, dt_bias, g, beta);

@@ -18,13 +18,15 @@ nvfp4_status validate_dims(const gdn_dims* d);
 nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, int64_t ld,
                              const nvfp4_tensor& out, int32_t flags, void* workspace, cudaStream_t st);
 nvfp4_status gemm_launch(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C, int64_t ldc, cudaStream_t st);
+nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
+                              const float* dt_bias, float* g, float* beta, cudaStream_t st);
 nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
                           const float* dt_bias, float* q_hat, float* k_hat, float* g, float* beta, cudaStream_t st);
 size_t scan_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo);
 nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                          const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form, int algo,
                          const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st,
-                         unsigned int* o_amax);
+                         unsigned int* o_amax, int64_t ld_qk, int normalize_qk);
 
 static int64_t n_in_of(const gdn_dims& d) { return 2ll * d.Hk * d.K + 2ll * d.Hv * d.V + 2ll * d.Hv; }
 static int64_t ld_proj_of(const gdn_dims& d) { return (n_in_of(d) + 3) / 4 * 4; }
@@ -118,15 +120,28 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
         NVFP4_OK)
         return s;
     if ((s = gemm_launch(xq, w->w_in, proj, ldp, st)) != NVFP4_OK) return s;
-    if ((s = gates_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, q_hat, k_hat, g, beta, st)) != NVFP4_OK) return s;
+    // T > 1: the chunked scan reads the raw q, k slices of the projection and
+    // normalises them while staging them, so only g and beta are formed here.
+    // T = 1 (decode): the recurrent scan reads normalised q_hat, k_hat.
+    const bool chunked = T > 1;
+    if (chunked) {
+        if ((s = gate_only_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, g, beta, st)) != NVFP4_OK) return s;
+    } else {
+        if ((s = gates_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, q_hat, k_hat, g, beta, st)) != NVFP4_OK)
+            return s;
+    }
+    const float* q_in = chunked ? proj : q_hat;
+    const float* k_in = chunked ? proj + static_cast<int64_t>(d.Hk) * d.K : k_hat;
+    const int64_t ld_qk = chunked ? ldp : static_cast<int64_t>(d.Hk) * d.K;
     const float scale = 1.0f / sqrtf(static_cast<float>(d.K));
     // the scan folds max|o| into the quantiser's amax word as it writes o, so the o
     // quantiser runs its quantisation pass only
     unsigned int* o_amax = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
     cudaError_t e = cudaMemsetAsync(o_amax, 0, sizeof(unsigned int), st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(o amax)");
-    if ((s = scan_launch(q_hat, k_hat, proj + 2ll * d.Hk * d.K, ldp, g, beta, B, T, d, scale, form, GDN_SCAN_AUTO,
-                         state_in, state_out, o, ws + L.scan_ws, st, o_amax)) != NVFP4_OK)
+    if ((s = scan_launch(q_in, k_in, proj + 2ll * d.Hk * d.K, ldp, g, beta, B, T, d, scale, form,
+                         chunked ? GDN_SCAN_CHUNKED : GDN_SCAN_RECURRENT, state_in, state_out, o, ws + L.scan_ws, st,
+                         o_amax, ld_qk, chunked ? 1 : 0)) != NVFP4_OK)
         return s;
     if ((s = quantize_launch(o, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, ws + L.quant_ws, st)) != NVFP4_OK)
         return s;

@@ -241,6 +241,7 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
 
 template <int K, int V>
 __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                                                         int64_t ld_qk, int normalize_qk,
                                                          const float* __restrict__ v, int64_t ld_v,
                                                          const float* __restrict__ g, const float* __restrict__ beta,
                                                          int64_t T, int Hk, int Hv, int form, int NC,
@@ -259,12 +260,13 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* rec = recs + ((static_cast<int64_t>(b) * Hv + h) * NC + c) * RC::BYTES;
 
-    // K, Q rows (zero past the end of the sequence) by asynchronous copies, g and beta
+    // K, Q rows (zero past the end of the sequence) by asynchronous copies, g and beta;
+    // token t's head hk row starts at (b T + t) ld_qk + hk K
     constexpr int V4 = K / 4;
     for (int idx = tid; idx < CH * V4; idx += 256) {
         const int r = idx / V4, c4 = idx - r * V4;
         const bool valid = r < n;
-        const int64_t off = valid ? ((static_cast<int64_t>(b) * T + t0 + r) * Hk + hk) * K + c4 * 4 : 0;
+        const int64_t off = valid ? (static_cast<int64_t>(b) * T + t0 + r) * ld_qk + static_cast<int64_t>(hk) * K + c4 * 4 : 0;
         cp_async16(&sm.ks[r * KS + c4 * 4], k + off, valid);
         cp_async16(&sm.qs[r * KS + c4 * 4], q + off, valid);
     }
@@ -276,6 +278,26 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     }
     cp_async_wait<0>();
     __syncthreads();
+    if (normalize_qk) {
+        // raw q, k rows: x / sqrt(sum x^2 + 1e-6), one warp per row, each lane K/32
+        // contiguous values (the same operation order as the standalone normalisation)
+        constexpr int PL = K / 32;
+        for (int row = warp; row < 2 * CH; row += 8) {
+            float* x = (row < CH ? sm.ks : sm.qs) + (row % CH) * KS + lane * PL;
+            float vv[PL];
+#pragma unroll
+            for (int i = 0; i < PL; ++i) vv[i] = x[i];
+            float ss = 0.0f;
+#pragma unroll
+            for (int i = 0; i < PL; ++i) ss = fmaf(vv[i], vv[i], ss);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float inv = 1.0f / sqrtf(ss + 1e-6f);
+#pragma unroll
+            for (int i = 0; i < PL; ++i) x[i] = vv[i] * inv;
+        }
+        __syncthreads();
+    }
     if (warp == 0) {
         // inclusive prefix sum of g over the chunk (2 values per lane)
         float a0 = sm.graw[2 * lane], a1 = sm.graw[2 * lane + 1];
@@ -781,7 +803,7 @@ template <int K, int V>
 nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                                const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form,
                                const float* s_in, float* s_out, float* o, void* ws, unsigned int* o_amax,
-                               cudaStream_t st) {
+                               int64_t ld_qk, int normalize_qk, cudaStream_t st) {
     const int NC = static_cast<int>((T + CH - 1) / CH);
     const int prep_smem = sizeof(PrepSmem<K, V>);
     const int seq_smem = SeqLayout<K>::BYTES;
@@ -799,7 +821,8 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     uint8_t* recs = static_cast<uint8_t*>(ws);
     const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
-    chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, recs);
+    chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, ld_qk, normalize_qk, v, ld_v, g, beta, T, d.Hk,
+                                                                 d.Hv, form, NC, recs);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
     chunk_seq_kernel<K, V><<<seq_blocks, 320, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, o_amax, err);
     cudaError_t e = cudaGetLastError();
@@ -828,8 +851,10 @@ size_t scan_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo) {
 nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                          const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form, int algo,
                          const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st,
-                         unsigned int* o_amax) {
+                         unsigned int* o_amax, int64_t ld_qk, int normalize_qk) {
     const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
+    if (!chunked && (normalize_qk || ld_qk != static_cast<int64_t>(d.Hk) * d.K))
+        return fail(NVFP4_ERR_INVALID_ARG, "raw q/k rows need the chunked scan");
     if (!chunked) {
         const unsigned blocks = static_cast<unsigned>(B * d.Hv * (d.V / 32));
         if (d.K == 128)
@@ -843,12 +868,12 @@ nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t
         return NVFP4_OK;
     }
     if (d.K == 128 && d.V == 128)
-        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
+        return launch_chunked_kv<128, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, ld_qk, normalize_qk, st);
     if (d.K == 128 && d.V == 64)
-        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
+        return launch_chunked_kv<128, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, ld_qk, normalize_qk, st);
     if (d.K == 64 && d.V == 128)
-        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
-    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, st);
+        return launch_chunked_kv<64, 128>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, ld_qk, normalize_qk, st);
+    return launch_chunked_kv<64, 64>(q, k, v, ld_v, g, beta, B, T, d, scale, form, s_in, s_out, o, ws, o_amax, ld_qk, normalize_qk, st);
 }
 
 }  // namespace nvg
@@ -878,5 +903,5 @@ extern "C" nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const f
     if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)))
         return fail(NVFP4_ERR_WORKSPACE, "scan workspace missing, too small or not 256-byte aligned");
     return scan_launch(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, algo, state_in, state_out, o,
-                       workspace, as_stream(stream), nullptr);
+                       workspace, as_stream(stream), nullptr, static_cast<int64_t>(dims->Hk) * dims->K, 0);
 }

@@ -20,7 +20,7 @@ nvfp4_status validate_dims(const gdn_dims* d);
 nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
                          const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form, int algo,
                          const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st,
-                         unsigned int* o_amax);
+                         unsigned int* o_amax, int64_t ld_qk, int normalize_qk);
 
 namespace {
 
@@ -77,5 +77,6 @@ extern "C" nvfp4_status gdn_scan_noalloc(const float* q_hat, const float* k_hat,
     void* scratch = nullptr;
     if ((s = scratch_address(&scratch)) != NVFP4_OK) return s;
     return scan_launch(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, GDN_SCAN_CHUNKED, state_in,
-                       state_out, o, scratch, as_stream(stream), nullptr);
+                       state_out, o, scratch, as_stream(stream), nullptr, static_cast<int64_t>(dims->Hk) * dims->K,
+                       0);
 }
