@@ -158,7 +158,7 @@ struct PrepSmem {
     static constexpr int TBS = 20;     // row stride of the diagonal-block inverses
     float ks[CH * KS];
     float qs[CH * KS];
-    float L[CH * LS];                  // strictly lower, scaled: b_t e^{Gd_t - G_i} k_t.k_i
+    float L[CH * LS];                  // -L (TF32): L strictly lower, L_ti = b_t e^{Gd_t - G_i} k_t.k_i
     float Tb[4 * 16 * TBS];            // (I + L_bb)^-1 for the four 16 x 16 diagonal blocks
     float gin[CH], gd[CH], bet[CH], graw[CH], df[CH];
     float eG[CH], eKh[CH];             // e^{G_t}, e^{G_C - G_t}
@@ -167,10 +167,11 @@ struct PrepSmem {
 // W = (I + L)^-1 diag(s) X for the 32-column strip c0..c0+31 of X [64 x N] (row
 // stride KS) in shared memory, by block forward substitution over 16-row blocks:
 //   W_b = T_bb (diag(s_b) X_b - sum_{k<b} L_bk W_k),   T_bb = (I + L_bb)^-1.
-// The strip is overwritten by W (float32) and each pair of adjacent outputs (t, col),
-// (t, col+1), col even, also goes to store(t, col, x0, x1).  One warp, which alone
-// touches these columns.  TF32 tensor cores (operands rounded to nearest), float32
-// accumulation.
+// Lm holds -L and Tb the T_bb, X the right-hand sides, all already rounded to TF32;
+// the strip is overwritten by W rounded to TF32 (it is only read again as an MMA
+// operand) and each pair of adjacent float32 outputs (t, col), (t, col+1), col even,
+// goes to store(t, col, x0, x1).  One warp, which alone touches these columns.
+// TF32 tensor cores, float32 accumulation.
 template <int KS, int LS, int TBS, typename Store>
 __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const float* __restrict__ Tb,
                                             const float* __restrict__ s, float* __restrict__ X, int c0, int lane,
@@ -193,13 +194,14 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
         }
 #pragma unroll
         for (int k0 = 0; k0 < r0; k0 += 8) {
-            const uint32_t a[4] = {to_tf32(-Lm[(r0 + grp) * LS + k0 + tig]), to_tf32(-Lm[(r0 + grp + 8) * LS + k0 + tig]),
-                                   to_tf32(-Lm[(r0 + grp) * LS + k0 + tig + 4]),
-                                   to_tf32(-Lm[(r0 + grp + 8) * LS + k0 + tig + 4])};
+            const uint32_t a[4] = {__float_as_uint(Lm[(r0 + grp) * LS + k0 + tig]),
+                                   __float_as_uint(Lm[(r0 + grp + 8) * LS + k0 + tig]),
+                                   __float_as_uint(Lm[(r0 + grp) * LS + k0 + tig + 4]),
+                                   __float_as_uint(Lm[(r0 + grp + 8) * LS + k0 + tig + 4])};
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                const uint32_t bb[2] = {to_tf32(X[(k0 + tig) * KS + c0 + nt * 8 + grp]),
-                                        to_tf32(X[(k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
+                const uint32_t bb[2] = {__float_as_uint(X[(k0 + tig) * KS + c0 + nt * 8 + grp]),
+                                        __float_as_uint(X[(k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
                 mma_tf32(acc[nt], a, bb);
             }
         }
@@ -207,8 +209,10 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
             const int col = c0 + nt * 8 + 2 * tig;
-            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) = make_float2(acc[nt][0], acc[nt][1]);
-            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) = make_float2(acc[nt][2], acc[nt][3]);
+            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) =
+                make_float2(__uint_as_float(to_tf32(acc[nt][0])), __uint_as_float(to_tf32(acc[nt][1])));
+            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) =
+                make_float2(__uint_as_float(to_tf32(acc[nt][2])), __uint_as_float(to_tf32(acc[nt][3])));
         }
         __syncwarp();
         float w[4][4];
@@ -217,12 +221,13 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
         const float* Tbb = Tb + b * 16 * TBS;
 #pragma unroll
         for (int k0 = 0; k0 < 16; k0 += 8) {
-            const uint32_t a[4] = {to_tf32(Tbb[grp * TBS + k0 + tig]), to_tf32(Tbb[(grp + 8) * TBS + k0 + tig]),
-                                   to_tf32(Tbb[grp * TBS + k0 + tig + 4]), to_tf32(Tbb[(grp + 8) * TBS + k0 + tig + 4])};
+            const uint32_t a[4] = {__float_as_uint(Tbb[grp * TBS + k0 + tig]), __float_as_uint(Tbb[(grp + 8) * TBS + k0 + tig]),
+                                   __float_as_uint(Tbb[grp * TBS + k0 + tig + 4]),
+                                   __float_as_uint(Tbb[(grp + 8) * TBS + k0 + tig + 4])};
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                const uint32_t bb[2] = {to_tf32(X[(r0 + k0 + tig) * KS + c0 + nt * 8 + grp]),
-                                        to_tf32(X[(r0 + k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
+                const uint32_t bb[2] = {__float_as_uint(X[(r0 + k0 + tig) * KS + c0 + nt * 8 + grp]),
+                                        __float_as_uint(X[(r0 + k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
                 mma_tf32(w[nt], a, bb);
             }
         }
@@ -230,8 +235,10 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
             const int col = c0 + nt * 8 + 2 * tig;
-            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) = make_float2(w[nt][0], w[nt][1]);
-            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) = make_float2(w[nt][2], w[nt][3]);
+            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) =
+                make_float2(__uint_as_float(to_tf32(w[nt][0])), __uint_as_float(to_tf32(w[nt][1])));
+            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) =
+                make_float2(__uint_as_float(to_tf32(w[nt][2])), __uint_as_float(to_tf32(w[nt][3])));
             store(r0 + grp, col, w[nt][0], w[nt][1]);
             store(r0 + grp + 8, col, w[nt][2], w[nt][3]);
         }
@@ -278,23 +285,28 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     }
     cp_async_wait<0>();
     __syncthreads();
-    if (normalize_qk) {
-        // raw q, k rows: x / sqrt(sum x^2 + 1e-6), one warp per row, each lane K/32
-        // contiguous values (the same operation order as the standalone normalisation)
+    {
+        // K and Q tiles are tensor-core operands only from here on: rounded to TF32
+        // in place.  With raw q, k rows (normalize_qk) each row is first scaled by
+        // 1 / sqrt(sum x^2 + 1e-6), one warp per row, each lane K/32 contiguous values
+        // (the same operation order as the standalone normalisation).
         constexpr int PL = K / 32;
         for (int row = warp; row < 2 * CH; row += 8) {
             float* x = (row < CH ? sm.ks : sm.qs) + (row % CH) * KS + lane * PL;
             float vv[PL];
 #pragma unroll
             for (int i = 0; i < PL; ++i) vv[i] = x[i];
-            float ss = 0.0f;
+            float inv = 1.0f;
+            if (normalize_qk) {
+                float ss = 0.0f;
 #pragma unroll
-            for (int i = 0; i < PL; ++i) ss = fmaf(vv[i], vv[i], ss);
+                for (int i = 0; i < PL; ++i) ss = fmaf(vv[i], vv[i], ss);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float inv = 1.0f / sqrtf(ss + 1e-6f);
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                inv = 1.0f / sqrtf(ss + 1e-6f);
+            }
 #pragma unroll
-            for (int i = 0; i < PL; ++i) x[i] = vv[i] * inv;
+            for (int i = 0; i < PL; ++i) x[i] = __uint_as_float(to_tf32(normalize_qk ? vv[i] * inv : vv[i]));
         }
         __syncthreads();
     }
@@ -337,13 +349,14 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         for (int k0 = 0; k0 < K; k0 += 8) {
             const float a[4] = {A[(r0 + grp) * KS + k0 + tig], A[(r0 + grp + 8) * KS + k0 + tig],
                                 A[(r0 + grp) * KS + k0 + tig + 4], A[(r0 + grp + 8) * KS + k0 + tig + 4]};
-            const uint32_t ai[4] = {to_tf32(a[0]), to_tf32(a[1]), to_tf32(a[2]), to_tf32(a[3])};
+            const uint32_t ai[4] = {__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                                    __float_as_uint(a[3])};
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 // tiles right of this warp's diagonal block are masked out afterwards
                 if (nt * 8 > r0 + 15) continue;
-                const uint32_t bb[2] = {to_tf32(sm.ks[(nt * 8 + grp) * KS + k0 + tig]),
-                                        to_tf32(sm.ks[(nt * 8 + grp) * KS + k0 + tig + 4])};
+                const uint32_t bb[2] = {__float_as_uint(sm.ks[(nt * 8 + grp) * KS + k0 + tig]),
+                                        __float_as_uint(sm.ks[(nt * 8 + grp) * KS + k0 + tig + 4])};
                 mma_tf32(acc[nt], ai, bb);
             }
         }
@@ -354,9 +367,12 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 const int t = r0 + grp + hh * 8;
                 const int i = nt * 8 + 2 * tig;
                 if (warp < 4) {
-                    sm.L[t * SM::LS + i] = (i < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
-                    sm.L[t * SM::LS + i + 1] =
+                    // stored negated and rounded to TF32: -L is a tensor-core operand
+                    const float l0 = (i < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
+                    const float l1 =
                         (i + 1 < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
+                    sm.L[t * SM::LS + i] = __uint_as_float(to_tf32(-l0));
+                    sm.L[t * SM::LS + i + 1] = __uint_as_float(to_tf32(-l1));
                 } else {
                     // rounded to TF32 here: it is only ever a tensor-core operand
                     const float m0 = (i <= t) ? __expf(sm.gin[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
@@ -413,15 +429,22 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
 #pragma unroll
             for (int j = 0; j <= i; ++j) {
                 const float tij = __shfl_sync(0xffffffffu, Tr[j], i);
-                Tr[j] = fmaf(-Lr[i], tij, Tr[j]);
+                Tr[j] = fmaf(Lr[i], tij, Tr[j]);   // Lr holds -L
             }
         }
         if (lane < 16) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) sm.Tb[warp * 16 * TBS + r * TBS + j] = Tr[j];
+            for (int j = 0; j < 16; ++j) sm.Tb[warp * 16 * TBS + r * TBS + j] = __uint_as_float(to_tf32(Tr[j]));
         }
     }
     cp_async_wait<0>();
+    __syncthreads();
+    for (int idx = tid; idx < CH * (V / 4); idx += 256) {
+        float4* p4 = reinterpret_cast<float4*>(&sm.qs[(idx / (V / 4)) * KS + 4 * (idx % (V / 4))]);
+        const float4 x = *p4;
+        *p4 = make_float4(__uint_as_float(to_tf32(x.x)), __uint_as_float(to_tf32(x.y)), __uint_as_float(to_tf32(x.z)),
+                          __uint_as_float(to_tf32(x.w)));
+    }
     __syncthreads();
     // W~ = (I + L)^-1 diag(b e^{Gd}) K (stored TF32-rounded: a tensor-core operand downstream),
     // U~ = (I + L)^-1 diag(beta) V; 32-column strips, W~ strips first, one warp each
