@@ -295,6 +295,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- standalone GEMM workload (M=8192, N=12288, K=5120), TFLOPS
     gemm = bench_gemm(nv, dev, args.steps, flush, stream)
+    # ---- batch-64 decode step (HBM-bound)
+    decode = bench_decode(nv, dev, w, sh, args.steps, stream)
 
     # ---- end to end through the public call with host buffers
     x_host = torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -355,12 +357,54 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": traffic, "peak_source": peak_note},
         "stages": stages,
         "gemm_standalone": gemm,
+        "decode": decode,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
     }
     return out
+
+
+def bench_decode(nv, dev, w, sh, steps, stream):
+    """Batch-64 decode: gdn_layer_forward with T = 1 and the 64 x 32 fp32 states
+    carried in place.  The states (268 MB) are larger than L2, so no flush is
+    needed between steps.  Algorithmic bytes per step: the states read and
+    written, both NVFP4 weights (codes + scales), x and y."""
+    import gdn_synth
+    B = 64
+    S = torch.from_numpy(gdn_synth.gaussian(9, (B, sh.Hv, sh.K, sh.V), std=0.3)).to(dev)
+    xs = [torch.from_numpy(gdn_synth.activations(2000 + i, B, sh.H, hot="none")[0].view(np.int16)).to(dev)
+          .view(torch.bfloat16) for i in range(4)]
+    y = torch.empty((B, sh.H), dtype=torch.float32, device=dev)
+    lay = nv.layer_workspace_layout(w, B, 1)
+    ws = torch.empty(lay["total"], dtype=torch.uint8, device=dev)
+
+    def step(i):
+        nv.gdn_layer_forward(w, xs[i % 4], B, 1, y=y, state_in=S, state_out=S, workspace=ws, stream=stream)
+
+    for i in range(5):
+        step(i)
+    n = max(steps, 32)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for i in range(n):
+        step(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    ms = s.elapsed_time(e) / n
+    pk = peaks()
+    state = 2 * B * sh.Hv * sh.K * sh.V * 4
+    weights = sh.n_in * sh.H // 2 + sh.n_in * sh.H // 16 + sh.H * sh.Hv * sh.V // 2 + sh.H * sh.Hv * sh.V // 16
+    io = B * sh.H * 2 + B * sh.H * 4
+    nbytes = state + weights + io
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": "gdn_decode_B64_h5120_hk16_hv32_k128_v128", "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(B / (ms / 1e3), 1), "bytes_per_step": nbytes, "GB/s": round(gbs, 1),
+            "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "steps": n,
+            "l2": "states (268 MB) larger than L2; no flush"}
 
 
 def bench_gemm(nv, dev, steps, flush, stream):
