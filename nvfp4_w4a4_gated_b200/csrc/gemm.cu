@@ -112,9 +112,8 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* empty = full + G::STAGES;
     uint64_t* acc_full = empty + G::STAGES;
     uint64_t* tmem_free = acc_full + 1;
-    uint64_t* sf_full = tmem_free + 1;   // [2] scale slot written (4 writer warps)
-    uint64_t* sf_free = sf_full + 2;     // [2] scale slot consumed (MMA commit)
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_free + 2);
+    uint64_t* sf_full = tmem_free + 1;   // [2] scale slot written (4 writer warps, after the stage landed)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_full + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
@@ -130,10 +129,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(tmem_free, 4);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&sf_full[i], 4);
-            mbar_init(&sf_free[i], 1);
-        }
+        for (int i = 0; i < 2; ++i) mbar_init(&sf_full[i], 4);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -196,10 +192,8 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 bool ok = true;
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    if (!mbar_wait(&full[stage], phase, err, kErrTimeoutMma)) {
-                        ok = false;
-                        break;
-                    }
+                    // the scale writers fill a slot only after this stage's copies landed,
+                    // so their signal covers the stage too
                     const int slot = static_cast<int>(kt_all & 1u);
                     if (!mbar_wait(&sf_full[slot], (kt_all >> 1) & 1u, err, kErrTimeoutMma)) {
                         ok = false;
@@ -216,7 +210,6 @@ __global__ void __launch_bounds__(320, 1)
                                  (kt > 0 || j > 0) ? 1u : 0u);
                     }
                     mma_commit(&empty[stage]);
-                    mma_commit(&sf_free[slot]);
                     if (++stage == G::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -260,9 +253,14 @@ __global__ void __launch_bounds__(320, 1)
                             wb[j][nb] = *reinterpret_cast<const uint4*>(b + nb * 2048 + j * 512);
                     }
                 }
-                if (kt_all >= 2 && !mbar_wait(&sf_free[slot], ((kt_all >> 1) - 1) & 1u, err, kErrTimeoutEpi)) {
-                    ok = false;
-                    break;
+                // the slot was last used by k-tile kt_all - 2, whose MMAs completing also
+                // released its stage: wait on that stage's empty barrier for that use
+                if (kt_all >= 2) {
+                    const uint32_t prev = kt_all - 2;
+                    if (!mbar_wait(&empty[prev % G::STAGES], (prev / G::STAGES) & 1u, err, kErrTimeoutEpi)) {
+                        ok = false;
+                        break;
+                    }
                 }
                 tc_fence_after();
 #pragma unroll
