@@ -476,9 +476,10 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
 // The recurrence runs through R1 -> U -> R2a -> S only; R2b and the output rows
 // drain while the next chunk's R1 and U run (D1 alternates between two TMEM
 // buffers).  Warp 0 copies the chunk records into shared memory (bulk copies,
-// [Q~; W~] and U~ double-buffered); warps 1..4 (one per TMEM lane quarter) form
-// U, the state and the output, and one lane of warp 2 issues the MMAs right
-// after the named barrier that publishes their operands.
+// [Q~; W~] and U~ double-buffered, L2 prefetch ahead) and issues R2b once R2a has
+// completed; warp 1 issues R1 and R2a; the compute warps, kSeqGroups per TMEM lane
+// quarter with kSeqCols columns each, form U, the state and the output.  Every
+// hand-off is an mbarrier (bounded waits).
 template <int K>
 struct SeqLayout {
     static constexpr uint32_t A1_BYTES = 128 * K * 4;
@@ -492,6 +493,12 @@ struct SeqLayout {
     static constexpr uint32_t BAR = B2 + CH * 128;
     static constexpr uint32_t BYTES = BAR + 256 + 1024;       // + alignment slack
 };
+
+// warp 0: producer, warp 1: MMA, then kSeqGroups groups of 4 compute warps (one per
+// TMEM lane quarter), group j owning columns 32 / kSeqGroups * j .. of the slice
+constexpr int kSeqGroups = 2;   // 4 measured slower (more arrivals per hand-off)
+constexpr int kSeqCols = 32 / kSeqGroups;
+constexpr int kSeqThreads = 64 + 128 * kSeqGroups;
 
 enum SeqBar : int {
     kA1Full = 0,   // [2] [Q~; W~] stage landed
@@ -513,7 +520,7 @@ enum SeqBar : int {
 };
 
 template <int K, int V>
-__global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
+__global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
                                                            float scale, int NC, const float* state_in,
                                                            float* state_out, float* __restrict__ o,
                                                            unsigned int* __restrict__ o_amax,
@@ -535,7 +542,9 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumSeqBars; ++i)
-            mbar_init(&bar[i], i == kSReady ? 8 : (i == kUtEmpty || i == kUtEmpty + 1 || i == kOFree || i == kUPub) ? 4 : 1);
+            mbar_init(&bar[i], i == kSReady                                                           ? 4 * kSeqGroups
+                               : (i == kUtEmpty || i == kUtEmpty + 1 || i == kOFree || i == kUPub) ? 2 * kSeqGroups
+                                                                                                     : 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -681,9 +690,9 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             mbar_wait(&bar[kFin], 0, err, kErrTimeoutSeq);
         }
     } else {
-        // ---- warps 2..9: TMEM lane quarter q = warp % 4, columns c0..c0+15 of the slice
+        // ---- compute warps: TMEM lane quarter q = warp % 4, columns c0..c0+kSeqCols-1 of the slice
         const int q = warp & 3;
-        const int c0 = 16 * ((warp - 2) >> 2);
+        const int c0 = kSeqCols * ((warp - 2) >> 2);
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int d = q * 32 + lane;             // state row
         const bool has_row = d < K;
@@ -715,8 +724,8 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar[kODone], c & 1, err, kErrTimeoutSeq));
             if (!ok) return false;
             tc_fence_after();
-            uint32_t x[16];
-            tmem_ld_32x32b_x16(tmem + 32 * (c & 1) + c0 + lane_base, x);
+            uint32_t x[kSeqCols];
+            tmem_ld_cols<kSeqCols>(tmem + 32 * (c & 1) + c0 + lane_base, x);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -726,7 +735,7 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             if (t < T) {
                 float* orow = o + ((static_cast<int64_t>(b) * T + t) * Hv + h) * V + vs0 + c0;
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4) {
+                for (int v4 = 0; v4 < kSeqCols / 4; ++v4) {
                     const float4 ov = make_float4(scale * __uint_as_float(x[4 * v4]), scale * __uint_as_float(x[4 * v4 + 1]),
                                                   scale * __uint_as_float(x[4 * v4 + 2]),
                                                   scale * __uint_as_float(x[4 * v4 + 3]));
@@ -741,9 +750,9 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             return true;
         };
 
-        float S[16];
+        float S[kSeqCols];
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
+        for (int v4 = 0; v4 < kSeqCols / 4; ++v4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (state_in && has_row)
                 x = *reinterpret_cast<const float4*>(state_in + sbase + static_cast<int64_t>(d) * V + vs0 + c0 + 4 * v4);
@@ -751,7 +760,7 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
         }
         if (has_row) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
+            for (int i = 0; i < kSeqCols; ++i)
                 *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) = __uint_as_float(to_tf32(S[i]));
         }
         publish(kSReady);
@@ -760,12 +769,12 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             const int s = c & 1;
             const float gc = *reinterpret_cast<const float*>(rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::GC);
             if (u_role) {
-                float ut[16];
+                float ut[kSeqCols];
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar[kUtFull + s], (c >> 1) & 1, err, kErrTimeoutSeq));
                 if (!ok) break;
                 const uint8_t* up = sm + L::UT + s * L::UT_BYTES + tu * 128;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
+                for (int jj = 0; jj < kSeqCols / 4; ++jj) {
                     const int j = (c0 >> 2) + jj;
                     const float4 x = *reinterpret_cast<const float4*>(up + ((j ^ (tu & 7)) << 4));
                     ut[4 * jj] = x.x; ut[4 * jj + 1] = x.y; ut[4 * jj + 2] = x.z; ut[4 * jj + 3] = x.w;
@@ -777,11 +786,11 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
                                                  (c == 0 || mbar_wait(&bar[kODone], (c - 1) & 1, err, kErrTimeoutSeq)));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t x[16];
-                tmem_ld_32x32b_x16(tmem + 32 * s + c0 + lane_base, x);
+                uint32_t x[kSeqCols];
+                tmem_ld_cols<kSeqCols>(tmem + 32 * s + c0 + lane_base, x);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
+                for (int i = 0; i < kSeqCols; ++i)
                     *reinterpret_cast<float*>(b2p + u_base + (i >> 3) * 1024 + u_xo[i & 7]) =
                         __uint_as_float(to_tf32(ut[i] - __uint_as_float(x[i])));
                 publish(kUPub);
@@ -792,13 +801,13 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
             ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR2Done], c & 1, err, kErrTimeoutSeq));
             if (!ok) break;
             tc_fence_after();
-            uint32_t x[16];
-            tmem_ld_32x32b_x16(tmem + 64 + c0 + lane_base, x);
+            uint32_t x[kSeqCols];
+            tmem_ld_cols<kSeqCols>(tmem + 64 + c0 + lane_base, x);
             tmem_wait_ld();
             if (has_row) {
                 const float eg = expf(gc);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < kSeqCols; ++i) {
                     S[i] = fmaf(eg, S[i], __uint_as_float(x[i]));
                     *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) =
                         __uint_as_float(to_tf32(S[i]));
@@ -809,7 +818,7 @@ __global__ void __launch_bounds__(320, 1) chunk_seq_kernel(const uint8_t* __rest
         if (ok && !u_role) ok = drain_o(NC - 1, ok);
         if (ok && state_out && has_row) {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
+            for (int v4 = 0; v4 < kSeqCols / 4; ++v4)
                 *reinterpret_cast<float4*>(state_out + sbase + static_cast<int64_t>(d) * V + vs0 + c0 + 4 * v4) =
                     make_float4(S[4 * v4], S[4 * v4 + 1], S[4 * v4 + 2], S[4 * v4 + 3]);
         }
@@ -847,7 +856,7 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, ld_qk, normalize_qk, v, ld_v, g, beta, T, d.Hk,
                                                                  d.Hv, form, NC, recs);
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    chunk_seq_kernel<K, V><<<seq_blocks, 320, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, o_amax, err);
+    chunk_seq_kernel<K, V><<<seq_blocks, kSeqThreads, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, o_amax, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     return NVFP4_OK;
