@@ -98,6 +98,14 @@ NVFP4_API const char* nvfp4_last_error(void);
 NVFP4_API nvfp4_status nvfp4_check_device_error(nvfp4_stream_t stream);
 /* Library version, "major.minor.patch". Host string, static storage. */
 NVFP4_API const char* nvfp4_version(void);
+/* Test hook for the failure path above (the pages have no counterpart): launches
+ * one thread on `stream` that waits on a barrier nothing ever arrives on, with a
+ * bounded wait of `budget_cycles` SM clocks (1 .. 2^30), after which it records a
+ * failure in the device error word and returns -- the same path every kernel of
+ * the library takes when a wait runs out.  The next nvfp4_check_device_error()
+ * then reports NVFP4_ERR_TIMEOUT and the CUDA context stays usable.
+ * NVFP4_ERR_INVALID_ARG for a budget outside the range. */
+NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(uint32_t budget_cycles, nvfp4_stream_t stream);
 
 /* ------------------------------------------------------------ quantiser -- */
 /* Bytes of the scale-factor buffer of an NVFP4 [rows x cols] matrix. */

@@ -19,7 +19,8 @@ from . import build as _build
 
 __all__ = [
     "NVFP4Error", "NVFP4Matrix", "GdnDims", "LayerWeights", "lib", "nvfp4_quantize", "w4a4_gemm", "gdn_gates",
-    "gdn_scan", "gdn_scan_noalloc", "gdn_layer_forward", "layer_workspace_layout", "check_device_error", "FORM_PAGES",
+    "gdn_scan", "gdn_scan_noalloc", "gdn_layer_forward", "layer_workspace_layout", "check_device_error",
+    "selftest_wait_timeout", "FORM_PAGES",
     "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
 ]
 
@@ -31,7 +32,7 @@ QUANT_COMPUTE_SCALE, QUANT_GIVEN_SCALE = 0, 1
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA", 5: "TIMEOUT", 6: "WORKSPACE"}
 
 EXPORTED_SYMBOLS = [
-    "nvfp4_last_error", "nvfp4_check_device_error", "nvfp4_version", "nvfp4_sf_bytes",
+    "nvfp4_last_error", "nvfp4_check_device_error", "nvfp4_version", "nvfp4_selftest_wait_timeout", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_size", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan_workspace_size",
     "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc",
 ]
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_last_error.restype = ctypes.c_char_p
         L.nvfp4_version.restype = ctypes.c_char_p
         L.nvfp4_check_device_error.argtypes = [P]
+        L.nvfp4_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
         L.nvfp4_sf_bytes.argtypes = [i64, i64]
         L.nvfp4_sf_bytes.restype = sz
         L.nvfp4_quantize_workspace_size.restype = sz
@@ -97,7 +99,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_scan_noalloc.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, P, P, P, P]
         L.gdn_layer_workspace_layout.argtypes = [ctypes.POINTER(_LayerWeights), i32, i64, ctypes.POINTER(_Layout)]
         L.gdn_layer_forward.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, i32, P, sz, P]
-        for f in ("nvfp4_check_device_error", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
+        for f in ("nvfp4_check_device_error", "nvfp4_selftest_wait_timeout", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
                   "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -173,6 +175,11 @@ class LayerWeights:
 
 def check_device_error(stream=None):
     _check(lib().nvfp4_check_device_error(_stream(stream)))
+
+
+def selftest_wait_timeout(budget_cycles: int = 1 << 22, stream=None):
+    """Exercise the bounded-wait failure path (see the C header)."""
+    _check(lib().nvfp4_selftest_wait_timeout(budget_cycles, _stream(stream)))
 
 
 # --------------------------------------------------------------- entry points --

@@ -99,6 +99,35 @@ nvfp4_status make_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t ro
 
 extern "C" const char* nvfp4_last_error(void) { return nvg::g_last_error.c_str(); }
 
+namespace nvg {
+namespace {
+// One thread waits, bounded, on an mbarrier no one arrives on (see the header).
+__global__ void selftest_wait_kernel(uint32_t budget_cycles, unsigned int* err) {
+    __shared__ uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bar, 0)) {
+        if (clock64() - t0 > static_cast<long long>(budget_cycles)) {
+            atomicOr(err, kErrTimeoutSelftest);
+            return;
+        }
+    }
+}
+}  // namespace
+}  // namespace nvg
+
+extern "C" nvfp4_status nvfp4_selftest_wait_timeout(uint32_t budget_cycles, nvfp4_stream_t stream) {
+    using namespace nvg;
+    if (budget_cycles < 1 || budget_cycles > (1u << 30)) return fail(NVFP4_ERR_INVALID_ARG, "budget_cycles out of range");
+    unsigned int* err = device_error_word();
+    if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
+    selftest_wait_kernel<<<1, 1, 0, as_stream(stream)>>>(budget_cycles, err);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+    return NVFP4_OK;
+}
+
 extern "C" const char* nvfp4_version(void) { return "0.1.0"; }
 
 extern "C" nvfp4_status nvfp4_check_device_error(nvfp4_stream_t stream) {

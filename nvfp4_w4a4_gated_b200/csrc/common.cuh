@@ -43,6 +43,7 @@ constexpr unsigned int kErrTimeoutTma = 1u;
 constexpr unsigned int kErrTimeoutMma = 2u;
 constexpr unsigned int kErrTimeoutEpi = 4u;
 constexpr unsigned int kErrTimeoutSeq = 8u;
+constexpr unsigned int kErrTimeoutSelftest = 16u;
 
 // ---------------------------------------------------------------- device ---
 // Bounded waits give up after this many SM clocks (about half a second);

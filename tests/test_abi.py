@@ -131,3 +131,10 @@ def test_layer_layout_and_validation():
     st, _ = _err(L.gdn_layer_forward(ctypes.byref(lw), FAKE, 1, 4096, FAKE, None, None, 3, FAKE, 1 << 40, None))
     assert st == 1
     del w_in
+
+
+def test_selftest_budget_validation():
+    L = nv.lib()
+    for budget in (0, (1 << 30) + 1):
+        st, msg = _err(L.nvfp4_selftest_wait_timeout(budget, None))
+        assert st == 1 and "budget" in msg

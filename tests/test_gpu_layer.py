@@ -32,8 +32,9 @@ def _make_layer(shape, seed, dev="cuda"):
 
 
 @pytest.mark.parametrize("form", [nv.FORM_PAGES, nv.FORM_STANDARD])
-def test_tiny_layer_stagewise(cuda_dev, form):
-    sh, B, T = gdn_synth.TINY, 1, 64
+@pytest.mark.parametrize("B,T", [(1, 64), (2, 100)])   # (2, 100): two sequences, a ragged last chunk
+def test_tiny_layer_stagewise(cuda_dev, form, B, T):
+    sh = gdn_synth.TINY
     bits, x = gdn_synth.activations(0, B * T, sh.H, hot="fixed")
     w, (W_in, W_out, A_log, dt_bias) = _make_layer(sh, 0)
     S_out = torch.empty((B, sh.Hv, sh.K, sh.V), device="cuda")
@@ -62,9 +63,12 @@ def test_tiny_layer_stagewise(cuda_dev, form):
     assert rel_fro(S_out.cpu().numpy(), ref["S"]) <= 2e-3
     # stage 5: o quantisation: nearly all codes agree (inputs differ at the 1e-4 level)
     oc = _view(ws, lay["o_codes"], BT * HvV // 2, torch.uint8).cpu().numpy().reshape(BT, HvV // 2)
-    assert np.mean(oc != ref["oq"][0]) < 0.02
-    # stage 6: layer output at the W4A4 noise level of the out_proj
-    assert rel_fro(y.cpu().numpy(), ref["y"]) <= 2e-2
+    flipped = np.mean(oc != ref["oq"][0])
+    assert flipped < 0.02
+    # stage 6: layer output.  A flipped code moves its element by one E2M1 step, at most
+    # half its magnitude, so the output moves by about 0.5 sqrt(flipped) relative; the
+    # out_proj itself is held to 1e-3 in the isolated test below.
+    assert rel_fro(y.cpu().numpy(), ref["y"]) <= max(2e-2, 0.5 * np.sqrt(flipped))
 
 
 def test_tiny_layer_out_proj_stage_isolated(cuda_dev):
