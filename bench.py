@@ -298,22 +298,48 @@ def run_ours(args, rank, world, local_rank):
     # ---- batch-64 decode step (HBM-bound)
     decode = bench_decode(nv, dev, w, sh, args.steps, stream)
 
-    # ---- end to end through the public call with host buffers
+    # ---- end to end through the public call with host buffers, pipelined over steps:
+    # the upload of step i+1 (pinned x -> device) and the download of step i's y
+    # (device -> pinned) run on their own streams while step i / i+1 computes; inputs
+    # and outputs are double-buffered, events order every reuse.  The L2 flush stays
+    # in front of every forward, on the compute stream.  Time = one window from the
+    # first upload to the last download.
     x_host = torch.empty(x.shape, dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(x.cpu())
-    y_host = torch.empty(y.shape, dtype=torch.float32, pin_memory=True)
-    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    x_dev2 = torch.empty_like(x)
-    for i in range(args.steps):
-        flush.zero_()
-        e_s[i].record(stream)
-        x_dev2.copy_(x_host, non_blocking=True)
-        nv.gdn_layer_forward(w, x_dev2, B, T, y=y, workspace=ws, stream=stream)
-        y_host.copy_(y, non_blocking=True)
-        e_e[i].record(stream)
+    y_host = [torch.empty(y.shape, dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    y_dev = [torch.empty_like(y) for _ in range(2)]
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    up_done = [ev() for _ in range(args.steps)]
+    comp_done = [ev() for _ in range(args.steps)]
+    down_done = [ev() for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+    t_start.record(stream)
+    s_up.wait_event(t_start)
+    s_down.wait_event(t_start)
+    for i in range(args.steps):
+        j = i % 2
+        with torch.cuda.stream(s_up):
+            if i >= 2:
+                s_up.wait_event(comp_done[i - 2])       # x_dev[j] read by step i-2
+            x_dev[j].copy_(x_host, non_blocking=True)
+            up_done[i].record(s_up)
+        stream.wait_event(up_done[i])
+        if i >= 2:
+            stream.wait_event(down_done[i - 2])          # y_dev[j] read back by step i-2
+        flush.zero_()
+        nv.gdn_layer_forward(w, x_dev[j], B, T, y=y_dev[j], workspace=ws, stream=stream)
+        comp_done[i].record(stream)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(comp_done[i])
+            y_host[j].copy_(y_dev[j], non_blocking=True)
+            down_done[i].record(s_down)
+    stream.wait_event(down_done[args.steps - 1])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t_start.elapsed_time(t_end)
 
     # ---- aggregate over ranks: max time
     tvec = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
