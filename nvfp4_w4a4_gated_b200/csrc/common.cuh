@@ -37,6 +37,9 @@ nvfp4_status make_tmap_f32_sw128(CUtensorMap* map, const void* base, uint64_t ro
 // amax of the input as float bits (for instance folded into the kernel that produced
 // the input), so only the quantisation pass runs.
 constexpr int32_t kQuantFromAmax = 0x100;
+// Internal quantiser mode: as NVFP4_QUANT_COMPUTE_SCALE, with the workspace's amax
+// and arrival words (two 32-bit words) already zeroed by the caller.
+constexpr int32_t kQuantComputeZeroedWs = 0x200;
 
 // Error codes recorded in the device error word.
 constexpr unsigned int kErrTimeoutTma = 1u;
@@ -44,6 +47,7 @@ constexpr unsigned int kErrTimeoutMma = 2u;
 constexpr unsigned int kErrTimeoutEpi = 4u;
 constexpr unsigned int kErrTimeoutSeq = 8u;
 constexpr unsigned int kErrTimeoutSelftest = 16u;
+constexpr unsigned int kErrTimeoutQuant = 32u;
 
 // ---------------------------------------------------------------- device ---
 // Bounded waits give up after this many SM clocks (about half a second);

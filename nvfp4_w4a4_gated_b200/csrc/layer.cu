@@ -116,8 +116,11 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
     float* beta = reinterpret_cast<float*>(ws + L.beta);
     float* o = reinterpret_cast<float*>(ws + L.o);
 
-    if ((s = quantize_launch(x_bf16, NVFP4_DTYPE_BF16, BT, H, H, xq, NVFP4_QUANT_COMPUTE_SCALE, ws + L.quant_ws, st)) !=
-        NVFP4_OK)
+    // quantiser words: [0] x amax, [1] x arrival counter, [2] o amax; one memset
+    unsigned int* qw = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
+    cudaError_t e = cudaMemsetAsync(qw, 0, 4 * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(quantiser words)");
+    if ((s = quantize_launch(x_bf16, NVFP4_DTYPE_BF16, BT, H, H, xq, kQuantComputeZeroedWs, qw, st)) != NVFP4_OK)
         return s;
     if ((s = gemm_launch(xq, w->w_in, proj, ldp, st)) != NVFP4_OK) return s;
     // T > 1: the chunked scan reads the raw q, k slices of the projection and
@@ -136,14 +139,12 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
     const float scale = 1.0f / sqrtf(static_cast<float>(d.K));
     // the scan folds max|o| into the quantiser's amax word as it writes o, so the o
     // quantiser runs its quantisation pass only
-    unsigned int* o_amax = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
-    cudaError_t e = cudaMemsetAsync(o_amax, 0, sizeof(unsigned int), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(o amax)");
+    unsigned int* o_amax = qw + 2;
     if ((s = scan_launch(q_in, k_in, proj + 2ll * d.Hk * d.K, ldp, g, beta, B, T, d, scale, form,
                          chunked ? GDN_SCAN_CHUNKED : GDN_SCAN_RECURRENT, state_in, state_out, o, ws + L.scan_ws, st,
                          o_amax, ld_qk, chunked ? 1 : 0)) != NVFP4_OK)
         return s;
-    if ((s = quantize_launch(o, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, ws + L.quant_ws, st)) != NVFP4_OK)
+    if ((s = quantize_launch(o, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, o_amax, st)) != NVFP4_OK)
         return s;
     return gemm_launch(oq, w->w_out, y, H, st);
 }

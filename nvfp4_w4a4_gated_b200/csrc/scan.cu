@@ -21,6 +21,8 @@
 //    Q K^T and G; kernel 2 (one CTA per head x 32-column V slice) walks the
 //    chunks in order.  Products run on the tensor cores in TF32 with float32
 //    accumulation (mma.sync m16n8k8).
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace nvg {
@@ -152,8 +154,9 @@ __device__ __forceinline__ void cp_async_wait() {
 // One CTA (256 threads) per (sequence, chunk, value head).
 template <int K, int V>
 struct PrepSmem {
-    // row stride of the K and Q tiles (== 4 mod 32); the Q tile later holds the V rows
-    static constexpr int KS = (K > V ? K : V) + 4;
+    // row stride of the K and Q tiles (a multiple of 32 floats; the columns are
+    // XOR-swizzled, see tile_off); the Q tile later holds the V rows
+    static constexpr int KS = (K > V ? K : V);
     static constexpr int LS = CH + 4;  // row stride of L (== 4 mod 32)
     static constexpr int TBS = 20;     // row stride of the diagonal-block inverses
     float ks[CH * KS];
@@ -172,6 +175,20 @@ struct PrepSmem {
 // operand) and each pair of adjacent float32 outputs (t, col), (t, col+1), col even,
 // goes to store(t, col, x0, x1).  One warp, which alone touches these columns.
 // TF32 tensor cores, float32 accumulation.
+// Float offset of element (r, c) of a K, Q or V tile with row stride KS (a
+// multiple of 32).  Bits 2..4 of the column are XORed with ((r & 3) << 3) | (r & 4),
+// which permutes the 4-float groups inside each 32-float segment of a row.  Every
+// access pattern of the tiles is then free of bank conflicts: the TF32 mma.sync A
+// and B fragments read with k along a row (rows grp, columns tig), the B
+// fragments read with k down the columns (rows tig, columns grp), the float2
+// accumulator accesses, and row-contiguous vector accesses.  Aligned 2- and
+// 4-float vectors stay contiguous.
+template <int KS>
+__device__ __forceinline__ int tile_off(int r, int c) {
+    static_assert(KS % 32 == 0, "tile stride must be a multiple of 32 floats");
+    return r * KS + (c ^ (((r & 3) << 3) | (r & 4)));
+}
+
 template <int KS, int LS, int TBS, typename Store>
 __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const float* __restrict__ Tb,
                                             const float* __restrict__ s, float* __restrict__ X, int c0, int lane,
@@ -185,8 +202,8 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
             const int col = c0 + nt * 8 + 2 * tig;
-            const float2 x0 = *reinterpret_cast<const float2*>(&X[(r0 + grp) * KS + col]);
-            const float2 x1 = *reinterpret_cast<const float2*>(&X[(r0 + grp + 8) * KS + col]);
+            const float2 x0 = *reinterpret_cast<const float2*>(&X[tile_off<KS>(r0 + grp, col)]);
+            const float2 x1 = *reinterpret_cast<const float2*>(&X[tile_off<KS>(r0 + grp + 8, col)]);
             acc[nt][0] = s0 * x0.x;
             acc[nt][1] = s0 * x0.y;
             acc[nt][2] = s1 * x1.x;
@@ -200,8 +217,8 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
                                    __float_as_uint(Lm[(r0 + grp + 8) * LS + k0 + tig + 4])};
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                const uint32_t bb[2] = {__float_as_uint(X[(k0 + tig) * KS + c0 + nt * 8 + grp]),
-                                        __float_as_uint(X[(k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
+                const uint32_t bb[2] = {__float_as_uint(X[tile_off<KS>(k0 + tig, c0 + nt * 8 + grp)]),
+                                        __float_as_uint(X[tile_off<KS>(k0 + tig + 4, c0 + nt * 8 + grp)])};
                 mma_tf32(acc[nt], a, bb);
             }
         }
@@ -209,9 +226,9 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
             const int col = c0 + nt * 8 + 2 * tig;
-            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) =
+            *reinterpret_cast<float2*>(&X[tile_off<KS>(r0 + grp, col)]) =
                 make_float2(__uint_as_float(to_tf32(acc[nt][0])), __uint_as_float(to_tf32(acc[nt][1])));
-            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) =
+            *reinterpret_cast<float2*>(&X[tile_off<KS>(r0 + grp + 8, col)]) =
                 make_float2(__uint_as_float(to_tf32(acc[nt][2])), __uint_as_float(to_tf32(acc[nt][3])));
         }
         __syncwarp();
@@ -226,8 +243,8 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
                                    __float_as_uint(Tbb[(grp + 8) * TBS + k0 + tig + 4])};
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                const uint32_t bb[2] = {__float_as_uint(X[(r0 + k0 + tig) * KS + c0 + nt * 8 + grp]),
-                                        __float_as_uint(X[(r0 + k0 + tig + 4) * KS + c0 + nt * 8 + grp])};
+                const uint32_t bb[2] = {__float_as_uint(X[tile_off<KS>(r0 + k0 + tig, c0 + nt * 8 + grp)]),
+                                        __float_as_uint(X[tile_off<KS>(r0 + k0 + tig + 4, c0 + nt * 8 + grp)])};
                 mma_tf32(w[nt], a, bb);
             }
         }
@@ -235,9 +252,9 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
             const int col = c0 + nt * 8 + 2 * tig;
-            *reinterpret_cast<float2*>(&X[(r0 + grp) * KS + col]) =
+            *reinterpret_cast<float2*>(&X[tile_off<KS>(r0 + grp, col)]) =
                 make_float2(__uint_as_float(to_tf32(w[nt][0])), __uint_as_float(to_tf32(w[nt][1])));
-            *reinterpret_cast<float2*>(&X[(r0 + grp + 8) * KS + col]) =
+            *reinterpret_cast<float2*>(&X[tile_off<KS>(r0 + grp + 8, col)]) =
                 make_float2(__uint_as_float(to_tf32(w[nt][2])), __uint_as_float(to_tf32(w[nt][3])));
             store(r0 + grp, col, w[nt][0], w[nt][1]);
             store(r0 + grp + 8, col, w[nt][2], w[nt][3]);
@@ -274,8 +291,8 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         const int r = idx / V4, c4 = idx - r * V4;
         const bool valid = r < n;
         const int64_t off = valid ? (static_cast<int64_t>(b) * T + t0 + r) * ld_qk + static_cast<int64_t>(hk) * K + c4 * 4 : 0;
-        cp_async16(&sm.ks[r * KS + c4 * 4], k + off, valid);
-        cp_async16(&sm.qs[r * KS + c4 * 4], q + off, valid);
+        cp_async16(&sm.ks[tile_off<KS>(r, c4 * 4)], k + off, valid);
+        cp_async16(&sm.qs[tile_off<KS>(r, c4 * 4)], q + off, valid);
     }
     cp_async_commit();
     if (tid < CH) {
@@ -290,12 +307,16 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         // in place.  With raw q, k rows (normalize_qk) each row is first scaled by
         // 1 / sqrt(sum x^2 + 1e-6), one warp per row, each lane K/32 contiguous values
         // (the same operation order as the standalone normalisation).
+        // (Each lane moves its K/32 values as one vector access, so a warp's row is
+        // contiguous in shared memory: no bank conflicts.)
         constexpr int PL = K / 32;
+        static_assert(PL == 2 || PL == 4, "K must be 64 or 128");
+        using VecT = typename std::conditional<PL == 4, float4, float2>::type;
         for (int row = warp; row < 2 * CH; row += 8) {
-            float* x = (row < CH ? sm.ks : sm.qs) + (row % CH) * KS + lane * PL;
+            VecT* x = reinterpret_cast<VecT*>((row < CH ? sm.ks : sm.qs) + tile_off<KS>(row % CH, lane * PL));
+            const VecT xv = *x;
             float vv[PL];
-#pragma unroll
-            for (int i = 0; i < PL; ++i) vv[i] = x[i];
+            memcpy(vv, &xv, sizeof(vv));
             float inv = 1.0f;
             if (normalize_qk) {
                 float ss = 0.0f;
@@ -306,7 +327,10 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 inv = 1.0f / sqrtf(ss + 1e-6f);
             }
 #pragma unroll
-            for (int i = 0; i < PL; ++i) x[i] = __uint_as_float(to_tf32(normalize_qk ? vv[i] * inv : vv[i]));
+            for (int i = 0; i < PL; ++i) vv[i] = __uint_as_float(to_tf32(normalize_qk ? vv[i] * inv : vv[i]));
+            VecT yv;
+            memcpy(&yv, vv, sizeof(vv));
+            *x = yv;
         }
         __syncthreads();
     }
@@ -347,16 +371,16 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll 4
         for (int k0 = 0; k0 < K; k0 += 8) {
-            const float a[4] = {A[(r0 + grp) * KS + k0 + tig], A[(r0 + grp + 8) * KS + k0 + tig],
-                                A[(r0 + grp) * KS + k0 + tig + 4], A[(r0 + grp + 8) * KS + k0 + tig + 4]};
+            const float a[4] = {A[tile_off<KS>(r0 + grp, k0 + tig)], A[tile_off<KS>(r0 + grp + 8, k0 + tig)],
+                                A[tile_off<KS>(r0 + grp, k0 + tig + 4)], A[tile_off<KS>(r0 + grp + 8, k0 + tig + 4)]};
             const uint32_t ai[4] = {__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
                                     __float_as_uint(a[3])};
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 // tiles right of this warp's diagonal block are masked out afterwards
                 if (nt * 8 > r0 + 15) continue;
-                const uint32_t bb[2] = {__float_as_uint(sm.ks[(nt * 8 + grp) * KS + k0 + tig]),
-                                        __float_as_uint(sm.ks[(nt * 8 + grp) * KS + k0 + tig + 4])};
+                const uint32_t bb[2] = {__float_as_uint(sm.ks[tile_off<KS>(nt * 8 + grp, k0 + tig)]),
+                                        __float_as_uint(sm.ks[tile_off<KS>(nt * 8 + grp, k0 + tig + 4)])};
                 mma_tf32(acc[nt], ai, bb);
             }
         }
@@ -371,8 +395,8 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                     const float l0 = (i < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
                     const float l1 =
                         (i + 1 < t) ? sm.bet[t] * __expf(sm.gd[t] - sm.gin[i + 1]) * acc[nt][2 * hh + 1] : 0.0f;
-                    sm.L[t * SM::LS + i] = __uint_as_float(to_tf32(-l0));
-                    sm.L[t * SM::LS + i + 1] = __uint_as_float(to_tf32(-l1));
+                    *reinterpret_cast<float2*>(&sm.L[t * SM::LS + i]) =
+                        make_float2(__uint_as_float(to_tf32(-l0)), __uint_as_float(to_tf32(-l1)));
                 } else {
                     // rounded to TF32 here: it is only ever a tensor-core operand
                     const float m0 = (i <= t) ? __expf(sm.gin[t] - sm.gin[i]) * acc[nt][2 * hh] : 0.0f;
@@ -388,7 +412,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     for (int idx = tid; idx < CH * (K / 4); idx += 256) {
         const int t = idx / (K / 4), c4 = idx - t * (K / 4);
         const float eg = sm.eG[t];
-        const float4 x = *reinterpret_cast<const float4*>(&sm.qs[t * KS + 4 * c4]);
+        const float4 x = *reinterpret_cast<const float4*>(&sm.qs[tile_off<KS>(t, 4 * c4)]);
         *reinterpret_cast<float4*>(rec + RC::A1 + sw128_off(t, 4 * c4, 128)) =
             make_float4(__uint_as_float(to_tf32(eg * x.x)), __uint_as_float(to_tf32(eg * x.y)),
                         __uint_as_float(to_tf32(eg * x.z)), __uint_as_float(to_tf32(eg * x.w)));
@@ -397,7 +421,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         const int dd = idx % K, t4 = idx / K;
         float x[4];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(to_tf32(sm.eKh[4 * t4 + w] * sm.ks[(4 * t4 + w) * KS + dd]));
+        for (int w = 0; w < 4; ++w) x[w] = __uint_as_float(to_tf32(sm.eKh[4 * t4 + w] * sm.ks[tile_off<KS>(4 * t4 + w, dd)]));
         *reinterpret_cast<float4*>(rec + RC::A3 + sw128_off(dd, 4 * t4, 128)) = make_float4(x[0], x[1], x[2], x[3]);
     }
     __syncthreads();
@@ -408,7 +432,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         const int r = idx / VV4, c4 = idx - r * VV4;
         const bool valid = r < n;
         const int64_t off = valid ? (static_cast<int64_t>(b) * T + t0 + r) * ld_v + static_cast<int64_t>(h) * V + c4 * 4 : 0;
-        cp_async16(&sm.qs[r * KS + c4 * 4], v + off, valid);
+        cp_async16(&sm.qs[tile_off<KS>(r, c4 * 4)], v + off, valid);
     }
     cp_async_commit();
 
@@ -440,7 +464,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     cp_async_wait<0>();
     __syncthreads();
     for (int idx = tid; idx < CH * (V / 4); idx += 256) {
-        float4* p4 = reinterpret_cast<float4*>(&sm.qs[(idx / (V / 4)) * KS + 4 * (idx % (V / 4))]);
+        float4* p4 = reinterpret_cast<float4*>(&sm.qs[tile_off<KS>(idx / (V / 4), 4 * (idx % (V / 4)))]);
         const float4 x = *p4;
         *p4 = make_float4(__uint_as_float(to_tf32(x.x)), __uint_as_float(to_tf32(x.y)), __uint_as_float(to_tf32(x.z)),
                           __uint_as_float(to_tf32(x.w)));

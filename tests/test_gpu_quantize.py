@@ -84,3 +84,34 @@ def test_quantize_full_size_weight(cuda_dev):
     sh = gdn_synth.FULL
     W = gdn_synth.weights(200, sh.n_in, sh.H)
     _check(f32_device(W), W)
+
+
+@pytest.mark.parametrize("amax", [2688.0, 1000.0, 3.3e-3, 7.77e5])
+def test_quantize_block_maxima_near_e4m3_midpoints(cuda_dev, amax):
+    """Blocks whose max m puts the quotient m / (6 S) within three fp32 ulps of
+    every rounding midpoint between consecutive E4M3 values, under four global
+    scales: the block scale bytes (and codes) must match the oracle's correctly
+    rounded division followed by E4M3 rounding."""
+    vals = sorted({oracle.e4m3_decode(b) for b in range(0x7F)})
+    S = np.float32(np.float32(amax) / np.float32(2688.0))
+    d6 = np.float32(np.float32(6.0) * S)
+    maxima = []
+    for lo, hi in zip(vals[:-1], vals[1:]):
+        m0 = np.float32(np.float32((lo + hi) / 2) * d6)
+        for k in range(-3, 4):
+            m = m0
+            for _ in range(abs(k)):
+                m = np.nextafter(m, np.float32(np.inf if k > 0 else 0), dtype=np.float32)
+            if 0 < m <= amax:
+                maxima.append(m)
+    blocks = np.zeros((len(maxima) + 1, 16), np.float32)
+    g = gdn_synth.rng(17)
+    for i, m in enumerate(maxima):
+        blocks[i, 1:] = (g.uniform(-1, 1, 15) * m).astype(np.float32)
+        blocks[i, 0] = -m if i % 2 else m
+    blocks[-1, 5] = np.float32(amax)
+    nblk = (blocks.shape[0] + 3) // 4 * 4
+    x = np.zeros((nblk, 16), np.float32)
+    x[:blocks.shape[0]] = blocks
+    x = x.reshape(-1, 64)
+    _check(f32_device(x), x)
