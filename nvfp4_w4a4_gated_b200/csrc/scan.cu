@@ -538,22 +538,10 @@ enum SeqBar : int {
     kUReady = 14,  // R2a issued (the producer then issues R2b)
     kFin = 15,     // completion of the MMA warp's MMAs
     kFinP = 16,    // completion of the producer's MMAs
-    kNumSeqBars = 17
+    kSReady = 17,  // S^T published (one arrival per compute warp)
+    kUPub = 18,    // U^T published (one arrival per U warp)
+    kNumSeqBars = 19
 };
-
-// Hand-offs between warps of the CTA go through named barriers, which measured
-// about a third of the latency of an mbarrier arrive/wait pair on this part.
-// Every participant executes bar.sync (no bar.arrive), and each executes the
-// barrier exactly once per chunk on every path, error paths included, so no
-// warp can run a generation ahead and no barrier can be left short.
-constexpr int kBarS = 1;   // S^T published: compute warps + MMA warp
-constexpr int kBarSThreads = 32 * (4 * kSeqGroups + 1);
-constexpr int kBarU = 2;   // U^T published: U warps + MMA warp
-constexpr int kBarUThreads = 32 * (2 * kSeqGroups + 1);
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 template <int K, int V>
 __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t* __restrict__ recs, int64_t T, int Hv,
@@ -578,7 +566,9 @@ __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumSeqBars; ++i)
-            mbar_init(&bar[i], (i == kUtEmpty || i == kUtEmpty + 1 || i == kOFree) ? 2 * kSeqGroups : 1);
+            mbar_init(&bar[i], i == kSReady                                                           ? 4 * kSeqGroups
+                               : (i == kUtEmpty || i == kUtEmpty + 1 || i == kOFree || i == kUPub) ? 2 * kSeqGroups
+                                                                                                     : 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -691,47 +681,34 @@ __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t
             }
         }
     } else if (warp == 1) {
-        // ---- MMA warp: R1 and R2a, the two products on the recurrence.  All lanes
-        // take the named barriers; lane 0 waits on the records and issues.
-        const uint32_t b1 = smem_u32(sm + L::B1), b2 = smem_u32(sm + L::B2);
-        const uint32_t a3 = smem_u32(sm + L::A23) + CH * CH * 4;
-        bool ok = true;
-        for (int c = 0; c < NC; ++c) {
-            const int s = c & 1;
-            __syncwarp();
-            named_bar_sync(kBarS, kBarSThreads);   // S^T of chunk c published
-            if (lane == 0 && ok) {
-                ok = mbar_wait(&bar[kA1Full + s], (c >> 1) & 1, err, kErrTimeoutSeq);
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t a1 = smem_u32(sm + L::A1 + s * L::A1_BYTES);
-#pragma unroll
-                    for (int j = 0; j < K / 8; ++j)
-                        mma_tf32_ss(tmem + 32 * s, sdesc_kmajor_sw128(a1 + (j >> 2) * 128 * 128 + (j & 3) * 32),
-                                    sdesc_kmajor_sw128(b1 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC,
-                                    j > 0 ? 1u : 0u);
-                    mma_commit(&bar[kA1Empty + s]);
-                    mma_commit(&bar[kR1Done]);
-                }
-            }
-            __syncwarp();
-            named_bar_sync(kBarU, kBarUThreads);   // U^T of chunk c published
-            if (lane == 0 && ok) {
-                ok = mbar_wait(&bar[kA3Full], c & 1, err, kErrTimeoutSeq);
-                if (ok) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int j = 0; j < CH / 8; ++j)
-                        mma_tf32_ss(tmem + 64, sdesc_kmajor_sw128(a3 + (j >> 2) * 128 * 128 + (j & 3) * 32),
-                                    sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC,
-                                    j > 0 ? 1u : 0u);
-                    mma_commit(&bar[kR2Done]);
-                    mbar_arrive(&bar[kUReady]);
-                }
-            }
-        }
-        __syncwarp();
         if (lane == 0) {
+            // ---- MMA warp: R1 and R2a, the two products on the recurrence
+            const uint32_t b1 = smem_u32(sm + L::B1), b2 = smem_u32(sm + L::B2);
+            const uint32_t a3 = smem_u32(sm + L::A23) + CH * CH * 4;
+            for (int c = 0; c < NC; ++c) {
+                const int s = c & 1;
+                if (!mbar_wait(&bar[kSReady], c & 1, err, kErrTimeoutSeq) ||
+                    !mbar_wait(&bar[kA1Full + s], (c >> 1) & 1, err, kErrTimeoutSeq))
+                    break;
+                tc_fence_after();
+                const uint32_t a1 = smem_u32(sm + L::A1 + s * L::A1_BYTES);
+#pragma unroll
+                for (int j = 0; j < K / 8; ++j)
+                    mma_tf32_ss(tmem + 32 * s, sdesc_kmajor_sw128(a1 + (j >> 2) * 128 * 128 + (j & 3) * 32),
+                                sdesc_kmajor_sw128(b1 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
+                mma_commit(&bar[kA1Empty + s]);
+                mma_commit(&bar[kR1Done]);
+                if (!mbar_wait(&bar[kUPub], c & 1, err, kErrTimeoutSeq) ||
+                    !mbar_wait(&bar[kA3Full], c & 1, err, kErrTimeoutSeq))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int j = 0; j < CH / 8; ++j)
+                    mma_tf32_ss(tmem + 64, sdesc_kmajor_sw128(a3 + (j >> 2) * 128 * 128 + (j & 3) * 32),
+                                sdesc_kmajor_sw128(b2 + (j >> 2) * 32 * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
+                mma_commit(&bar[kR2Done]);
+                mbar_arrive(&bar[kUReady]);
+            }
             // all MMAs issued here have completed before TMEM is released
             mma_commit(&bar[kFin]);
             mbar_wait(&bar[kFin], 0, err, kErrTimeoutSeq);
@@ -760,13 +737,11 @@ __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t
         uint32_t u_base = 0, u_xo[8];
         swz_cols(u_role ? tu : 0, u_base, u_xo);
 
-        // shared-memory writes of this warp -> visible to the tensor core, then the
-        // named barrier with the MMA warp
-        auto publish = [&](int bar_id, int nthreads) {
+        auto publish = [&](int bar_id) {
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            named_bar_sync(bar_id, nthreads);
+            if (lane == 0) mbar_arrive(&bar[bar_id]);
         };
         // output rows t = d (lanes 0..63) of chunk c from D1
         auto drain_o = [&](int c, bool ok) -> bool {
@@ -812,61 +787,57 @@ __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t
             for (int i = 0; i < kSeqCols; ++i)
                 *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) = __uint_as_float(to_tf32(S[i]));
         }
-        publish(kBarS, kBarSThreads);
-        // After a failed wait the warp stops waiting and computing but still takes
-        // every named barrier, so that the MMA warp is never left at one.
+        publish(kSReady);
         bool ok = true;
-        for (int c = 0; c < NC; ++c) {
+        for (int c = 0; c < NC && ok; ++c) {
             const int s = c & 1;
             const float gc = *reinterpret_cast<const float*>(rec0 + static_cast<int64_t>(c) * RC::BYTES + RC::GC);
             if (u_role) {
                 float ut[kSeqCols];
-                ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar[kUtFull + s], (c >> 1) & 1, err, kErrTimeoutSeq));
-                if (ok) {
-                    const uint8_t* up = sm + L::UT + s * L::UT_BYTES + tu * 128;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar[kUtFull + s], (c >> 1) & 1, err, kErrTimeoutSeq));
+                if (!ok) break;
+                const uint8_t* up = sm + L::UT + s * L::UT_BYTES + tu * 128;
 #pragma unroll
-                    for (int jj = 0; jj < kSeqCols / 4; ++jj) {
-                        const int j = (c0 >> 2) + jj;
-                        const float4 x = *reinterpret_cast<const float4*>(up + ((j ^ (tu & 7)) << 4));
-                        ut[4 * jj] = x.x; ut[4 * jj + 1] = x.y; ut[4 * jj + 2] = x.z; ut[4 * jj + 3] = x.w;
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[kUtEmpty + s]);
+                for (int jj = 0; jj < kSeqCols / 4; ++jj) {
+                    const int j = (c0 >> 2) + jj;
+                    const float4 x = *reinterpret_cast<const float4*>(up + ((j ^ (tu & 7)) << 4));
+                    ut[4 * jj] = x.x; ut[4 * jj + 1] = x.y; ut[4 * jj + 2] = x.z; ut[4 * jj + 3] = x.w;
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kUtEmpty + s]);
                 // R1 done; R2b of the previous chunk has finished reading U^T
-                ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar[kR1Done], c & 1, err, kErrTimeoutSeq) &&
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR1Done], c & 1, err, kErrTimeoutSeq) &&
                                                  (c == 0 || mbar_wait(&bar[kODone], (c - 1) & 1, err, kErrTimeoutSeq)));
-                if (ok) {
-                    tc_fence_after();
-                    uint32_t x[kSeqCols];
-                    tmem_ld_cols<kSeqCols>(tmem + 32 * s + c0 + lane_base, x);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < kSeqCols; ++i)
-                        *reinterpret_cast<float*>(b2p + u_base + (i >> 3) * 1024 + u_xo[i & 7]) =
-                            __uint_as_float(to_tf32(ut[i] - __uint_as_float(x[i])));
-                }
-                publish(kBarU, kBarUThreads);
-            } else if (c > 0) {
-                ok = drain_o(c - 1, ok);
-            }
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar[kR2Done], c & 1, err, kErrTimeoutSeq));
-            if (ok) {
+                if (!ok) break;
                 tc_fence_after();
                 uint32_t x[kSeqCols];
-                tmem_ld_cols<kSeqCols>(tmem + 64 + c0 + lane_base, x);
+                tmem_ld_cols<kSeqCols>(tmem + 32 * s + c0 + lane_base, x);
                 tmem_wait_ld();
-                if (has_row) {
-                    const float eg = expf(gc);
 #pragma unroll
-                    for (int i = 0; i < kSeqCols; ++i) {
-                        S[i] = fmaf(eg, S[i], __uint_as_float(x[i]));
-                        *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) =
-                            __uint_as_float(to_tf32(S[i]));
-                    }
+                for (int i = 0; i < kSeqCols; ++i)
+                    *reinterpret_cast<float*>(b2p + u_base + (i >> 3) * 1024 + u_xo[i & 7]) =
+                        __uint_as_float(to_tf32(ut[i] - __uint_as_float(x[i])));
+                publish(kUPub);
+            } else if (c > 0) {
+                ok = drain_o(c - 1, ok);
+                if (!ok) break;
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar[kR2Done], c & 1, err, kErrTimeoutSeq));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t x[kSeqCols];
+            tmem_ld_cols<kSeqCols>(tmem + 64 + c0 + lane_base, x);
+            tmem_wait_ld();
+            if (has_row) {
+                const float eg = expf(gc);
+#pragma unroll
+                for (int i = 0; i < kSeqCols; ++i) {
+                    S[i] = fmaf(eg, S[i], __uint_as_float(x[i]));
+                    *reinterpret_cast<float*>(b1p + s_base + (i >> 3) * 1024 + s_xo[i & 7]) =
+                        __uint_as_float(to_tf32(S[i]));
                 }
             }
-            if (c + 1 < NC) publish(kBarS, kBarSThreads);
+            publish(kSReady);
         }
         if (ok && !u_role) ok = drain_o(NC - 1, ok);
         if (ok && state_out && has_row) {
