@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include <string>
 
 #include "../../include/nvfp4_gdn.h"
@@ -53,6 +55,17 @@ constexpr unsigned int kErrTimeoutQuant = 32u;
 // Bounded waits give up after this many SM clocks (about half a second);
 // they then record a failure in the device error word and the kernel returns.
 constexpr long long kWaitBudgetCycles = 1ll << 30;
+
+// Programmatic dependent launch.  Kernels launched by launch_pdl may start while
+// the previous kernel of the stream is still finishing.  pdl_wait_and_trigger()
+// blocks until that kernel has completed and its memory is visible (a no-op when
+// the kernel was launched without the attribute), then lets the next kernel of
+// the stream begin its own launch.  Every kernel calls it before its first access
+// to global memory that another kernel may write or read.
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -398,6 +411,23 @@ __device__ __forceinline__ uint32_t elect_one() {
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(pred));
     return pred;
+}
+
+// Launch with programmatic stream serialization (see pdl_wait_and_trigger).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace nvg

@@ -18,6 +18,7 @@ namespace {
 template <int D>
 __global__ void __launch_bounds__(256) l2norm_kernel(const float* __restrict__ proj, int64_t ld, int64_t n_tokens,
                                                      int Hk, float* __restrict__ q_hat, float* __restrict__ k_hat) {
+    pdl_wait_and_trigger();
     constexpr int PER_LANE = D / 32;  // 2 or 4 contiguous floats per lane
     const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -54,6 +55,7 @@ __global__ void __launch_bounds__(256) gate_kernel(const float* __restrict__ pro
                                                    int64_t col_a, int64_t col_b, const float* __restrict__ A_log,
                                                    const float* __restrict__ dt_bias, float* __restrict__ g,
                                                    float* __restrict__ beta) {
+    pdl_wait_and_trigger();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= n_tokens * Hv) return;
     const int64_t t = i / Hv;
@@ -83,10 +85,12 @@ nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_di
                           const float* dt_bias, float* q_hat, float* k_hat, float* g, float* beta, cudaStream_t st) {
     const int64_t warps = n * d.Hk * 2;
     const unsigned blocks_n = static_cast<unsigned>((warps * 32 + 255) / 256);
+    cudaError_t e;
     if (d.K == 128)
-        l2norm_kernel<128><<<blocks_n, 256, 0, st>>>(proj, ld, n, d.Hk, q_hat, k_hat);
+        e = launch_pdl(l2norm_kernel<128>, dim3(blocks_n), dim3(256), 0, st, proj, ld, n, d.Hk, q_hat, k_hat);
     else
-        l2norm_kernel<64><<<blocks_n, 256, 0, st>>>(proj, ld, n, d.Hk, q_hat, k_hat);
+        e = launch_pdl(l2norm_kernel<64>, dim3(blocks_n), dim3(256), 0, st, proj, ld, n, d.Hk, q_hat, k_hat);
+    if (e != cudaSuccess) return cuda_fail(e, "l2norm launch");
     return gate_only_launch(proj, ld, n, d, A_log, dt_bias, g, beta, st);
 }
 
@@ -95,8 +99,8 @@ nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gd
                               const float* dt_bias, float* g, float* beta, cudaStream_t st) {
     const int64_t col_a = 2ll * d.Hk * d.K + 2ll * d.Hv * d.V;
     const unsigned blocks_g = static_cast<unsigned>((n * d.Hv + 255) / 256);
-    gate_kernel<<<blocks_g, 256, 0, st>>>(proj, ld, n, d.Hv, col_a, col_a + d.Hv, A_log, dt_bias, g, beta);
-    cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(gate_kernel, dim3(blocks_g), dim3(256), 0, st, proj, ld, n, d.Hv, col_a,
+                                     col_a + d.Hv, A_log, dt_bias, g, beta);
     if (e != cudaSuccess) return cuda_fail(e, "gates launch");
     return NVFP4_OK;
 }

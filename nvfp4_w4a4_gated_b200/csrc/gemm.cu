@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    pdl_wait_and_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -675,9 +676,8 @@ nvfp4_status launch_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C,
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_kernel<BN><<<grid, 320, G::SMEM, st>>>(ta, tb, tc, A.sf, B.sf, A.global_scale, B.global_scale, M, N, K,
-                                                     err);
-    cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(w4a4_gemm_kernel<BN>, dim3(grid), dim3(320), G::SMEM, st, ta, tb, tc, A.sf, B.sf,
+                                     A.global_scale, B.global_scale, M, N, K, err);
     if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm launch");
     return NVFP4_OK;
 }

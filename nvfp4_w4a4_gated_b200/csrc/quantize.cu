@@ -39,21 +39,6 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float s) {
     return static_cast<uint32_t>(r) & 0xFFu;
 }
 
-// Eight fp32 values -> eight E2M1 codes packed in 32 bits, element 0 in the
-// lowest nibble; round to nearest even, saturating at +-6.
-__device__ __forceinline__ uint32_t f32x8_to_e2m1(const float (&y)[8]) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}\n"
-        : "=r"(r)
-        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
-    return r;
-}
-
 __device__ __forceinline__ float global_scale_from_amax(float amax) {
     return (amax < kTwoPowMinus100) ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
@@ -91,6 +76,7 @@ __device__ __forceinline__ void unpack16B(const uint4& u, float* out, const floa
 template <typename T>
 __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                                                    unsigned int* __restrict__ amax_bits) {
+    pdl_wait_and_trigger();
     constexpr int P = Vec<T>::kPer16B;
     constexpr int U = 8;
     const int lane = threadIdx.x & 31;
@@ -301,6 +287,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const T* __restric
                                                               float* __restrict__ global_scale, int scale_mode,
                                                               uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
                                                               unsigned int* __restrict__ err) {
+    pdl_wait_and_trigger();
     const int64_t k_atoms = cols / 64;
     const int64_t natoms = ((rows + 127) / 128) * k_atoms;
     const int t = threadIdx.x % kQuantGroupThreads;
@@ -428,11 +415,11 @@ nvfp4_status quant_dispatch(const T* x, int64_t rows, int64_t cols, int64_t ld, 
     }
     int64_t grid = static_cast<int64_t>(num_sms()) * quant_blocks_per_sm<T, false>();
     if (grid > groups_needed) grid = groups_needed;
-    quant_kernel<T, false><<<(unsigned)grid, kQuantThreads, 0, st>>>(
-        x, rows, cols, ld, ws, out.global_scale,
-        flags == NVFP4_QUANT_GIVEN_SCALE ? static_cast<int>(kScaleGiven) : static_cast<int>(kScaleFromAmaxWord),
-        out.codes, out.sf, err);
-    e = cudaGetLastError();
+    e = launch_pdl(quant_kernel<T, false>, dim3(static_cast<unsigned>(grid)), dim3(kQuantThreads), 0, st, x, rows,
+                   cols, ld, ws, out.global_scale,
+                   flags == NVFP4_QUANT_GIVEN_SCALE ? static_cast<int>(kScaleGiven)
+                                                    : static_cast<int>(kScaleFromAmaxWord),
+                   out.codes, out.sf, err);
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     return NVFP4_OK;
 }

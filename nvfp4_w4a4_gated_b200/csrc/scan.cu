@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(128) scan_recurrent_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, int64_t ld_v,
     const float* __restrict__ g, const float* __restrict__ beta, int B, int64_t T, int Hk, int Hv, int V, float scale,
     int form, const float* state_in, float* state_out, float* __restrict__ o, unsigned int* __restrict__ o_amax) {
+    pdl_wait_and_trigger();
     constexpr int RW = K / 4;
     const int nslice = V / 32;
     const int bh = blockIdx.x / nslice, slice = blockIdx.x - bh * nslice;
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                                                          const float* __restrict__ g, const float* __restrict__ beta,
                                                          int64_t T, int Hk, int Hv, int form, int NC,
                                                          uint8_t* __restrict__ recs) {
+    pdl_wait_and_trigger();
     using SM = PrepSmem<K, V>;
     using RC = ChunkRec<K, V>;
     constexpr int KS = SM::KS;
@@ -579,6 +581,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    pdl_wait_and_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -877,11 +880,12 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     uint8_t* recs = static_cast<uint8_t*>(ws);
     const unsigned prep_blocks = static_cast<unsigned>(static_cast<int64_t>(B) * NC * d.Hv);
-    chunk_prep_kernel<K, V><<<prep_blocks, 256, prep_smem, st>>>(q, k, ld_qk, normalize_qk, v, ld_v, g, beta, T, d.Hk,
-                                                                 d.Hv, form, NC, recs);
+    cudaError_t e = launch_pdl(chunk_prep_kernel<K, V>, dim3(prep_blocks), dim3(256), prep_smem, st, q, k, ld_qk,
+                               normalize_qk, v, ld_v, g, beta, T, d.Hk, d.Hv, form, NC, recs);
+    if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     const unsigned seq_blocks = static_cast<unsigned>(B * d.Hv * (V / 32));
-    chunk_seq_kernel<K, V><<<seq_blocks, kSeqThreads, seq_smem, st>>>(recs, T, d.Hv, scale, NC, s_in, s_out, o, o_amax, err);
-    cudaError_t e = cudaGetLastError();
+    e = launch_pdl(chunk_seq_kernel<K, V>, dim3(seq_blocks), dim3(kSeqThreads), seq_smem, st, recs, T, d.Hv, scale, NC,
+                   s_in, s_out, o, o_amax, err);
     if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
     return NVFP4_OK;
 }
@@ -913,13 +917,11 @@ nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t
         return fail(NVFP4_ERR_INVALID_ARG, "raw q/k rows need the chunked scan");
     if (!chunked) {
         const unsigned blocks = static_cast<unsigned>(B * d.Hv * (d.V / 32));
-        if (d.K == 128)
-            scan_recurrent_kernel<128><<<blocks, 128, 0, st>>>(q, k, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form,
-                                                               s_in, s_out, o, o_amax);
-        else
-            scan_recurrent_kernel<64><<<blocks, 128, 0, st>>>(q, k, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form,
-                                                              s_in, s_out, o, o_amax);
-        cudaError_t e = cudaGetLastError();
+        const cudaError_t e =
+            d.K == 128 ? launch_pdl(scan_recurrent_kernel<128>, dim3(blocks), dim3(128), 0, st, q, k, v, ld_v, g, beta,
+                                    B, T, d.Hk, d.Hv, d.V, scale, form, s_in, s_out, o, o_amax)
+                       : launch_pdl(scan_recurrent_kernel<64>, dim3(blocks), dim3(128), 0, st, q, k, v, ld_v, g, beta, B,
+                                    T, d.Hk, d.Hv, d.V, scale, form, s_in, s_out, o, o_amax);
         if (e != cudaSuccess) return cuda_fail(e, "recurrent scan launch");
         return NVFP4_OK;
     }
