@@ -15,6 +15,7 @@ namespace nvg {
 
 nvfp4_status validate_tensor(const nvfp4_tensor* t, const char* name);
 nvfp4_status validate_dims(const gdn_dims* d);
+nvfp4_status zero_words_launch(unsigned int* w, int n, cudaStream_t st);
 nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, int64_t ld,
                              const nvfp4_tensor& out, int32_t flags, void* workspace, cudaStream_t st);
 nvfp4_status gemm_launch(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C, int64_t ldc, cudaStream_t st);
@@ -118,8 +119,7 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
 
     // quantiser words: [0] x amax, [1] x arrival counter, [2] o amax; one memset
     unsigned int* qw = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
-    cudaError_t e = cudaMemsetAsync(qw, 0, 4 * sizeof(unsigned int), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(quantiser words)");
+    if ((s = zero_words_launch(qw, 4, st)) != NVFP4_OK) return s;
     if ((s = quantize_launch(x_bf16, NVFP4_DTYPE_BF16, BT, H, H, xq, kQuantComputeZeroedWs, qw, st)) != NVFP4_OK)
         return s;
     if ((s = gemm_launch(xq, w->w_in, proj, ldp, st)) != NVFP4_OK) return s;

@@ -118,6 +118,13 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     }
 }
 
+// Zeroes n 32-bit words (the quantiser's amax and arrival words).  A kernel rather
+// than a memset, so that it chains with its neighbours by programmatic launch.
+__global__ void __launch_bounds__(32) zero_words_kernel(unsigned int* __restrict__ w, int n) {
+    pdl_wait_and_trigger();
+    if (static_cast<int>(threadIdx.x) < n) w[threadIdx.x] = 0u;
+}
+
 // Pass 2 (and, fused, pass 1): the matrix is cut into scale atoms (128 rows x
 // 64 columns, 512 blocks of 16).  A group of 128 threads handles one atom at a
 // time: thread t owns atom bytes t, t+128, t+256, t+384, i.e. the blocks (r, j)
@@ -385,8 +392,8 @@ nvfp4_status quant_dispatch(const T* x, int64_t rows, int64_t cols, int64_t ld, 
     cudaError_t e;
     if (flags == NVFP4_QUANT_COMPUTE_SCALE || flags == kQuantComputeZeroedWs) {
         if (flags == NVFP4_QUANT_COMPUTE_SCALE) {
-            e = cudaMemsetAsync(ws, 0, 2 * sizeof(unsigned int), st);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(amax)");
+            e = launch_pdl(zero_words_kernel, dim3(1), dim3(32), 0, st, ws, 2);
+            if (e != cudaSuccess) return cuda_fail(e, "zero amax words");
         }
         // one launch: every CTA resident at once (cooperative launch), at most one
         // atom group per thread group
@@ -396,11 +403,13 @@ nvfp4_status quant_dispatch(const T* x, int64_t rows, int64_t cols, int64_t ld, 
         cfg.gridDim = dim3(static_cast<unsigned>(grid));
         cfg.blockDim = dim3(kQuantThreads);
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         e = cudaLaunchKernelEx(&cfg, quant_kernel<T, true>, x, rows, cols, ld, ws, out.global_scale,
                                static_cast<int>(kScaleFromAmaxWord), out.codes, out.sf, err);
         if (e == cudaSuccess) return NVFP4_OK;
@@ -411,7 +420,8 @@ nvfp4_status quant_dispatch(const T* x, int64_t rows, int64_t cols, int64_t ld, 
         int64_t blocks = (rows + 7) / 8;
         const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
         if (blocks > cap) blocks = cap;
-        amax_kernel<T><<<(unsigned)blocks, 256, 0, st>>>(x, rows, cols, ld, ws);
+        e = launch_pdl(amax_kernel<T>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, x, rows, cols, ld, ws);
+        if (e != cudaSuccess) return cuda_fail(e, "amax launch");
     }
     int64_t grid = static_cast<int64_t>(num_sms()) * quant_blocks_per_sm<T, false>();
     if (grid > groups_needed) grid = groups_needed;
@@ -425,6 +435,12 @@ nvfp4_status quant_dispatch(const T* x, int64_t rows, int64_t cols, int64_t ld, 
 }
 
 }  // namespace
+
+nvfp4_status zero_words_launch(unsigned int* w, int n, cudaStream_t st) {
+    const cudaError_t e = launch_pdl(zero_words_kernel, dim3(1), dim3(32), 0, st, w, n);
+    if (e != cudaSuccess) return cuda_fail(e, "zero words");
+    return NVFP4_OK;
+}
 
 // flags: NVFP4_QUANT_COMPUTE_SCALE (amax and quantisation, one cooperative
 // launch; kQuantComputeZeroedWs when the caller has zeroed workspace[0..1]),
