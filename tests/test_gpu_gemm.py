@@ -8,7 +8,7 @@ import torch
 import gdn_synth
 import nvfp4_w4a4_gated_b200 as nv
 import oracle
-from gpu_util import rel_fro, upload_oracle_nvfp4
+from gpu_util import bf16_device, f32_device, rel_fro, upload_oracle_nvfp4
 
 pytestmark = pytest.mark.gpu
 
@@ -122,4 +122,29 @@ def test_gemm_decode_shape(cuda_dev):
     Aq, Bq = _operands(44, M, N, K)
     got = _run(Aq, Bq, M, N, K)
     ref = oracle.w4a4_gemm(Aq, Bq)
+    assert rel_fro(got, ref) <= TOL
+
+
+def test_out_proj_in_decode_layer(cuda_dev):
+    """Batch-64 decode step through the layer (out_proj: M = 64, 40 output tiles,
+    K = 4096): y must match the oracle's float64 product of the quantised o and
+    W_out."""
+    sh = gdn_synth.FULL
+    B, T = 64, 1
+    W_in = gdn_synth.weights(300, sh.n_in, sh.H)
+    W_out = gdn_synth.weights(301, sh.H, sh.Hv * sh.V)
+    A_log, dt_bias = gdn_synth.gate_params(302, sh.Hv)
+    dims = nv.GdnDims(sh.Hk, sh.Hv, sh.K, sh.V)
+    w = nv.LayerWeights(nv.nvfp4_quantize(f32_device(W_in)), nv.nvfp4_quantize(f32_device(W_out)),
+                        f32_device(A_log), f32_device(dt_bias), dims, sh.H)
+    bits, _ = gdn_synth.activations(303, B * T, sh.H, hot="none")
+    S0 = f32_device(gdn_synth.gaussian(304, (B, sh.Hv, sh.K, sh.V), std=0.5))
+    y, ws, lay = nv.gdn_layer_forward(w, bf16_device(bits), B, T, state_in=S0)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    HvV = sh.Hv * sh.V
+    o = ws[lay["o"]:lay["o"] + B * T * HvV * 4].view(torch.float32).view(B * T, HvV).cpu().numpy()
+    ref = oracle.w4a4_gemm(oracle.quantize(o), oracle.quantize(W_out))
+    got = y.cpu().numpy()
+    assert np.all(np.isfinite(got))
     assert rel_fro(got, ref) <= TOL
