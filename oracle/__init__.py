@@ -14,7 +14,7 @@ composes the steps in the order the pages give them:
    harmonised weight scale (review page, paper sec.6; abstract page);
 3. gates, Eq.(1) (review page, paper sec.2) and q/k L2 normalisation;
 4. the delta-rule recurrence, Eq.(2) (review page, paper sec.1), then the
-   NVFP4 out_proj.
+   NVFP4 out_proj; optionally through the output gate of reading O1.
 
 Every function states the reading it follows where the pages are silent.
 """
@@ -61,6 +61,8 @@ def _L():
         lib.orc_sf_linear_to_mma.argtypes = [P, i64, i64, P]; lib.orc_sf_linear_to_mma.restype = None
         lib.orc_gemm_nt.argtypes = [P, P, i64, i64, i64, P]; lib.orc_gemm_nt.restype = None
         lib.orc_softplus.argtypes = [f64]; lib.orc_softplus.restype = f64
+        lib.orc_output_gate.argtypes = [P, P, P, i64, i32, i32, f64, P]
+        lib.orc_output_gate.restype = None
         lib.orc_gates.argtypes = [P, P, P, P, i64, i32, P, P]; lib.orc_gates.restype = None
         lib.orc_l2norm.argtypes = [P, i64, i32, f64]; lib.orc_l2norm.restype = None
         lib.orc_scan.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, f64, i32, P, P, P]
@@ -195,6 +197,19 @@ def l2norm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     return y
 
 
+def output_gate(o: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """Optional output gate (reading O1 in oracle.c): per token and value head,
+    o / sqrt(mean(o^2) + eps) * w * SiLU(z).  o, z: [..., Hv, V] (any leading
+    shape); w: [V].  Returns float64 of o's shape."""
+    o64 = _c(o, np.float64)
+    z64 = _c(z, np.float64).reshape(o64.shape)
+    V = o64.shape[-1]
+    Hv = o64.shape[-2]
+    out = np.empty_like(o64)
+    _L().orc_output_gate(_p(o64), _p(z64), _p(_c(w, np.float64)), o64.size // (Hv * V), Hv, V, float(eps), _p(out))
+    return out
+
+
 # --------------------------------------------------------------------- scan --
 def scan(q, k, v, g, beta, scale=None, form=FORM_PAGES, S0=None):
     """Eq.(2) token by token.  q, k: [B,T,Hk,K]; v: [B,T,Hv,V]; g, beta: [B,T,Hv];
@@ -242,27 +257,33 @@ def split_projection(P: np.ndarray, Hk: int, Hv: int, K: int, V: int):
 
 def layer_forward(x: np.ndarray, W_in_q, W_out_q, A_log, dt_bias, B: int, T: int, Hk: int, Hv: int,
                   K: int, V: int, form=FORM_PAGES, S0=None, stages: bool = False, W_in_deq=None,
-                  W_out_deq=None):
+                  W_out_deq=None, out_norm=None):
     """The four steps composed.  x: float32 [B*T, H] (bf16 values);
     W_in_q, W_out_q: (codes, sf_linear, S) of the fused in_proj [N_in, H] and
     out_proj [H, Hv*V] (or their dequantised float64 matrices in W_in_deq /
-    W_out_deq, to skip re-dequantising fixed weights).  Returns y [B*T, H]
-    float64 and the final state (and every intermediate when ``stages``)."""
+    W_out_deq, to skip re-dequantising fixed weights).  With ``out_norm`` (the
+    weight w of V entries) the output gate of reading O1 is applied to o before
+    out_proj.  Returns y [B*T, H] float64 and the final state (and every
+    intermediate when ``stages``)."""
     xq = quantize(x)                                            # step 1
     if W_in_deq is None:
         W_in_deq = dequantize(*W_in_q)
     if W_out_deq is None:
         W_out_deq = dequantize(*W_out_q)
     P = gemm_nt(dequantize(*xq), W_in_deq)                      # step 2
-    q, k, v, _z, a, b = split_projection(P, Hk, Hv, K, V)
+    q, k, v, z, a, b = split_projection(P, Hk, Hv, K, V)
     g, beta = gates(a, b, A_log, dt_bias)                       # step 3
     qh = l2norm(q.reshape(B, T, Hk, K))
     kh = l2norm(k.reshape(B, T, Hk, K))
     o, S = scan(qh, kh, v.reshape(B, T, Hv, V), g.reshape(B, T, Hv), beta.reshape(B, T, Hv),
                 form=form, S0=S0)                               # step 4
     o2 = o.reshape(B * T, Hv * V).astype(np.float32)            # the out_proj reads fp32 o
+    G = None
+    if out_norm is not None:                                    # optional output gate
+        G = output_gate(o2.reshape(B * T, Hv, V), z.reshape(B * T, Hv, V), out_norm)
+        o2 = G.reshape(B * T, Hv * V).astype(np.float32)
     oq = quantize(o2)
     y = gemm_nt(dequantize(*oq), W_out_deq)
     if stages:
-        return dict(xq=xq, P=P, g=g, beta=beta, q_hat=qh, k_hat=kh, o=o, S=S, oq=oq, y=y)
+        return dict(xq=xq, P=P, g=g, beta=beta, q_hat=qh, k_hat=kh, o=o, S=S, G=G, oq=oq, y=y)
     return y, S

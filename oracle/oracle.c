@@ -35,6 +35,11 @@
  *   S1 form PAGES:    S_t = a S + b k (v - S^T k)^T         (the pages' Eq.(2))
  *      form STANDARD: S_t = a S + b k (v - a S^T k)^T       (decay inside)
  *   S2 value head h reads key head floor(h * Hk / Hv); zero initial state.
+ *   O1 output gate (optional; [R] names the z projection as one that moves the
+ *      output y, Table 3 discussion, and keeps the norms unquantised, "Minima"
+ *      section, but gives no formula): per token and value head,
+ *      G = o / sqrt(mean(o^2) + 1e-6) * w * z * sigmoid(z), w a learned weight
+ *      of V entries shared by the heads; out_proj then reads G instead of o.
  */
 #include <math.h>
 #include <stdint.h>
@@ -222,6 +227,23 @@ ORC_EXPORT void orc_l2norm(double* x, int64_t nrows, int32_t D, double eps) {
         for (int32_t i = 0; i < D; ++i) s += x[r * D + i] * x[r * D + i];
         double inv = 1.0 / sqrt(s + eps);
         for (int32_t i = 0; i < D; ++i) x[r * D + i] *= inv;
+    }
+}
+
+/* Output gate (reading O1).  o, z, out: [n x Hv x V]; w: [V]. */
+ORC_EXPORT void orc_output_gate(const double* o, const double* z, const double* w, int64_t n, int32_t Hv,
+                                int32_t V, double eps, double* out) {
+    for (int64_t r = 0; r < n * Hv; ++r) {
+        const double* orow = o + r * V;
+        const double* zrow = z + r * V;
+        double ms = 0.0;
+        for (int32_t i = 0; i < V; ++i) ms += orow[i] * orow[i];
+        ms /= V;
+        double inv_rms = 1.0 / sqrt(ms + eps);
+        for (int32_t i = 0; i < V; ++i) {
+            double silu = zrow[i] / (1.0 + exp(-zrow[i]));
+            out[r * V + i] = orow[i] * inv_rms * w[i] * silu;
+        }
     }
 }
 

@@ -414,3 +414,63 @@ def test_layer_oracle_composes_on_tiny_shapes():
     y = o.reshape(64, -1) @ W_out.astype(np.float64).T
     rel = np.linalg.norm(st["y"] - y) / np.linalg.norm(y)
     assert rel < 0.5
+
+
+# ------------------------------------------------------------- output gate --
+# Reading O1 (the pages name the z projection as one that moves y and keep the
+# norms unquantised, but give no formula): G = RMSNorm(o) * w * SiLU(z) per token
+# and value head.  Pinned by closed forms and invariants, not by its formula.
+def test_output_gate_silu_closed_forms():
+    """o = ones (RMS 1, eps 0), w = 1: G = SiLU(z); sigmoid(+-ln 3) = 3/4, 1/4."""
+    ln3 = np.log(3.0)
+    z = np.array([[[ln3, -ln3, 0.0, 60.0]]])
+    G = oracle.output_gate(np.ones((1, 1, 4)), z, np.ones(4), eps=0.0)
+    np.testing.assert_allclose(G[0, 0], [0.75 * ln3, -0.25 * ln3, 0.0, 60.0], rtol=1e-15, atol=1e-15)
+
+
+def test_output_gate_normalises_by_the_mean_square():
+    """One-hot o over V = 4 channels: mean square 1/4, so the normalised row is 2 e_1;
+    with z = 60 (SiLU(z) = z to double precision) and w = 1/z the gate output is
+    that row, and any row's output has mean square 1."""
+    z = np.full((1, 1, 4), 60.0)
+    w = np.full(4, 1.0 / 60.0)
+    G = oracle.output_gate(np.array([[[0.0, 1.0, 0.0, 0.0]]]), z, w, eps=0.0)
+    np.testing.assert_allclose(G[0, 0], [0.0, 2.0, 0.0, 0.0], rtol=1e-14, atol=1e-15)
+    o = gdn_synth.gaussian(7, (3, 2, 4), std=5.0)
+    G = oracle.output_gate(o, np.full(o.shape, 60.0), w, eps=0.0)
+    np.testing.assert_allclose((G ** 2).mean(axis=-1), 1.0, rtol=1e-13)
+
+
+def test_output_gate_scale_invariance_and_zero_gate():
+    """RMSNorm ignores a positive scale of o (eps 0); z = 0 closes the gate; the
+    per-channel weight multiplies channel i of every head."""
+    o = gdn_synth.gaussian(8, (5, 3, 8), std=1.0).astype(np.float64)
+    z = gdn_synth.gaussian(9, (5, 3, 8), std=2.0).astype(np.float64)
+    w = gdn_synth.gaussian(10, (8,), std=1.0).astype(np.float64)
+    G = oracle.output_gate(o, z, w, eps=0.0)
+    np.testing.assert_allclose(oracle.output_gate(3.7 * o, z, w, eps=0.0), G, rtol=1e-13, atol=1e-14)
+    assert np.all(oracle.output_gate(o, np.zeros_like(z), w) == 0.0)
+    G1 = oracle.output_gate(o, z, np.ones(8), eps=0.0)
+    np.testing.assert_allclose(G, G1 * w, rtol=1e-13, atol=1e-14)
+    # a zero row stays zero (eps keeps it finite)
+    o[2, 1] = 0.0
+    assert np.all(oracle.output_gate(o, z, w)[2, 1] == 0.0)
+
+
+def test_layer_oracle_gate_option_routes_z():
+    """With the gate, the layer's out_proj input is G computed from the scan output
+    and the projection's z slice; a gate weight of zero gives y = 0."""
+    sh = gdn_synth.TINY
+    _, x = gdn_synth.activations(1, 64, sh.H, hot="fixed")
+    W_in = oracle.quantize(gdn_synth.weights(110, sh.n_in, sh.H))
+    W_out = oracle.quantize(gdn_synth.weights(111, sh.H, sh.Hv * sh.V))
+    A_log, dt_bias = gdn_synth.gate_params(112, sh.Hv)
+    w = gdn_synth.gaussian(113, (sh.V,), std=1.0)
+    st = oracle.layer_forward(x, W_in, W_out, A_log, dt_bias, 1, 64, sh.Hk, sh.Hv, sh.K, sh.V, stages=True,
+                              out_norm=w)
+    z = oracle.split_projection(st["P"], sh.Hk, sh.Hv, sh.K, sh.V)[3]
+    o32 = st["o"].reshape(64, sh.Hv, sh.V).astype(np.float32)
+    np.testing.assert_allclose(st["G"], oracle.output_gate(o32, z.reshape(64, sh.Hv, sh.V), w), rtol=0, atol=0)
+    y0 = oracle.layer_forward(x, W_in, W_out, A_log, dt_bias, 1, 64, sh.Hk, sh.Hv, sh.K, sh.V,
+                              out_norm=np.zeros(sh.V))[0]
+    assert np.all(y0 == 0.0)
