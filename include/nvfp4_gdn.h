@@ -207,6 +207,24 @@ NVFP4_API nvfp4_status gdn_scan_noalloc(const float* q_hat, const float* k_hat, 
                                         const gdn_dims* dims, float scale, int32_t form, const float* state_in,
                                         float* state_out, float* o, nvfp4_stream_t stream);
 
+/* ---------------------------------------------------------- output gate -- */
+/* Optional output gate before out_proj.  The pages name z as one of the
+ * projections that move the layer output y (review page, Table 3 discussion)
+ * and keep the layer's norms unquantised ("Minima" section) but give no
+ * formula; this library reads it as the usual gated RMSNorm, per token t and
+ * value head h:
+ *   out[t,h,:] = o[t,h,:] / sqrt(mean_i o[t,h,i]^2 + 1e-6) * w[:] * SiLU(z[t,h,:]),
+ *   SiLU(z) = z / (1 + exp(-z)).
+ * o, out: device float32 [n_tokens x Hv x V] (out may equal o); z: device, token
+ * t's row at z + t * ld_z, head h at + h*V (the z slice of the fused projection);
+ * w: device float32 [V], shared by the heads.  V must be 64 or 128; ld_z a
+ * multiple of 4 and z 16-byte aligned.  amax_word (device, nullable): the
+ * maximum |out| is folded into it with atomicMax on the float bits (it must hold
+ * a non-negative float, e.g. 0, beforehand). */
+NVFP4_API nvfp4_status gdn_output_gate(const float* o, const float* z, int64_t ld_z, const float* w,
+                                       int64_t n_tokens, int32_t Hv, int32_t V, float* out,
+                                       unsigned int* amax_word, nvfp4_stream_t stream);
+
 /* ---------------------------------------------------------------- layer -- */
 typedef struct {
     nvfp4_tensor w_in;    /* [N_in x hidden], N_in = 2*Hk*K + 2*Hv*V + 2*Hv, one global scale */
@@ -215,6 +233,8 @@ typedef struct {
     const float* dt_bias; /* device [Hv] */
     gdn_dims dims;
     int32_t hidden;
+    const float* out_norm; /* device [V]: weight of the output gate (see
+                              gdn_output_gate); NULL: o goes to out_proj as is */
 } gdn_layer_weights;
 
 /* Byte offsets of the intermediates gdn_layer_forward leaves in its
@@ -224,6 +244,8 @@ typedef struct {
     size_t proj;                   /* float32 [B*T x N_in] fused projection */
     size_t q_hat, k_hat, g, beta;  /* gate / normalisation outputs */
     size_t o;                      /* float32 [B*T x Hv*V] scan output */
+    size_t o_gated;                /* float32 [B*T x Hv*V] gated output (an empty
+                                      region when out_norm is NULL) */
     size_t o_codes, o_sf, o_scale; /* quantised scan output */
     size_t quant_ws;               /* quantiser scratch */
     size_t scan_ws;                /* scan scratch */
@@ -234,7 +256,8 @@ NVFP4_API nvfp4_status gdn_layer_workspace_layout(const gdn_layer_weights* w, in
                                         gdn_layer_ws_layout* out /* host */);
 
 /* One GDN layer forward under NVFP4 W4A4 (the four steps above, then the
- * NVFP4 out_proj):
+ * NVFP4 out_proj; with w->out_norm set, out_proj reads the output gate's G
+ * instead of o):
  *   x_bf16: device bf16 [B*T x hidden]; y: device float32 [B*T x hidden].
  *   state_in (NULL = zeros) / state_out (NULL = not written): device float32
  *   [B x Hv x K x V].  form: GDN_FORM_PAGES or GDN_FORM_STANDARD.

@@ -19,7 +19,8 @@ from . import build as _build
 
 __all__ = [
     "NVFP4Error", "NVFP4Matrix", "GdnDims", "LayerWeights", "lib", "nvfp4_quantize", "w4a4_gemm", "gdn_gates",
-    "gdn_scan", "gdn_scan_noalloc", "gdn_layer_forward", "layer_workspace_layout", "check_device_error",
+    "gdn_scan", "gdn_scan_noalloc", "gdn_output_gate", "gdn_layer_forward", "layer_workspace_layout",
+    "check_device_error",
     "selftest_wait_timeout", "FORM_PAGES",
     "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
 ]
@@ -34,7 +35,7 @@ STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4:
 EXPORTED_SYMBOLS = [
     "nvfp4_last_error", "nvfp4_check_device_error", "nvfp4_version", "nvfp4_selftest_wait_timeout", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_size", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan_workspace_size",
-    "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc",
+    "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc", "gdn_output_gate",
 ]
 
 # Size of the fixed scratch array gdn_scan_noalloc uses (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
@@ -58,11 +59,11 @@ class _Dims(ctypes.Structure):
 
 class _LayerWeights(ctypes.Structure):
     _fields_ = [("w_in", _Tensor), ("w_out", _Tensor), ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
-                ("dims", _Dims), ("hidden", ctypes.c_int32)]
+                ("dims", _Dims), ("hidden", ctypes.c_int32), ("out_norm", ctypes.c_void_p)]
 
 
-_LAYOUT_FIELDS = ["x_codes", "x_sf", "x_scale", "proj", "q_hat", "k_hat", "g", "beta", "o", "o_codes", "o_sf",
-                  "o_scale", "quant_ws", "scan_ws", "total"]
+_LAYOUT_FIELDS = ["x_codes", "x_sf", "x_scale", "proj", "q_hat", "k_hat", "g", "beta", "o", "o_gated", "o_codes",
+                  "o_sf", "o_scale", "quant_ws", "scan_ws", "total"]
 
 
 class _Layout(ctypes.Structure):
@@ -93,6 +94,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize.argtypes = [P, i32, i64, i64, i64, TP, i32, P, sz, P]
         L.w4a4_gemm.argtypes = [TP, TP, P, i64, P]
         L.gdn_gates.argtypes = [P, i64, i64, DP, P, P, P, P, P, P, P]
+        L.gdn_output_gate.argtypes = [P, P, i64, P, i64, i32, i32, P, P, P]
         L.gdn_scan_workspace_size.argtypes = [i32, i64, DP, i32]
         L.gdn_scan_workspace_size.restype = sz
         L.gdn_scan.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, i32, P, P, P, P, sz, P]
@@ -167,10 +169,11 @@ class LayerWeights:
     dt_bias: torch.Tensor
     dims: GdnDims
     hidden: int
+    out_norm: torch.Tensor | None = None   # [V] weight of the optional output gate
 
     def c(self) -> _LayerWeights:
         return _LayerWeights(self.w_in.c(), self.w_out.c(), self.A_log.data_ptr(), self.dt_bias.data_ptr(),
-                             self.dims.c(), self.hidden)
+                             self.dims.c(), self.hidden, _ptr(self.out_norm))
 
 
 def check_device_error(stream=None):
@@ -234,6 +237,18 @@ def gdn_gates(proj: torch.Tensor, dims: GdnDims, A_log: torch.Tensor, dt_bias: t
     _check(lib().gdn_gates(_ptr(proj), proj.stride(0), n, ctypes.byref(d), _ptr(A_log), _ptr(dt_bias), _ptr(q_hat),
                            _ptr(k_hat), _ptr(g), _ptr(beta), _stream(stream)))
     return q_hat, k_hat, g, beta
+
+
+def gdn_output_gate(o: torch.Tensor, z: torch.Tensor, w: torch.Tensor, out=None, amax_word=None, stream=None):
+    """Output gate: out = o / sqrt(mean(o^2) + 1e-6) * w * SiLU(z) per (token, value
+    head).  o: [n, Hv, V] contiguous; z: a [n, >= Hv*V] view (row stride ld_z);
+    w: [V].  Returns out (a new tensor unless given; may be o)."""
+    n, Hv, V = o.shape
+    if out is None:
+        out = torch.empty_like(o)
+    _check(lib().gdn_output_gate(_ptr(o), _ptr(z), z.stride(0), _ptr(w), n, Hv, V, _ptr(out), _ptr(amax_word),
+                                 _stream(stream)))
+    return out
 
 
 def gdn_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,

@@ -9,6 +9,15 @@
 // Element-wise and HBM-bound: one warp per (token, head) row for the
 // normalisation (coalesced 16-byte loads), one thread per (token, value head)
 // for the gates.
+//
+// Also the optional output gate before out_proj (the pages name z as moving the
+// output y, review page Table 3 discussion, and keep the norms unquantised,
+// "Minima" section; the formula is this library's reading, the usual gated
+// RMSNorm): out = o / sqrt(mean(o^2) + 1e-6) * w * SiLU(z) per (token, value
+// head), one warp per row, its |out| maximum folded into an amax word for the
+// quantiser that follows.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace nvg {
@@ -68,6 +77,50 @@ __global__ void __launch_bounds__(256) gate_kernel(const float* __restrict__ pro
     beta[i] = 1.0f / (1.0f + expf(-b));
 }
 
+// One warp per (token, value head) row of V values, V/32 per lane.
+template <int V>
+__global__ void __launch_bounds__(256) output_gate_kernel(const float* o, const float* __restrict__ z, int64_t ld_z,
+                                                          const float* __restrict__ w, int64_t n_tokens, int Hv,
+                                                          float* out, unsigned int* __restrict__ amax_word) {
+    pdl_wait_and_trigger();
+    constexpr int PL = V / 32;
+    using VecT = typename std::conditional<PL == 4, float4, float2>::type;
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= n_tokens * Hv) return;   // whole warps leave together
+    const int64_t t = row / Hv;
+    const int h = static_cast<int>(row - t * Hv);
+    float ov[PL], zv[PL], wv[PL];
+    {
+        const VecT a = *reinterpret_cast<const VecT*>(o + row * V + lane * PL);
+        const VecT b = *reinterpret_cast<const VecT*>(z + t * ld_z + static_cast<int64_t>(h) * V + lane * PL);
+        const VecT c = *reinterpret_cast<const VecT*>(w + lane * PL);
+        memcpy(ov, &a, sizeof(ov));
+        memcpy(zv, &b, sizeof(zv));
+        memcpy(wv, &c, sizeof(wv));
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) ss = fmaf(ov[i], ov[i], ss);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv_rms = 1.0f / sqrtf(ss / static_cast<float>(V) + 1e-6f);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+        const float silu = zv[i] / (1.0f + expf(-zv[i]));
+        ov[i] = ov[i] * inv_rms * wv[i] * silu;
+        m = fmaxf(m, fabsf(ov[i]));
+    }
+    VecT r;
+    memcpy(&r, ov, sizeof(ov));
+    *reinterpret_cast<VecT*>(out + row * V + lane * PL) = r;
+    if (amax_word) {
+        const unsigned int mb = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+        if (lane == 0) atomicMax(amax_word, mb);
+    }
+}
+
 }  // namespace
 
 nvfp4_status validate_dims(const gdn_dims* d) {
@@ -105,6 +158,17 @@ nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gd
     return NVFP4_OK;
 }
 
+nvfp4_status output_gate_launch(const float* o, const float* z, int64_t ld_z, const float* w, int64_t n, int Hv, int V,
+                                float* out, unsigned int* amax_word, cudaStream_t st) {
+    const int64_t rows = n * Hv;
+    const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+    const cudaError_t e =
+        V == 128 ? launch_pdl(output_gate_kernel<128>, dim3(blocks), dim3(256), 0, st, o, z, ld_z, w, n, Hv, out, amax_word)
+                 : launch_pdl(output_gate_kernel<64>, dim3(blocks), dim3(256), 0, st, o, z, ld_z, w, n, Hv, out, amax_word);
+    if (e != cudaSuccess) return cuda_fail(e, "output gate launch");
+    return NVFP4_OK;
+}
+
 }  // namespace nvg
 
 extern "C" nvfp4_status gdn_gates(const float* proj, int64_t ld_proj, int64_t n_tokens, const gdn_dims* dims,
@@ -121,4 +185,17 @@ extern "C" nvfp4_status gdn_gates(const float* proj, int64_t ld_proj, int64_t n_
     if (!aligned16(proj) || ld_proj % 4 || !aligned16(q_hat) || !aligned16(k_hat))
         return fail(NVFP4_ERR_MISALIGNED, "proj / q_hat / k_hat must be 16-byte aligned, ld_proj % 4 == 0");
     return gates_launch(proj, ld_proj, n_tokens, *dims, A_log, dt_bias, q_hat, k_hat, g, beta, as_stream(stream));
+}
+
+extern "C" nvfp4_status gdn_output_gate(const float* o, const float* z, int64_t ld_z, const float* w, int64_t n_tokens,
+                                        int32_t Hv, int32_t V, float* out, unsigned int* amax_word,
+                                        nvfp4_stream_t stream) {
+    using namespace nvg;
+    if (!o || !z || !w || !out) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+    if (n_tokens < 1 || Hv < 1) return fail(NVFP4_ERR_INVALID_ARG, "n_tokens and Hv must be >= 1");
+    if (V != 64 && V != 128) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "V must be 64 or 128");
+    if (ld_z < static_cast<int64_t>(Hv) * V) return fail(NVFP4_ERR_INVALID_ARG, "ld_z smaller than Hv*V");
+    if (!aligned16(o) || !aligned16(z) || !aligned16(w) || !aligned16(out) || ld_z % 4)
+        return fail(NVFP4_ERR_MISALIGNED, "o / z / w / out must be 16-byte aligned, ld_z % 4 == 0");
+    return output_gate_launch(o, z, ld_z, w, n_tokens, Hv, V, out, amax_word, as_stream(stream));
 }

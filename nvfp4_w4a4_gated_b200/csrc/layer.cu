@@ -16,6 +16,8 @@ namespace nvg {
 nvfp4_status validate_tensor(const nvfp4_tensor* t, const char* name);
 nvfp4_status validate_dims(const gdn_dims* d);
 nvfp4_status zero_words_launch(unsigned int* w, int n, cudaStream_t st);
+nvfp4_status output_gate_launch(const float* o, const float* z, int64_t ld_z, const float* w, int64_t n, int Hv, int V,
+                                float* out, unsigned int* amax_word, cudaStream_t st);
 nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, int64_t ld,
                              const nvfp4_tensor& out, int32_t flags, void* workspace, cudaStream_t st);
 nvfp4_status gemm_launch(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C, int64_t ldc, cudaStream_t st);
@@ -50,6 +52,7 @@ static nvfp4_status layout_of(const gdn_layer_weights* w, int32_t B, int64_t T, 
     L->g = take(BT * d.Hv * 4);
     L->beta = take(BT * d.Hv * 4);
     L->o = take(BT * HvV * 4);
+    L->o_gated = take(w->out_norm ? BT * HvV * 4 : 0);
     L->o_codes = take(BT * HvV / 2);
     L->o_sf = take(nvfp4_sf_bytes(BT, HvV));
     L->o_scale = take(4);
@@ -66,6 +69,7 @@ static nvfp4_status validate_layer(const gdn_layer_weights* w, int32_t B, int64_
     if ((s = validate_tensor(&w->w_in, "w_in")) != NVFP4_OK) return s;
     if ((s = validate_tensor(&w->w_out, "w_out")) != NVFP4_OK) return s;
     if (!w->A_log || !w->dt_bias) return fail(NVFP4_ERR_INVALID_ARG, "A_log / dt_bias null");
+    if (w->out_norm && !aligned16(w->out_norm)) return fail(NVFP4_ERR_MISALIGNED, "out_norm must be 16-byte aligned");
     if (w->hidden < 64 || w->hidden % 64) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "hidden must be a multiple of 64");
     if (w->w_in.rows != n_in_of(w->dims) || w->w_in.cols != w->hidden)
         return fail(NVFP4_ERR_INVALID_ARG, "w_in must be [2HkK + 2HvV + 2Hv, hidden]");
@@ -144,7 +148,17 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
                          chunked ? GDN_SCAN_CHUNKED : GDN_SCAN_RECURRENT, state_in, state_out, o, ws + L.scan_ws, st,
                          o_amax, ld_qk, chunked ? 1 : 0)) != NVFP4_OK)
         return s;
-    if ((s = quantize_launch(o, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, o_amax, st)) != NVFP4_OK)
+    const float* oq_in = o;
+    unsigned int* oq_amax = o_amax;
+    if (w->out_norm) {
+        // output gate: G = RMSNorm(o) * w * SiLU(z), its amax into the fourth word
+        float* og = reinterpret_cast<float*>(ws + L.o_gated);
+        const float* z = proj + 2ll * d.Hk * d.K + static_cast<int64_t>(d.Hv) * d.V;
+        if ((s = output_gate_launch(o, z, ldp, w->out_norm, BT, d.Hv, d.V, og, qw + 3, st)) != NVFP4_OK) return s;
+        oq_in = og;
+        oq_amax = qw + 3;
+    }
+    if ((s = quantize_launch(oq_in, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, oq_amax, st)) != NVFP4_OK)
         return s;
     return gemm_launch(oq, w->w_out, y, H, st);
 }

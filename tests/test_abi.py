@@ -138,3 +138,24 @@ def test_selftest_budget_validation():
     for budget in (0, (1 << 30) + 1):
         st, msg = _err(L.nvfp4_selftest_wait_timeout(budget, None))
         assert st == 1 and "budget" in msg
+
+
+def test_output_gate_validation_and_layout():
+    L = nv.lib()
+    st, _ = _err(L.gdn_output_gate(None, FAKE, 4096, FAKE, 10, 32, 128, FAKE, None, None))
+    assert st == 1
+    st, _ = _err(L.gdn_output_gate(FAKE, FAKE, 4096, FAKE, 10, 32, 96, FAKE, None, None))
+    assert st == 2
+    st, _ = _err(L.gdn_output_gate(FAKE, FAKE, 4000, FAKE, 10, 32, 128, FAKE, None, None))
+    assert st == 1
+    st, _ = _err(L.gdn_output_gate(FAKE, FAKE, 4098, FAKE, 10, 32, 128, FAKE, None, None))
+    assert st == 3
+    # the layout reserves a gated-output region only when the gate weight is set
+    dims = nv.GdnDims(16, 32, 128, 128)
+    lay0, lay1 = nv._Layout(), nv._Layout()
+    lw0 = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120, None)
+    lw1 = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120, FAKE)
+    assert L.gdn_layer_workspace_layout(ctypes.byref(lw0), 1, 4096, ctypes.byref(lay0)) == 0
+    assert L.gdn_layer_workspace_layout(ctypes.byref(lw1), 1, 4096, ctypes.byref(lay1)) == 0
+    assert lay0.o_codes == lay0.o_gated and lay1.o_codes - lay1.o_gated >= 4096 * 4096 * 4
+    assert lay1.total - lay0.total == lay1.o_codes - lay1.o_gated
