@@ -297,6 +297,8 @@ def run_ours(args, rank, world, local_rank):
     gemm = bench_gemm(nv, dev, args.steps, flush, stream)
     # ---- batch-64 decode step (HBM-bound)
     decode = bench_decode(nv, dev, w, sh, args.steps, stream)
+    # ---- the prefill step with the optional output gate
+    gated = bench_gated(nv, dev, w, sh, x, B, T, args.steps, flush, stream)
 
     # ---- end to end through the public call with host buffers, pipelined over steps:
     # the upload of step i+1 (pinned x -> device) and the download of step i's y
@@ -384,12 +386,61 @@ def run_ours(args, rank, world, local_rank):
         "stages": stages,
         "gemm_standalone": gemm,
         "decode": decode,
+        "output_gate": gated,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
     }
     return out
+
+
+def bench_gated(nv, dev, w, sh, x, B, T, steps, flush, stream):
+    """The same prefill step with the optional output gate (out_proj reads
+    RMSNorm(o) * w * SiLU(z)), and the gate kernel alone.  Algorithmic bytes of
+    the gate: o and z read, the gated output written, 12 B per element."""
+    import dataclasses
+    import gdn_synth
+    w_norm = torch.from_numpy(gdn_synth.gaussian(9, (sh.V,), std=1.0)).to(dev)
+    wg = dataclasses.replace(w, out_norm=w_norm)
+    lay = nv.layer_workspace_layout(wg, B, T)
+    ws = torch.empty(lay["total"], dtype=torch.uint8, device=dev)
+    y = torch.empty((B * T, sh.H), dtype=torch.float32, device=dev)
+    for _ in range(3):
+        nv.gdn_layer_forward(wg, x, B, T, y=y, workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        nv.gdn_layer_forward(wg, x, B, T, y=y, workspace=ws, stream=stream)
+        e.record(stream)
+        ts.append((s, e))
+    # the gate kernel alone, on the step's own o and z
+    BT, HvV = B * T, sh.Hv * sh.V
+    ldp = (sh.n_in + 3) // 4 * 4
+    o = ws[lay["o"]:lay["o"] + BT * HvV * 4].view(torch.float32).view(BT, sh.Hv, sh.V)
+    P = ws[lay["proj"]:lay["proj"] + BT * ldp * 4].view(torch.float32).view(BT, ldp)
+    z = P[:, 2 * sh.Hk * sh.K + HvV:]
+    G = ws[lay["o_gated"]:lay["o_gated"] + BT * HvV * 4].view(torch.float32).view(BT, sh.Hv, sh.V)
+    gt = []
+    for _ in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        nv.gdn_output_gate(o, z, w_norm, out=G, stream=stream)
+        e.record(stream)
+        gt.append((s, e))
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    ms = statistics.mean(s.elapsed_time(e) for s, e in ts)
+    gms = statistics.mean(s.elapsed_time(e) for s, e in gt)
+    gbs = BT * HvV * 12 / (gms / 1e3) / 1e9
+    return {"workload": WORKLOAD + "_output_gate", "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(B * T / (ms / 1e3), 1),
+            "output_gate_kernel": {"ms": round(gms, 4), "GB/s": round(gbs, 1),
+                                   "frac_of_hbm": round(gbs / peaks()["hbm_gbs"], 4)}}
 
 
 def bench_decode(nv, dev, w, sh, steps, stream):

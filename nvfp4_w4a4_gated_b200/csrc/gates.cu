@@ -14,7 +14,7 @@
 // output y, review page Table 3 discussion, and keep the norms unquantised,
 // "Minima" section; the formula is this library's reading, the usual gated
 // RMSNorm): out = o / sqrt(mean(o^2) + 1e-6) * w * SiLU(z) per (token, value
-// head), one warp per row, its |out| maximum folded into an amax word for the
+// head), warps walking rows, the |out| maximum folded into an amax word for the
 // quantiser that follows.
 #include <type_traits>
 
@@ -77,7 +77,9 @@ __global__ void __launch_bounds__(256) gate_kernel(const float* __restrict__ pro
     beta[i] = 1.0f / (1.0f + expf(-b));
 }
 
-// One warp per (token, value head) row of V values, V/32 per lane.
+// Each warp walks (token, value head) rows of V values, V/32 per lane, in a
+// grid-stride loop; one atomicMax per CTA folds the |out| maximum into the amax
+// word (one per row would serialise on that word).
 template <int V>
 __global__ void __launch_bounds__(256) output_gate_kernel(const float* o, const float* __restrict__ z, int64_t ld_z,
                                                           const float* __restrict__ w, int64_t n_tokens, int Hv,
@@ -85,39 +87,50 @@ __global__ void __launch_bounds__(256) output_gate_kernel(const float* o, const 
     pdl_wait_and_trigger();
     constexpr int PL = V / 32;
     using VecT = typename std::conditional<PL == 4, float4, float2>::type;
-    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (row >= n_tokens * Hv) return;   // whole warps leave together
-    const int64_t t = row / Hv;
-    const int h = static_cast<int>(row - t * Hv);
-    float ov[PL], zv[PL], wv[PL];
+    const int64_t rows = n_tokens * Hv;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    float wv[PL];
     {
-        const VecT a = *reinterpret_cast<const VecT*>(o + row * V + lane * PL);
-        const VecT b = *reinterpret_cast<const VecT*>(z + t * ld_z + static_cast<int64_t>(h) * V + lane * PL);
         const VecT c = *reinterpret_cast<const VecT*>(w + lane * PL);
-        memcpy(ov, &a, sizeof(ov));
-        memcpy(zv, &b, sizeof(zv));
         memcpy(wv, &c, sizeof(wv));
     }
-    float ss = 0.0f;
-#pragma unroll
-    for (int i = 0; i < PL; ++i) ss = fmaf(ov[i], ov[i], ss);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float inv_rms = 1.0f / sqrtf(ss / static_cast<float>(V) + 1e-6f);
     float m = 0.0f;
+    for (int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
+         row += nwarps) {
+        const int64_t t = row / Hv;
+        const int h = static_cast<int>(row - t * Hv);
+        float ov[PL], zv[PL];
+        const VecT a = *reinterpret_cast<const VecT*>(o + row * V + lane * PL);
+        const VecT b = *reinterpret_cast<const VecT*>(z + t * ld_z + static_cast<int64_t>(h) * V + lane * PL);
+        memcpy(ov, &a, sizeof(ov));
+        memcpy(zv, &b, sizeof(zv));
+        float ss = 0.0f;
 #pragma unroll
-    for (int i = 0; i < PL; ++i) {
-        const float silu = zv[i] / (1.0f + expf(-zv[i]));
-        ov[i] = ov[i] * inv_rms * wv[i] * silu;
-        m = fmaxf(m, fabsf(ov[i]));
+        for (int i = 0; i < PL; ++i) ss = fmaf(ov[i], ov[i], ss);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv_rms = 1.0f / sqrtf(ss / static_cast<float>(V) + 1e-6f);
+#pragma unroll
+        for (int i = 0; i < PL; ++i) {
+            const float silu = zv[i] / (1.0f + expf(-zv[i]));
+            ov[i] = ov[i] * inv_rms * wv[i] * silu;
+            m = fmaxf(m, fabsf(ov[i]));
+        }
+        VecT r;
+        memcpy(&r, ov, sizeof(ov));
+        *reinterpret_cast<VecT*>(out + row * V + lane * PL) = r;
     }
-    VecT r;
-    memcpy(&r, ov, sizeof(ov));
-    *reinterpret_cast<VecT*>(out + row * V + lane * PL) = r;
     if (amax_word) {
+        __shared__ unsigned int warp_max[8];
         const unsigned int mb = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
-        if (lane == 0) atomicMax(amax_word, mb);
+        if (lane == 0) warp_max[threadIdx.x >> 5] = mb;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            unsigned int v = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0u;
+            v = __reduce_max_sync(0xffffffffu, v);
+            if (threadIdx.x == 0) atomicMax(amax_word, v);
+        }
     }
 }
 
@@ -161,7 +174,10 @@ nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gd
 nvfp4_status output_gate_launch(const float* o, const float* z, int64_t ld_z, const float* w, int64_t n, int Hv, int V,
                                 float* out, unsigned int* amax_word, cudaStream_t st) {
     const int64_t rows = n * Hv;
-    const unsigned blocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+    int64_t blocks64 = (rows + 7) / 8;                         // one row per warp at most
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;  // resident CTAs of 8 warps
+    if (blocks64 > cap) blocks64 = cap;
+    const unsigned blocks = static_cast<unsigned>(blocks64);
     const cudaError_t e =
         V == 128 ? launch_pdl(output_gate_kernel<128>, dim3(blocks), dim3(256), 0, st, o, z, ld_z, w, n, Hv, out, amax_word)
                  : launch_pdl(output_gate_kernel<64>, dim3(blocks), dim3(256), 0, st, o, z, ld_z, w, n, Hv, out, amax_word);
