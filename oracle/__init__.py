@@ -63,6 +63,8 @@ def _L():
         lib.orc_softplus.argtypes = [f64]; lib.orc_softplus.restype = f64
         lib.orc_output_gate.argtypes = [P, P, P, i64, i32, i32, f64, P]
         lib.orc_output_gate.restype = None
+        lib.orc_short_conv.argtypes = [P, i64, i32, i64, i32, i32, P, P, P, P, i32]
+        lib.orc_short_conv.restype = None
         lib.orc_gates.argtypes = [P, P, P, P, i64, i32, P, P]; lib.orc_gates.restype = None
         lib.orc_l2norm.argtypes = [P, i64, i32, f64]; lib.orc_l2norm.restype = None
         lib.orc_scan.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, f64, i32, P, P, P]
@@ -210,6 +212,22 @@ def output_gate(o: np.ndarray, z: np.ndarray, w: np.ndarray, eps: float = 1e-6) 
     return out
 
 
+def short_conv(x: np.ndarray, w: np.ndarray, B: int, T: int, state_in=None, silu: bool = True,
+               return_state: bool = False):
+    """Optional short causal convolution (reading C1 in oracle.c).  x: [B*T, C]
+    (a column slice is fine); w: [C, W]; state_in: [B, C, W-1] or None.
+    Returns out [B*T, C] float64 (and the new state [B, C, W-1])."""
+    x64 = _c(x, np.float64)
+    C, W = w.shape
+    assert x64.shape == (B * T, C)
+    out = np.empty((B * T, C), np.float64)
+    st_out = np.empty((B, C, W - 1), np.float64) if return_state else None
+    st_in = None if state_in is None else _c(state_in, np.float64)
+    _L().orc_short_conv(_p(x64), C, B, T, C, W, _p(_c(w, np.float64)), None if st_in is None else _p(st_in),
+                        None if st_out is None else _p(st_out), _p(out), 1 if silu else 0)
+    return (out, st_out) if return_state else out
+
+
 # --------------------------------------------------------------------- scan --
 def scan(q, k, v, g, beta, scale=None, form=FORM_PAGES, S0=None):
     """Eq.(2) token by token.  q, k: [B,T,Hk,K]; v: [B,T,Hv,V]; g, beta: [B,T,Hv];
@@ -257,21 +275,31 @@ def split_projection(P: np.ndarray, Hk: int, Hv: int, K: int, V: int):
 
 def layer_forward(x: np.ndarray, W_in_q, W_out_q, A_log, dt_bias, B: int, T: int, Hk: int, Hv: int,
                   K: int, V: int, form=FORM_PAGES, S0=None, stages: bool = False, W_in_deq=None,
-                  W_out_deq=None, out_norm=None):
+                  W_out_deq=None, out_norm=None, conv_w=None, conv_state=None):
     """The four steps composed.  x: float32 [B*T, H] (bf16 values);
     W_in_q, W_out_q: (codes, sf_linear, S) of the fused in_proj [N_in, H] and
     out_proj [H, Hv*V] (or their dequantised float64 matrices in W_in_deq /
     W_out_deq, to skip re-dequantising fixed weights).  With ``out_norm`` (the
     weight w of V entries) the output gate of reading O1 is applied to o before
-    out_proj.  Returns y [B*T, H] float64 and the final state (and every
-    intermediate when ``stages``)."""
+    out_proj.  With ``conv_w`` ([2 Hk K + Hv V, W]) the q|k|v columns of the
+    projection first pass through the short convolution of reading C1, with
+    ``conv_state`` ([B, C, W-1] or None) as the carried inputs.  Returns y
+    [B*T, H] float64 and the final state (and every intermediate, with the new
+    convolution state, when ``stages``)."""
     xq = quantize(x)                                            # step 1
     if W_in_deq is None:
         W_in_deq = dequantize(*W_in_q)
     if W_out_deq is None:
         W_out_deq = dequantize(*W_out_q)
     P = gemm_nt(dequantize(*xq), W_in_deq)                      # step 2
-    q, k, v, z, a, b = split_projection(P, Hk, Hv, K, V)
+    conv_state_out = None
+    Pc = P
+    if conv_w is not None:                                      # optional short convolution
+        C = 2 * Hk * K + Hv * V
+        Pc = P.copy()
+        Pc[:, :C], conv_state_out = short_conv(P[:, :C], conv_w, B, T, state_in=conv_state, return_state=True)
+    q, k, v, _, _, _ = split_projection(Pc, Hk, Hv, K, V)
+    _, _, _, z, a, b = split_projection(P, Hk, Hv, K, V)
     g, beta = gates(a, b, A_log, dt_bias)                       # step 3
     qh = l2norm(q.reshape(B, T, Hk, K))
     kh = l2norm(k.reshape(B, T, Hk, K))
@@ -285,5 +313,6 @@ def layer_forward(x: np.ndarray, W_in_q, W_out_q, A_log, dt_bias, B: int, T: int
     oq = quantize(o2)
     y = gemm_nt(dequantize(*oq), W_out_deq)
     if stages:
-        return dict(xq=xq, P=P, g=g, beta=beta, q_hat=qh, k_hat=kh, o=o, S=S, G=G, oq=oq, y=y)
+        return dict(xq=xq, P=P, Pc=Pc, conv_state=conv_state_out, g=g, beta=beta, q_hat=qh, k_hat=kh, o=o, S=S,
+                    G=G, oq=oq, y=y)
     return y, S

@@ -40,6 +40,12 @@
  *      section, but gives no formula): per token and value head,
  *      G = o / sqrt(mean(o^2) + 1e-6) * w * z * sigmoid(z), w a learned weight
  *      of V entries shared by the heads; out_proj then reads G instead of o.
+ *   C1 short convolution (optional; [R] lists convolutions among the layers kept
+ *      unquantised, "Minima" section, and gives nothing else): per channel c of
+ *      the q|k|v slices, a causal depthwise convolution of width W followed by
+ *      SiLU, out_t[c] = SiLU(sum_j w[c][j] x_{t-W+1+j}[c]); inputs before the
+ *      first token come from a carried state (the previous W-1 inputs, zero when
+ *      absent), and the new state is the last W-1 inputs.
  */
 #include <math.h>
 #include <stdint.h>
@@ -245,6 +251,41 @@ ORC_EXPORT void orc_output_gate(const double* o, const double* z, const double* 
             out[r * V + i] = orow[i] * inv_rms * w[i] * silu;
         }
     }
+}
+
+/* Short causal convolution (reading C1).  x: token (b, t) row at x + (b*T + t)*ldx,
+ * channels 0..C-1; w: [C x W]; state_in, state_out: [B x C x (W-1)] (NULL: zeros /
+ * not written); out: [B*T x C].  silu = 0 returns the pre-activation. */
+ORC_EXPORT void orc_short_conv(const double* x, int64_t ldx, int32_t B, int64_t T, int32_t C, int32_t W,
+                               const double* w, const double* state_in, double* state_out, double* out,
+                               int32_t silu) {
+    for (int32_t b = 0; b < B; ++b)
+        for (int32_t c = 0; c < C; ++c) {
+            /* input at token index u (u may be negative: from the state) */
+            for (int64_t t = 0; t < T; ++t) {
+                double acc = 0.0;
+                for (int32_t j = 0; j < W; ++j) {
+                    int64_t u = t - (W - 1) + j;
+                    double xv;
+                    if (u >= 0)
+                        xv = x[(b * T + u) * ldx + c];
+                    else
+                        xv = state_in ? state_in[((int64_t)b * C + c) * (W - 1) + (u + (W - 1))] : 0.0;
+                    acc += w[(int64_t)c * W + j] * xv;
+                }
+                out[(b * T + t) * C + c] = silu ? acc / (1.0 + exp(-acc)) : acc;
+            }
+            if (state_out)
+                for (int32_t i = 0; i < W - 1; ++i) {
+                    int64_t u = T - (W - 1) + i;
+                    double xv;
+                    if (u >= 0)
+                        xv = x[(b * T + u) * ldx + c];
+                    else
+                        xv = state_in ? state_in[((int64_t)b * C + c) * (W - 1) + (u + (W - 1))] : 0.0;
+                    state_out[((int64_t)b * C + c) * (W - 1) + i] = xv;
+                }
+        }
 }
 
 /* ------------------------------------------------------------------------ */

@@ -474,3 +474,70 @@ def test_layer_oracle_gate_option_routes_z():
     y0 = oracle.layer_forward(x, W_in, W_out, A_log, dt_bias, 1, 64, sh.Hk, sh.Hv, sh.K, sh.V,
                               out_norm=np.zeros(sh.V))[0]
     assert np.all(y0 == 0.0)
+
+
+# -------------------------------------------------------- short convolution --
+# Reading C1 (the pages keep convolutions unquantised and say nothing else): a
+# causal depthwise convolution of width W on the q|k|v channels, then SiLU.
+def test_short_conv_matches_numpy_convolve():
+    """Pre-activation per channel = the first T terms of numpy.convolve with the
+    reversed taps (zero history)."""
+    B, T, C, W = 2, 11, 5, 4
+    x = gdn_synth.gaussian(30, (B * T, C), std=1.0).astype(np.float64)
+    w = gdn_synth.gaussian(31, (C, W), std=1.0).astype(np.float64)
+    out = oracle.short_conv(x, w, B, T, silu=False)
+    for b in range(B):
+        for c in range(C):
+            ref = np.convolve(x[b * T:(b + 1) * T, c], w[c, ::-1])[:T]
+            np.testing.assert_allclose(out[b * T:(b + 1) * T, c], ref, rtol=1e-14, atol=1e-14)
+
+
+def test_short_conv_taps_and_silu_closed_form():
+    """The last tap alone gives SiLU(x_t) (SiLU(ln 3) = 0.75 ln 3); the first tap
+    alone gives SiLU(x_{t-3}), zero for the first three tokens."""
+    ln3 = np.log(3.0)
+    x = np.full((6, 1), ln3)
+    out = oracle.short_conv(x, np.array([[0.0, 0.0, 0.0, 1.0]]), 1, 6)
+    np.testing.assert_allclose(out[:, 0], 0.75 * ln3, rtol=1e-15)
+    x = np.arange(1, 7, dtype=np.float64).reshape(6, 1)
+    out = oracle.short_conv(x, np.array([[1.0, 0.0, 0.0, 0.0]]), 1, 6, silu=False)
+    np.testing.assert_array_equal(out[:, 0], [0.0, 0.0, 0.0, 1.0, 2.0, 3.0])
+
+
+def test_short_conv_is_causal_and_chains():
+    """Changing token 7 leaves tokens 0..6 alone; convolving T1 then T2 tokens with
+    the carried state equals convolving T1 + T2 at once (T2 shorter than the
+    window included), and the state holds the last W-1 inputs."""
+    T, C, W = 16, 6, 4
+    x = gdn_synth.gaussian(32, (T, C), std=1.0).astype(np.float64)
+    w = gdn_synth.gaussian(33, (C, W), std=1.0).astype(np.float64)
+    full, st_full = oracle.short_conv(x, w, 1, T, return_state=True)
+    x2 = x.copy()
+    x2[7] += 5.0
+    out2 = oracle.short_conv(x2, w, 1, T)
+    np.testing.assert_array_equal(out2[:7], full[:7])
+    assert np.all(out2[7] != full[7])
+    for t1 in (1, 2, 9, 15):
+        a, st = oracle.short_conv(x[:t1], w, 1, t1, return_state=True)
+        b, st2 = oracle.short_conv(x[t1:], w, 1, T - t1, state_in=st, return_state=True)
+        np.testing.assert_array_equal(np.concatenate([a, b]), full)
+        np.testing.assert_array_equal(st2, st_full)
+    np.testing.assert_array_equal(st_full[0], x[T - (W - 1):].T)
+
+
+def test_layer_oracle_conv_option():
+    """The convolution feeds q|k|v only: z, a, b and the gates see the raw projection;
+    an identity-tap convolution equals applying SiLU to q|k|v."""
+    sh = gdn_synth.TINY
+    _, x = gdn_synth.activations(2, 32, sh.H, hot="fixed")
+    W_in = oracle.quantize(gdn_synth.weights(120, sh.n_in, sh.H))
+    W_out = oracle.quantize(gdn_synth.weights(121, sh.H, sh.Hv * sh.V))
+    A_log, dt_bias = gdn_synth.gate_params(122, sh.Hv)
+    C = 2 * sh.Hk * sh.K + sh.Hv * sh.V
+    taps = np.zeros((C, 4))
+    taps[:, 3] = 1.0
+    st = oracle.layer_forward(x, W_in, W_out, A_log, dt_bias, 1, 32, sh.Hk, sh.Hv, sh.K, sh.V, stages=True,
+                              conv_w=taps)
+    P = st["P"]
+    np.testing.assert_allclose(st["Pc"][:, :C], P[:, :C] / (1.0 + np.exp(-P[:, :C])), rtol=1e-15)
+    np.testing.assert_array_equal(st["Pc"][:, C:], P[:, C:])
