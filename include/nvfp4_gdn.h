@@ -225,6 +225,22 @@ NVFP4_API nvfp4_status gdn_output_gate(const float* o, const float* z, int64_t l
                                        int64_t n_tokens, int32_t Hv, int32_t V, float* out,
                                        unsigned int* amax_word, nvfp4_stream_t stream);
 
+/* ------------------------------------------------------ short convolution -- */
+/* Optional short causal convolution on the q|k|v channels.  The pages list
+ * convolutions among the layers kept unquantised (review page, "Minima"
+ * section) and give nothing more; this library reads it as the usual Gated
+ * DeltaNet short convolution, per sequence b, token t and channel c:
+ *   out[b,t,c] = SiLU(sum_{j<W} w[c*W + j] * x[b, t-W+1+j, c]),
+ * with inputs before token 0 taken from state_in[b, c, 0..W-2] (NULL: zeros).
+ * x: device float32, token (b, t) row at x + (b*T + t)*ld_x, channels 0..C-1;
+ * out: device float32, row at out + (b*T + t)*ld_out, must not overlap x;
+ * w: device float32 [C x W], 2 <= W <= 4;
+ * state_out (nullable): device float32 [B x C x (W-1)], the last W-1 inputs of
+ * each sequence; it may equal state_in. */
+NVFP4_API nvfp4_status gdn_short_conv(const float* x, int64_t ld_x, int32_t B, int64_t T, int32_t C, int32_t W,
+                                      const float* w, const float* state_in, float* state_out, float* out,
+                                      int64_t ld_out, nvfp4_stream_t stream);
+
 /* ---------------------------------------------------------------- layer -- */
 typedef struct {
     nvfp4_tensor w_in;    /* [N_in x hidden], N_in = 2*Hk*K + 2*Hv*V + 2*Hv, one global scale */
@@ -235,6 +251,9 @@ typedef struct {
     int32_t hidden;
     const float* out_norm; /* device [V]: weight of the output gate (see
                               gdn_output_gate); NULL: o goes to out_proj as is */
+    const float* conv_weight; /* device [(2*Hk*K + Hv*V) x conv_width]: short
+                                 convolution on q|k|v (see gdn_short_conv); NULL: none */
+    int32_t conv_width;       /* 2..4 when conv_weight is set */
 } gdn_layer_weights;
 
 /* Byte offsets of the intermediates gdn_layer_forward leaves in its
@@ -246,6 +265,8 @@ typedef struct {
     size_t o;                      /* float32 [B*T x Hv*V] scan output */
     size_t o_gated;                /* float32 [B*T x Hv*V] gated output (an empty
                                       region when out_norm is NULL) */
+    size_t qkv_conv;               /* float32 [B*T x (2*Hk*K + Hv*V)] convolved q|k|v
+                                      (an empty region when conv_weight is NULL) */
     size_t o_codes, o_sf, o_scale; /* quantised scan output */
     size_t quant_ws;               /* quantiser scratch */
     size_t scan_ws;                /* scan scratch */
@@ -256,7 +277,8 @@ NVFP4_API nvfp4_status gdn_layer_workspace_layout(const gdn_layer_weights* w, in
                                         gdn_layer_ws_layout* out /* host */);
 
 /* One GDN layer forward under NVFP4 W4A4 (the four steps above, then the
- * NVFP4 out_proj; with w->out_norm set, out_proj reads the output gate's G
+ * NVFP4 out_proj; with w->conv_weight set, q|k|v first pass through the short
+ * convolution; with w->out_norm set, out_proj reads the output gate's G
  * instead of o):
  *   x_bf16: device bf16 [B*T x hidden]; y: device float32 [B*T x hidden].
  *   state_in (NULL = zeros) / state_out (NULL = not written): device float32
@@ -265,6 +287,15 @@ NVFP4_API nvfp4_status gdn_layer_workspace_layout(const gdn_layer_weights* w, in
 NVFP4_API nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void* x_bf16, int32_t B, int64_t T,
                                float* y, const float* state_in, float* state_out, int32_t form,
                                void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* gdn_layer_forward with the short convolution's carried inputs (used only when
+ * w->conv_weight is set): conv_state_in (NULL: zeros) and conv_state_out (NULL:
+ * not written), device float32 [B x (2*Hk*K + Hv*V) x (conv_width-1)]; they may
+ * be the same buffer.  gdn_layer_forward is this call with both NULL. */
+NVFP4_API nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, const void* x_bf16, int32_t B,
+                                                  int64_t T, float* y, const float* state_in, float* state_out,
+                                                  const float* conv_state_in, float* conv_state_out, int32_t form,
+                                                  void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
 
 #ifdef __cplusplus
 }

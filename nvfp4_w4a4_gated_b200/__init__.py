@@ -19,7 +19,7 @@ from . import build as _build
 
 __all__ = [
     "NVFP4Error", "NVFP4Matrix", "GdnDims", "LayerWeights", "lib", "nvfp4_quantize", "w4a4_gemm", "gdn_gates",
-    "gdn_scan", "gdn_scan_noalloc", "gdn_output_gate", "gdn_layer_forward", "layer_workspace_layout",
+    "gdn_scan", "gdn_scan_noalloc", "gdn_output_gate", "gdn_short_conv", "gdn_layer_forward", "layer_workspace_layout",
     "check_device_error",
     "selftest_wait_timeout", "FORM_PAGES",
     "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
@@ -36,6 +36,7 @@ EXPORTED_SYMBOLS = [
     "nvfp4_last_error", "nvfp4_check_device_error", "nvfp4_version", "nvfp4_selftest_wait_timeout", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_size", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan_workspace_size",
     "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc", "gdn_output_gate",
+    "gdn_short_conv", "gdn_layer_forward_stateful",
 ]
 
 # Size of the fixed scratch array gdn_scan_noalloc uses (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
@@ -59,11 +60,12 @@ class _Dims(ctypes.Structure):
 
 class _LayerWeights(ctypes.Structure):
     _fields_ = [("w_in", _Tensor), ("w_out", _Tensor), ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
-                ("dims", _Dims), ("hidden", ctypes.c_int32), ("out_norm", ctypes.c_void_p)]
+                ("dims", _Dims), ("hidden", ctypes.c_int32), ("out_norm", ctypes.c_void_p),
+                ("conv_weight", ctypes.c_void_p), ("conv_width", ctypes.c_int32)]
 
 
-_LAYOUT_FIELDS = ["x_codes", "x_sf", "x_scale", "proj", "q_hat", "k_hat", "g", "beta", "o", "o_gated", "o_codes",
-                  "o_sf", "o_scale", "quant_ws", "scan_ws", "total"]
+_LAYOUT_FIELDS = ["x_codes", "x_sf", "x_scale", "proj", "q_hat", "k_hat", "g", "beta", "o", "o_gated", "qkv_conv",
+                  "o_codes", "o_sf", "o_scale", "quant_ws", "scan_ws", "total"]
 
 
 class _Layout(ctypes.Structure):
@@ -101,6 +103,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_scan_noalloc.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, P, P, P, P]
         L.gdn_layer_workspace_layout.argtypes = [ctypes.POINTER(_LayerWeights), i32, i64, ctypes.POINTER(_Layout)]
         L.gdn_layer_forward.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, i32, P, sz, P]
+        L.gdn_layer_forward_stateful.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, P, P, i32, P,
+                                                 sz, P]
+        L.gdn_short_conv.argtypes = [P, i64, i32, i64, i32, i32, P, P, P, P, i64, P]
         for f in ("nvfp4_check_device_error", "nvfp4_selftest_wait_timeout", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
                   "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc"):
             getattr(L, f).restype = ctypes.c_int
@@ -169,11 +174,14 @@ class LayerWeights:
     dt_bias: torch.Tensor
     dims: GdnDims
     hidden: int
-    out_norm: torch.Tensor | None = None   # [V] weight of the optional output gate
+    out_norm: torch.Tensor | None = None      # [V] weight of the optional output gate
+    conv_weight: torch.Tensor | None = None   # [2 Hk K + Hv V, conv_width] optional short convolution
+    conv_width: int = 4
 
     def c(self) -> _LayerWeights:
         return _LayerWeights(self.w_in.c(), self.w_out.c(), self.A_log.data_ptr(), self.dt_bias.data_ptr(),
-                             self.dims.c(), self.hidden, _ptr(self.out_norm))
+                             self.dims.c(), self.hidden, _ptr(self.out_norm), _ptr(self.conv_weight),
+                             self.conv_width)
 
 
 def check_device_error(stream=None):
@@ -251,6 +259,19 @@ def gdn_output_gate(o: torch.Tensor, z: torch.Tensor, w: torch.Tensor, out=None,
     return out
 
 
+def gdn_short_conv(x: torch.Tensor, w: torch.Tensor, B: int, T: int, out=None, state_in=None, state_out=None,
+                   stream=None):
+    """Short causal convolution + SiLU per channel.  x: a [B*T, >= C] view (row
+    stride ld_x); w: [C, W]; state_in / state_out: [B, C, W-1] or None.
+    Returns out [B*T, C] (a new tensor unless given)."""
+    C, W = w.shape
+    if out is None:
+        out = torch.empty((B * T, C), dtype=torch.float32, device=x.device)
+    _check(lib().gdn_short_conv(_ptr(x), x.stride(0), B, T, C, W, _ptr(w), _ptr(state_in), _ptr(state_out), _ptr(out),
+                                out.stride(0), _stream(stream)))
+    return out
+
+
 def gdn_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
              form: int = FORM_PAGES, algo: int = SCAN_AUTO, state_in=None, state_out=None, o=None,
              workspace=None, stream=None):
@@ -296,8 +317,10 @@ def layer_workspace_layout(w: LayerWeights, B: int, T: int) -> dict:
 
 
 def gdn_layer_forward(w: LayerWeights, x: torch.Tensor, B: int, T: int, y=None, state_in=None, state_out=None,
-                      form: int = FORM_PAGES, workspace=None, stream=None):
-    """y = GDN layer(x) under NVFP4 W4A4.  x: bf16 [B*T, hidden] on the device."""
+                      form: int = FORM_PAGES, workspace=None, stream=None, conv_state_in=None, conv_state_out=None):
+    """y = GDN layer(x) under NVFP4 W4A4.  x: bf16 [B*T, hidden] on the device.
+    conv_state_in / conv_state_out: the short convolution's carried inputs
+    [B, 2 Hk K + Hv V, conv_width - 1] (used only when w.conv_weight is set)."""
     assert x.dtype == torch.bfloat16 and x.is_contiguous()
     if y is None:
         y = torch.empty((B * T, w.hidden), dtype=torch.float32, device=x.device)
@@ -305,6 +328,7 @@ def gdn_layer_forward(w: LayerWeights, x: torch.Tensor, B: int, T: int, y=None, 
     if workspace is None:
         workspace = torch.empty(lay["total"], dtype=torch.uint8, device=x.device)
     lw = w.c()
-    _check(lib().gdn_layer_forward(ctypes.byref(lw), _ptr(x), B, T, _ptr(y), _ptr(state_in), _ptr(state_out), form,
-                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+    _check(lib().gdn_layer_forward_stateful(ctypes.byref(lw), _ptr(x), B, T, _ptr(y), _ptr(state_in), _ptr(state_out),
+                                            _ptr(conv_state_in), _ptr(conv_state_out), form, _ptr(workspace),
+                                            workspace.numel(), _stream(stream)))
     return y, workspace, lay

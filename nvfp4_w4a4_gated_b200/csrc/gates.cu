@@ -147,8 +147,9 @@ nvfp4_status validate_dims(const gdn_dims* d) {
 nvfp4_status gate_only_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
                               const float* dt_bias, float* g, float* beta, cudaStream_t st);
 
-nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
-                          const float* dt_bias, float* q_hat, float* k_hat, float* g, float* beta, cudaStream_t st) {
+// q_hat, k_hat from rows whose first 2 Hk K columns are q | k (row stride ld).
+nvfp4_status l2norm_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, float* q_hat, float* k_hat,
+                           cudaStream_t st) {
     const int64_t warps = n * d.Hk * 2;
     const unsigned blocks_n = static_cast<unsigned>((warps * 32 + 255) / 256);
     cudaError_t e;
@@ -157,6 +158,13 @@ nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_di
     else
         e = launch_pdl(l2norm_kernel<64>, dim3(blocks_n), dim3(256), 0, st, proj, ld, n, d.Hk, q_hat, k_hat);
     if (e != cudaSuccess) return cuda_fail(e, "l2norm launch");
+    return NVFP4_OK;
+}
+
+nvfp4_status gates_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, const float* A_log,
+                          const float* dt_bias, float* q_hat, float* k_hat, float* g, float* beta, cudaStream_t st) {
+    nvfp4_status s = l2norm_launch(proj, ld, n, d, q_hat, k_hat, st);
+    if (s != NVFP4_OK) return s;
     return gate_only_launch(proj, ld, n, d, A_log, dt_bias, g, beta, st);
 }
 

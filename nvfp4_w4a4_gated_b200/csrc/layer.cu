@@ -16,6 +16,10 @@ namespace nvg {
 nvfp4_status validate_tensor(const nvfp4_tensor* t, const char* name);
 nvfp4_status validate_dims(const gdn_dims* d);
 nvfp4_status zero_words_launch(unsigned int* w, int n, cudaStream_t st);
+nvfp4_status short_conv_launch(const float* x, int64_t ld_x, int B, int64_t T, int C, int W, const float* w,
+                               const float* state_in, float* state_out, float* out, int64_t ld_out, cudaStream_t st);
+nvfp4_status l2norm_launch(const float* proj, int64_t ld, int64_t n, const gdn_dims& d, float* q_hat, float* k_hat,
+                           cudaStream_t st);
 nvfp4_status output_gate_launch(const float* o, const float* z, int64_t ld_z, const float* w, int64_t n, int Hv, int V,
                                 float* out, unsigned int* amax_word, cudaStream_t st);
 nvfp4_status quantize_launch(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, int64_t ld,
@@ -33,6 +37,7 @@ nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t
 
 static int64_t n_in_of(const gdn_dims& d) { return 2ll * d.Hk * d.K + 2ll * d.Hv * d.V + 2ll * d.Hv; }
 static int64_t ld_proj_of(const gdn_dims& d) { return (n_in_of(d) + 3) / 4 * 4; }
+static int64_t qkv_width(const gdn_dims& d) { return 2ll * d.Hk * d.K + static_cast<int64_t>(d.Hv) * d.V; }
 
 static nvfp4_status layout_of(const gdn_layer_weights* w, int32_t B, int64_t T, gdn_layer_ws_layout* L) {
     const gdn_dims& d = w->dims;
@@ -53,6 +58,7 @@ static nvfp4_status layout_of(const gdn_layer_weights* w, int32_t B, int64_t T, 
     L->beta = take(BT * d.Hv * 4);
     L->o = take(BT * HvV * 4);
     L->o_gated = take(w->out_norm ? BT * HvV * 4 : 0);
+    L->qkv_conv = take(w->conv_weight ? BT * qkv_width(d) * 4 : 0);
     L->o_codes = take(BT * HvV / 2);
     L->o_sf = take(nvfp4_sf_bytes(BT, HvV));
     L->o_scale = take(4);
@@ -70,6 +76,8 @@ static nvfp4_status validate_layer(const gdn_layer_weights* w, int32_t B, int64_
     if ((s = validate_tensor(&w->w_out, "w_out")) != NVFP4_OK) return s;
     if (!w->A_log || !w->dt_bias) return fail(NVFP4_ERR_INVALID_ARG, "A_log / dt_bias null");
     if (w->out_norm && !aligned16(w->out_norm)) return fail(NVFP4_ERR_MISALIGNED, "out_norm must be 16-byte aligned");
+    if (w->conv_weight && (w->conv_width < 2 || w->conv_width > 4))
+        return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "conv_width must be 2, 3 or 4");
     if (w->hidden < 64 || w->hidden % 64) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "hidden must be a multiple of 64");
     if (w->w_in.rows != n_in_of(w->dims) || w->w_in.cols != w->hidden)
         return fail(NVFP4_ERR_INVALID_ARG, "w_in must be [2HkK + 2HvV + 2Hv, hidden]");
@@ -94,6 +102,14 @@ extern "C" nvfp4_status gdn_layer_workspace_layout(const gdn_layer_weights* w, i
 extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void* x_bf16, int32_t B, int64_t T,
                                           float* y, const float* state_in, float* state_out, int32_t form,
                                           void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+    return gdn_layer_forward_stateful(w, x_bf16, B, T, y, state_in, state_out, nullptr, nullptr, form, workspace,
+                                      workspace_bytes, stream);
+}
+
+extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, const void* x_bf16, int32_t B,
+                                                   int64_t T, float* y, const float* state_in, float* state_out,
+                                                   const float* conv_state_in, float* conv_state_out, int32_t form,
+                                                   void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
     using namespace nvg;
     nvfp4_status s = validate_layer(w, B, T);
     if (s != NVFP4_OK) return s;
@@ -127,24 +143,31 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
     if ((s = quantize_launch(x_bf16, NVFP4_DTYPE_BF16, BT, H, H, xq, kQuantComputeZeroedWs, qw, st)) != NVFP4_OK)
         return s;
     if ((s = gemm_launch(xq, w->w_in, proj, ldp, st)) != NVFP4_OK) return s;
-    // T > 1: the chunked scan reads the raw q, k slices of the projection and
-    // normalises them while staging them, so only g and beta are formed here.
+    // q|k|v come from the projection, or from its short convolution when one is set
+    const float* qkv = proj;
+    int64_t ld_qkv = ldp;
+    if (w->conv_weight) {
+        float* cv = reinterpret_cast<float*>(ws + L.qkv_conv);
+        if ((s = short_conv_launch(proj, ldp, B, T, static_cast<int>(qkv_width(d)), w->conv_width, w->conv_weight,
+                                   conv_state_in, conv_state_out, cv, qkv_width(d), st)) != NVFP4_OK)
+            return s;
+        qkv = cv;
+        ld_qkv = qkv_width(d);
+    }
+    // T > 1: the chunked scan reads the raw q, k slices and normalises them while
+    // staging them, so only g and beta are formed here.
     // T = 1 (decode): the recurrent scan reads normalised q_hat, k_hat.
     const bool chunked = T > 1;
-    if (chunked) {
-        if ((s = gate_only_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, g, beta, st)) != NVFP4_OK) return s;
-    } else {
-        if ((s = gates_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, q_hat, k_hat, g, beta, st)) != NVFP4_OK)
-            return s;
-    }
-    const float* q_in = chunked ? proj : q_hat;
-    const float* k_in = chunked ? proj + static_cast<int64_t>(d.Hk) * d.K : k_hat;
-    const int64_t ld_qk = chunked ? ldp : static_cast<int64_t>(d.Hk) * d.K;
+    if (!chunked && (s = l2norm_launch(qkv, ld_qkv, BT, d, q_hat, k_hat, st)) != NVFP4_OK) return s;
+    if ((s = gate_only_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, g, beta, st)) != NVFP4_OK) return s;
+    const float* q_in = chunked ? qkv : q_hat;
+    const float* k_in = chunked ? qkv + static_cast<int64_t>(d.Hk) * d.K : k_hat;
+    const int64_t ld_qk = chunked ? ld_qkv : static_cast<int64_t>(d.Hk) * d.K;
     const float scale = 1.0f / sqrtf(static_cast<float>(d.K));
     // the scan folds max|o| into the quantiser's amax word as it writes o, so the o
     // quantiser runs its quantisation pass only
     unsigned int* o_amax = qw + 2;
-    if ((s = scan_launch(q_in, k_in, proj + 2ll * d.Hk * d.K, ldp, g, beta, B, T, d, scale, form,
+    if ((s = scan_launch(q_in, k_in, qkv + 2ll * d.Hk * d.K, ld_qkv, g, beta, B, T, d, scale, form,
                          chunked ? GDN_SCAN_CHUNKED : GDN_SCAN_RECURRENT, state_in, state_out, o, ws + L.scan_ws, st,
                          o_amax, ld_qk, chunked ? 1 : 0)) != NVFP4_OK)
         return s;

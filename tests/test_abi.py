@@ -159,3 +159,24 @@ def test_output_gate_validation_and_layout():
     assert L.gdn_layer_workspace_layout(ctypes.byref(lw1), 1, 4096, ctypes.byref(lay1)) == 0
     assert lay0.o_codes == lay0.o_gated and lay1.o_codes - lay1.o_gated >= 4096 * 4096 * 4
     assert lay1.total - lay0.total == lay1.o_codes - lay1.o_gated
+
+
+def test_short_conv_validation_and_layout():
+    L = nv.lib()
+    st, _ = _err(L.gdn_short_conv(None, 8192, 1, 64, 8192, 4, FAKE, None, None, FAKE, 8192, None))
+    assert st == 1
+    st, _ = _err(L.gdn_short_conv(FAKE, 8192, 1, 64, 8192, 5, FAKE, None, None, 0x4000000, 8192, None))
+    assert st == 2
+    st, msg = _err(L.gdn_short_conv(FAKE, 8192, 1, 64, 8192, 4, FAKE, None, None, FAKE + 4096, 8192, None))
+    assert st == 1 and "overlap" in msg
+    dims = nv.GdnDims(16, 32, 128, 128)
+    C = 2 * 16 * 128 + 32 * 128
+    lay0, lay1 = nv._Layout(), nv._Layout()
+    lw0 = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120, None, None, 4)
+    lw1 = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120, None, FAKE, 4)
+    assert L.gdn_layer_workspace_layout(ctypes.byref(lw0), 1, 4096, ctypes.byref(lay0)) == 0
+    assert L.gdn_layer_workspace_layout(ctypes.byref(lw1), 1, 4096, ctypes.byref(lay1)) == 0
+    assert lay1.o_codes - lay1.qkv_conv >= 4096 * C * 4 and lay0.o_codes == lay0.qkv_conv
+    lw_bad = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120, None, FAKE, 7)
+    st, msg = _err(L.gdn_layer_workspace_layout(ctypes.byref(lw_bad), 1, 4096, ctypes.byref(lay1)))
+    assert st == 2 and "conv_width" in msg
