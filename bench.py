@@ -437,10 +437,46 @@ def bench_gated(nv, dev, w, sh, x, B, T, steps, flush, stream):
     ms = statistics.mean(s.elapsed_time(e) for s, e in ts)
     gms = statistics.mean(s.elapsed_time(e) for s, e in gt)
     gbs = BT * HvV * 12 / (gms / 1e3) / 1e9
+    # the whole block: short convolution on q|k|v (width 4) and the output gate
+    C = 2 * sh.Hk * sh.K + HvV
+    conv_w = torch.from_numpy(gdn_synth.gaussian(10, (C, 4), std=0.5)).to(dev)
+    wf = dataclasses.replace(wg, conv_weight=conv_w, conv_width=4)
+    layf = nv.layer_workspace_layout(wf, B, T)
+    wsf = torch.empty(layf["total"], dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        nv.gdn_layer_forward(wf, x, B, T, y=y, workspace=wsf, stream=stream)
+    torch.cuda.synchronize()
+    tf, ct = [], []
+    for _ in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        nv.gdn_layer_forward(wf, x, B, T, y=y, workspace=wsf, stream=stream)
+        e.record(stream)
+        tf.append((s, e))
+    # the convolution kernel alone on the step's projection (4 B read + 4 B written per element)
+    Pf = wsf[layf["proj"]:layf["proj"] + BT * ldp * 4].view(torch.float32).view(BT, ldp)
+    qkv = wsf[layf["qkv_conv"]:layf["qkv_conv"] + BT * C * 4].view(torch.float32).view(BT, C)
+    for _ in range(steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        nv.gdn_short_conv(Pf, conv_w, B, T, out=qkv, stream=stream)
+        e.record(stream)
+        ct.append((s, e))
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    fms = statistics.mean(s.elapsed_time(e) for s, e in tf)
+    cms = statistics.mean(s.elapsed_time(e) for s, e in ct)
+    cgbs = BT * C * 8 / (cms / 1e3) / 1e9
     return {"workload": WORKLOAD + "_output_gate", "ms_per_step": round(ms, 4),
             "tokens_per_s": round(B * T / (ms / 1e3), 1),
             "output_gate_kernel": {"ms": round(gms, 4), "GB/s": round(gbs, 1),
-                                   "frac_of_hbm": round(gbs / peaks()["hbm_gbs"], 4)}}
+                                   "frac_of_hbm": round(gbs / peaks()["hbm_gbs"], 4)},
+            "with_short_conv": {"workload": WORKLOAD + "_short_conv4_output_gate", "ms_per_step": round(fms, 4),
+                                "tokens_per_s": round(B * T / (fms / 1e3), 1),
+                                "short_conv_kernel": {"ms": round(cms, 4), "GB/s": round(cgbs, 1),
+                                                      "frac_of_hbm": round(cgbs / peaks()["hbm_gbs"], 4)}}}
 
 
 def bench_decode(nv, dev, w, sh, steps, stream):

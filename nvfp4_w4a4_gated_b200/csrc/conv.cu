@@ -9,10 +9,12 @@
 // with the inputs before a call's first token taken from a carried state (the
 // previous W-1 inputs of the sequence, zero when absent).
 //
-// HBM-bound: one thread per channel over a block of tokens, keeping the last
-// W-1 inputs in registers; a warp's loads and stores are consecutive channels
-// (coalesced).  A second small kernel writes the new state after the first has
-// read the old one, so the state may be updated in place.
+// HBM-bound.  When the channel count and the row strides allow 16-byte access,
+// each thread takes four channels over a block of 16 tokens with all of the
+// block's inputs loaded before any is used; otherwise one thread per channel
+// slides a window of W inputs over 32 tokens.  A warp's loads and stores are
+// consecutive channels (coalesced).  A second small kernel writes the new state
+// after the first has read the old one, so the state may be updated in place.
 #include "common.cuh"
 
 namespace nvg {
@@ -57,6 +59,63 @@ __global__ void __launch_bounds__(kConvThreads) short_conv_kernel(const float* _
     }
 }
 
+// Four channels per thread (16-byte loads and stores) over a block of kConvTokens4
+// tokens, whose inputs are all loaded before any is used.  Needs C, ld_x and
+// ld_out multiples of 4 and 16-byte aligned x, out.
+constexpr int kConvTokens4 = 16;
+template <int W>
+__global__ void __launch_bounds__(kConvThreads) short_conv4_kernel(const float* __restrict__ x, int64_t ld_x, int64_t T,
+                                                                   int C, const float* __restrict__ w,
+                                                                   const float* __restrict__ state_in,
+                                                                   float* __restrict__ out, int64_t ld_out) {
+    pdl_wait_and_trigger();
+    const int c0 = (blockIdx.x * kConvThreads + threadIdx.x) * 4;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kConvTokens4;
+    const int b = blockIdx.z;
+    if (c0 >= C || t0 >= T) return;
+    const int n = static_cast<int>(T - t0 < kConvTokens4 ? T - t0 : kConvTokens4);
+    float tap[4][W];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int j = 0; j < W; ++j) tap[k][j] = w[static_cast<int64_t>(c0 + k) * W + j];
+    float4 in[W - 1 + kConvTokens4];
+#pragma unroll
+    for (int j = 0; j < W - 1; ++j) {
+        const int64_t u = t0 - (W - 1) + j;
+        if (u >= 0) {
+            in[j] = *reinterpret_cast<const float4*>(x + (static_cast<int64_t>(b) * T + u) * ld_x + c0);
+        } else if (state_in) {
+            const float* sp = state_in + static_cast<int64_t>(b) * C * (W - 1) + (u + (W - 1));
+            in[j] = make_float4(sp[static_cast<int64_t>(c0) * (W - 1)], sp[static_cast<int64_t>(c0 + 1) * (W - 1)],
+                                sp[static_cast<int64_t>(c0 + 2) * (W - 1)], sp[static_cast<int64_t>(c0 + 3) * (W - 1)]);
+        } else {
+            in[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kConvTokens4; ++i)
+        in[W - 1 + i] = i < n ? *reinterpret_cast<const float4*>(x + (static_cast<int64_t>(b) * T + t0 + i) * ld_x + c0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kConvTokens4; ++i) {
+        if (i < n) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < W; ++j) {
+                const float4 v = in[i + j];
+                acc[0] = fmaf(tap[0][j], v.x, acc[0]);
+                acc[1] = fmaf(tap[1][j], v.y, acc[1]);
+                acc[2] = fmaf(tap[2][j], v.z, acc[2]);
+                acc[3] = fmaf(tap[3][j], v.w, acc[3]);
+            }
+            *reinterpret_cast<float4*>(out + (static_cast<int64_t>(b) * T + t0 + i) * ld_out + c0) =
+                make_float4(acc[0] / (1.0f + expf(-acc[0])), acc[1] / (1.0f + expf(-acc[1])),
+                            acc[2] / (1.0f + expf(-acc[2])), acc[3] / (1.0f + expf(-acc[3])));
+        }
+    }
+}
+
 // New state: the last W-1 inputs of each sequence (some from the old state when
 // T < W-1).  Each thread reads all it needs before writing, so in place is safe.
 template <int W>
@@ -83,10 +142,16 @@ __global__ void __launch_bounds__(kConvThreads) short_conv_state_kernel(const fl
 template <int W>
 nvfp4_status launch_conv(const float* x, int64_t ld_x, int B, int64_t T, int C, const float* w, const float* state_in,
                          float* state_out, float* out, int64_t ld_out, cudaStream_t st) {
-    const dim3 grid((C + kConvThreads - 1) / kConvThreads, static_cast<unsigned>((T + kConvTokens - 1) / kConvTokens),
-                    B);
-    cudaError_t e = launch_pdl(short_conv_kernel<W>, grid, dim3(kConvThreads), 0, st, x, ld_x, T, C, w, state_in, out,
-                               ld_out);
+    cudaError_t e;
+    if (C % 4 == 0 && ld_x % 4 == 0 && ld_out % 4 == 0 && aligned16(x) && aligned16(out)) {
+        const dim3 grid((C / 4 + kConvThreads - 1) / kConvThreads,
+                        static_cast<unsigned>((T + kConvTokens4 - 1) / kConvTokens4), B);
+        e = launch_pdl(short_conv4_kernel<W>, grid, dim3(kConvThreads), 0, st, x, ld_x, T, C, w, state_in, out, ld_out);
+    } else {
+        const dim3 grid((C + kConvThreads - 1) / kConvThreads,
+                        static_cast<unsigned>((T + kConvTokens - 1) / kConvTokens), B);
+        e = launch_pdl(short_conv_kernel<W>, grid, dim3(kConvThreads), 0, st, x, ld_x, T, C, w, state_in, out, ld_out);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "short conv launch");
     if (state_out) {
         const dim3 g2((C + kConvThreads - 1) / kConvThreads, B);
@@ -118,7 +183,7 @@ extern "C" nvfp4_status gdn_short_conv(const float* x, int64_t ld_x, int32_t B, 
     if (B < 1 || T < 1 || C < 1) return fail(NVFP4_ERR_INVALID_ARG, "B, T and C must be >= 1");
     if (W < 2 || W > 4) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "conv width must be 2, 3 or 4");
     if (ld_x < C || ld_out < C) return fail(NVFP4_ERR_INVALID_ARG, "ld_x / ld_out smaller than C");
-    if (static_cast<int64_t>(B) * T > (int64_t(1) << 31) || (T + kConvTokens - 1) / kConvTokens > 65535 || B > 65535)
+    if (static_cast<int64_t>(B) * T > (int64_t(1) << 31) || (T + kConvTokens4 - 1) / kConvTokens4 > 65535 || B > 65535)
         return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "B or T too large");
     const char* xb = reinterpret_cast<const char*>(x);
     const char* ob = reinterpret_cast<const char*>(out);

@@ -96,30 +96,45 @@ __global__ void __launch_bounds__(256) output_gate_kernel(const float* o, const 
         memcpy(wv, &c, sizeof(wv));
     }
     float m = 0.0f;
-    for (int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
-         row += nwarps) {
-        const int64_t t = row / Hv;
-        const int h = static_cast<int>(row - t * Hv);
-        float ov[PL], zv[PL];
-        const VecT a = *reinterpret_cast<const VecT*>(o + row * V + lane * PL);
-        const VecT b = *reinterpret_cast<const VecT*>(z + t * ld_z + static_cast<int64_t>(h) * V + lane * PL);
-        memcpy(ov, &a, sizeof(ov));
-        memcpy(zv, &b, sizeof(zv));
-        float ss = 0.0f;
+    // two rows per iteration, both rows' loads issued before either is used
+    constexpr int R = 2;
+    for (int64_t row0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row0 < rows;
+         row0 += R * nwarps) {
+        float ov[R][PL], zv[R][PL];
 #pragma unroll
-        for (int i = 0; i < PL; ++i) ss = fmaf(ov[i], ov[i], ss);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv_rms = 1.0f / sqrtf(ss / static_cast<float>(V) + 1e-6f);
-#pragma unroll
-        for (int i = 0; i < PL; ++i) {
-            const float silu = zv[i] / (1.0f + expf(-zv[i]));
-            ov[i] = ov[i] * inv_rms * wv[i] * silu;
-            m = fmaxf(m, fabsf(ov[i]));
+        for (int r = 0; r < R; ++r) {
+            const int64_t row = row0 + r * nwarps;
+            VecT a{}, b{};
+            if (row < rows) {
+                const int64_t t = row / Hv;
+                const int h = static_cast<int>(row - t * Hv);
+                a = *reinterpret_cast<const VecT*>(o + row * V + lane * PL);
+                b = *reinterpret_cast<const VecT*>(z + t * ld_z + static_cast<int64_t>(h) * V + lane * PL);
+            }
+            memcpy(ov[r], &a, sizeof(ov[r]));
+            memcpy(zv[r], &b, sizeof(zv[r]));
         }
-        VecT r;
-        memcpy(&r, ov, sizeof(ov));
-        *reinterpret_cast<VecT*>(out + row * V + lane * PL) = r;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t row = row0 + r * nwarps;
+            float ss = 0.0f;
+#pragma unroll
+            for (int i = 0; i < PL; ++i) ss = fmaf(ov[r][i], ov[r][i], ss);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const float inv_rms = 1.0f / sqrtf(ss / static_cast<float>(V) + 1e-6f);
+#pragma unroll
+            for (int i = 0; i < PL; ++i) {
+                const float silu = zv[r][i] / (1.0f + expf(-zv[r][i]));
+                ov[r][i] = ov[r][i] * inv_rms * wv[i] * silu;
+                m = fmaxf(m, fabsf(ov[r][i]));
+            }
+            if (row < rows) {
+                VecT res;
+                memcpy(&res, ov[r], sizeof(ov[r]));
+                *reinterpret_cast<VecT*>(out + row * V + lane * PL) = res;
+            }
+        }
     }
     if (amax_word) {
         __shared__ unsigned int warp_max[8];

@@ -24,8 +24,9 @@ def _close(got, ref):
 
 @pytest.mark.parametrize("W", [2, 3, 4])
 @pytest.mark.parametrize("with_state", [False, True])
-def test_short_conv_matches_oracle(cuda_dev, W, with_state):
-    B, T, C, extra = 2, 45, 300, 12          # ragged: tokens past one 32-token block, channels past 2 x 128
+@pytest.mark.parametrize("C", [300, 301])   # 301: no 16-byte access, the one-channel-per-thread kernel
+def test_short_conv_matches_oracle(cuda_dev, W, with_state, C):
+    B, T, extra = 2, 45, 12                  # ragged: tokens past one 32-token block, channels past 2 x 128
     xbig = gdn_synth.gaussian(40 + W, (B * T, C + extra), std=2.0)
     w = gdn_synth.gaussian(41 + W, (C, W), std=0.7)
     s0 = gdn_synth.gaussian(42 + W, (B, C, W - 1), std=2.0) if with_state else None
