@@ -634,6 +634,21 @@ def kernel_case(args):
         ws = torch.empty(nv.lib().gdn_scan_workspace_size(B, T, __import__("ctypes").byref(dims.c()), 0),
                          dtype=torch.uint8, device=dev)
         fn = lambda: nv.gdn_scan(qh, kh, v, gg, bt, B, T, dims, o=o, workspace=ws)
+    elif args.kernel_case in ("gate", "conv"):
+        # the optional output gate / short convolution on the layer-sized operands
+        B, T, Hk, Hv, Kd = 1, args.T, 16, 32, 128
+        C = 2 * Hk * Kd + Hv * Kd
+        ldp = 2 * C                              # projection-like row stride
+        P = torch.randn((B * T, ldp), generator=g, device=dev)
+        if args.kernel_case == "gate":
+            o = torch.randn((B * T, Hv, Kd), generator=g, device=dev)
+            wn = torch.randn((Kd,), generator=g, device=dev)
+            G = torch.empty_like(o)
+            fn = lambda: nv.gdn_output_gate(o, P[:, C:], wn, out=G)
+        else:
+            wc = torch.randn((C, 4), generator=g, device=dev) * 0.5
+            out = torch.empty((B * T, C), device=dev)
+            fn = lambda: nv.gdn_short_conv(P, wc, B, T, out=out)
     else:
         raise SystemExit("unknown kernel case")
     for _ in range(args.warmup):
@@ -659,7 +674,7 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     ap.add_argument("--ref-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan"], default=None,
+    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv"], default=None,
                     help="profile helper: run one kernel on a fixed case and exit")
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
