@@ -72,6 +72,8 @@ def _L():
         lib.orc_scan_chunked.argtypes = [P, P, P, P, P, i32, i64, i32, i32, i32, i32, f64, i32, i32,
                                          P, P, P]
         lib.orc_scan_chunked.restype = None
+        lib.orc_scan_transition.argtypes = [P, P, P, P, i32, i64, i32, i32, i32, f64, i32, P, P]
+        lib.orc_scan_transition.restype = None
         lib.orc_num_threads.argtypes = []; lib.orc_num_threads.restype = i32
         _lib = lib
     return _lib
@@ -259,6 +261,61 @@ def scan_chunked(q, k, v, g, beta, chunk=64, scale=None, form=FORM_PAGES, S0=Non
     s0 = None if S0 is None else _c(S0, np.float64)
     _L().orc_scan_chunked(_p(q), _p(k), _p(v), _p(g), _p(beta), B, T, Hk, Hv, K, V, float(scale),
                           int(form), int(chunk), None if s0 is None else _p(s0), _p(S), _p(o))
+    return o, S
+
+
+# ----------------------------------------------------------- state passing --
+def scan_transition(q, k, g, beta, scale=None, form=FORM_PAGES):
+    """Reading P1: the span's state map P = A_T...A_1 (A_t = a_t I - b_t k_t k_t^T,
+    or a_t (I - b_t k_t k_t^T) in the STANDARD form) and the query map
+    m_t = scale P_t^T q_t, formed token by token from the product itself.
+    q, k: [B,T,Hk,K]; g, beta: [B,T,Hv].  Returns (P [B,Hv,K,K], m [B,T,Hv,K]).
+    A span started from S_in then ends in P S_in + S_loc and its outputs gain
+    S_in^T m_t (Eq.(2) is affine in the state; review page, background)."""
+    q, k = _c(q, np.float64), _c(k, np.float64)
+    g, beta = _c(g, np.float64), _c(beta, np.float64)
+    B, T, Hk, K = q.shape
+    Hv = g.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(K)
+    P = np.empty((B, Hv, K, K), np.float64)
+    m = np.empty((B, T, Hv, K), np.float64)
+    _L().orc_scan_transition(_p(q), _p(k), _p(g), _p(beta), B, T, Hk, Hv, K, float(scale), int(form), _p(P), _p(m))
+    return P, m
+
+
+def state_combine(P, S_loc, S_in):
+    """State at the end of a span that started from S_in: P S_in + S_loc, per
+    (sequence, value head).  P: [...,K,K]; S_loc, S_in: [...,K,V]."""
+    return np.matmul(np.asarray(P, np.float64), np.asarray(S_in, np.float64)) + np.asarray(S_loc, np.float64)
+
+
+def output_correct(o_loc, m, S_in):
+    """Outputs of a span that started from S_in, given its zero-start outputs
+    o_loc [B,T,Hv,V] and query map m [B,T,Hv,K]: o_t = o_loc_t + S_in^T m_t,
+    S_in [B,Hv,K,V]."""
+    return np.asarray(o_loc, np.float64) + np.einsum("bthi,bhij->bthj", np.asarray(m, np.float64),
+                                                     np.asarray(S_in, np.float64))
+
+
+def scan_segmented(q, k, v, g, beta, bounds, scale=None, form=FORM_PAGES, S0=None):
+    """Reading P1: the scan of each span [bounds[i], bounds[i+1]) from a zero
+    state, the span maps, the spans' initial states by composing the maps in
+    order from S0, then each span's outputs corrected by its initial state.
+    Returns (o [B,T,Hv,V], S [B,Hv,K,V]) like scan()."""
+    q, k, v = _c(q, np.float64), _c(k, np.float64), _c(v, np.float64)
+    g, beta = _c(g, np.float64), _c(beta, np.float64)
+    B, T, Hk, K = q.shape
+    Hv, V = v.shape[2], v.shape[3]
+    assert bounds[0] == 0 and bounds[-1] == T and all(a < b for a, b in zip(bounds, bounds[1:]))
+    S = np.zeros((B, Hv, K, V)) if S0 is None else _c(S0, np.float64).copy()
+    o = np.empty((B, T, Hv, V), np.float64)
+    for a, b in zip(bounds, bounds[1:]):
+        sl = slice(a, b)
+        o_loc, S_loc = scan(q[:, sl], k[:, sl], v[:, sl], g[:, sl], beta[:, sl], scale=scale, form=form)
+        P, m = scan_transition(q[:, sl], k[:, sl], g[:, sl], beta[:, sl], scale=scale, form=form)
+        o[:, sl] = output_correct(o_loc, m, S)
+        S = state_combine(P, S_loc, S)
     return o, S
 
 

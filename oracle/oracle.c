@@ -40,6 +40,11 @@
  *      section, but gives no formula): per token and value head,
  *      G = o / sqrt(mean(o^2) + 1e-6) * w * z * sigmoid(z), w a learned weight
  *      of V entries shared by the heads; out_proj then reads G instead of o.
+ *   P1 state passing (the sequence-sharded scan): the pages run the recurrence
+ *      over windows of up to 32K tokens ([R] sec.5.3) in one pass and say
+ *      nothing about splitting it; here a sequence is split into spans that
+ *      are joined through the affinity of Eq.(2) in the state
+ *      (orc_scan_transition).
  *   C1 short convolution (optional; [R] lists convolutions among the layers kept
  *      unquantised, "Minima" section, and gives nothing else): per channel c of
  *      the q|k|v slices, a causal depthwise convolution of width W followed by
@@ -404,6 +409,58 @@ ORC_EXPORT void orc_scan_chunked(const double* q, const double* k, const double*
 #undef VV
             }
             free(G); free(U); free(Sn);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* State passing (reading P1).  Eq.(2) is affine in the state: with           */
+/*   A_t = a_t I - b_t k_t k_t^T          (form PAGES)                        */
+/*   A_t = a_t (I - b_t k_t k_t^T)        (form STANDARD)                     */
+/* one token maps S to A_t S + b_t k_t v_t^T, so a span of tokens maps an     */
+/* initial state S_in to P S_in + S_loc, with P = A_T ... A_1 and S_loc the   */
+/* span's final state from a zero start, and each output of the span gains   */
+/* S_in^T (scale P_t^T q_t), P_t = A_t ... A_1.  This function forms P and    */
+/* the query map m_t = scale P_t^T q_t straight from that product, one token  */
+/* at a time: A_t P = a_t P - b_t k_t (k_t^T P) for PAGES and                 */
+/* a_t (P - b_t k_t (k_t^T P)) for STANDARD.                                  */
+/*   q, k: [B, T, Hk, K]; g, beta: [B, T, Hv]; P: [B, Hv, K, K];              */
+/*   qmap: [B, T, Hv, K].                                                     */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_scan_transition(const double* q, const double* k, const double* g, const double* beta,
+                                    int32_t B, int64_t T, int32_t Hk, int32_t Hv, int32_t K, double scale,
+                                    int32_t form, double* P, double* qmap) {
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int32_t bb = 0; bb < B; ++bb)
+        for (int32_t h = 0; h < Hv; ++h) {
+            const int32_t hk = (int32_t)(((int64_t)h * Hk) / Hv);
+            double* Pt = P + ((int64_t)bb * Hv + h) * K * K;
+            for (int32_t i = 0; i < K; ++i)
+                for (int32_t j = 0; j < K; ++j) Pt[(int64_t)i * K + j] = (i == j) ? 1.0 : 0.0;
+            double* kP = (double*)malloc(sizeof(double) * K);
+            for (int64_t t = 0; t < T; ++t) {
+                const double* kt = k + (((int64_t)bb * T + t) * Hk + hk) * K;
+                const double* qt = q + (((int64_t)bb * T + t) * Hk + hk) * K;
+                const double alpha = exp(g[((int64_t)bb * T + t) * Hv + h]);
+                const double bt = beta[((int64_t)bb * T + t) * Hv + h];
+                for (int32_t j = 0; j < K; ++j) {           /* k_t^T P, a row vector */
+                    double s = 0.0;
+                    for (int32_t i = 0; i < K; ++i) s += kt[i] * Pt[(int64_t)i * K + j];
+                    kP[j] = s;
+                }
+                for (int32_t i = 0; i < K; ++i)
+                    for (int32_t j = 0; j < K; ++j) {
+                        const double rank1 = bt * kt[i] * kP[j];
+                        double* e = &Pt[(int64_t)i * K + j];
+                        *e = (form == 1) ? alpha * (*e - rank1) : alpha * (*e) - rank1;
+                    }
+                double* mt = qmap + (((int64_t)bb * T + t) * Hv + h) * K;
+                for (int32_t j = 0; j < K; ++j) {           /* scale P_t^T q_t */
+                    double s = 0.0;
+                    for (int32_t i = 0; i < K; ++i) s += Pt[(int64_t)i * K + j] * qt[i];
+                    mt[j] = s * scale;
+                }
+            }
+            free(kP);
         }
 }
 

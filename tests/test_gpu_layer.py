@@ -129,3 +129,40 @@ def test_full_size_prefill_layer_stage_checks(cuda_dev):
     P = _view(ws, lay["proj"], BT * ldp * 4, torch.float32).view(BT, ldp)[torch.from_numpy(rows).cuda(), :n_in]
     assert rel_fro(P.cpu().numpy(), ref) <= 1e-3
     assert torch.isfinite(y).all() and torch.isfinite(S_out).all()
+
+
+def _check_o_quantised_exactly(ws, lay, BT, HvV, o_field="o"):
+    """The o quantiser in the layer takes its amax from the word the scan (or the
+    output gate) filled, and runs only its quantisation pass.  Codes, block scales
+    and the global scale must equal the oracle's quantisation of the same o."""
+    o = _view(ws, lay[o_field], BT * HvV * 4, torch.float32).cpu().numpy().reshape(BT, HvV)
+    codes, sf, S = oracle.quantize(o)
+    oc = _view(ws, lay["o_codes"], BT * HvV // 2, torch.uint8).cpu().numpy().reshape(BT, HvV // 2)
+    osf = ws[lay["o_sf"]:lay["o_sf"] + nv.lib().nvfp4_sf_bytes(BT, HvV)].cpu().numpy()
+    oS = _view(ws, lay["o_scale"], 4, torch.float32).cpu().numpy()[0]
+    assert np.float32(oS) == np.float32(S)
+    assert np.array_equal(oc, codes)
+    assert np.array_equal(osf, oracle.sf_linear_to_mma(sf, BT, HvV))
+
+
+@pytest.mark.parametrize("B,T", [(1, 64), (2, 100), (3, 1)])   # chunked scan twice, then the one-token scan
+def test_o_quantised_from_the_producer_amax(cuda_dev, B, T):
+    sh = gdn_synth.TINY
+    bits, _ = gdn_synth.activations(5, B * T, sh.H, hot="fixed")
+    w, _ = _make_layer(sh, 5)
+    S0 = f32_device(gdn_synth.gaussian(6, (B, sh.Hv, sh.K, sh.V), std=0.5))
+    _, ws, lay = nv.gdn_layer_forward(w, bf16_device(bits), B, T, state_in=S0)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    _check_o_quantised_exactly(ws, lay, B * T, sh.Hv * sh.V)
+
+
+def test_o_quantised_from_the_producer_amax_full_size(cuda_dev):
+    """The T = 4096 layer-prefill workload as the benchmark runs it."""
+    sh, B, T = gdn_synth.FULL, 1, 4096
+    bits, _ = gdn_synth.activations(7, B * T, sh.H, hot="percent")
+    w, _ = _make_layer(sh, 7)
+    _, ws, lay = nv.gdn_layer_forward(w, bf16_device(bits), B, T)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    _check_o_quantised_exactly(ws, lay, B * T, sh.Hv * sh.V)

@@ -541,3 +541,90 @@ def test_layer_oracle_conv_option():
     P = st["P"]
     np.testing.assert_allclose(st["Pc"][:, :C], P[:, :C] / (1.0 + np.exp(-P[:, :C])), rtol=1e-15)
     np.testing.assert_array_equal(st["Pc"][:, C:], P[:, C:])
+
+
+# ------------------------------------------------------ state passing (P1) --
+@pytest.mark.parametrize("form", [oracle.FORM_PAGES, oracle.FORM_STANDARD])
+def test_transition_of_one_token_is_the_closed_form(form):
+    """One token: P = a I - b k k^T (PAGES) or a (I - b k k^T) (STANDARD), and
+    the query map is scale P^T q (Eq.(2) written as a map of the state)."""
+    B, T, Hk, Hv, K = 1, 1, 1, 2, 6
+    q, k, _, g, beta = gdn_synth.scan_inputs(200, B, T, Hk, Hv, K, 4, alpha_lo=0.5)
+    P, m = oracle.scan_transition(q, k, g, beta, scale=0.3, form=form)
+    kt = k[0, 0, 0].astype(np.float64)
+    for h in range(Hv):
+        a, bt = math.exp(g[0, 0, h]), float(beta[0, 0, h])
+        want = (a * np.eye(K) - bt * np.outer(kt, kt)) if form == oracle.FORM_PAGES else \
+            a * (np.eye(K) - bt * np.outer(kt, kt))
+        assert np.allclose(P[0, h], want, rtol=0, atol=1e-15)
+        assert np.allclose(m[0, 0, h], 0.3 * want.T @ q[0, 0, 0], rtol=0, atol=1e-15)
+
+
+def test_transition_without_writes_is_the_decay():
+    """beta = 0: nothing is written, the state only decays, so P_t is the
+    running product of the alphas times I and m_t = scale (prod alpha) q_t."""
+    B, T, Hk, Hv, K = 1, 9, 1, 1, 5
+    q, k, _, g, beta = gdn_synth.scan_inputs(201, B, T, Hk, Hv, K, 4, alpha_lo=0.6)
+    beta[:] = 0.0
+    P, m = oracle.scan_transition(q, k, g, beta, scale=1.0)
+    run = np.cumprod(np.exp(g[0, :, 0].astype(np.float64)))
+    assert np.allclose(P[0, 0], run[-1] * np.eye(K), rtol=1e-14, atol=0)
+    for t in range(T):
+        assert np.allclose(m[0, t, 0], run[t] * q[0, t, 0], rtol=1e-14, atol=1e-16)
+
+
+def test_transition_full_overwrite_is_a_projector():
+    """alpha = 1, beta = 1, unit k: each token erases the state along k
+    (review page, sec.5.3, the overwrite along the key direction), so the map
+    of a token is the projector I - k k^T; repeating the same key changes
+    nothing, and two orthogonal keys erase both directions."""
+    B, T, Hk, Hv, K = 1, 3, 1, 1, 6
+    q, k, _, g, beta = gdn_synth.scan_inputs(202, B, T, Hk, Hv, K, 4)
+    g[:] = 0.0
+    beta[:] = 1.0
+    k[0, :, 0] = k[0, 0, 0]
+    P, _ = oracle.scan_transition(q, k, g, beta)
+    k0 = k[0, 0, 0].astype(np.float64)
+    proj = np.eye(K) - np.outer(k0, k0)
+    assert np.allclose(P[0, 0], proj, atol=1e-15) and np.allclose(P[0, 0] @ P[0, 0], P[0, 0], atol=1e-15)
+    e = np.eye(K)
+    k2 = np.zeros((B, 2, Hk, K), np.float32)
+    k2[0, 0, 0], k2[0, 1, 0] = e[1], e[4]
+    P2, _ = oracle.scan_transition(q[:, :2], k2, g[:, :2], beta[:, :2])
+    want = np.eye(K)
+    want[1, 1] = want[4, 4] = 0.0
+    assert np.array_equal(P2[0, 0], want)
+
+
+@pytest.mark.parametrize("form", [oracle.FORM_PAGES, oracle.FORM_STANDARD])
+@pytest.mark.parametrize("bounds", [[0, 50], [0, 1, 50], [0, 17, 18, 40, 50], [0, 25, 50]])
+def test_segmented_scan_equals_the_recurrence(form, bounds):
+    """Spans scanned from zero, joined through their maps, give the recurrence
+    over the whole sequence (outputs and final state), with a random start."""
+    B, T, Hk, Hv, K, V = 2, 50, 2, 4, 8, 6
+    q, k, v, g, beta = gdn_synth.scan_inputs(203, B, T, Hk, Hv, K, V, alpha_lo=0.7)
+    S0 = gdn_synth.gaussian(204, (B, Hv, K, V))
+    o1, S1 = oracle.scan(q, k, v, g, beta, form=form, S0=S0)
+    o2, S2 = oracle.scan_segmented(q, k, v, g, beta, bounds, form=form, S0=S0)
+    assert np.max(np.abs(o1 - o2)) < 1e-12 * max(1, np.abs(o1).max())
+    assert np.max(np.abs(S1 - S2)) < 1e-12 * max(1, np.abs(S1).max())
+
+
+def test_state_combine_and_correction_by_hand():
+    """The two joining steps written out with explicit loops on a tiny case."""
+    r = np.random.default_rng(205)
+    P, S_loc, S_in = r.standard_normal((2, 3, 3)), r.standard_normal((2, 3, 2)), r.standard_normal((2, 3, 2))
+    got = oracle.state_combine(P, S_loc, S_in)
+    for n in range(2):
+        for i in range(3):
+            for j in range(2):
+                assert math.isclose(got[n, i, j], sum(P[n, i, l] * S_in[n, l, j] for l in range(3)) + S_loc[n, i, j],
+                                    rel_tol=1e-14, abs_tol=1e-14)
+    o_loc, m = r.standard_normal((1, 2, 2, 2)), r.standard_normal((1, 2, 2, 3))
+    S = r.standard_normal((1, 2, 3, 2))
+    got = oracle.output_correct(o_loc, m, S)
+    for t in range(2):
+        for h in range(2):
+            for j in range(2):
+                want = o_loc[0, t, h, j] + sum(S[0, h, i, j] * m[0, t, h, i] for i in range(3))
+                assert math.isclose(got[0, t, h, j], want, rel_tol=1e-14, abs_tol=1e-14)
