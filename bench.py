@@ -18,6 +18,7 @@ and the reported time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -299,6 +300,8 @@ def run_ours(args, rank, world, local_rank):
     decode = bench_decode(nv, dev, w, sh, args.steps, stream)
     # ---- the prefill step with the optional output gate
     gated = bench_gated(nv, dev, w, sh, x, B, T, args.steps, flush, stream)
+    # ---- the 32K-token scan split into eight spans (one sequence-parallel rank's work)
+    seqpar = bench_seqpar(nv, dev, args.steps, flush, stream, clk.get("sm_max_mhz"))
 
     # ---- end to end through the public call with host buffers, pipelined over steps:
     # the upload of step i+1 (pinned x -> device) and the download of step i's y
@@ -387,6 +390,7 @@ def run_ours(args, rank, world, local_rank):
         "gemm_standalone": gemm,
         "decode": decode,
         "output_gate": gated,
+        "sequence_parallel_scan": seqpar,
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * 2), "d2h_bytes_per_step": int(y.numel() * 4)},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
@@ -477,6 +481,100 @@ def bench_gated(nv, dev, w, sh, x, B, T, steps, flush, stream):
                                 "tokens_per_s": round(B * T / (fms / 1e3), 1),
                                 "short_conv_kernel": {"ms": round(cms, 4), "GB/s": round(cgbs, 1),
                                                       "frac_of_hbm": round(cgbs / peaks()["hbm_gbs"], 4)}}}
+
+
+def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
+    """The 32K-token scan (B = 1, 16 key / 32 value heads of 128) split into
+    eight spans of 4096 tokens, as eight ranks of a sequence-parallel scan run
+    it, timed on one GPU: one rank's steps (zero-start scan of its span, the
+    span maps, the last rank's seven state combines, the output correction)
+    against the unsplit scan.  The all-gather of (P, S_loc), 4 MiB per rank,
+    is not measured on one GPU.  The correction kernel does 2 T Hv K V FLOP on
+    the CUDA cores (peak: SMs x 128 FP32 lanes x 2 x the maximum SM clock) and
+    moves (T Hv (K + 2 V) + Hv K V) x 4 bytes."""
+    B, T, Hk, Hv, K, V, n = 1, 32768, 16, 32, 128, 128, 8
+    Ts = T // n
+    dims = nv.GdnDims(Hk, Hv, K, V)
+    g_ = torch.Generator(device=dev)
+    g_.manual_seed(11)
+    q = torch.nn.functional.normalize(torch.randn((T, Hk, K), generator=g_, device=dev), dim=-1)
+    k = torch.nn.functional.normalize(torch.randn((T, Hk, K), generator=g_, device=dev), dim=-1)
+    v = torch.randn((T, Hv * V), generator=g_, device=dev)
+    g = torch.log(torch.rand((T, Hv), generator=g_, device=dev) * (0.9999 - 0.99) + 0.99)
+    beta = torch.rand((T, Hv), generator=g_, device=dev)
+    o = torch.empty((T, Hv, V), device=dev)
+    S = torch.empty((B, Hv, K, V), device=dev)
+    ws = torch.empty(nv.lib().gdn_scan_workspace_size(B, T, ctypes.byref(dims.c()), nv.SCAN_AUTO),
+                     dtype=torch.uint8, device=dev)
+    a = T - Ts                                   # the last rank's span
+    span = (q[a:], k[a:], v[a:], g[a:], beta[a:])
+    o_s = torch.empty((Ts, Hv, V), device=dev)
+    S_loc = torch.empty((B, Hv, K, V), device=dev)
+    ws_s = torch.empty(nv.lib().gdn_scan_workspace_size(B, Ts, ctypes.byref(dims.c()), nv.SCAN_AUTO),
+                       dtype=torch.uint8, device=dev)
+    P = torch.empty((B, Hv, K, K), device=dev)
+    qmap = torch.empty((Ts, Hv, K), device=dev)
+    ws_t = torch.empty(nv.lib().gdn_scan_transition_workspace_size(B, Ts, ctypes.byref(dims.c()), nv.SCAN_AUTO),
+                       dtype=torch.uint8, device=dev)
+    Ps = torch.randn((n - 1, B, Hv, K, K), generator=g_, device=dev) * (K ** -0.5)
+    Sl = torch.randn((n - 1, B, Hv, K, V), generator=g_, device=dev)
+    S_run = [torch.empty((B, Hv, K, V), device=dev) for _ in range(n)]
+    S_run[0].zero_()
+
+    def whole():
+        nv.gdn_scan(q, k, v, g, beta, B, T, dims, o=o, state_out=S, workspace=ws, stream=stream)
+
+    def rank_steps(ev):
+        ev[0].record(stream)
+        nv.gdn_scan(*span, B, Ts, dims, o=o_s, state_out=S_loc, workspace=ws_s, stream=stream)
+        ev[1].record(stream)
+        nv.gdn_scan_transition(*span[:2], *span[3:], B, Ts, dims, P=P, qmap=qmap, workspace=ws_t, stream=stream)
+        ev[2].record(stream)
+        for r in range(n - 1):
+            nv.gdn_state_combine(Ps[r], Sl[r], S_run[r] if r else None, out=S_run[r + 1], stream=stream)
+        ev[3].record(stream)
+        nv.gdn_scan_correct(qmap, S_run[n - 1], o_s, B, Ts, stream=stream)
+        ev[4].record(stream)
+
+    mk = lambda m: [torch.cuda.Event(enable_timing=True) for _ in range(m)]
+    for _ in range(3):
+        whole()
+        rank_steps(mk(5))
+    torch.cuda.synchronize()
+    tw, tr = [], []
+    for _ in range(steps):
+        flush.zero_()
+        ev = mk(2)
+        ev[0].record(stream)
+        whole()
+        ev[1].record(stream)
+        tw.append(ev)
+        flush.zero_()
+        ev = mk(5)
+        rank_steps(ev)
+        tr.append(ev)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    mean = lambda evs, i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
+    whole_ms, rank_ms = mean(tw, 0, 1), mean(tr, 0, 4)
+    corr_ms = mean(tr, 3, 4)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    clk = sm_max_mhz or 1965.0
+    alu_peak = sms * 128 * 2 * clk * 1e6 / 1e12
+    flop = 2.0 * Ts * Hv * K * V
+    byt = (Ts * Hv * (K + 2 * V) + Hv * K * V) * 4
+    return {"workload": "gdn_scan_B1_T32768_hk16_hv32_k128_v128_in_8_spans_of_4096",
+            "whole_scan_ms": round(whole_ms, 4), "per_rank_ms": round(rank_ms, 4),
+            "per_rank_speedup_without_exchange": round(whole_ms / rank_ms, 2),
+            "rank_steps_ms": {"span_scan": round(mean(tr, 0, 1), 4), "span_maps": round(mean(tr, 1, 2), 4),
+                              "seven_combines": round(mean(tr, 2, 3), 4), "correct": round(corr_ms, 4)},
+            "exchange": "all-gather of P and S_loc (4 MiB per rank): not measured on one GPU",
+            "correct_kernel": {"bound": "alu", "TFLOP/s": round(flop / (corr_ms / 1e3) / 1e12, 2),
+                               "peak_TFLOP/s": round(alu_peak, 1),
+                               "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 x {clk:g} MHz",
+                               "frac": round(flop / (corr_ms / 1e3) / 1e12 / alu_peak, 4),
+                               "GB/s": round(byt / (corr_ms / 1e3) / 1e9, 1),
+                               "frac_of_hbm": round(byt / (corr_ms / 1e3) / 1e9 / peaks()["hbm_gbs"], 4)}}
 
 
 def bench_decode(nv, dev, w, sh, steps, stream):
@@ -649,6 +747,13 @@ def kernel_case(args):
             wc = torch.randn((C, 4), generator=g, device=dev) * 0.5
             out = torch.empty((B * T, C), device=dev)
             fn = lambda: nv.gdn_short_conv(P, wc, B, T, out=out)
+    elif args.kernel_case == "correct":
+        # the sequence-parallel scan's output correction over one span of T tokens
+        B, T, Hv, Kd = 1, args.T, 32, 128
+        qm = torch.randn((B * T, Hv, Kd), generator=g, device=dev) * 0.1
+        S_in = torch.randn((B, Hv, Kd, Kd), generator=g, device=dev)
+        o = torch.randn((B * T, Hv, Kd), generator=g, device=dev)
+        fn = lambda: nv.gdn_scan_correct(qm, S_in, o, B, T)
     else:
         raise SystemExit("unknown kernel case")
     for _ in range(args.warmup):
@@ -674,7 +779,7 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     ap.add_argument("--ref-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv"], default=None,
+    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct"], default=None,
                     help="profile helper: run one kernel on a fixed case and exit")
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)

@@ -207,6 +207,59 @@ NVFP4_API nvfp4_status gdn_scan_noalloc(const float* q_hat, const float* k_hat, 
                                         const gdn_dims* dims, float scale, int32_t form, const float* state_in,
                                         float* state_out, float* o, nvfp4_stream_t stream);
 
+/* ------------------------------------------------------- state passing -- */
+/* Joining spans of one sequence (for a sequence split across GPUs, or into
+ * independent spans on one).  Eq.(2) (review page, background) is affine in
+ * the state: a token maps S to A_t S + b_t k_t v_t^T with
+ *   A_t = a_t I - b_t k_t k_t^T        (GDN_FORM_PAGES)
+ *   A_t = a_t (I - b_t k_t k_t^T)      (GDN_FORM_STANDARD),
+ * so a span started from S_in ends in P S_in + S_loc, P = A_T ... A_1, S_loc its
+ * final state from a zero start, and its outputs are o_t = o_loc_t + S_in^T m_t
+ * with m_t = scale P_t^T q_t (P_t = A_t ... A_1) and o_loc the zero-start
+ * outputs.  The pages scan each window in one pass and say nothing about
+ * splitting it; this is the plain reading of the recurrence's algebra.
+ * Recipe: gdn_scan every span from a zero state (o_loc, S_loc) and
+ * gdn_scan_transition every span (P, m), in any order or in parallel; then in
+ * span order S_in(next) = gdn_state_combine(P, S_loc, S_in) and
+ * gdn_scan_correct(m, S_in, o_loc) for every span whose S_in is not zero. */
+
+/* Bytes of workspace gdn_scan_transition needs. */
+NVFP4_API size_t gdn_scan_transition_workspace_size(int32_t B, int64_t T, const gdn_dims* dims, int32_t algo);
+
+/* The span map P and the query map m of B spans of T tokens each (the
+ * recurrence run on v = 0 from S = I).  q_hat, k_hat, g, beta, scale, form,
+ * algo: as for gdn_scan (the same inputs the span's gdn_scan takes; dims->V is
+ * not used).  P: device float32 [B x Hv x K x K] (written); qmap: device float32
+ * [B x T x Hv x K] (written).  P, qmap and the workspace must not overlap;
+ * pointers 16-byte aligned; workspace 256-byte aligned, >=
+ * gdn_scan_transition_workspace_size(B, T, dims, algo) bytes.  Costs one scan
+ * of the span with V = K. */
+NVFP4_API nvfp4_status gdn_scan_transition(const float* q_hat, const float* k_hat, const float* g,
+                                           const float* beta, int32_t B, int64_t T, const gdn_dims* dims,
+                                           float scale, int32_t form, int32_t algo, float* P, float* qmap,
+                                           void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* S_out[i] = P[i] S_in[i] + S_loc[i] for i < n (n = spans x value heads):
+ * P device float32 [n x K x K]; S_loc, S_in, S_out device float32 [n x K x V].
+ * S_in NULL means zero (P is then not read), S_loc NULL means zero.  S_out may
+ * be S_loc itself but must not overlap P or S_in.  K, V multiples of 32 in
+ * [32, 256]. */
+NVFP4_API nvfp4_status gdn_state_combine(const float* P, const float* S_loc, const float* S_in, float* S_out,
+                                         int64_t n, int32_t K, int32_t V, nvfp4_stream_t stream);
+
+/* o[b,t,h,:] += S_in[b,h]^T qmap[b,t,h,:]: the outputs of B spans of T tokens
+ * that started from S_in instead of zero.  qmap: device float32 [B x T x Hv x K]
+ * (from gdn_scan_transition); S_in: device float32 [B x Hv x K x V]; o: device
+ * float32 [B x T x Hv x V], updated in place, not overlapping the others.  K, V
+ * must be 64 or 128; pointers 16-byte aligned.  o_amax (device, nullable): the
+ * maximum |o| after the update is folded into it with atomicMax on the float
+ * bits (it must hold a non-negative float, e.g. 0, beforehand).  With the spans
+ * on several GPUs, a max all-reduce of the word gives the whole sequence's
+ * amax, from which S = amax / 2688 goes to nvfp4_quantize as a given scale. */
+NVFP4_API nvfp4_status gdn_scan_correct(const float* qmap, const float* S_in, float* o, int32_t B, int64_t T,
+                                        int32_t Hv, int32_t K, int32_t V, unsigned int* o_amax,
+                                        nvfp4_stream_t stream);
+
 /* ---------------------------------------------------------- output gate -- */
 /* Optional output gate before out_proj.  The pages name z as one of the
  * projections that move the layer output y (review page, Table 3 discussion)

@@ -20,7 +20,7 @@ from . import build as _build
 __all__ = [
     "NVFP4Error", "NVFP4Matrix", "GdnDims", "LayerWeights", "lib", "nvfp4_quantize", "w4a4_gemm", "gdn_gates",
     "gdn_scan", "gdn_scan_noalloc", "gdn_output_gate", "gdn_short_conv", "gdn_layer_forward", "layer_workspace_layout",
-    "check_device_error",
+    "check_device_error", "gdn_scan_transition", "gdn_state_combine", "gdn_scan_correct",
     "selftest_wait_timeout", "FORM_PAGES",
     "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
 ]
@@ -36,7 +36,8 @@ EXPORTED_SYMBOLS = [
     "nvfp4_last_error", "nvfp4_check_device_error", "nvfp4_version", "nvfp4_selftest_wait_timeout", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_size", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan_workspace_size",
     "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc", "gdn_output_gate",
-    "gdn_short_conv", "gdn_layer_forward_stateful",
+    "gdn_short_conv", "gdn_layer_forward_stateful", "gdn_scan_transition_workspace_size", "gdn_scan_transition",
+    "gdn_state_combine", "gdn_scan_correct",
 ]
 
 # Size of the fixed scratch array gdn_scan_noalloc uses (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
@@ -106,6 +107,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_layer_forward_stateful.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, P, P, i32, P,
                                                  sz, P]
         L.gdn_short_conv.argtypes = [P, i64, i32, i64, i32, i32, P, P, P, P, i64, P]
+        L.gdn_scan_transition_workspace_size.argtypes = [i32, i64, DP, i32]
+        L.gdn_scan_transition_workspace_size.restype = sz
+        L.gdn_scan_transition.argtypes = [P, P, P, P, i32, i64, DP, ctypes.c_float, i32, i32, P, P, P, sz, P]
+        L.gdn_state_combine.argtypes = [P, P, P, P, i64, i32, i32, P]
+        L.gdn_scan_correct.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, P]
         for f in ("nvfp4_check_device_error", "nvfp4_selftest_wait_timeout", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
                   "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc"):
             getattr(L, f).restype = ctypes.c_int
@@ -291,6 +297,50 @@ def gdn_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: flo
                           float(scale), form, algo, _ptr(state_in), _ptr(state_out), _ptr(o), _ptr(workspace),
                           0 if workspace is None else workspace.numel(), _stream(stream)))
     return o, state_out
+
+
+def gdn_scan_transition(q_hat, k_hat, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
+                        form: int = FORM_PAGES, algo: int = SCAN_AUTO, P=None, qmap=None, workspace=None,
+                        stream=None):
+    """Span map P [B, Hv, K, K] and query map [B*T, Hv, K] of B spans of T
+    tokens: a span started from S_in ends in P S_in + S_loc and its outputs
+    gain S_in^T qmap_t.  Inputs as for gdn_scan."""
+    dev = q_hat.device
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.K)
+    if P is None:
+        P = torch.empty((B, dims.Hv, dims.K, dims.K), dtype=torch.float32, device=dev)
+    if qmap is None:
+        qmap = torch.empty((B * T, dims.Hv, dims.K), dtype=torch.float32, device=dev)
+    d = dims.c()
+    need = lib().gdn_scan_transition_workspace_size(B, T, ctypes.byref(d), algo)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(lib().gdn_scan_transition(_ptr(q_hat), _ptr(k_hat), _ptr(g), _ptr(beta), B, T, ctypes.byref(d),
+                                     float(scale), form, algo, _ptr(P), _ptr(qmap), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)))
+    return P, qmap
+
+
+def gdn_state_combine(P, S_loc, S_in, out=None, stream=None):
+    """P S_in + S_loc per leading index: P [..., K, K], S_loc / S_in [..., K, V]
+    (S_in or S_loc None = zero).  out may be S_loc."""
+    ref = S_loc if S_loc is not None else S_in
+    K, V = ref.shape[-2], ref.shape[-1]
+    n = ref.numel() // (K * V)
+    if out is None:
+        out = torch.empty_like(ref)
+    _check(lib().gdn_state_combine(_ptr(P), _ptr(S_loc), _ptr(S_in), _ptr(out), n, K, V, _stream(stream)))
+    return out
+
+
+def gdn_scan_correct(qmap, S_in, o, B: int, T: int, amax_word=None, stream=None):
+    """o += S_in^T qmap per (sequence, token, value head), in place: qmap
+    [B*T, Hv, K], S_in [B, Hv, K, V], o [B*T, Hv, V]."""
+    Hv, K, V = S_in.shape[1], S_in.shape[2], S_in.shape[3]
+    _check(lib().gdn_scan_correct(_ptr(qmap), _ptr(S_in), _ptr(o), B, T, Hv, K, V, _ptr(amax_word),
+                                  _stream(stream)))
+    return o
 
 
 def gdn_scan_noalloc(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,

@@ -1,0 +1,123 @@
+"""Sequence-parallel delta-rule scan: each rank holds one span of every
+sequence, and the spans are joined through the recurrence's state.
+
+Eq.(2) of the review page "Why Gated DeltaNet Survives 4-Bit Quantization"
+(background) is affine in the state, so a span started from S_in ends in
+P S_in + S_loc and its outputs are o_loc + S_in^T m (P, m: the span's maps;
+o_loc, S_loc: its zero-start scan).  Per rank:
+
+1. scan the local span from a zero state (o_loc, S_loc) and form its maps
+   (P, m): two independent launches on the local tokens;
+2. all-gather (P, S_loc): the one exchange, B x Hv x K x (K + V) floats per
+   rank, whatever the span length;
+3. compose the maps of the ranks before this one, in rank order, starting from
+   the sequence's initial state: this rank's S_in;
+4. correct the outputs, o = o_loc + S_in^T m, and form the state at the end of
+   the span, P S_in + S_loc (the last rank's is the sequence's final state).
+
+The compute steps are the library's kernels (``gdn_scan``,
+``gdn_scan_transition``, ``gdn_state_combine``, ``gdn_scan_correct``);
+torch.distributed carries the exchange.  ``ops`` lets the host logic run
+against another implementation of the four steps (the multi-rank CPU tests
+use it); the default is the CUDA library and nothing else.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+import torch.distributed as dist
+
+from . import (FORM_PAGES, SCAN_AUTO, GdnDims, gdn_scan, gdn_scan_correct, gdn_scan_transition,
+               gdn_state_combine)
+
+
+class CudaSpanOps:
+    """The four steps on the GPU, through the C-ABI library."""
+
+    def __init__(self, algo: int = SCAN_AUTO, stream=None):
+        self.algo, self.stream = algo, stream
+
+    def scan(self, q_hat, k_hat, v, g, beta, B, T, dims, scale, form):
+        S_loc = torch.empty((B, dims.Hv, dims.K, dims.V), dtype=torch.float32, device=q_hat.device)
+        o, _ = gdn_scan(q_hat, k_hat, v, g, beta, B, T, dims, scale=scale, form=form, algo=self.algo,
+                        state_out=S_loc, stream=self.stream)
+        return o, S_loc
+
+    def transition(self, q_hat, k_hat, g, beta, B, T, dims, scale, form):
+        return gdn_scan_transition(q_hat, k_hat, g, beta, B, T, dims, scale=scale, form=form, algo=self.algo,
+                                   stream=self.stream)
+
+    def combine(self, P, S_loc, S_in):
+        return gdn_state_combine(P, S_loc, S_in, stream=self.stream)
+
+    def correct(self, qmap, S_in, o, B, T):
+        return gdn_scan_correct(qmap, S_in, o, B, T, stream=self.stream)
+
+
+@dataclass
+class SpanLocal:
+    """Step 1's results for one span."""
+    o: torch.Tensor        # [B*T, Hv, V], zero-start outputs (corrected in place by join)
+    S_loc: torch.Tensor    # [B, Hv, K, V]
+    P: torch.Tensor        # [B, Hv, K, K]
+    qmap: torch.Tensor     # [B*T, Hv, K]
+
+
+def span_local(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
+               form: int = FORM_PAGES, ops=None) -> SpanLocal:
+    """Step 1: the span's zero-start scan and its maps."""
+    ops = ops or CudaSpanOps()
+    o, S_loc = ops.scan(q_hat, k_hat, v, g, beta, B, T, dims, scale, form)
+    P, qmap = ops.transition(q_hat, k_hat, g, beta, B, T, dims, scale, form)
+    return SpanLocal(o, S_loc, P, qmap)
+
+
+def span_join(local: SpanLocal, P_before, S_loc_before, B: int, T: int, state_in=None, ops=None):
+    """Steps 3 and 4 for one span, given the maps of the spans before it in
+    order (lists, possibly empty) and the sequence's initial state (None =
+    zero).  Returns (o, state at the end of the span)."""
+    ops = ops or CudaSpanOps()
+    S_in = state_in
+    for P_r, S_r in zip(P_before, S_loc_before):
+        S_in = ops.combine(P_r, S_r, S_in)
+    o = local.o
+    if S_in is not None:
+        o = ops.correct(local.qmap, S_in, o, B, T)
+    return o, ops.combine(local.P, local.S_loc, S_in)
+
+
+def sequence_parallel_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
+                           form: int = FORM_PAGES, state_in=None, group=None, ops=None):
+    """The delta-rule scan of B sequences whose tokens are split across the
+    ranks of ``group`` in rank order: this rank holds T consecutive tokens of
+    every sequence (q_hat, k_hat [B*T, Hk, K]; v [B*T, >=Hv*V]; g, beta
+    [B*T, Hv]), and every rank passes the same ``state_in`` (the sequences'
+    initial state, or None).  Returns (o [B*T, Hv, V] for the local tokens, the
+    state after the local span [B, Hv, K, V]).  Every rank must call it with
+    the same B and dims; span lengths may differ."""
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    local = span_local(q_hat, k_hat, v, g, beta, B, T, dims, scale, form, ops)
+    if world == 1:
+        return span_join(local, [], [], B, T, state_in, ops)
+    Ps = [torch.empty_like(local.P) for _ in range(world)]
+    Ss = [torch.empty_like(local.S_loc) for _ in range(world)]
+    dist.all_gather(Ps, local.P.contiguous(), group=group)
+    dist.all_gather(Ss, local.S_loc.contiguous(), group=group)
+    return span_join(local, Ps[:rank], Ss[:rank], B, T, state_in, ops)
+
+
+def segmented_scan(spans, B: int, dims: GdnDims, scale: float | None = None, form: int = FORM_PAGES,
+                   state_in=None, ops=None):
+    """The same algorithm on one device, with the spans of every sequence given
+    as a list of (q_hat, k_hat, v, g, beta, T) tuples in order: all spans'
+    step 1 first (independent), then the joins in order, each span starting
+    from the state the previous join produced.  Returns the list of span
+    outputs and the final state."""
+    locals_ = [span_local(q, k, v, g, b, B, T, dims, scale, form, ops) for (q, k, v, g, b, T) in spans]
+    outs, S = [], state_in
+    for loc, span in zip(locals_, spans):
+        o, S = span_join(loc, [], [], B, span[5], S, ops)
+        outs.append(o)
+    return outs, S

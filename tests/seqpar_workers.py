@@ -1,0 +1,84 @@
+"""Rank bodies for the multi-process CPU tests of the sequence-parallel scan
+(run under torch.multiprocessing.spawn with the gloo backend).  The four span
+steps are the oracle's, on float64 CPU tensors; what runs under test is the
+host logic of nvfp4_w4a4_gated_b200.seqpar: rank order, the all-gather, the
+composition of the maps and the corrections."""
+import os
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+import gdn_synth
+import oracle
+
+
+class OracleSpanOps:
+    """gdn_scan / gdn_scan_transition / gdn_state_combine / gdn_scan_correct
+    restated with the oracle, in the binding's tensor shapes."""
+
+    def scan(self, q, k, v, g, beta, B, T, dims, scale, form):
+        Hk, Hv, K, V = dims.Hk, dims.Hv, dims.K, dims.V
+        o, S = oracle.scan(q.numpy().reshape(B, T, Hk, K), k.numpy().reshape(B, T, Hk, K),
+                           v.numpy()[:, :Hv * V].reshape(B, T, Hv, V), g.numpy().reshape(B, T, Hv),
+                           beta.numpy().reshape(B, T, Hv), scale=scale, form=form)
+        return torch.from_numpy(o.reshape(B * T, Hv, V)), torch.from_numpy(S)
+
+    def transition(self, q, k, g, beta, B, T, dims, scale, form):
+        Hk, Hv, K = dims.Hk, dims.Hv, dims.K
+        P, m = oracle.scan_transition(q.numpy().reshape(B, T, Hk, K), k.numpy().reshape(B, T, Hk, K),
+                                      g.numpy().reshape(B, T, Hv), beta.numpy().reshape(B, T, Hv), scale=scale,
+                                      form=form)
+        return torch.from_numpy(P), torch.from_numpy(m.reshape(B * T, Hv, K))
+
+    def combine(self, P, S_loc, S_in):
+        if S_in is None:
+            return S_loc.clone()
+        return torch.from_numpy(oracle.state_combine(P.numpy(), S_loc.numpy(), S_in.numpy()))
+
+    def correct(self, qmap, S_in, o, B, T):
+        Hv, K, V = S_in.shape[1], S_in.shape[2], S_in.shape[3]
+        out = oracle.output_correct(o.numpy().reshape(B, T, Hv, V), qmap.numpy().reshape(B, T, Hv, K), S_in.numpy())
+        return torch.from_numpy(out.reshape(B * T, Hv, V))
+
+
+def problem(form):
+    """One seeded problem shared by every rank: 2 sequences of 90 tokens."""
+    from nvfp4_w4a4_gated_b200 import GdnDims
+    B, T, Hk, Hv, K, V = 2, 90, 2, 4, 8, 6
+    q, k, v, g, beta = gdn_synth.scan_inputs(300, B, T, Hk, Hv, K, V, alpha_lo=0.7)
+    S0 = gdn_synth.gaussian(301, (B, Hv, K, V)).astype(np.float64)
+    return GdnDims(Hk, Hv, K, V), (q, k, v, g, beta), S0
+
+
+def span_tensors(arrs, a, e, dims):
+    """This rank's tokens [a, e) of every sequence, in the binding's shapes."""
+    q, k, v, g, beta = (x[:, a:e].astype(np.float64) for x in arrs)
+    B, T = q.shape[0], e - a
+    t = lambda x, *shape: torch.from_numpy(np.ascontiguousarray(x).reshape(*shape))
+    return (t(q, B * T, dims.Hk, dims.K), t(k, B * T, dims.Hk, dims.K), t(v, B * T, dims.Hv * dims.V),
+            t(g, B * T, dims.Hv), t(beta, B * T, dims.Hv))
+
+
+def rank_main(rank, world, port, bounds, form, with_state, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from nvfp4_w4a4_gated_b200.seqpar import sequence_parallel_scan
+        dims, arrs, S0 = problem(form)
+        a, e = bounds[rank], bounds[rank + 1]
+        q, k, v, g, beta = span_tensors(arrs, a, e, dims)
+        B = q.shape[0] // (e - a)
+        o, S_end = sequence_parallel_scan(q, k, v, g, beta, B, e - a, dims, scale=None, form=form,
+                                          state_in=torch.from_numpy(S0) if with_state else None,
+                                          ops=OracleSpanOps())
+        o_ref, _ = oracle.scan(*arrs, form=form, S0=S0 if with_state else None)
+        _, S_ref = oracle.scan(*(x[:, :e] for x in arrs), form=form, S0=S0 if with_state else None)
+        o_ref = o_ref[:, a:e].reshape(B * (e - a), dims.Hv, dims.V)
+        err_o = float(np.max(np.abs(o.numpy() - o_ref)) / max(1.0, np.abs(o_ref).max()))
+        err_S = float(np.max(np.abs(S_end.numpy() - S_ref)) / max(1.0, np.abs(S_ref).max()))
+        with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+            f.write(f"{err_o} {err_S}\n")
+    finally:
+        dist.destroy_process_group()

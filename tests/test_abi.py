@@ -180,3 +180,49 @@ def test_short_conv_validation_and_layout():
     lw_bad = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120, None, FAKE, 7)
     st, msg = _err(L.gdn_layer_workspace_layout(ctypes.byref(lw_bad), 1, 4096, ctypes.byref(lay1)))
     assert st == 2 and "conv_width" in msg
+
+
+def test_state_passing_validation_and_sizes():
+    L = nv.lib()
+    d = nv.GdnDims(16, 32, 128, 64).c()
+    # the transition runs the scan with V = K plus one zero row of Hv*K floats
+    dk = nv.GdnDims(16, 32, 128, 128).c()
+    scan_ws = L.gdn_scan_workspace_size(1, 4096, ctypes.byref(dk), nv.SCAN_CHUNKED)
+    tw = L.gdn_scan_transition_workspace_size(1, 4096, ctypes.byref(d), nv.SCAN_CHUNKED)
+    assert tw >= scan_ws + 32 * 128 * 4 and tw % 256 == 0
+    assert L.gdn_scan_transition_workspace_size(1, 1, ctypes.byref(d), nv.SCAN_AUTO) == 256 * ((32 * 128 * 4 + 255) // 256)
+    big = 0x40000000
+    st, _ = _err(L.gdn_scan_transition(None, FAKE, FAKE, FAKE, 1, 64, ctypes.byref(d), 1.0, 0, 0, FAKE, FAKE,
+                                       FAKE, 1 << 30, None))
+    assert st == 1
+    st, msg = _err(L.gdn_scan_transition(FAKE, FAKE, FAKE, FAKE, 1, 4096, ctypes.byref(d), 1.0, 0, 2, big,
+                                         2 * big, 3 * big, tw - 1, None))
+    assert st == 6
+    st, msg = _err(L.gdn_scan_transition(FAKE, FAKE, FAKE, FAKE, 1, 4096, ctypes.byref(d), 1.0, 0, 2, big, big,
+                                         3 * big, tw, None))
+    assert st == 1 and "overlap" in msg
+    st, _ = _err(L.gdn_scan_transition(FAKE, FAKE, FAKE, FAKE, 1, 64, ctypes.byref(d), 1.0, 5, 0, big, 2 * big,
+                                       3 * big, tw, None))
+    assert st == 1
+    # combine: shapes, aliasing
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, None, 4, 128, 128, None))
+    assert st == 1
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 4, 48, 128, None))
+    assert st == 2
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 4, 128, 512, None))
+    assert st == 2
+    st, msg = _err(L.gdn_state_combine(big, 2 * big, 3 * big, 3 * big + 4096, 4, 128, 128, None))
+    assert st == 1 and "overlap" in msg
+    st, msg = _err(L.gdn_state_combine(big, 2 * big + 4096, 3 * big, 2 * big, 4, 128, 128, None))
+    assert st == 1 and "S_loc" in msg
+    st, _ = _err(L.gdn_state_combine(None, FAKE, FAKE, big, 4, 128, 128, None))
+    assert st == 1
+    # correct: head dims, alignment, aliasing
+    st, _ = _err(L.gdn_scan_correct(FAKE, FAKE, big, 1, 64, 32, 96, 128, None, None))
+    assert st == 2
+    st, _ = _err(L.gdn_scan_correct(FAKE + 4, FAKE, big, 1, 64, 32, 128, 128, None, None))
+    assert st == 3
+    st, msg = _err(L.gdn_scan_correct(big, 2 * big, big + 4096, 1, 64, 32, 128, 128, None, None))
+    assert st == 1 and "overlap" in msg
+    st, _ = _err(L.gdn_scan_correct(FAKE, FAKE, big, 70000, 64, 32, 128, 128, None, None))
+    assert st == 2
