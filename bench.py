@@ -486,12 +486,13 @@ def bench_gated(nv, dev, w, sh, x, B, T, steps, flush, stream):
 def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
     """The 32K-token scan (B = 1, 16 key / 32 value heads of 128) split into
     eight spans of 4096 tokens, as eight ranks of a sequence-parallel scan run
-    it, timed on one GPU: one rank's steps (zero-start scan of its span, the
-    span maps, the last rank's seven state combines, the output correction)
-    against the unsplit scan.  The all-gather of (P, S_loc), 4 MiB per rank,
-    is not measured on one GPU.  The correction kernel does 2 T Hv K V FLOP on
-    the CUDA cores (peak: SMs x 128 FP32 lanes x 2 x the maximum SM clock) and
-    moves (T Hv (K + 2 V) + Hv K V) x 4 bytes."""
+    it, timed on one GPU: the last rank's steps (its span's zero-start scan and
+    maps in one gdn_scan_span call, the seven earlier maps composed in one
+    gdn_state_combine launch, the output correction) against the unsplit scan.
+    The all-gather of (P, S_loc), 4 MiB per rank, is not measured on one GPU.
+    The correction kernel does 2 T Hv K V FLOP on the CUDA cores (peak: SMs x
+    128 FP32 lanes x 2 x the maximum SM clock) and moves
+    (T Hv (K + 2 V) + Hv K V) x 4 bytes."""
     B, T, Hk, Hv, K, V, n = 1, 32768, 16, 32, 128, 128, 8
     Ts = T // n
     dims = nv.GdnDims(Hk, Hv, K, V)
@@ -508,32 +509,24 @@ def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
                      dtype=torch.uint8, device=dev)
     a = T - Ts                                   # the last rank's span
     span = (q[a:], k[a:], v[a:], g[a:], beta[a:])
-    o_s = torch.empty((Ts, Hv, V), device=dev)
-    S_loc = torch.empty((B, Hv, K, V), device=dev)
-    ws_s = torch.empty(nv.lib().gdn_scan_workspace_size(B, Ts, ctypes.byref(dims.c()), nv.SCAN_AUTO),
-                       dtype=torch.uint8, device=dev)
-    P = torch.empty((B, Hv, K, K), device=dev)
-    qmap = torch.empty((Ts, Hv, K), device=dev)
-    ws_t = torch.empty(nv.lib().gdn_scan_transition_workspace_size(B, Ts, ctypes.byref(dims.c()), nv.SCAN_AUTO),
+    ws_s = torch.empty(nv.lib().gdn_scan_span_workspace_size(B, Ts, ctypes.byref(dims.c()), nv.SCAN_AUTO),
                        dtype=torch.uint8, device=dev)
     Ps = torch.randn((n - 1, B, Hv, K, K), generator=g_, device=dev) * (K ** -0.5)
     Sl = torch.randn((n - 1, B, Hv, K, V), generator=g_, device=dev)
-    S_run = [torch.empty((B, Hv, K, V), device=dev) for _ in range(n)]
-    S_run[0].zero_()
+    S_in = torch.empty((B, Hv, K, V), device=dev)
 
     def whole():
         nv.gdn_scan(q, k, v, g, beta, B, T, dims, o=o, state_out=S, workspace=ws, stream=stream)
 
     def rank_steps(ev):
         ev[0].record(stream)
-        nv.gdn_scan(*span, B, Ts, dims, o=o_s, state_out=S_loc, workspace=ws_s, stream=stream)
+        o_s, S_loc, P, qmap = nv.gdn_scan_span(*span, B, Ts, dims, workspace=ws_s, stream=stream)
         ev[1].record(stream)
-        nv.gdn_scan_transition(*span[:2], *span[3:], B, Ts, dims, P=P, qmap=qmap, workspace=ws_t, stream=stream)
+        nv.gdn_state_combine(Ps, Sl, None, out=S_in, stream=stream)
         ev[2].record(stream)
-        for r in range(n - 1):
-            nv.gdn_state_combine(Ps[r], Sl[r], S_run[r] if r else None, out=S_run[r + 1], stream=stream)
+        nv.gdn_scan_correct(qmap, S_in, o_s, B, Ts, stream=stream)
         ev[3].record(stream)
-        nv.gdn_scan_correct(qmap, S_run[n - 1], o_s, B, Ts, stream=stream)
+        nv.gdn_state_combine(P, S_loc, S_in, out=S_loc, stream=stream)   # the state after the span
         ev[4].record(stream)
 
     mk = lambda m: [torch.cuda.Event(enable_timing=True) for _ in range(m)]
@@ -557,7 +550,7 @@ def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
     nv.check_device_error()
     mean = lambda evs, i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
     whole_ms, rank_ms = mean(tw, 0, 1), mean(tr, 0, 4)
-    corr_ms = mean(tr, 3, 4)
+    corr_ms = mean(tr, 2, 3)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     clk = sm_max_mhz or 1965.0
     alu_peak = sms * 128 * 2 * clk * 1e6 / 1e12
@@ -566,8 +559,9 @@ def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
     return {"workload": "gdn_scan_B1_T32768_hk16_hv32_k128_v128_in_8_spans_of_4096",
             "whole_scan_ms": round(whole_ms, 4), "per_rank_ms": round(rank_ms, 4),
             "per_rank_speedup_without_exchange": round(whole_ms / rank_ms, 2),
-            "rank_steps_ms": {"span_scan": round(mean(tr, 0, 1), 4), "span_maps": round(mean(tr, 1, 2), 4),
-                              "seven_combines": round(mean(tr, 2, 3), 4), "correct": round(corr_ms, 4)},
+            "rank_steps_ms": {"span_scan_and_maps": round(mean(tr, 0, 1), 4),
+                              "combine_7_maps": round(mean(tr, 1, 2), 4), "correct": round(corr_ms, 4),
+                              "end_state": round(mean(tr, 3, 4), 4)},
             "exchange": "all-gather of P and S_loc (4 MiB per rank): not measured on one GPU",
             "correct_kernel": {"bound": "alu", "TFLOP/s": round(flop / (corr_ms / 1e3) / 1e12, 2),
                                "peak_TFLOP/s": round(alu_peak, 1),

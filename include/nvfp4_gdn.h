@@ -218,9 +218,9 @@ NVFP4_API nvfp4_status gdn_scan_noalloc(const float* q_hat, const float* k_hat, 
  * with m_t = scale P_t^T q_t (P_t = A_t ... A_1) and o_loc the zero-start
  * outputs.  The pages scan each window in one pass and say nothing about
  * splitting it; this is the plain reading of the recurrence's algebra.
- * Recipe: gdn_scan every span from a zero state (o_loc, S_loc) and
- * gdn_scan_transition every span (P, m), in any order or in parallel; then in
- * span order S_in(next) = gdn_state_combine(P, S_loc, S_in) and
+ * Recipe: gdn_scan_span on every span (its zero-start scan o_loc, S_loc and
+ * its maps P, m; the spans are independent), then for each span its initial
+ * state S_in = gdn_state_combine over the maps of the spans before it, and
  * gdn_scan_correct(m, S_in, o_loc) for every span whose S_in is not zero. */
 
 /* Bytes of workspace gdn_scan_transition needs. */
@@ -239,13 +239,33 @@ NVFP4_API nvfp4_status gdn_scan_transition(const float* q_hat, const float* k_ha
                                            float scale, int32_t form, int32_t algo, float* P, float* qmap,
                                            void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
 
-/* S_out[i] = P[i] S_in[i] + S_loc[i] for i < n (n = spans x value heads):
- * P device float32 [n x K x K]; S_loc, S_in, S_out device float32 [n x K x V].
- * S_in NULL means zero (P is then not read), S_loc NULL means zero.  S_out may
- * be S_loc itself but must not overlap P or S_in.  K, V multiples of 32 in
- * [32, 256]. */
+/* Bytes of workspace gdn_scan_span needs. */
+NVFP4_API size_t gdn_scan_span_workspace_size(int32_t B, int64_t T, const gdn_dims* dims, int32_t algo);
+
+/* One call for a span's independent step: the zero-start scan (o as gdn_scan's
+ * output, S_loc its final state) and the span maps (P, qmap as
+ * gdn_scan_transition's).  With the chunked algorithm and K == V the two share
+ * one chunk preparation (the maps' chunk records are the scan's with the
+ * v-dependent part zeroed); otherwise it runs gdn_scan then
+ * gdn_scan_transition.  Inputs as for gdn_scan; o [B x T x Hv x V], S_loc
+ * [B x Hv x K x V], P [B x Hv x K x K], qmap [B x T x Hv x K], all device
+ * float32, 16-byte aligned, not overlapping each other or the workspace
+ * (256-byte aligned, >= gdn_scan_span_workspace_size bytes). */
+NVFP4_API nvfp4_status gdn_scan_span(const float* q_hat, const float* k_hat, const float* v, int64_t ld_v,
+                                     const float* g, const float* beta, int32_t B, int64_t T, const gdn_dims* dims,
+                                     float scale, int32_t form, int32_t algo, float* o, float* S_loc, float* P,
+                                     float* qmap, void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* The composition of m spans' maps in order, per (sequence, value head) i < n
+ * (n = sequences x value heads):
+ *   S = S_in[i];  S = P[j][i] S + S_loc[j][i] for j = 0 .. m-1;  S_out[i] = S.
+ * P: device float32 [m x n x K x K]; S_loc: device float32 [m x n x K x V]
+ * (NULL: zero); S_in, S_out: device float32 [n x K x V] (S_in NULL: zero).
+ * S_out may be S_in, or the last S_loc (S_loc + (m-1) n K V), and must not
+ * overlap P or any other part of S_loc.  m >= 1; K = 32, 64 or 128; V a
+ * multiple of 32; P 16-byte aligned.  One launch for the whole chain. */
 NVFP4_API nvfp4_status gdn_state_combine(const float* P, const float* S_loc, const float* S_in, float* S_out,
-                                         int64_t n, int32_t K, int32_t V, nvfp4_stream_t stream);
+                                         int32_t m, int64_t n, int32_t K, int32_t V, nvfp4_stream_t stream);
 
 /* o[b,t,h,:] += S_in[b,h]^T qmap[b,t,h,:]: the outputs of B spans of T tokens
  * that started from S_in instead of zero.  qmap: device float32 [B x T x Hv x K]

@@ -20,7 +20,7 @@ from . import build as _build
 __all__ = [
     "NVFP4Error", "NVFP4Matrix", "GdnDims", "LayerWeights", "lib", "nvfp4_quantize", "w4a4_gemm", "gdn_gates",
     "gdn_scan", "gdn_scan_noalloc", "gdn_output_gate", "gdn_short_conv", "gdn_layer_forward", "layer_workspace_layout",
-    "check_device_error", "gdn_scan_transition", "gdn_state_combine", "gdn_scan_correct",
+    "check_device_error", "gdn_scan_transition", "gdn_state_combine", "gdn_scan_correct", "gdn_scan_span",
     "selftest_wait_timeout", "FORM_PAGES",
     "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
 ]
@@ -37,7 +37,7 @@ EXPORTED_SYMBOLS = [
     "nvfp4_quantize_workspace_size", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan_workspace_size",
     "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc", "gdn_output_gate",
     "gdn_short_conv", "gdn_layer_forward_stateful", "gdn_scan_transition_workspace_size", "gdn_scan_transition",
-    "gdn_state_combine", "gdn_scan_correct",
+    "gdn_state_combine", "gdn_scan_correct", "gdn_scan_span_workspace_size", "gdn_scan_span",
 ]
 
 # Size of the fixed scratch array gdn_scan_noalloc uses (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
@@ -110,7 +110,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_scan_transition_workspace_size.argtypes = [i32, i64, DP, i32]
         L.gdn_scan_transition_workspace_size.restype = sz
         L.gdn_scan_transition.argtypes = [P, P, P, P, i32, i64, DP, ctypes.c_float, i32, i32, P, P, P, sz, P]
-        L.gdn_state_combine.argtypes = [P, P, P, P, i64, i32, i32, P]
+        L.gdn_state_combine.argtypes = [P, P, P, P, i32, i64, i32, i32, P]
+        L.gdn_scan_span_workspace_size.argtypes = [i32, i64, DP, i32]
+        L.gdn_scan_span_workspace_size.restype = sz
+        L.gdn_scan_span.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, i32, P, P, P, P, P, sz, P]
         L.gdn_scan_correct.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, P]
         for f in ("nvfp4_check_device_error", "nvfp4_selftest_wait_timeout", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
                   "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc"):
@@ -323,15 +326,40 @@ def gdn_scan_transition(q_hat, k_hat, g, beta, B: int, T: int, dims: GdnDims, sc
 
 
 def gdn_state_combine(P, S_loc, S_in, out=None, stream=None):
-    """P S_in + S_loc per leading index: P [..., K, K], S_loc / S_in [..., K, V]
-    (S_in or S_loc None = zero).  out may be S_loc."""
-    ref = S_loc if S_loc is not None else S_in
-    K, V = ref.shape[-2], ref.shape[-1]
-    n = ref.numel() // (K * V)
+    """The maps of m spans composed in order: S = S_in, then S = P[j] S +
+    S_loc[j] for each j; returns S [B, Hv, K, V].  P [m, B, Hv, K, K] (or
+    [B, Hv, K, K]: one step), S_loc shaped like P with V columns (None = zero),
+    S_in [B, Hv, K, V] (None = zero).  out may be S_in."""
+    B, Hv, K = P.shape[-4], P.shape[-3], P.shape[-1]
+    n = B * Hv
+    m = P.numel() // (n * K * K)
+    V = (S_in if S_in is not None else S_loc).shape[-1]
     if out is None:
-        out = torch.empty_like(ref)
-    _check(lib().gdn_state_combine(_ptr(P), _ptr(S_loc), _ptr(S_in), _ptr(out), n, K, V, _stream(stream)))
+        out = torch.empty((B, Hv, K, V), dtype=torch.float32, device=P.device)
+    _check(lib().gdn_state_combine(_ptr(P), _ptr(S_loc), _ptr(S_in), _ptr(out), m, n, K, V, _stream(stream)))
     return out
+
+
+def gdn_scan_span(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
+                  form: int = FORM_PAGES, algo: int = SCAN_AUTO, workspace=None, stream=None):
+    """A span's zero-start scan and its maps in one call: returns (o [B*T, Hv, V],
+    S_loc [B, Hv, K, V], P [B, Hv, K, K], qmap [B*T, Hv, K])."""
+    dev = q_hat.device
+    if scale is None:
+        scale = 1.0 / math.sqrt(dims.K)
+    f32 = dict(dtype=torch.float32, device=dev)
+    o = torch.empty((B * T, dims.Hv, dims.V), **f32)
+    S_loc = torch.empty((B, dims.Hv, dims.K, dims.V), **f32)
+    P = torch.empty((B, dims.Hv, dims.K, dims.K), **f32)
+    qmap = torch.empty((B * T, dims.Hv, dims.K), **f32)
+    d = dims.c()
+    need = lib().gdn_scan_span_workspace_size(B, T, ctypes.byref(d), algo)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _check(lib().gdn_scan_span(_ptr(q_hat), _ptr(k_hat), _ptr(v), v.stride(0), _ptr(g), _ptr(beta), B, T,
+                               ctypes.byref(d), float(scale), form, algo, _ptr(o), _ptr(S_loc), _ptr(P), _ptr(qmap),
+                               _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, S_loc, P, qmap
 
 
 def gdn_scan_correct(qmap, S_in, o, B: int, T: int, amax_word=None, stream=None):

@@ -21,11 +21,15 @@
 //    Q K^T and G; kernel 2 (one CTA per head x 32-column V slice) walks the
 //    chunks in order.  Products run on the tensor cores in TF32 with float32
 //    accumulation (mma.sync m16n8k8).
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
 
 namespace nvg {
+
+nvfp4_status identity_fill_launch(float* P, int64_t n_mat, int K, float* zero_row, int64_t n_zero, cudaStream_t st);
+size_t transition_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo);
 
 namespace {
 
@@ -139,16 +143,6 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------ chunk preparation --
@@ -890,6 +884,48 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     return NVFP4_OK;
 }
 
+// Zero the U~ sections of n_rec records: only U~ = T diag(beta) V depends on v,
+// so the records become those of the same span with v = 0.
+template <int K, int V>
+__global__ void __launch_bounds__(256) zero_ut_kernel(uint8_t* __restrict__ recs, int64_t n_rec) {
+    pdl_wait_and_trigger();
+    using RC = ChunkRec<K, V>;
+    constexpr int64_t per = static_cast<int64_t>(V / 32) * RC::UT_SLICE / 16;   // 16-byte words per record
+    const int64_t total = n_rec * per;
+    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = e / per, i = e - r * per;
+        reinterpret_cast<float4*>(recs + r * RC::BYTES + RC::UT)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// One span's zero-start scan (o, S_loc) and its maps (P, qmap) with one chunk
+// preparation: the sequential kernel runs on the records as prepared, then on
+// the same records with U~ zeroed, from P = I (K == V only).
+template <int K>
+nvfp4_status launch_span_chunked(const float* q, const float* k, const float* v, int64_t ld_v, const float* g,
+                                 const float* beta, int B, int64_t T, const gdn_dims& d, float scale, int form,
+                                 float* o, float* S_loc, float* P, float* qmap, void* ws, cudaStream_t st) {
+    nvfp4_status s = launch_chunked_kv<K, K>(q, k, v, ld_v, g, beta, B, T, d, scale, form, nullptr, S_loc, o, ws,
+                                             nullptr, static_cast<int64_t>(d.Hk) * K, 0, st);
+    if (s != NVFP4_OK) return s;
+    const int NC = static_cast<int>((T + CH - 1) / CH);
+    const int64_t n_rec = static_cast<int64_t>(B) * d.Hv * NC;
+    uint8_t* recs = static_cast<uint8_t*>(ws);
+    const int64_t words = n_rec * (K / 32) * ChunkRec<K, K>::UT_SLICE / 16;
+    const unsigned zb = static_cast<unsigned>(std::min<int64_t>((words + 255) / 256, int64_t(num_sms()) * 8));
+    cudaError_t e = launch_pdl(zero_ut_kernel<K, K>, dim3(zb), dim3(256), 0, st, recs, n_rec);
+    if (e != cudaSuccess) return cuda_fail(e, "record U~ zero launch");
+    if ((s = identity_fill_launch(P, static_cast<int64_t>(B) * d.Hv, K, nullptr, 0, st)) != NVFP4_OK) return s;
+    unsigned int* err = device_error_word();
+    if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
+    e = launch_pdl(chunk_seq_kernel<K, K>, dim3(static_cast<unsigned>(B * d.Hv * (K / 32))), dim3(kSeqThreads),
+                   static_cast<int>(SeqLayout<K>::BYTES), st, recs, T, d.Hv, scale, NC, P, P, qmap,
+                   static_cast<unsigned int*>(nullptr), err);
+    if (e != cudaSuccess) return cuda_fail(e, "chunked scan launch");
+    return NVFP4_OK;
+}
+
 size_t chunk_rec_bytes(const gdn_dims& d) {
     if (d.K == 128 && d.V == 128) return ChunkRec<128, 128>::BYTES;
     if (d.K == 128 && d.V == 64) return ChunkRec<128, 64>::BYTES;
@@ -962,4 +998,66 @@ extern "C" nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const f
         return fail(NVFP4_ERR_WORKSPACE, "scan workspace missing, too small or not 256-byte aligned");
     return scan_launch(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, algo, state_in, state_out, o,
                        workspace, as_stream(stream), nullptr, static_cast<int64_t>(dims->Hk) * dims->K, 0);
+}
+
+extern "C" size_t gdn_scan_span_workspace_size(int32_t B, int64_t T, const gdn_dims* dims, int32_t algo) {
+    if (!dims || nvg::validate_dims(dims) != NVFP4_OK || B < 1 || T < 1) return 0;
+    return std::max(nvg::scan_workspace_bytes(B, T, *dims, algo), nvg::transition_workspace_bytes(B, T, *dims, algo));
+}
+
+extern "C" nvfp4_status gdn_scan_span(const float* q_hat, const float* k_hat, const float* v, int64_t ld_v,
+                                      const float* g, const float* beta, int32_t B, int64_t T, const gdn_dims* dims,
+                                      float scale, int32_t form, int32_t algo, float* o, float* S_loc, float* P,
+                                      float* qmap, void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+    using namespace nvg;
+    nvfp4_status s = validate_dims(dims);
+    if (s != NVFP4_OK) return s;
+    if (!q_hat || !k_hat || !v || !g || !beta || !o || !S_loc || !P || !qmap)
+        return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+    if (B < 1 || T < 1) return fail(NVFP4_ERR_INVALID_ARG, "B and T must be >= 1");
+    if (form != GDN_FORM_PAGES && form != GDN_FORM_STANDARD) return fail(NVFP4_ERR_INVALID_ARG, "bad form");
+    if (algo != GDN_SCAN_AUTO && algo != GDN_SCAN_RECURRENT && algo != GDN_SCAN_CHUNKED)
+        return fail(NVFP4_ERR_INVALID_ARG, "bad algo");
+    if (ld_v < static_cast<int64_t>(dims->Hv) * dims->V) return fail(NVFP4_ERR_INVALID_ARG, "ld_v < Hv*V");
+    if (static_cast<int64_t>(B) * T > (int64_t(1) << 31)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "B*T too large");
+    if (!aligned16(q_hat) || !aligned16(k_hat) || !aligned16(v) || ld_v % 4 || !aligned16(o) || !aligned16(S_loc) ||
+        !aligned16(P) || !aligned16(qmap))
+        return fail(NVFP4_ERR_MISALIGNED, "pointers must be 16-byte aligned and ld_v % 4 == 0");
+    const size_t need = std::max(scan_workspace_bytes(B, T, *dims, algo), transition_workspace_bytes(B, T, *dims, algo));
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return fail(NVFP4_ERR_WORKSPACE, "span workspace missing, too small or not 256-byte aligned");
+    const size_t nbytes[5] = {static_cast<size_t>(B) * T * dims->Hv * dims->V * 4,
+                              static_cast<size_t>(B) * dims->Hv * dims->K * dims->V * 4,
+                              static_cast<size_t>(B) * dims->Hv * dims->K * dims->K * 4,
+                              static_cast<size_t>(B) * T * dims->Hv * dims->K * 4, need};
+    const char* ptrs[5] = {reinterpret_cast<const char*>(o), reinterpret_cast<const char*>(S_loc),
+                           reinterpret_cast<const char*>(P), reinterpret_cast<const char*>(qmap),
+                           static_cast<const char*>(workspace)};
+    for (int i = 0; i < 5; ++i)
+        for (int j = i + 1; j < 5; ++j)
+            if (ptrs[i] < ptrs[j] + nbytes[j] && ptrs[j] < ptrs[i] + nbytes[i])
+                return fail(NVFP4_ERR_INVALID_ARG, "o, S_loc, P, qmap and the workspace must not overlap");
+    const cudaStream_t st = as_stream(stream);
+    const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
+    const int64_t ld_qk = static_cast<int64_t>(dims->Hk) * dims->K;
+    if (chunked && dims->K == dims->V) {
+        if (dims->K == 128)
+            return launch_span_chunked<128>(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, o, S_loc, P,
+                                            qmap, workspace, st);
+        return launch_span_chunked<64>(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, o, S_loc, P, qmap,
+                                       workspace, st);
+    }
+    // the zero-start scan, then the maps (the scan on v = 0 from P = I with V = K) in the same workspace
+    if ((s = scan_launch(q_hat, k_hat, v, ld_v, g, beta, B, T, *dims, scale, form, algo, nullptr, S_loc, o,
+                         workspace, st, nullptr, ld_qk, 0)) != NVFP4_OK)
+        return s;
+    gdn_dims dk = *dims;
+    dk.V = dims->K;
+    const size_t zero_off = (scan_workspace_bytes(B, T, dk, algo) + 255) / 256 * 256;
+    float* zero_row = reinterpret_cast<float*>(static_cast<char*>(workspace) + zero_off);
+    if ((s = identity_fill_launch(P, static_cast<int64_t>(B) * dims->Hv, dims->K, zero_row,
+                                  static_cast<int64_t>(dims->Hv) * dims->K, st)) != NVFP4_OK)
+        return s;
+    return scan_launch(q_hat, k_hat, zero_row, 0, g, beta, B, T, dk, scale, form, algo, P, P, qmap, workspace, st,
+                       nullptr, ld_qk, 0);
 }

@@ -14,7 +14,8 @@
 //   gdn_scan_transition   P and m of a span: the chunked (or one-token) scan
 //                         run on v = 0 from S_in = I with V = K, so P is its
 //                         final state and m its output;
-//   gdn_state_combine     S_out = P S_in + S_loc per (sequence, value head);
+//   gdn_state_combine     S_out = P S_in + S_loc per (sequence, value head),
+//                         or a chain of m such steps in one launch;
 //   gdn_scan_correct      o_t += S_in^T m_t over a span's tokens, with the
 //                         quantiser's amax of the corrected o folded in.
 #include <algorithm>
@@ -49,130 +50,188 @@ __global__ void __launch_bounds__(256) identity_fill_kernel(float* __restrict__ 
         zero_row[e] = 0.0f;
 }
 
-// S_out[n] = P[n] S_in[n] + S_loc[n].  One CTA per (n, 32 rows of the output);
-// warp w owns rows 4w..4w+3 of the block, lane l the columns l + 32c.  The 32
-// rows of P sit in shared memory and are read as broadcasts; the rows of S_in
-// are read coalesced (the CTAs of one n share them through L1/L2).
-constexpr int kCombRows = 32;
-__global__ void __launch_bounds__(256) state_combine_kernel(const float* __restrict__ P,
-                                                            const float* S_loc,
-                                                            const float* __restrict__ S_in, float* S_out,
-                                                            int K, int V) {
+// The chain S = S_in; S = P[j] S + S_loc[j] for j = 0..m-1; S_out = S, per
+// (sequence, value head) n.  The columns of S evolve independently, so one CTA
+// per (n, 32 columns) carries its K x 32 slice through the whole chain in
+// shared memory; each step stages P[j][n] (K x K) in shared memory, warp w owns
+// rows w + 8r and lane l column c0 + l, and P is read as warp-wide broadcasts.
+template <int K>
+__global__ void __launch_bounds__(256) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
+                                                          const float* S_in, float* S_out, int m, int64_t n_total,
+                                                          int V) {
     pdl_wait_and_trigger();
-    __shared__ float Ps[kCombRows][256];
+    constexpr int R = K / 8;
+    extern __shared__ __align__(16) float smem[];
+    float* Ps = smem;            // [K][K]
+    float* Ss = smem + K * K;    // [K][32]
     const int64_t n = blockIdx.x;
-    const int i0 = blockIdx.y * kCombRows;
+    const int c0 = blockIdx.y * 32;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int VC = V >> 5;
-    float acc[4][8];
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
-    if (S_in) {
-        const float* Pn = P + n * K * K;
-        for (int e = threadIdx.x; e < kCombRows * K; e += blockDim.x) Ps[e / K][e % K] = Pn[static_cast<int64_t>(i0 + e / K) * K + e % K];
+    for (int i = w; i < K; i += 8)
+        Ss[i * 32 + lane] = S_in ? S_in[(n * K + i) * V + c0 + lane] : 0.0f;
+    for (int j = 0; j < m; ++j) {
+        const float4* Pj = reinterpret_cast<const float4*>(P + (static_cast<int64_t>(j) * n_total + n) * K * K);
+        __syncthreads();   // the slice is written; the previous step's P is no longer read
+        for (int e = threadIdx.x; e < K * K / 4; e += 256) reinterpret_cast<float4*>(Ps)[e] = Pj[e];
         __syncthreads();
-        const float* Sn = S_in + n * K * V;
-        for (int l = 0; l < K; ++l) {
-            float s[8];
+        float acc[R];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) s[c] = c < VC ? Sn[static_cast<int64_t>(l) * V + lane + 32 * c] : 0.0f;
+        for (int r = 0; r < R; ++r) acc[r] = 0.0f;
+#pragma unroll 2
+        for (int l = 0; l < K; l += 4) {
+            const float s0 = Ss[(l + 0) * 32 + lane], s1 = Ss[(l + 1) * 32 + lane];
+            const float s2 = Ss[(l + 2) * 32 + lane], s3 = Ss[(l + 3) * 32 + lane];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float p = Ps[4 * w + r][l];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(p, s[c], acc[r][c]);
+            for (int r = 0; r < R; ++r) {
+                const float4 p = *reinterpret_cast<const float4*>(Ps + (w + 8 * r) * K + l);
+                acc[r] = fmaf(p.x, s0, acc[r]);
+                acc[r] = fmaf(p.y, s1, acc[r]);
+                acc[r] = fmaf(p.z, s2, acc[r]);
+                acc[r] = fmaf(p.w, s3, acc[r]);
             }
         }
-    }
+        __syncthreads();   // every warp has read the old slice
+        const float* Lj = S_loc ? S_loc + (static_cast<int64_t>(j) * n_total + n) * K * V : nullptr;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int64_t row = n * K * V + static_cast<int64_t>(i0 + 4 * w + r) * V;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            if (c < VC) {
-                const int64_t e = row + lane + 32 * c;
-                S_out[e] = acc[r][c] + (S_loc ? S_loc[e] : 0.0f);
-            }
+        for (int r = 0; r < R; ++r) {
+            const int i = w + 8 * r;
+            Ss[i * 32 + lane] = acc[r] + (Lj ? Lj[static_cast<int64_t>(i) * V + c0 + lane] : 0.0f);
+        }
     }
+    __syncthreads();
+    for (int i = w; i < K; i += 8) S_out[(n * K + i) * V + c0 + lane] = Ss[i * 32 + lane];
 }
 
-// o[b,t,h,:] += S_in[b,h]^T m[b,t,h,:] over a tile of 64 tokens of one (b, h).
-// S_in[b,h] (K x V) and the tile's m rows (64 x K) are staged in shared memory;
-// thread (ty, tx) of a 16 x 16 grid owns tokens 4ty..4ty+3 and the columns
-// 4tx + 64c .. +3 (c < V/64), so each step over 4 values of k takes 4 + 4 V/64
-// 16-byte shared loads for 64 V/64 FMAs.  The largest |o| of the CTA goes into
-// the quantiser's amax word with one atomicMax.
-constexpr int kCorrTok = 64;
+template <int K>
+nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in, float* S_out, int m, int64_t n,
+                          int V, cudaStream_t st) {
+    constexpr int smem = (K * K + K * 32) * 4;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(state_chain_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chain)");
+        attr_done[dev] = true;
+    }
+    const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / 32), dim3(256), smem,
+                                     st, P, S_loc, S_in, S_out, m, n, V);
+    if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
+    return NVFP4_OK;
+}
+
+// o[b,t,h,:] += S_in[b,h]^T m[b,t,h,:].  The work is a list of items (b, h,
+// tile of 32 tokens) in that order; each CTA takes a contiguous run of items,
+// so it stages S_in[b,h] (K x V) in shared memory once per head it meets.  The
+// m rows of the next item are copied asynchronously (double buffer) while the
+// current item computes, and each thread loads its o values before the k loop.
+// Thread (ty, tx) of a 16 x 16 grid owns tokens 2ty, 2ty+1 and the columns
+// 4tx + 64c .. +3 (c < V/64).  The largest |o| of the CTA goes into the
+// quantiser's amax word with one atomicMax.
+constexpr int kCorrTok = 32;
 template <int K, int V>
-__global__ void __launch_bounds__(256) scan_correct_kernel(const float* __restrict__ m, const float* __restrict__ S_in,
-                                                           float* __restrict__ o, int64_t T, int Hv,
-                                                           unsigned int* __restrict__ o_amax) {
+__global__ void __launch_bounds__(256, 2) scan_correct_kernel(const float* __restrict__ m,
+                                                              const float* __restrict__ S_in, float* __restrict__ o,
+                                                              int64_t T, int Hv, int64_t n_items, int per_cta,
+                                                              unsigned int* __restrict__ o_amax) {
     pdl_wait_and_trigger();
     constexpr int VC = V / 64;
     extern __shared__ __align__(16) float smem[];
     float* Ss = smem;              // [K][V]
-    float* Ms = smem + K * V;      // [kCorrTok][K]
-    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kCorrTok;
-    const int h = blockIdx.y, b = blockIdx.z;
-    const float4* S4 = reinterpret_cast<const float4*>(S_in + (static_cast<int64_t>(b) * Hv + h) * K * V);
-    for (int e = threadIdx.x; e < K * V / 4; e += 256) reinterpret_cast<float4*>(Ss)[e] = S4[e];
-    for (int e = threadIdx.x; e < kCorrTok * K / 4; e += 256) {
-        const int r = e / (K / 4), c4 = e % (K / 4);
-        const int64_t t = t0 + r;
-        reinterpret_cast<float4*>(Ms)[e] =
-            t < T ? *reinterpret_cast<const float4*>(m + ((static_cast<int64_t>(b) * T + t) * Hv + h) * K + 4 * c4)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
+    float* Mb = smem + K * V;      // [2][kCorrTok][K]
+    const int64_t tiles = (T + kCorrTok - 1) / kCorrTok;
+    const int64_t i0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+    const int64_t i1 = i0 + per_cta < n_items ? i0 + per_cta : n_items;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][4 * VC];
+    float mx = 0.0f;
+    if (i0 < i1) {
+        auto stage_S = [&](int64_t bh) {
+            const float4* S4 = reinterpret_cast<const float4*>(S_in + bh * K * V);
+            for (int e = threadIdx.x; e < K * V / 4; e += 256) reinterpret_cast<float4*>(Ss)[e] = S4[e];
+        };
+        auto issue_m = [&](int64_t item, int buf) {
+            const int64_t bh = item / tiles, t0 = (item - bh * tiles) * kCorrTok;
+            const int64_t b = bh / Hv, h = bh - b * Hv;
+            float* dst = Mb + buf * kCorrTok * K;
+            for (int e = threadIdx.x; e < kCorrTok * K / 4; e += 256) {
+                const int r = e / (K / 4), c4 = e - r * (K / 4);
+                const int64_t t = t0 + r;
+                const bool valid = t < T;
+                cp_async16(dst + 4 * e, valid ? m + ((b * T + t) * Hv + h) * K + 4 * c4 : m, valid);
+            }
+            cp_async_commit();
+        };
+        int64_t cur_bh = i0 / tiles;
+        stage_S(cur_bh);
+        issue_m(i0, 0);
+        for (int64_t it = i0; it < i1; ++it) {
+            const int buf = static_cast<int>((it - i0) & 1);
+            if (it + 1 < i1) issue_m(it + 1, buf ^ 1);
+            else cp_async_commit();                    // one group per iteration
+            cp_async_wait<1>();                          // this item's rows have landed
+            __syncthreads();
+            const int64_t bh = it / tiles, t0 = (it - bh * tiles) * kCorrTok;
+            const int64_t b = bh / Hv, h = bh - b * Hv;
+            float4 ov[2][VC];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 2; ++r) {
+                const int64_t t = t0 + 2 * ty + r;
 #pragma unroll
-        for (int c = 0; c < 4 * VC; ++c) acc[r][c] = 0.0f;
-#pragma unroll 2
-    for (int kk = 0; kk < K; kk += 4) {
-        float4 a[4];
+                for (int c = 0; c < VC; ++c)
+                    ov[r][c] = t < T ? *reinterpret_cast<const float4*>(o + ((b * T + t) * Hv + h) * V + 4 * tx + 64 * c)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            const float* Ms = Mb + buf * kCorrTok * K;
+            float acc[2][4 * VC];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) a[r] = *reinterpret_cast<const float4*>(Ms + (4 * ty + r) * K + kk);
+            for (int r = 0; r < 2; ++r)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float4 s[VC];
+                for (int c = 0; c < 4 * VC; ++c) acc[r][c] = 0.0f;
+#pragma unroll 4
+            for (int kk = 0; kk < K; kk += 4) {
+                const float4 a0 = *reinterpret_cast<const float4*>(Ms + (2 * ty) * K + kk);
+                const float4 a1 = *reinterpret_cast<const float4*>(Ms + (2 * ty + 1) * K + kk);
 #pragma unroll
-            for (int c = 0; c < VC; ++c) s[c] = *reinterpret_cast<const float4*>(Ss + (kk + q) * V + 4 * tx + 64 * c);
+                for (int q = 0; q < 4; ++q) {
+                    const float x0 = q == 0 ? a0.x : q == 1 ? a0.y : q == 2 ? a0.z : a0.w;
+                    const float x1 = q == 0 ? a1.x : q == 1 ? a1.y : q == 2 ? a1.z : a1.w;
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float av = q == 0 ? a[r].x : q == 1 ? a[r].y : q == 2 ? a[r].z : a[r].w;
-#pragma unroll
-                for (int c = 0; c < VC; ++c) {
-                    acc[r][4 * c + 0] = fmaf(av, s[c].x, acc[r][4 * c + 0]);
-                    acc[r][4 * c + 1] = fmaf(av, s[c].y, acc[r][4 * c + 1]);
-                    acc[r][4 * c + 2] = fmaf(av, s[c].z, acc[r][4 * c + 2]);
-                    acc[r][4 * c + 3] = fmaf(av, s[c].w, acc[r][4 * c + 3]);
+                    for (int c = 0; c < VC; ++c) {
+                        const float4 sv = *reinterpret_cast<const float4*>(Ss + (kk + q) * V + 4 * tx + 64 * c);
+                        acc[0][4 * c + 0] = fmaf(x0, sv.x, acc[0][4 * c + 0]);
+                        acc[0][4 * c + 1] = fmaf(x0, sv.y, acc[0][4 * c + 1]);
+                        acc[0][4 * c + 2] = fmaf(x0, sv.z, acc[0][4 * c + 2]);
+                        acc[0][4 * c + 3] = fmaf(x0, sv.w, acc[0][4 * c + 3]);
+                        acc[1][4 * c + 0] = fmaf(x1, sv.x, acc[1][4 * c + 0]);
+                        acc[1][4 * c + 1] = fmaf(x1, sv.y, acc[1][4 * c + 1]);
+                        acc[1][4 * c + 2] = fmaf(x1, sv.z, acc[1][4 * c + 2]);
+                        acc[1][4 * c + 3] = fmaf(x1, sv.w, acc[1][4 * c + 3]);
+                    }
                 }
             }
-        }
-    }
-    float mx = 0.0f;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int64_t t = t0 + 4 * ty + r;
-        if (t < T) {
-            float* orow = o + ((static_cast<int64_t>(b) * T + t) * Hv + h) * V;
+            for (int r = 0; r < 2; ++r) {
+                const int64_t t = t0 + 2 * ty + r;
+                if (t < T) {
 #pragma unroll
-            for (int c = 0; c < VC; ++c) {
-                float4* p = reinterpret_cast<float4*>(orow + 4 * tx + 64 * c);
-                float4 x = *p;
-                x.x += acc[r][4 * c + 0];
-                x.y += acc[r][4 * c + 1];
-                x.z += acc[r][4 * c + 2];
-                x.w += acc[r][4 * c + 3];
-                *p = x;
-                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+                    for (int c = 0; c < VC; ++c) {
+                        float4 x = ov[r][c];
+                        x.x += acc[r][4 * c + 0];
+                        x.y += acc[r][4 * c + 1];
+                        x.z += acc[r][4 * c + 2];
+                        x.w += acc[r][4 * c + 3];
+                        *reinterpret_cast<float4*>(o + ((b * T + t) * Hv + h) * V + 4 * tx + 64 * c) = x;
+                        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+                    }
+                }
+            }
+            __syncthreads();                             // this item's rows and S are no longer read
+            if (it + 1 < i1 && (it + 1) / tiles != cur_bh) {
+                cur_bh = (it + 1) / tiles;
+                stage_S(cur_bh);                         // visible after the next iteration's barrier
             }
         }
+        cp_async_wait<0>();
     }
     if (o_amax) {
         __shared__ unsigned int wmax[8];
@@ -191,7 +250,7 @@ __global__ void __launch_bounds__(256) scan_correct_kernel(const float* __restri
 template <int K, int V>
 nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, int64_t T, int Hv,
                             unsigned int* o_amax, cudaStream_t st) {
-    constexpr int smem = (K * V + kCorrTok * K) * 4;
+    constexpr int smem = (K * V + 2 * kCorrTok * K) * 4;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -200,8 +259,12 @@ nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, 
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(correct)");
         attr_done[dev] = true;
     }
-    const dim3 grid(static_cast<unsigned>((T + kCorrTok - 1) / kCorrTok), Hv, B);
-    const cudaError_t e = launch_pdl(scan_correct_kernel<K, V>, grid, dim3(256), smem, st, m, S_in, o, T, Hv, o_amax);
+    const int64_t n_items = static_cast<int64_t>(B) * Hv * ((T + kCorrTok - 1) / kCorrTok);
+    const int64_t slots = int64_t(num_sms()) * 2;
+    const int per_cta = static_cast<int>((n_items + slots - 1) / slots);
+    const unsigned grid = static_cast<unsigned>((n_items + per_cta - 1) / per_cta);
+    const cudaError_t e = launch_pdl(scan_correct_kernel<K, V>, dim3(grid), dim3(256), smem, st, m, S_in, o, T, Hv,
+                                     n_items, per_cta, o_amax);
     if (e != cudaSuccess) return cuda_fail(e, "scan correct launch");
     return NVFP4_OK;
 }
@@ -213,6 +276,15 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 }  // namespace
+
+nvfp4_status identity_fill_launch(float* P, int64_t n_mat, int K, float* zero_row, int64_t n_zero,
+                                  cudaStream_t st) {
+    const int64_t total = n_mat * K * K;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, int64_t(num_sms()) * 8));
+    const cudaError_t e = launch_pdl(identity_fill_kernel, dim3(blocks), dim3(256), 0, st, P, n_mat, K, zero_row, n_zero);
+    if (e != cudaSuccess) return cuda_fail(e, "identity fill launch");
+    return NVFP4_OK;
+}
 
 size_t transition_workspace_bytes(int B, int64_t T, const gdn_dims& d, int algo) {
     gdn_dims dk = d;
@@ -255,35 +327,35 @@ extern "C" nvfp4_status gdn_scan_transition(const float* q_hat, const float* k_h
     const size_t zero_off = round_up(scan_workspace_bytes(B, T, dk, algo));
     float* zero_row = reinterpret_cast<float*>(static_cast<char*>(workspace) + zero_off);
     const cudaStream_t st = as_stream(stream);
-    const int64_t n_mat = static_cast<int64_t>(B) * dims->Hv;
-    const int64_t total = n_mat * dims->K * dims->K;
-    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, int64_t(num_sms()) * 8));
-    const cudaError_t e = launch_pdl(identity_fill_kernel, dim3(blocks), dim3(256), 0, st, P, n_mat, dims->K, zero_row,
-                                     static_cast<int64_t>(dims->Hv) * dims->K);
-    if (e != cudaSuccess) return cuda_fail(e, "identity fill launch");
+    if ((s = identity_fill_launch(P, static_cast<int64_t>(B) * dims->Hv, dims->K, zero_row,
+                                  static_cast<int64_t>(dims->Hv) * dims->K, st)) != NVFP4_OK)
+        return s;
     // v = 0 (every token reads the same zero row: row stride 0), state P in place
     return scan_launch(q_hat, k_hat, zero_row, 0, g, beta, B, T, dk, scale, form, algo, P, P, qmap, workspace, st,
                        nullptr, static_cast<int64_t>(dims->Hk) * dims->K, 0);
 }
 
 extern "C" nvfp4_status gdn_state_combine(const float* P, const float* S_loc, const float* S_in, float* S_out,
-                                          int64_t n, int32_t K, int32_t V, nvfp4_stream_t stream) {
+                                          int32_t m, int64_t n, int32_t K, int32_t V, nvfp4_stream_t stream) {
     using namespace nvg;
-    if (!S_out || (S_in && !P)) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
-    if (n < 1) return fail(NVFP4_ERR_INVALID_ARG, "n must be >= 1");
-    if (K < 32 || K > 256 || K % 32 || V < 32 || V > 256 || V % 32)
-        return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K and V must be multiples of 32 in [32, 256]");
+    if (!S_out || !P) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+    if (m < 1 || n < 1) return fail(NVFP4_ERR_INVALID_ARG, "m and n must be >= 1");
+    if ((K != 32 && K != 64 && K != 128) || V < 32 || V % 32 || V / 32 > 65535)
+        return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be 32, 64 or 128 and V a multiple of 32");
     if (n > 2147483647) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "n too large");
+    if (!aligned16(P)) return fail(NVFP4_ERR_MISALIGNED, "P must be 16-byte aligned");
     const size_t s_bytes = static_cast<size_t>(n) * K * V * 4;
-    const size_t p_bytes = static_cast<size_t>(n) * K * K * 4;
-    if (overlaps(S_out, s_bytes, S_in, s_bytes) || overlaps(S_out, s_bytes, P, p_bytes))
-        return fail(NVFP4_ERR_INVALID_ARG, "S_out must not overlap P or S_in");
-    if (S_loc && S_loc != S_out && overlaps(S_out, s_bytes, S_loc, s_bytes))
-        return fail(NVFP4_ERR_INVALID_ARG, "S_out must be S_loc or not overlap it");
-    const cudaError_t e = launch_pdl(state_combine_kernel, dim3(static_cast<unsigned>(n), K / kCombRows), dim3(256), 0,
-                                     as_stream(stream), P, S_loc, S_in, S_out, K, V);
-    if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
-    return NVFP4_OK;
+    const size_t p_bytes = static_cast<size_t>(m) * n * K * K * 4;
+    if (overlaps(S_out, s_bytes, P, p_bytes)) return fail(NVFP4_ERR_INVALID_ARG, "S_out must not overlap P");
+    if (S_in && S_in != S_out && overlaps(S_out, s_bytes, S_in, s_bytes))
+        return fail(NVFP4_ERR_INVALID_ARG, "S_out must be S_in or not overlap it");
+    const float* last = S_loc ? S_loc + static_cast<int64_t>(m - 1) * n * K * V : nullptr;
+    if (S_loc && S_out != last && overlaps(S_out, s_bytes, S_loc, static_cast<size_t>(m) * s_bytes))
+        return fail(NVFP4_ERR_INVALID_ARG, "S_out must be the last S_loc or not overlap S_loc");
+    const cudaStream_t st = as_stream(stream);
+    if (K == 128) return launch_chain<128>(P, S_loc, S_in, S_out, m, n, V, st);
+    if (K == 64) return launch_chain<64>(P, S_loc, S_in, S_out, m, n, V, st);
+    return launch_chain<32>(P, S_loc, S_in, S_out, m, n, V, st);
 }
 
 extern "C" nvfp4_status gdn_scan_correct(const float* qmap, const float* S_in, float* o, int32_t B, int64_t T,

@@ -15,11 +15,11 @@ o_loc, S_loc: its zero-start scan).  Per rank:
 4. correct the outputs, o = o_loc + S_in^T m, and form the state at the end of
    the span, P S_in + S_loc (the last rank's is the sequence's final state).
 
-The compute steps are the library's kernels (``gdn_scan``,
-``gdn_scan_transition``, ``gdn_state_combine``, ``gdn_scan_correct``);
+The compute steps are the library's kernels (``gdn_scan_span`` for step 1,
+``gdn_state_combine`` for step 3 in one launch, ``gdn_scan_correct``);
 torch.distributed carries the exchange.  ``ops`` lets the host logic run
-against another implementation of the four steps (the multi-rank CPU tests
-use it); the default is the CUDA library and nothing else.
+against another implementation of the steps (the multi-rank CPU tests use
+it); the default is the CUDA library and nothing else.
 """
 from __future__ import annotations
 
@@ -28,27 +28,22 @@ from dataclasses import dataclass
 import torch
 import torch.distributed as dist
 
-from . import (FORM_PAGES, SCAN_AUTO, GdnDims, gdn_scan, gdn_scan_correct, gdn_scan_transition,
-               gdn_state_combine)
+from . import FORM_PAGES, SCAN_AUTO, GdnDims, gdn_scan_correct, gdn_scan_span, gdn_state_combine
 
 
 class CudaSpanOps:
-    """The four steps on the GPU, through the C-ABI library."""
+    """The steps on the GPU, through the C-ABI library."""
 
     def __init__(self, algo: int = SCAN_AUTO, stream=None):
         self.algo, self.stream = algo, stream
 
-    def scan(self, q_hat, k_hat, v, g, beta, B, T, dims, scale, form):
-        S_loc = torch.empty((B, dims.Hv, dims.K, dims.V), dtype=torch.float32, device=q_hat.device)
-        o, _ = gdn_scan(q_hat, k_hat, v, g, beta, B, T, dims, scale=scale, form=form, algo=self.algo,
-                        state_out=S_loc, stream=self.stream)
-        return o, S_loc
-
-    def transition(self, q_hat, k_hat, g, beta, B, T, dims, scale, form):
-        return gdn_scan_transition(q_hat, k_hat, g, beta, B, T, dims, scale=scale, form=form, algo=self.algo,
-                                   stream=self.stream)
+    def local(self, q_hat, k_hat, v, g, beta, B, T, dims, scale, form):
+        """Zero-start scan and span maps, one chunk preparation (gdn_scan_span)."""
+        return gdn_scan_span(q_hat, k_hat, v, g, beta, B, T, dims, scale=scale, form=form, algo=self.algo,
+                             stream=self.stream)
 
     def combine(self, P, S_loc, S_in):
+        """P [m, B, Hv, K, K], S_loc [m, B, Hv, K, V]: the m maps in order, one launch."""
         return gdn_state_combine(P, S_loc, S_in, stream=self.stream)
 
     def correct(self, qmap, S_in, o, B, T):
@@ -68,23 +63,22 @@ def span_local(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: f
                form: int = FORM_PAGES, ops=None) -> SpanLocal:
     """Step 1: the span's zero-start scan and its maps."""
     ops = ops or CudaSpanOps()
-    o, S_loc = ops.scan(q_hat, k_hat, v, g, beta, B, T, dims, scale, form)
-    P, qmap = ops.transition(q_hat, k_hat, g, beta, B, T, dims, scale, form)
-    return SpanLocal(o, S_loc, P, qmap)
+    return SpanLocal(*ops.local(q_hat, k_hat, v, g, beta, B, T, dims, scale, form))
 
 
 def span_join(local: SpanLocal, P_before, S_loc_before, B: int, T: int, state_in=None, ops=None):
     """Steps 3 and 4 for one span, given the maps of the spans before it in
-    order (lists, possibly empty) and the sequence's initial state (None =
-    zero).  Returns (o, state at the end of the span)."""
+    order, stacked (P_before [m, B, Hv, K, K], S_loc_before [m, B, Hv, K, V];
+    None or m = 0 when it is the first span), and the sequence's initial state
+    (None = zero).  Returns (o, state at the end of the span)."""
     ops = ops or CudaSpanOps()
     S_in = state_in
-    for P_r, S_r in zip(P_before, S_loc_before):
-        S_in = ops.combine(P_r, S_r, S_in)
+    if P_before is not None and len(P_before):
+        S_in = ops.combine(P_before, S_loc_before, S_in)
     o = local.o
     if S_in is not None:
         o = ops.correct(local.qmap, S_in, o, B, T)
-    return o, ops.combine(local.P, local.S_loc, S_in)
+    return o, ops.combine(local.P[None], local.S_loc[None], S_in)
 
 
 def sequence_parallel_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDims, scale: float | None = None,
@@ -100,12 +94,12 @@ def sequence_parallel_scan(q_hat, k_hat, v, g, beta, B: int, T: int, dims: GdnDi
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     local = span_local(q_hat, k_hat, v, g, beta, B, T, dims, scale, form, ops)
     if world == 1:
-        return span_join(local, [], [], B, T, state_in, ops)
-    Ps = [torch.empty_like(local.P) for _ in range(world)]
-    Ss = [torch.empty_like(local.S_loc) for _ in range(world)]
-    dist.all_gather(Ps, local.P.contiguous(), group=group)
-    dist.all_gather(Ss, local.S_loc.contiguous(), group=group)
-    return span_join(local, Ps[:rank], Ss[:rank], B, T, state_in, ops)
+        return span_join(local, None, None, B, T, state_in, ops)
+    P_all = torch.empty((world,) + tuple(local.P.shape), dtype=local.P.dtype, device=local.P.device)
+    S_all = torch.empty((world,) + tuple(local.S_loc.shape), dtype=local.S_loc.dtype, device=local.S_loc.device)
+    dist.all_gather(list(P_all.unbind(0)), local.P.contiguous(), group=group)
+    dist.all_gather(list(S_all.unbind(0)), local.S_loc.contiguous(), group=group)
+    return span_join(local, P_all[:rank], S_all[:rank], B, T, state_in, ops)
 
 
 def segmented_scan(spans, B: int, dims: GdnDims, scale: float | None = None, form: int = FORM_PAGES,
@@ -118,6 +112,6 @@ def segmented_scan(spans, B: int, dims: GdnDims, scale: float | None = None, for
     locals_ = [span_local(q, k, v, g, b, B, T, dims, scale, form, ops) for (q, k, v, g, b, T) in spans]
     outs, S = [], state_in
     for loc, span in zip(locals_, spans):
-        o, S = span_join(loc, [], [], B, span[5], S, ops)
+        o, S = span_join(loc, None, None, B, span[5], S, ops)
         outs.append(o)
     return outs, S

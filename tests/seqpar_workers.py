@@ -1,5 +1,5 @@
 """Rank bodies for the multi-process CPU tests of the sequence-parallel scan
-(run under torch.multiprocessing.spawn with the gloo backend).  The four span
+(run under torch.multiprocessing.spawn with the gloo backend).  The span
 steps are the oracle's, on float64 CPU tensors; what runs under test is the
 host logic of nvfp4_w4a4_gated_b200.seqpar: rank order, the all-gather, the
 composition of the maps and the corrections."""
@@ -14,27 +14,24 @@ import oracle
 
 
 class OracleSpanOps:
-    """gdn_scan / gdn_scan_transition / gdn_state_combine / gdn_scan_correct
-    restated with the oracle, in the binding's tensor shapes."""
+    """gdn_scan_span / gdn_state_combine / gdn_scan_correct restated with the
+    oracle, in the binding's tensor shapes."""
 
-    def scan(self, q, k, v, g, beta, B, T, dims, scale, form):
+    def local(self, q, k, v, g, beta, B, T, dims, scale, form):
         Hk, Hv, K, V = dims.Hk, dims.Hv, dims.K, dims.V
-        o, S = oracle.scan(q.numpy().reshape(B, T, Hk, K), k.numpy().reshape(B, T, Hk, K),
-                           v.numpy()[:, :Hv * V].reshape(B, T, Hv, V), g.numpy().reshape(B, T, Hv),
-                           beta.numpy().reshape(B, T, Hv), scale=scale, form=form)
-        return torch.from_numpy(o.reshape(B * T, Hv, V)), torch.from_numpy(S)
-
-    def transition(self, q, k, g, beta, B, T, dims, scale, form):
-        Hk, Hv, K = dims.Hk, dims.Hv, dims.K
-        P, m = oracle.scan_transition(q.numpy().reshape(B, T, Hk, K), k.numpy().reshape(B, T, Hk, K),
-                                      g.numpy().reshape(B, T, Hv), beta.numpy().reshape(B, T, Hv), scale=scale,
-                                      form=form)
-        return torch.from_numpy(P), torch.from_numpy(m.reshape(B * T, Hv, K))
+        qa, ka = q.numpy().reshape(B, T, Hk, K), k.numpy().reshape(B, T, Hk, K)
+        ga, ba = g.numpy().reshape(B, T, Hv), beta.numpy().reshape(B, T, Hv)
+        o, S = oracle.scan(qa, ka, v.numpy()[:, :Hv * V].reshape(B, T, Hv, V), ga, ba, scale=scale, form=form)
+        P, m = oracle.scan_transition(qa, ka, ga, ba, scale=scale, form=form)
+        return (torch.from_numpy(o.reshape(B * T, Hv, V)), torch.from_numpy(S), torch.from_numpy(P),
+                torch.from_numpy(m.reshape(B * T, Hv, K)))
 
     def combine(self, P, S_loc, S_in):
-        if S_in is None:
-            return S_loc.clone()
-        return torch.from_numpy(oracle.state_combine(P.numpy(), S_loc.numpy(), S_in.numpy()))
+        """P [m, ...], S_loc [m, ...]: fold the maps in order."""
+        S = None if S_in is None else S_in.numpy()
+        for j in range(P.shape[0]):
+            S = S_loc[j].numpy().copy() if S is None else oracle.state_combine(P[j].numpy(), S_loc[j].numpy(), S)
+        return torch.from_numpy(S)
 
     def correct(self, qmap, S_in, o, B, T):
         Hv, K, V = S_in.shape[1], S_in.shape[2], S_in.shape[3]

@@ -204,19 +204,39 @@ def test_state_passing_validation_and_sizes():
     st, _ = _err(L.gdn_scan_transition(FAKE, FAKE, FAKE, FAKE, 1, 64, ctypes.byref(d), 1.0, 5, 0, big, 2 * big,
                                        3 * big, tw, None))
     assert st == 1
-    # combine: shapes, aliasing
-    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, None, 4, 128, 128, None))
+    # combine (a chain of m maps): shapes, aliasing
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, None, 1, 4, 128, 128, None))
     assert st == 1
-    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 4, 48, 128, None))
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 0, 4, 128, 128, None))
+    assert st == 1
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 1, 4, 48, 128, None))
     assert st == 2
-    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 4, 128, 512, None))
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 1, 4, 256, 128, None))
     assert st == 2
-    st, msg = _err(L.gdn_state_combine(big, 2 * big, 3 * big, 3 * big + 4096, 4, 128, 128, None))
-    assert st == 1 and "overlap" in msg
-    st, msg = _err(L.gdn_state_combine(big, 2 * big + 4096, 3 * big, 2 * big, 4, 128, 128, None))
+    st, _ = _err(L.gdn_state_combine(FAKE, FAKE, FAKE, big, 1, 4, 128, 100, None))
+    assert st == 2
+    st, _ = _err(L.gdn_state_combine(FAKE + 4, FAKE, FAKE, big, 1, 4, 128, 128, None))
+    assert st == 3
+    st, msg = _err(L.gdn_state_combine(big, 2 * big, 3 * big, 3 * big + 4096, 1, 4, 128, 128, None))
+    assert st == 1 and "S_in" in msg
+    sb = 4 * 128 * 128 * 4          # one state block of n = 4
+    st, msg = _err(L.gdn_state_combine(big, 2 * big, 3 * big, 2 * big, 3, 4, 128, 128, None))
     assert st == 1 and "S_loc" in msg
-    st, _ = _err(L.gdn_state_combine(None, FAKE, FAKE, big, 4, 128, 128, None))
+    st, msg = _err(L.gdn_state_combine(big, 2 * big, 3 * big, big + 1024, 1, 4, 128, 128, None))
+    assert st == 1 and "P" in msg
+    # the span step
+    tws = L.gdn_scan_span_workspace_size(1, 4096, ctypes.byref(dk), nv.SCAN_CHUNKED)
+    assert tws >= max(scan_ws, L.gdn_scan_transition_workspace_size(1, 4096, ctypes.byref(dk), nv.SCAN_CHUNKED))
+    st, _ = _err(L.gdn_scan_span(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 4096, ctypes.byref(dk), 1.0, 0, 0, None,
+                                 big, 2 * big, 3 * big, 4 * big, tws, None))
     assert st == 1
+    st, _ = _err(L.gdn_scan_span(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 4096, ctypes.byref(dk), 1.0, 0, 0, big,
+                                 2 * big, 3 * big, 4 * big, 5 * big, tws - 1, None))
+    assert st == 6
+    st, msg = _err(L.gdn_scan_span(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 4096, ctypes.byref(dk), 1.0, 0, 0, big,
+                                   big + 4096, 3 * big, 4 * big, 5 * big, tws, None))
+    assert st == 1 and "overlap" in msg
+    assert sb > 0
     # correct: head dims, alignment, aliasing
     st, _ = _err(L.gdn_scan_correct(FAKE, FAKE, big, 1, 64, 32, 96, 128, None, None))
     assert st == 2

@@ -48,23 +48,68 @@ def test_transition_matches_oracle(cuda_dev, algo, form, B, T, Hk, Hv, K, V):
     assert rel_fro(m.cpu().numpy().reshape(B, T, Hv, K), m_ref) <= SCAN_TOL
 
 
-@pytest.mark.parametrize("K,V", [(32, 32), (64, 128), (128, 128), (256, 64), (128, 256)])
+@pytest.mark.parametrize("K,V", [(32, 32), (64, 128), (128, 128), (128, 64), (64, 256), (128, 96)])
 def test_state_combine_matches_oracle(cuda_dev, K, V):
-    n = 6
-    P = gdn_synth.gaussian(410, (n, K, K), std=K ** -0.5)
-    S_loc, S_in = gdn_synth.gaussian(411, (n, K, V)), gdn_synth.gaussian(412, (n, K, V))
+    B, Hv = 2, 3
+    P = gdn_synth.gaussian(410, (B, Hv, K, K), std=K ** -0.5)
+    S_loc, S_in = gdn_synth.gaussian(411, (B, Hv, K, V)), gdn_synth.gaussian(412, (B, Hv, K, V))
     dP, dL, dI = f32_device(P), f32_device(S_loc), f32_device(S_in)
     out = nv.gdn_state_combine(dP, dL, dI)
     ref = oracle.state_combine(P, S_loc, S_in)
     assert rel_fro(out.cpu().numpy(), ref) <= F32_TOL
     # S_in absent: the local state itself; S_loc absent: the map applied alone
-    assert torch.equal(nv.gdn_state_combine(None, dL, None), dL)
+    assert torch.equal(nv.gdn_state_combine(dP, dL, None), dL)
     only = nv.gdn_state_combine(dP, None, dI)
     assert rel_fro(only.cpu().numpy(), oracle.state_combine(P, np.zeros_like(S_loc), S_in)) <= F32_TOL
-    # in place on S_loc
-    nv.gdn_state_combine(dP, dL, dI, out=dL)
+    # in place on S_in
+    nv.gdn_state_combine(dP, dL, dI, out=dI)
     torch.cuda.synchronize()
-    assert torch.equal(dL, out)
+    assert torch.equal(dI, out)
+
+
+@pytest.mark.parametrize("K,V", [(64, 64), (128, 128)])
+def test_state_combine_chain(cuda_dev, K, V):
+    """Five maps composed in one launch equal the oracle's fold, with and
+    without a starting state; the result may overwrite the last S_loc."""
+    m, B, Hv = 5, 1, 4
+    P = gdn_synth.gaussian(415, (m, B, Hv, K, K), std=K ** -0.5)
+    S_loc = gdn_synth.gaussian(416, (m, B, Hv, K, V))
+    S0 = gdn_synth.gaussian(417, (B, Hv, K, V))
+    for start in (None, S0):
+        want = None if start is None else start.astype(np.float64)
+        for j in range(m):
+            want = S_loc[j].astype(np.float64) if want is None else oracle.state_combine(P[j], S_loc[j], want)
+        dL = f32_device(S_loc)
+        got = nv.gdn_state_combine(f32_device(P), dL, None if start is None else f32_device(start))
+        assert rel_fro(got.cpu().numpy(), want) <= F32_TOL
+        again = nv.gdn_state_combine(f32_device(P), dL, None if start is None else f32_device(start), out=dL[m - 1])
+        torch.cuda.synchronize()
+        assert torch.equal(again, got)
+
+
+@pytest.mark.parametrize("form", [nv.FORM_PAGES, nv.FORM_STANDARD])
+@pytest.mark.parametrize("B,T,Hk,Hv,K,V", [
+    (2, 200, 2, 4, 128, 128),    # chunked, K == V: one chunk preparation for both
+    (1, 64, 1, 2, 64, 64),
+    (1, 130, 2, 2, 128, 64),     # K != V: the scan, then the maps
+    (2, 1, 1, 2, 128, 128),      # one token
+])
+def test_scan_span_equals_scan_and_maps(cuda_dev, form, B, T, Hk, Hv, K, V):
+    arrs = gdn_synth.scan_inputs(418 + T, B, T, Hk, Hv, K, V, alpha_lo=0.9, alpha_hi=0.9999)
+    dims = nv.GdnDims(Hk, Hv, K, V)
+    q, k, v, g, beta, _ = _dev_span(arrs, 0, T, dims)
+    o, S_loc, P, m = nv.gdn_scan_span(q, k, v, g, beta, B, T, dims, form=form)
+    S_ref = torch.empty_like(S_loc)
+    o_ref, _ = nv.gdn_scan(q, k, v, g, beta, B, T, dims, form=form, state_out=S_ref)
+    P_ref, m_ref = nv.gdn_scan_transition(q, k, g, beta, B, T, dims, form=form)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    assert torch.equal(o, o_ref) and torch.equal(S_loc, S_ref)
+    assert rel_fro(P.cpu().numpy(), P_ref.cpu().numpy()) <= 1e-6
+    assert rel_fro(m.cpu().numpy(), m_ref.cpu().numpy()) <= 1e-6
+    Po, mo = oracle.scan_transition(arrs[0], arrs[1], arrs[3], arrs[4], form=form)
+    assert rel_fro(P.cpu().numpy(), Po) <= SCAN_TOL
+    assert rel_fro(m.cpu().numpy().reshape(B, T, Hv, K), mo) <= SCAN_TOL
 
 
 @pytest.mark.parametrize("B,T,Hv,K,V", [
