@@ -490,9 +490,8 @@ def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
     maps in one gdn_scan_span call, the seven earlier maps composed in one
     gdn_state_combine launch, the output correction) against the unsplit scan.
     The all-gather of (P, S_loc), 4 MiB per rank, is not measured on one GPU.
-    The correction kernel does 2 T Hv K V FLOP on the CUDA cores (peak: SMs x
-    128 FP32 lanes x 2 x the maximum SM clock) and moves
-    (T Hv (K + 2 V) + Hv K V) x 4 bytes."""
+    The correction kernel (tcgen05, TF32) does 2 T Hv K V FLOP and moves
+    (T Hv (K + 2 V) + Hv K V) x 4 bytes: HBM-bound."""
     B, T, Hk, Hv, K, V, n = 1, 32768, 16, 32, 128, 128, 8
     Ts = T // n
     dims = nv.GdnDims(Hk, Hv, K, V)
@@ -551,9 +550,25 @@ def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
     mean = lambda evs, i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
     whole_ms, rank_ms = mean(tw, 0, 1), mean(tr, 0, 4)
     corr_ms = mean(tr, 2, 3)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    clk = sm_max_mhz or 1965.0
-    alu_peak = sms * 128 * 2 * clk * 1e6 / 1e12
+    # the correction alone, tensor-core kernel and the CUDA-core one (same launch, same inputs)
+    o_c = torch.randn((Ts, Hv, V), generator=g_, device=dev)
+    m_c = torch.randn((Ts, Hv, K), generator=g_, device=dev) * 0.1
+    alone = {}
+    for variant in ("tcgen05", "cuda_core"):
+        if variant == "cuda_core":
+            os.environ["NVFP4_CORRECT_VARIANT"] = "cuda_core"
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            ev = mk(2)
+            ev[0].record(stream)
+            nv.gdn_scan_correct(m_c, S_in, o_c, B, Ts, stream=stream)
+            ev[1].record(stream)
+            ts.append(ev)
+        torch.cuda.synchronize()
+        os.environ.pop("NVFP4_CORRECT_VARIANT", None)
+        alone[variant] = mean(ts, 0, 1)
+    nv.check_device_error()
     flop = 2.0 * Ts * Hv * K * V
     byt = (Ts * Hv * (K + 2 * V) + Hv * K * V) * 4
     return {"workload": "gdn_scan_B1_T32768_hk16_hv32_k128_v128_in_8_spans_of_4096",
@@ -563,12 +578,12 @@ def bench_seqpar(nv, dev, steps, flush, stream, sm_max_mhz):
                               "combine_7_maps": round(mean(tr, 1, 2), 4), "correct": round(corr_ms, 4),
                               "end_state": round(mean(tr, 3, 4), 4)},
             "exchange": "all-gather of P and S_loc (4 MiB per rank): not measured on one GPU",
-            "correct_kernel": {"bound": "alu", "TFLOP/s": round(flop / (corr_ms / 1e3) / 1e12, 2),
-                               "peak_TFLOP/s": round(alu_peak, 1),
-                               "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 x {clk:g} MHz",
-                               "frac": round(flop / (corr_ms / 1e3) / 1e12 / alu_peak, 4),
-                               "GB/s": round(byt / (corr_ms / 1e3) / 1e9, 1),
-                               "frac_of_hbm": round(byt / (corr_ms / 1e3) / 1e9 / peaks()["hbm_gbs"], 4)}}
+            "correct_kernel": {"bound": "hbm", "GB/s": round(byt / (corr_ms / 1e3) / 1e9, 1),
+                               "frac": round(byt / (corr_ms / 1e3) / 1e9 / peaks()["hbm_gbs"], 4),
+                               "peak_source": "measured HBM copy",
+                               "TFLOP/s": round(flop / (corr_ms / 1e3) / 1e12, 2),
+                               "note": "tcgen05 kind::tf32; 2 T Hv K V FLOP, (T Hv (K + 2 V) + Hv K V) x 4 bytes",
+                               "alone_ms": {k_: round(v_, 4) for k_, v_ in alone.items()}}}
 
 
 def bench_decode(nv, dev, w, sh, steps, stream):

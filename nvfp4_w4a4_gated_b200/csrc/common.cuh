@@ -50,6 +50,7 @@ constexpr unsigned int kErrTimeoutEpi = 4u;
 constexpr unsigned int kErrTimeoutSeq = 8u;
 constexpr unsigned int kErrTimeoutSelftest = 16u;
 constexpr unsigned int kErrTimeoutQuant = 32u;
+constexpr unsigned int kErrTimeoutCorrect = 64u;
 
 // ---------------------------------------------------------------- device ---
 // Bounded waits give up after this many SM clocks (about half a second);

@@ -19,6 +19,8 @@
 //   gdn_scan_correct      o_t += S_in^T m_t over a span's tokens, with the
 //                         quantiser's amax of the corrected o folded in.
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -269,6 +271,206 @@ nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, 
     return NVFP4_OK;
 }
 
+// The same correction on the tcgen05 tensor cores (kind::tf32, float32
+// accumulation in TMEM): per item (b, h, 64 columns of V, tile of 128 tokens)
+//   D[t, j] = sum_i m[t, i] S_in[i, j]     (M = 128 tokens, N = 64, K)
+// with A = the tile's m rows and B = S_in^T (the 64 columns as rows), both
+// rounded to TF32 (nearest) while staged into 128-byte-swizzled K-major images.
+// A CTA takes a contiguous run of items (tile fastest), so it stages S_in^T once
+// per (b, h, column half); two CTAs share an SM.  Each thread loads its o values
+// before waiting for the MMAs; warp w reads TMEM lanes 32 (w % 4) .. + 31 (its
+// tokens) and columns 32 (w / 4) .. + 31.  The MMA completion wait is bounded;
+// on expiry the CTA records kErrTimeoutCorrect and stops.
+__device__ __forceinline__ uint32_t sw128_off(int r, int col, int rows) {
+    return static_cast<uint32_t>((col >> 5) * rows * 128 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) +
+                                 ((col & 3) << 2));
+}
+__device__ __forceinline__ float tf32_rn(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+constexpr int kTcTok = 128;     // tokens per item (MMA M)
+constexpr int kTcCols = 64;     // columns of V per item (MMA N)
+
+template <int K>
+struct CorrTcLayout {
+    static constexpr uint32_t A = 0;                          // [128 tokens x K] image
+    static constexpr uint32_t A_BYTES = kTcTok * K * 4;
+    static constexpr uint32_t Bm = A + A_BYTES;                // [64 columns x K] image
+    static constexpr uint32_t B_BYTES = kTcCols * K * 4;
+    static constexpr uint32_t BAR = Bm + B_BYTES;
+    static constexpr uint32_t BYTES = BAR + 64 + 1024;         // + alignment slack
+};
+
+template <int K, int V>
+__global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __restrict__ m,
+                                                                 const float* __restrict__ S_in,
+                                                                 float* __restrict__ o, int64_t T, int Hv,
+                                                                 int64_t n_items, int per_cta,
+                                                                 unsigned int* __restrict__ o_amax,
+                                                                 unsigned int* __restrict__ err) {
+    using L = CorrTcLayout<K>;
+    constexpr int NH = V / kTcCols;
+    constexpr uint32_t IDESC = idesc_tf32(kTcTok, kTcCols, false, false);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::BAR + 16);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_holder, kTcCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    pdl_wait_and_trigger();
+
+    const int64_t tiles = (T + kTcTok - 1) / kTcTok;
+    const int64_t i0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+    const int64_t i1 = i0 + per_cta < n_items ? i0 + per_cta : n_items;
+    const int q = warp & 3, ch = warp >> 2;
+    float mx = 0.0f;
+    int64_t cur = -1;       // (b, h, half) whose S_in^T is staged
+    uint32_t phase = 0;
+    bool all_ok = true;
+    for (int64_t it = i0; it < i1; ++it) {
+        const int64_t bhh = it / tiles, t0 = (it - bhh * tiles) * kTcTok;
+        const int64_t bh = bhh / NH;
+        const int half = static_cast<int>(bhh - bh * NH);
+        const int64_t b = bh / Hv, h = bh - b * Hv;
+        if (bhh != cur) {   // stage B = S_in[b,h][:, 64 half .. +63]^T, TF32
+            cur = bhh;
+            const float* Sb = S_in + bh * K * V + half * kTcCols;
+            for (int e = threadIdx.x; e < K * kTcCols / 4; e += 256) {
+                const int i = e / (kTcCols / 4), j4 = (e - i * (kTcCols / 4)) * 4;
+                const float4 v = *reinterpret_cast<const float4*>(Sb + static_cast<int64_t>(i) * V + j4);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 0, i, kTcCols)) = tf32_rn(v.x);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 1, i, kTcCols)) = tf32_rn(v.y);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 2, i, kTcCols)) = tf32_rn(v.z);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 3, i, kTcCols)) = tf32_rn(v.w);
+            }
+        }
+        // stage A = the tile's m rows, TF32; rows past T are zero
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            constexpr int PER = kTcTok * K / 4 / 256 / 2;       // float4 per thread per pass
+            float4 vals[PER];
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = (pass * PER + u) * 256 + threadIdx.x;
+                const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
+                const int64_t t = t0 + r;
+                vals[u] = t < T ? *reinterpret_cast<const float4*>(m + ((b * T + t) * Hv + h) * K + c4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = (pass * PER + u) * 256 + threadIdx.x;
+                const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
+                *reinterpret_cast<float4*>(sm + L::A + sw128_off(r, c4, kTcTok)) =
+                    make_float4(tf32_rn(vals[u].x), tf32_rn(vals[u].y), tf32_rn(vals[u].z), tf32_rn(vals[u].w));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (threadIdx.x == 0) {
+            const uint32_t a = smem_u32(sm + L::A), bb = smem_u32(sm + L::Bm);
+#pragma unroll
+            for (int j = 0; j < K / 8; ++j)
+                mma_tf32_ss(tmem, sdesc_kmajor_sw128(a + (j >> 2) * kTcTok * 128 + (j & 3) * 32),
+                            sdesc_kmajor_sw128(bb + (j >> 2) * kTcCols * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
+            mma_commit(bar);
+        }
+        // this thread's token and 32 columns; o loaded while the MMAs run
+        const int r = 32 * q + lane;
+        const int64_t t = t0 + r;
+        float* orow = o + ((b * T + t) * Hv + h) * V + half * kTcCols + 32 * ch;
+        float4 ov[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            ov[c] = t < T ? *reinterpret_cast<const float4*>(orow + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool ok = __syncthreads_and(mbar_wait(bar, phase, err, kErrTimeoutCorrect));
+        if (!ok) {
+            all_ok = false;
+            break;
+        }
+        phase ^= 1;
+        tc_fence_after();
+        uint32_t x[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * ch, x);
+        tmem_wait_ld();
+        tc_fence_before();
+        if (t < T) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float4 y = ov[c];
+                y.x += __uint_as_float(x[4 * c + 0]);
+                y.y += __uint_as_float(x[4 * c + 1]);
+                y.z += __uint_as_float(x[4 * c + 2]);
+                y.w += __uint_as_float(x[4 * c + 3]);
+                *reinterpret_cast<float4*>(orow + 4 * c) = y;
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))));
+            }
+        }
+        __syncthreads();    // TMEM read and the images free before the next item
+    }
+    if (o_amax) {
+        __shared__ unsigned int wmax[8];
+        const unsigned int wm = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+        if (lane == 0) wmax[warp] = wm;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            unsigned int bm = wmax[0];
+#pragma unroll
+            for (int i = 1; i < 8; ++i) bm = bm > wmax[i] ? bm : wmax[i];
+            atomicMax(o_amax, bm);
+        }
+    }
+    // after an expired wait, wait once more (bounded) for the MMAs in flight before TMEM is released
+    if (!all_ok && threadIdx.x == 0) mbar_wait(bar, phase, err, kErrTimeoutCorrect);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTcCols);
+    }
+}
+
+template <int K, int V>
+nvfp4_status launch_correct_tc(const float* m, const float* S_in, float* o, int B, int64_t T, int Hv,
+                               unsigned int* o_amax, cudaStream_t st) {
+    constexpr int smem = static_cast<int>(CorrTcLayout<K>::BYTES);
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(scan_correct_tc_kernel<K, V>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(correct tc)");
+        attr_done[dev] = true;
+    }
+    unsigned int* err = device_error_word();
+    if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
+    const int64_t n_items = static_cast<int64_t>(B) * Hv * (V / kTcCols) * ((T + kTcTok - 1) / kTcTok);
+    const int64_t slots = int64_t(num_sms()) * 2;
+    const int per_cta = static_cast<int>((n_items + slots - 1) / slots);
+    const unsigned grid = static_cast<unsigned>((n_items + per_cta - 1) / per_cta);
+    const cudaError_t e = launch_pdl(scan_correct_tc_kernel<K, V>, dim3(grid), dim3(256), smem, st, m, S_in, o, T,
+                                     Hv, n_items, per_cta, o_amax, err);
+    if (e != cudaSuccess) return cuda_fail(e, "scan correct launch");
+    return NVFP4_OK;
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const char* pa = static_cast<const char*>(a);
     const char* pb = static_cast<const char*>(b);
@@ -376,8 +578,15 @@ extern "C" nvfp4_status gdn_scan_correct(const float* qmap, const float* S_in, f
         return fail(NVFP4_ERR_INVALID_ARG, "o must not overlap qmap or S_in");
     const cudaStream_t st = as_stream(stream);
     unsigned int* amax = o_amax;
-    if (K == 128 && V == 128) return launch_correct<128, 128>(qmap, S_in, o, B, T, Hv, amax, st);
-    if (K == 128 && V == 64) return launch_correct<128, 64>(qmap, S_in, o, B, T, Hv, amax, st);
-    if (K == 64 && V == 128) return launch_correct<64, 128>(qmap, S_in, o, B, T, Hv, amax, st);
-    return launch_correct<64, 64>(qmap, S_in, o, B, T, Hv, amax, st);
+    const char* var = getenv("NVFP4_CORRECT_VARIANT");
+    if (var && strcmp(var, "cuda_core") == 0) {
+        if (K == 128 && V == 128) return launch_correct<128, 128>(qmap, S_in, o, B, T, Hv, amax, st);
+        if (K == 128 && V == 64) return launch_correct<128, 64>(qmap, S_in, o, B, T, Hv, amax, st);
+        if (K == 64 && V == 128) return launch_correct<64, 128>(qmap, S_in, o, B, T, Hv, amax, st);
+        return launch_correct<64, 64>(qmap, S_in, o, B, T, Hv, amax, st);
+    }
+    if (K == 128 && V == 128) return launch_correct_tc<128, 128>(qmap, S_in, o, B, T, Hv, amax, st);
+    if (K == 128 && V == 64) return launch_correct_tc<128, 64>(qmap, S_in, o, B, T, Hv, amax, st);
+    if (K == 64 && V == 128) return launch_correct_tc<64, 128>(qmap, S_in, o, B, T, Hv, amax, st);
+    return launch_correct_tc<64, 64>(qmap, S_in, o, B, T, Hv, amax, st);
 }

@@ -112,10 +112,16 @@ def test_scan_span_equals_scan_and_maps(cuda_dev, form, B, T, Hk, Hv, K, V):
     assert rel_fro(m.cpu().numpy().reshape(B, T, Hv, K), mo) <= SCAN_TOL
 
 
+@pytest.mark.parametrize("variant,tol", [("tcgen05", SCAN_TOL), ("cuda_core", F32_TOL)])
 @pytest.mark.parametrize("B,T,Hv,K,V", [
     (1, 1, 2, 128, 128), (2, 100, 4, 128, 128), (1, 64, 3, 64, 128), (2, 65, 2, 128, 64), (1, 130, 2, 64, 64),
+    (1, 1000, 5, 128, 128),      # several 128-token tiles per CTA run, heads changing inside a run
 ])
-def test_scan_correct_matches_oracle(cuda_dev, B, T, Hv, K, V):
+def test_scan_correct_matches_oracle(cuda_dev, monkeypatch, variant, tol, B, T, Hv, K, V):
+    """The tensor-core kernel (TF32 operands, the scan's bar) and the CUDA-core
+    kernel (float32) against the oracle; the amax word equals max |o| exactly."""
+    if variant == "cuda_core":
+        monkeypatch.setenv("NVFP4_CORRECT_VARIANT", "cuda_core")
     o_loc = gdn_synth.gaussian(420, (B, T, Hv, V))
     m = gdn_synth.gaussian(421, (B, T, Hv, K), std=0.1)
     S_in = gdn_synth.gaussian(422, (B, Hv, K, V))
@@ -123,9 +129,12 @@ def test_scan_correct_matches_oracle(cuda_dev, B, T, Hv, K, V):
     word = torch.zeros(1, dtype=torch.int32, device="cuda")
     nv.gdn_scan_correct(f32_device(m.reshape(B * T, Hv, K)), f32_device(S_in), o, B, T, amax_word=word)
     torch.cuda.synchronize()
+    nv.check_device_error()
     ref = oracle.output_correct(o_loc, m, S_in)
     got = o.cpu().numpy().reshape(B, T, Hv, V)
-    assert rel_fro(got, ref) <= F32_TOL
+    assert rel_fro(got, ref) <= tol
+    corr = ref - o_loc                 # the correction alone, to its own bar as well
+    assert rel_fro(got - o_loc, corr) <= tol
     assert word.view(torch.float32).item() == float(np.abs(got).max())
 
 
