@@ -54,60 +54,72 @@ __global__ void __launch_bounds__(256) identity_fill_kernel(float* __restrict__ 
 
 // The chain S = S_in; S = P[j] S + S_loc[j] for j = 0..m-1; S_out = S, per
 // (sequence, value head) n.  The columns of S evolve independently, so one CTA
-// per (n, 32 columns) carries its K x 32 slice through the whole chain in
-// shared memory; each step stages P[j][n] (K x K) in shared memory, warp w owns
-// rows w + 8r and lane l column c0 + l, and P is read as warp-wide broadcasts.
+// per (n, 8 columns) carries its K x 8 slice through the whole chain in shared
+// memory; each step stages P[j][n] (K x K, rows padded by 4 floats so that the
+// four consecutive rows a warp reads at once fall in different banks) in shared
+// memory.  Thread (g, c) owns column c0 + c and rows g + 32 r (r < K / 32).
+constexpr int kChainCols = 8;
 template <int K>
 __global__ void __launch_bounds__(256) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
                                                           const float* S_in, float* S_out, int m, int64_t n_total,
                                                           int V) {
     pdl_wait_and_trigger();
-    constexpr int R = K / 8;
+    constexpr int R = K / 32;
+    constexpr int PK = K + 4;
     extern __shared__ __align__(16) float smem[];
-    float* Ps = smem;            // [K][K]
-    float* Ss = smem + K * K;    // [K][32]
+    float* Ps = smem;                  // [K][K + 4]
+    float* Ss = smem + K * PK;         // [K][8]
     const int64_t n = blockIdx.x;
-    const int c0 = blockIdx.y * 32;
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = w; i < K; i += 8)
-        Ss[i * 32 + lane] = S_in ? S_in[(n * K + i) * V + c0 + lane] : 0.0f;
+    const int c0 = blockIdx.y * kChainCols;
+    const int c = threadIdx.x & 7, g = threadIdx.x >> 3;
+    for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
+        const int i = e >> 3, cc = e & 7;
+        Ss[e] = S_in ? S_in[(n * K + i) * V + c0 + cc] : 0.0f;
+    }
     for (int j = 0; j < m; ++j) {
         const float4* Pj = reinterpret_cast<const float4*>(P + (static_cast<int64_t>(j) * n_total + n) * K * K);
         __syncthreads();   // the slice is written; the previous step's P is no longer read
-        for (int e = threadIdx.x; e < K * K / 4; e += 256) reinterpret_cast<float4*>(Ps)[e] = Pj[e];
+#pragma unroll 4
+        for (int e = threadIdx.x; e < K * K / 4; e += 256) {
+            const int i = e / (K / 4), l4 = e - i * (K / 4);
+            *reinterpret_cast<float4*>(Ps + i * PK + 4 * l4) = Pj[e];
+        }
         __syncthreads();
         float acc[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) acc[r] = 0.0f;
-#pragma unroll 2
+#pragma unroll 4
         for (int l = 0; l < K; l += 4) {
-            const float s0 = Ss[(l + 0) * 32 + lane], s1 = Ss[(l + 1) * 32 + lane];
-            const float s2 = Ss[(l + 2) * 32 + lane], s3 = Ss[(l + 3) * 32 + lane];
+            const float s0 = Ss[(l + 0) * 8 + c], s1 = Ss[(l + 1) * 8 + c];
+            const float s2 = Ss[(l + 2) * 8 + c], s3 = Ss[(l + 3) * 8 + c];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float4 p = *reinterpret_cast<const float4*>(Ps + (w + 8 * r) * K + l);
+                const float4 p = *reinterpret_cast<const float4*>(Ps + (g + 32 * r) * PK + l);
                 acc[r] = fmaf(p.x, s0, acc[r]);
                 acc[r] = fmaf(p.y, s1, acc[r]);
                 acc[r] = fmaf(p.z, s2, acc[r]);
                 acc[r] = fmaf(p.w, s3, acc[r]);
             }
         }
-        __syncthreads();   // every warp has read the old slice
+        __syncthreads();   // every thread has read the old slice
         const float* Lj = S_loc ? S_loc + (static_cast<int64_t>(j) * n_total + n) * K * V : nullptr;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int i = w + 8 * r;
-            Ss[i * 32 + lane] = acc[r] + (Lj ? Lj[static_cast<int64_t>(i) * V + c0 + lane] : 0.0f);
+            const int i = g + 32 * r;
+            Ss[i * 8 + c] = acc[r] + (Lj ? Lj[static_cast<int64_t>(i) * V + c0 + c] : 0.0f);
         }
     }
     __syncthreads();
-    for (int i = w; i < K; i += 8) S_out[(n * K + i) * V + c0 + lane] = Ss[i * 32 + lane];
+    for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
+        const int i = e >> 3, cc = e & 7;
+        S_out[(n * K + i) * V + c0 + cc] = Ss[e];
+    }
 }
 
 template <int K>
 nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in, float* S_out, int m, int64_t n,
                           int V, cudaStream_t st) {
-    constexpr int smem = (K * K + K * 32) * 4;
+    constexpr int smem = (K * (K + 4) + K * kChainCols) * 4;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -116,8 +128,8 @@ nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in,
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chain)");
         attr_done[dev] = true;
     }
-    const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / 32), dim3(256), smem,
-                                     st, P, S_loc, S_in, S_out, m, n, V);
+    const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / kChainCols), dim3(256),
+                                     smem, st, P, S_loc, S_in, S_out, m, n, V);
     if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
     return NVFP4_OK;
 }
@@ -272,15 +284,16 @@ nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, 
 }
 
 // The same correction on the tcgen05 tensor cores (kind::tf32, float32
-// accumulation in TMEM): per item (b, h, 64 columns of V, tile of 128 tokens)
-//   D[t, j] = sum_i m[t, i] S_in[i, j]     (M = 128 tokens, N = 64, K)
-// with A = the tile's m rows and B = S_in^T (the 64 columns as rows), both
-// rounded to TF32 (nearest) while staged into 128-byte-swizzled K-major images.
-// A CTA takes a contiguous run of items (tile fastest), so it stages S_in^T once
-// per (b, h, column half); two CTAs share an SM.  Each thread loads its o values
-// before waiting for the MMAs; warp w reads TMEM lanes 32 (w % 4) .. + 31 (its
-// tokens) and columns 32 (w / 4) .. + 31.  The MMA completion wait is bounded;
-// on expiry the CTA records kErrTimeoutCorrect and stops.
+// accumulation in TMEM): per item (b, h, tile of 128 tokens)
+//   D[t, j] = sum_i m[t, i] S_in[i, j]     (M = 128 tokens, N = V, K)
+// with A = the tile's m rows and B = S_in^T (the V columns as rows), both in
+// 128-byte-swizzled K-major images and rounded to TF32 (nearest).  One CTA per
+// SM takes a contiguous run of items (tile fastest) and stages S_in^T once per
+// head; the m rows of the next item are copied asynchronously into the other A
+// buffer while the current item's MMAs and epilogue run, and each thread loads
+// its o values while the MMAs run.  Warp w reads TMEM lanes 32 (w % 4) .. + 31
+// (its token) and columns V/2 (w / 4) .. + V/2 - 1.  The MMA completion wait is
+// bounded; on expiry the CTA records kErrTimeoutCorrect and stops.
 __device__ __forceinline__ uint32_t sw128_off(int r, int col, int rows) {
     return static_cast<uint32_t>((col >> 5) * rows * 128 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) +
                                  ((col & 3) << 2));
@@ -292,28 +305,28 @@ __device__ __forceinline__ float tf32_rn(float x) {
 }
 
 constexpr int kTcTok = 128;     // tokens per item (MMA M)
-constexpr int kTcCols = 64;     // columns of V per item (MMA N)
 
-template <int K>
+template <int K, int V>
 struct CorrTcLayout {
-    static constexpr uint32_t A = 0;                          // [128 tokens x K] image
     static constexpr uint32_t A_BYTES = kTcTok * K * 4;
-    static constexpr uint32_t Bm = A + A_BYTES;                // [64 columns x K] image
-    static constexpr uint32_t B_BYTES = kTcCols * K * 4;
+    static constexpr uint32_t A = 0;                           // two [128 tokens x K] images
+    static constexpr uint32_t Bm = A + 2 * A_BYTES;            // [V columns x K] image
+    static constexpr uint32_t B_BYTES = V * K * 4;
     static constexpr uint32_t BAR = Bm + B_BYTES;
     static constexpr uint32_t BYTES = BAR + 64 + 1024;         // + alignment slack
 };
 
 template <int K, int V>
-__global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __restrict__ m,
+__global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __restrict__ m,
                                                                  const float* __restrict__ S_in,
                                                                  float* __restrict__ o, int64_t T, int Hv,
                                                                  int64_t n_items, int per_cta,
                                                                  unsigned int* __restrict__ o_amax,
                                                                  unsigned int* __restrict__ err) {
-    using L = CorrTcLayout<K>;
-    constexpr int NH = V / kTcCols;
-    constexpr uint32_t IDESC = idesc_tf32(kTcTok, kTcCols, false, false);
+    using L = CorrTcLayout<K, V>;
+    constexpr uint32_t IDESC = idesc_tf32(kTcTok, V, false, false);
+    constexpr int CPT = kTcTok * K / 4 / 256;       // 16-byte chunks of A per thread
+    constexpr int HALF = V / 2;                     // columns per warp
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
@@ -324,7 +337,7 @@ __global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_holder, kTcCols);
+        tmem_alloc(tmem_holder, V);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -337,46 +350,56 @@ __global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __
     const int64_t i0 = static_cast<int64_t>(blockIdx.x) * per_cta;
     const int64_t i1 = i0 + per_cta < n_items ? i0 + per_cta : n_items;
     const int q = warp & 3, ch = warp >> 2;
+    // this thread's A chunks: e = u * 256 + tid -> row e / (K/4), column 4 (e % (K/4))
+    auto issue_a = [&](int64_t item, int buf) {
+        const int64_t bh = item / tiles, t0 = (item - bh * tiles) * kTcTok;
+        const int64_t b = bh / Hv, h = bh - b * Hv;
+        uint8_t* dst = sm + L::A + buf * L::A_BYTES;
+#pragma unroll
+        for (int u = 0; u < CPT; ++u) {
+            const int e = u * 256 + threadIdx.x;
+            const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
+            const int64_t t = t0 + r;
+            const bool valid = t < T;
+            cp_async16(dst + sw128_off(r, c4, kTcTok), valid ? m + ((b * T + t) * Hv + h) * K + c4 : m, valid);
+        }
+        cp_async_commit();
+    };
     float mx = 0.0f;
-    int64_t cur = -1;       // (b, h, half) whose S_in^T is staged
+    int64_t cur = -1;       // (b, h) whose S_in^T is staged
     uint32_t phase = 0;
     bool all_ok = true;
+    if (i0 < i1) issue_a(i0, 0);
     for (int64_t it = i0; it < i1; ++it) {
-        const int64_t bhh = it / tiles, t0 = (it - bhh * tiles) * kTcTok;
-        const int64_t bh = bhh / NH;
-        const int half = static_cast<int>(bhh - bh * NH);
+        const int buf = static_cast<int>((it - i0) & 1);
+        const int64_t bh = it / tiles, t0 = (it - bh * tiles) * kTcTok;
         const int64_t b = bh / Hv, h = bh - b * Hv;
-        if (bhh != cur) {   // stage B = S_in[b,h][:, 64 half .. +63]^T, TF32
-            cur = bhh;
-            const float* Sb = S_in + bh * K * V + half * kTcCols;
-            for (int e = threadIdx.x; e < K * kTcCols / 4; e += 256) {
-                const int i = e / (kTcCols / 4), j4 = (e - i * (kTcCols / 4)) * 4;
+        if (bh != cur) {    // stage B = S_in[b,h]^T, TF32
+            cur = bh;
+            const float* Sb = S_in + bh * K * V;
+            for (int e = threadIdx.x; e < K * V / 4; e += 256) {
+                const int i = e / (V / 4), j4 = (e - i * (V / 4)) * 4;
                 const float4 v = *reinterpret_cast<const float4*>(Sb + static_cast<int64_t>(i) * V + j4);
-                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 0, i, kTcCols)) = tf32_rn(v.x);
-                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 1, i, kTcCols)) = tf32_rn(v.y);
-                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 2, i, kTcCols)) = tf32_rn(v.z);
-                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 3, i, kTcCols)) = tf32_rn(v.w);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 0, i, V)) = tf32_rn(v.x);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 1, i, V)) = tf32_rn(v.y);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 2, i, V)) = tf32_rn(v.z);
+                *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 3, i, V)) = tf32_rn(v.w);
             }
         }
-        // stage A = the tile's m rows, TF32; rows past T are zero
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            constexpr int PER = kTcTok * K / 4 / 256 / 2;       // float4 per thread per pass
-            float4 vals[PER];
+        // the next item's rows go into the other buffer (its last reader, the
+        // previous item's MMAs, has completed)
+        if (it + 1 < i1) issue_a(it + 1, buf ^ 1);
+        else cp_async_commit();
+        cp_async_wait<1>();
+        {   // round this thread's own chunks of the current buffer to TF32
+            uint8_t* a = sm + L::A + buf * L::A_BYTES;
 #pragma unroll
-            for (int u = 0; u < PER; ++u) {
-                const int e = (pass * PER + u) * 256 + threadIdx.x;
+            for (int u = 0; u < CPT; ++u) {
+                const int e = u * 256 + threadIdx.x;
                 const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
-                const int64_t t = t0 + r;
-                vals[u] = t < T ? *reinterpret_cast<const float4*>(m + ((b * T + t) * Hv + h) * K + c4)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < PER; ++u) {
-                const int e = (pass * PER + u) * 256 + threadIdx.x;
-                const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
-                *reinterpret_cast<float4*>(sm + L::A + sw128_off(r, c4, kTcTok)) =
-                    make_float4(tf32_rn(vals[u].x), tf32_rn(vals[u].y), tf32_rn(vals[u].z), tf32_rn(vals[u].w));
+                float4* p = reinterpret_cast<float4*>(a + sw128_off(r, c4, kTcTok));
+                const float4 v = *p;
+                *p = make_float4(tf32_rn(v.x), tf32_rn(v.y), tf32_rn(v.z), tf32_rn(v.w));
             }
         }
         fence_proxy_async_smem();
@@ -384,20 +407,20 @@ __global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __
         __syncthreads();
         tc_fence_after();
         if (threadIdx.x == 0) {
-            const uint32_t a = smem_u32(sm + L::A), bb = smem_u32(sm + L::Bm);
+            const uint32_t a = smem_u32(sm + L::A + buf * L::A_BYTES), bb = smem_u32(sm + L::Bm);
 #pragma unroll
             for (int j = 0; j < K / 8; ++j)
                 mma_tf32_ss(tmem, sdesc_kmajor_sw128(a + (j >> 2) * kTcTok * 128 + (j & 3) * 32),
-                            sdesc_kmajor_sw128(bb + (j >> 2) * kTcCols * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
+                            sdesc_kmajor_sw128(bb + (j >> 2) * V * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
             mma_commit(bar);
         }
-        // this thread's token and 32 columns; o loaded while the MMAs run
+        // this thread's token and HALF columns; o loaded while the MMAs run
         const int r = 32 * q + lane;
         const int64_t t = t0 + r;
-        float* orow = o + ((b * T + t) * Hv + h) * V + half * kTcCols + 32 * ch;
-        float4 ov[8];
+        float* orow = o + ((b * T + t) * Hv + h) * V + HALF * ch;
+        float4 ov[HALF / 4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < HALF / 4; ++c)
             ov[c] = t < T ? *reinterpret_cast<const float4*>(orow + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
         const bool ok = __syncthreads_and(mbar_wait(bar, phase, err, kErrTimeoutCorrect));
         if (!ok) {
@@ -406,24 +429,28 @@ __global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __
         }
         phase ^= 1;
         tc_fence_after();
-        uint32_t x[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * ch, x);
-        tmem_wait_ld();
-        tc_fence_before();
-        if (t < T) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float4 y = ov[c];
-                y.x += __uint_as_float(x[4 * c + 0]);
-                y.y += __uint_as_float(x[4 * c + 1]);
-                y.z += __uint_as_float(x[4 * c + 2]);
-                y.w += __uint_as_float(x[4 * c + 3]);
-                *reinterpret_cast<float4*>(orow + 4 * c) = y;
-                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))));
+        for (int cc = 0; cc < HALF / 32; ++cc) {
+            uint32_t x[32];
+            tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + HALF * ch + 32 * cc, x);
+            tmem_wait_ld();
+            if (t < T) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float4 y = ov[8 * cc + c];
+                    y.x += __uint_as_float(x[4 * c + 0]);
+                    y.y += __uint_as_float(x[4 * c + 1]);
+                    y.z += __uint_as_float(x[4 * c + 2]);
+                    y.w += __uint_as_float(x[4 * c + 3]);
+                    *reinterpret_cast<float4*>(orow + 32 * cc + 4 * c) = y;
+                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))));
+                }
             }
         }
-        __syncthreads();    // TMEM read and the images free before the next item
+        tc_fence_before();
+        __syncthreads();    // TMEM read and B free before the next item
     }
+    cp_async_wait<0>();
     if (o_amax) {
         __shared__ unsigned int wmax[8];
         const unsigned int wm = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
@@ -442,14 +469,14 @@ __global__ void __launch_bounds__(256, 2) scan_correct_tc_kernel(const float* __
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTcCols);
+        tmem_dealloc(tmem, V);
     }
 }
 
 template <int K, int V>
 nvfp4_status launch_correct_tc(const float* m, const float* S_in, float* o, int B, int64_t T, int Hv,
                                unsigned int* o_amax, cudaStream_t st) {
-    constexpr int smem = static_cast<int>(CorrTcLayout<K>::BYTES);
+    constexpr int smem = static_cast<int>(CorrTcLayout<K, V>::BYTES);
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -461,8 +488,8 @@ nvfp4_status launch_correct_tc(const float* m, const float* S_in, float* o, int 
     }
     unsigned int* err = device_error_word();
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
-    const int64_t n_items = static_cast<int64_t>(B) * Hv * (V / kTcCols) * ((T + kTcTok - 1) / kTcTok);
-    const int64_t slots = int64_t(num_sms()) * 2;
+    const int64_t n_items = static_cast<int64_t>(B) * Hv * ((T + kTcTok - 1) / kTcTok);
+    const int64_t slots = num_sms();
     const int per_cta = static_cast<int>((n_items + slots - 1) / slots);
     const unsigned grid = static_cast<unsigned>((n_items + per_cta - 1) / per_cta);
     const cudaError_t e = launch_pdl(scan_correct_tc_kernel<K, V>, dim3(grid), dim3(256), smem, st, m, S_in, o, T,
@@ -542,7 +569,7 @@ extern "C" nvfp4_status gdn_state_combine(const float* P, const float* S_loc, co
     using namespace nvg;
     if (!S_out || !P) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
     if (m < 1 || n < 1) return fail(NVFP4_ERR_INVALID_ARG, "m and n must be >= 1");
-    if ((K != 32 && K != 64 && K != 128) || V < 32 || V % 32 || V / 32 > 65535)
+    if ((K != 32 && K != 64 && K != 128) || V < 32 || V % 32 || V / 8 > 65535)
         return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be 32, 64 or 128 and V a multiple of 32");
     if (n > 2147483647) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "n too large");
     if (!aligned16(P)) return fail(NVFP4_ERR_MISALIGNED, "P must be 16-byte aligned");
