@@ -54,64 +54,87 @@ __global__ void __launch_bounds__(256) identity_fill_kernel(float* __restrict__ 
 
 // The chain S = S_in; S = P[j] S + S_loc[j] for j = 0..m-1; S_out = S, per
 // (sequence, value head) n.  The columns of S evolve independently, so one CTA
-// per (n, 8 columns) carries its K x 8 slice through the whole chain in shared
-// memory; each step stages P[j][n] (K x K, rows padded by 4 floats so that the
-// four consecutive rows a warp reads at once fall in different banks) in shared
-// memory.  Thread (g, c) owns column c0 + c and rows g + 32 r (r < K / 32).
-constexpr int kChainCols = 8;
+// per (n, 32 columns) carries its K x 32 slice through the whole chain in
+// shared memory.  P[j+1][n] (K x K) is copied asynchronously into the second of
+// two shared buffers while step j computes; rows are padded by 4 floats so the
+// four consecutive rows a warp reads at once fall in different banks.  Thread
+// (tr, tc) owns rows tr + 32 r (r < K / 32) and columns 4 tc .. 4 tc + 3.
+constexpr int kChainCols = 32;
 template <int K>
-__global__ void __launch_bounds__(256) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
-                                                          const float* S_in, float* S_out, int m, int64_t n_total,
-                                                          int V) {
+__global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
+                                                             const float* S_in, float* S_out, int m,
+                                                             int64_t n_total, int V) {
     pdl_wait_and_trigger();
     constexpr int R = K / 32;
     constexpr int PK = K + 4;
     extern __shared__ __align__(16) float smem[];
-    float* Ps = smem;                  // [K][K + 4]
-    float* Ss = smem + K * PK;         // [K][8]
+    float* Pb = smem;                      // [2][K][K + 4]
+    float* Ss = smem + 2 * K * PK;         // [K][32]
     const int64_t n = blockIdx.x;
     const int c0 = blockIdx.y * kChainCols;
-    const int c = threadIdx.x & 7, g = threadIdx.x >> 3;
-    for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
-        const int i = e >> 3, cc = e & 7;
-        Ss[e] = S_in ? S_in[(n * K + i) * V + c0 + cc] : 0.0f;
-    }
-    for (int j = 0; j < m; ++j) {
-        const float4* Pj = reinterpret_cast<const float4*>(P + (static_cast<int64_t>(j) * n_total + n) * K * K);
-        __syncthreads();   // the slice is written; the previous step's P is no longer read
+    const int tc = threadIdx.x & 7, tr = threadIdx.x >> 3;
+    auto issue_p = [&](int j, int buf) {
+        const float* Pj = P + (static_cast<int64_t>(j) * n_total + n) * K * K;
+        float* dst = Pb + buf * K * PK;
 #pragma unroll 4
         for (int e = threadIdx.x; e < K * K / 4; e += 256) {
             const int i = e / (K / 4), l4 = e - i * (K / 4);
-            *reinterpret_cast<float4*>(Ps + i * PK + 4 * l4) = Pj[e];
+            cp_async16(dst + i * PK + 4 * l4, Pj + 4 * static_cast<int64_t>(e), true);
         }
-        __syncthreads();
-        float acc[R];
+        cp_async_commit();
+    };
+    issue_p(0, 0);
+    for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
+        const int i = e >> 5, cc = e & 31;
+        Ss[e] = S_in ? S_in[(n * K + i) * V + c0 + cc] : 0.0f;
+    }
+    for (int j = 0; j < m; ++j) {
+        if (j + 1 < m) issue_p(j + 1, (j + 1) & 1);
+        else cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();   // P[j] landed everywhere; the slice of the previous step is written
+        const float* Ps = Pb + (j & 1) * K * PK;
+        float acc[R][4];
 #pragma unroll
-        for (int r = 0; r < R; ++r) acc[r] = 0.0f;
-#pragma unroll 4
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) acc[r][cc] = 0.0f;
+#pragma unroll 2
         for (int l = 0; l < K; l += 4) {
-            const float s0 = Ss[(l + 0) * 8 + c], s1 = Ss[(l + 1) * 8 + c];
-            const float s2 = Ss[(l + 2) * 8 + c], s3 = Ss[(l + 3) * 8 + c];
+            float4 p[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const float4 p = *reinterpret_cast<const float4*>(Ps + (g + 32 * r) * PK + l);
-                acc[r] = fmaf(p.x, s0, acc[r]);
-                acc[r] = fmaf(p.y, s1, acc[r]);
-                acc[r] = fmaf(p.z, s2, acc[r]);
-                acc[r] = fmaf(p.w, s3, acc[r]);
+            for (int r = 0; r < R; ++r) p[r] = *reinterpret_cast<const float4*>(Ps + (tr + 32 * r) * PK + l);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 sv = *reinterpret_cast<const float4*>(Ss + (l + q) * kChainCols + 4 * tc);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float pv = q == 0 ? p[r].x : q == 1 ? p[r].y : q == 2 ? p[r].z : p[r].w;
+                    acc[r][0] = fmaf(pv, sv.x, acc[r][0]);
+                    acc[r][1] = fmaf(pv, sv.y, acc[r][1]);
+                    acc[r][2] = fmaf(pv, sv.z, acc[r][2]);
+                    acc[r][3] = fmaf(pv, sv.w, acc[r][3]);
+                }
             }
         }
-        __syncthreads();   // every thread has read the old slice
+        __syncthreads();   // every thread has read the old slice and P[j]
         const float* Lj = S_loc ? S_loc + (static_cast<int64_t>(j) * n_total + n) * K * V : nullptr;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int i = g + 32 * r;
-            Ss[i * 8 + c] = acc[r] + (Lj ? Lj[static_cast<int64_t>(i) * V + c0 + c] : 0.0f);
+            const int i = tr + 32 * r;
+            float4 add = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (Lj) {
+                const float* lp = Lj + static_cast<int64_t>(i) * V + c0 + 4 * tc;
+                add = make_float4(lp[0], lp[1], lp[2], lp[3]);
+            }
+            *reinterpret_cast<float4*>(Ss + i * kChainCols + 4 * tc) =
+                make_float4(acc[r][0] + add.x, acc[r][1] + add.y, acc[r][2] + add.z, acc[r][3] + add.w);
         }
     }
+    cp_async_wait<0>();
     __syncthreads();
     for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
-        const int i = e >> 3, cc = e & 7;
+        const int i = e >> 5, cc = e & 31;
         S_out[(n * K + i) * V + c0 + cc] = Ss[e];
     }
 }
@@ -119,7 +142,7 @@ __global__ void __launch_bounds__(256) state_chain_kernel(const float* __restric
 template <int K>
 nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in, float* S_out, int m, int64_t n,
                           int V, cudaStream_t st) {
-    constexpr int smem = (K * (K + 4) + K * kChainCols) * 4;
+    constexpr int smem = (2 * K * (K + 4) + K * kChainCols) * 4;
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -291,7 +314,7 @@ nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, 
 // SM takes a contiguous run of items (tile fastest) and stages S_in^T once per
 // head; the m rows of the next item are copied asynchronously into the other A
 // buffer while the current item's MMAs and epilogue run, and each thread loads
-// its o values while the MMAs run.  Warp w reads TMEM lanes 32 (w % 4) .. + 31
+// its o values before the current A is rounded and multiplied.  Warp w reads TMEM lanes 32 (w % 4) .. + 31
 // (its token) and columns V/2 (w / 4) .. + V/2 - 1.  The MMA completion wait is
 // bounded; on expiry the CTA records kErrTimeoutCorrect and stops.
 __device__ __forceinline__ uint32_t sw128_off(int r, int col, int rows) {
@@ -390,6 +413,14 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
         // previous item's MMAs, has completed)
         if (it + 1 < i1) issue_a(it + 1, buf ^ 1);
         else cp_async_commit();
+        // this thread's token and HALF columns of o, loaded while A is rounded and the MMAs run
+        const int r = 32 * q + lane;
+        const int64_t t = t0 + r;
+        float* orow = o + ((b * T + t) * Hv + h) * V + HALF * ch;
+        float4 ov[HALF / 4];
+#pragma unroll
+        for (int c = 0; c < HALF / 4; ++c)
+            ov[c] = t < T ? *reinterpret_cast<const float4*>(orow + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
         cp_async_wait<1>();
         {   // round this thread's own chunks of the current buffer to TF32
             uint8_t* a = sm + L::A + buf * L::A_BYTES;
@@ -414,14 +445,6 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
                             sdesc_kmajor_sw128(bb + (j >> 2) * V * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
             mma_commit(bar);
         }
-        // this thread's token and HALF columns; o loaded while the MMAs run
-        const int r = 32 * q + lane;
-        const int64_t t = t0 + r;
-        float* orow = o + ((b * T + t) * Hv + h) * V + HALF * ch;
-        float4 ov[HALF / 4];
-#pragma unroll
-        for (int c = 0; c < HALF / 4; ++c)
-            ov[c] = t < T ? *reinterpret_cast<const float4*>(orow + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
         const bool ok = __syncthreads_and(mbar_wait(bar, phase, err, kErrTimeoutCorrect));
         if (!ok) {
             all_ok = false;
@@ -569,7 +592,7 @@ extern "C" nvfp4_status gdn_state_combine(const float* P, const float* S_loc, co
     using namespace nvg;
     if (!S_out || !P) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
     if (m < 1 || n < 1) return fail(NVFP4_ERR_INVALID_ARG, "m and n must be >= 1");
-    if ((K != 32 && K != 64 && K != 128) || V < 32 || V % 32 || V / 8 > 65535)
+    if ((K != 32 && K != 64 && K != 128) || V < 32 || V % 32 || V / 32 > 65535)
         return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be 32, 64 or 128 and V a multiple of 32");
     if (n > 2147483647) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "n too large");
     if (!aligned16(P)) return fail(NVFP4_ERR_MISALIGNED, "P must be 16-byte aligned");
