@@ -763,6 +763,18 @@ def kernel_case(args):
         S_in = torch.randn((B, Hv, Kd, Kd), generator=g, device=dev)
         o = torch.randn((B * T, Hv, Kd), generator=g, device=dev)
         fn = lambda: nv.gdn_scan_correct(qm, S_in, o, B, T)
+    elif args.kernel_case == "statepass":
+        # one rank's joining steps over a span of T tokens: seven maps composed, then the correction
+        B, T, Hv, Kd = 1, args.T, 32, 128
+        Ps = torch.randn((7, B, Hv, Kd, Kd), generator=g, device=dev) * (Kd ** -0.5)
+        Sl = torch.randn((7, B, Hv, Kd, Kd), generator=g, device=dev)
+        S_in = torch.empty((B, Hv, Kd, Kd), device=dev)
+        qm = torch.randn((B * T, Hv, Kd), generator=g, device=dev) * 0.1
+        o = torch.randn((B * T, Hv, Kd), generator=g, device=dev)
+
+        def fn():
+            nv.gdn_state_combine(Ps, Sl, None, out=S_in)
+            nv.gdn_scan_correct(qm, S_in, o, B, T)
     else:
         raise SystemExit("unknown kernel case")
     for _ in range(args.warmup):
@@ -788,7 +800,7 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     ap.add_argument("--ref-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct"], default=None,
+    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct", "statepass"], default=None,
                     help="profile helper: run one kernel on a fixed case and exit")
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
