@@ -57,15 +57,17 @@ __global__ void __launch_bounds__(256) identity_fill_kernel(float* __restrict__ 
 // per (n, 32 columns) carries its K x 32 slice through the whole chain in
 // shared memory.  P[j+1][n] (K x K) is copied asynchronously into the second of
 // two shared buffers while step j computes; rows are padded by 4 floats so the
-// four consecutive rows a warp reads at once fall in different banks.  Thread
-// (tr, tc) owns rows tr + 32 r (r < K / 32) and columns 4 tc .. 4 tc + 3.
+// four consecutive rows a warp reads at once fall in different banks.  4K
+// threads; thread (tr, tc) owns rows tr and tr + K/2 and columns 4 tc .. 4 tc + 3.
 constexpr int kChainCols = 32;
 template <int K>
-__global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
-                                                             const float* S_in, float* S_out, int m,
-                                                             int64_t n_total, int V) {
+__global__ void __launch_bounds__(4 * K, 1) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
+                                                               const float* S_in, float* S_out, int m,
+                                                               int64_t n_total, int V) {
     pdl_wait_and_trigger();
-    constexpr int R = K / 32;
+    constexpr int NT = 4 * K;          // threads
+    constexpr int R = 2;
+    constexpr int RS = K / 2;          // row stride between a thread's rows
     constexpr int PK = K + 4;
     extern __shared__ __align__(16) float smem[];
     float* Pb = smem;                      // [2][K][K + 4]
@@ -77,14 +79,14 @@ __global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __rest
         const float* Pj = P + (static_cast<int64_t>(j) * n_total + n) * K * K;
         float* dst = Pb + buf * K * PK;
 #pragma unroll 4
-        for (int e = threadIdx.x; e < K * K / 4; e += 256) {
+        for (int e = threadIdx.x; e < K * K / 4; e += NT) {
             const int i = e / (K / 4), l4 = e - i * (K / 4);
             cp_async16(dst + i * PK + 4 * l4, Pj + 4 * static_cast<int64_t>(e), true);
         }
         cp_async_commit();
     };
     issue_p(0, 0);
-    for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
+    for (int e = threadIdx.x; e < K * kChainCols; e += NT) {
         const int i = e >> 5, cc = e & 31;
         Ss[e] = S_in ? S_in[(n * K + i) * V + c0 + cc] : 0.0f;
     }
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __rest
         for (int l = 0; l < K; l += 4) {
             float4 p[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) p[r] = *reinterpret_cast<const float4*>(Ps + (tr + 32 * r) * PK + l);
+            for (int r = 0; r < R; ++r) p[r] = *reinterpret_cast<const float4*>(Ps + (tr + RS * r) * PK + l);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 sv = *reinterpret_cast<const float4*>(Ss + (l + q) * kChainCols + 4 * tc);
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __rest
         const float* Lj = S_loc ? S_loc + (static_cast<int64_t>(j) * n_total + n) * K * V : nullptr;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const int i = tr + 32 * r;
+            const int i = tr + RS * r;
             float4 add = make_float4(0.f, 0.f, 0.f, 0.f);
             if (Lj) {
                 const float* lp = Lj + static_cast<int64_t>(i) * V + c0 + 4 * tc;
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __rest
     }
     cp_async_wait<0>();
     __syncthreads();
-    for (int e = threadIdx.x; e < K * kChainCols; e += 256) {
+    for (int e = threadIdx.x; e < K * kChainCols; e += NT) {
         const int i = e >> 5, cc = e & 31;
         S_out[(n * K + i) * V + c0 + cc] = Ss[e];
     }
@@ -151,8 +153,8 @@ nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in,
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chain)");
         attr_done[dev] = true;
     }
-    const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / kChainCols), dim3(256),
-                                     smem, st, P, S_loc, S_in, S_out, m, n, V);
+    const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / kChainCols),
+                                     dim3(4 * K), smem, st, P, S_loc, S_in, S_out, m, n, V);
     if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
     return NVFP4_OK;
 }
@@ -314,8 +316,8 @@ nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, 
 // SM takes a contiguous run of items (tile fastest) and stages S_in^T once per
 // head; the m rows of the next item are copied asynchronously into the other A
 // buffer while the current item's MMAs and epilogue run, and each thread loads
-// its o values before the current A is rounded and multiplied.  Warp w reads TMEM lanes 32 (w % 4) .. + 31
-// (its token) and columns V/2 (w / 4) .. + V/2 - 1.  The MMA completion wait is
+// its o values before the current A is rounded and multiplied.  Warp w of 16 reads TMEM lanes
+// 32 (w % 4) .. + 31 (its token) and columns V/4 (w / 4) .. + V/4 - 1.  The MMA completion wait is
 // bounded; on expiry the CTA records kErrTimeoutCorrect and stops.
 __device__ __forceinline__ uint32_t sw128_off(int r, int col, int rows) {
     return static_cast<uint32_t>((col >> 5) * rows * 128 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) +
@@ -340,7 +342,7 @@ struct CorrTcLayout {
 };
 
 template <int K, int V>
-__global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __restrict__ m,
+__global__ void __launch_bounds__(512, 1) scan_correct_tc_kernel(const float* __restrict__ m,
                                                                  const float* __restrict__ S_in,
                                                                  float* __restrict__ o, int64_t T, int Hv,
                                                                  int64_t n_items, int per_cta,
@@ -348,8 +350,9 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
                                                                  unsigned int* __restrict__ err) {
     using L = CorrTcLayout<K, V>;
     constexpr uint32_t IDESC = idesc_tf32(kTcTok, V, false, false);
-    constexpr int CPT = kTcTok * K / 4 / 256;       // 16-byte chunks of A per thread
-    constexpr int HALF = V / 2;                     // columns per warp
+    constexpr int NT = 512;
+    constexpr int CPT = kTcTok * K / 4 / NT;        // 16-byte chunks of A per thread
+    constexpr int COLS = V / 4;                     // columns per warp
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
     const int64_t tiles = (T + kTcTok - 1) / kTcTok;
     const int64_t i0 = static_cast<int64_t>(blockIdx.x) * per_cta;
     const int64_t i1 = i0 + per_cta < n_items ? i0 + per_cta : n_items;
-    const int q = warp & 3, ch = warp >> 2;
+    const int q = warp & 3, cg = warp >> 2;
     // this thread's A chunks: e = u * 256 + tid -> row e / (K/4), column 4 (e % (K/4))
     auto issue_a = [&](int64_t item, int buf) {
         const int64_t bh = item / tiles, t0 = (item - bh * tiles) * kTcTok;
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
         uint8_t* dst = sm + L::A + buf * L::A_BYTES;
 #pragma unroll
         for (int u = 0; u < CPT; ++u) {
-            const int e = u * 256 + threadIdx.x;
+            const int e = u * NT + threadIdx.x;
             const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
             const int64_t t = t0 + r;
             const bool valid = t < T;
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
         if (bh != cur) {    // stage B = S_in[b,h]^T, TF32
             cur = bh;
             const float* Sb = S_in + bh * K * V;
-            for (int e = threadIdx.x; e < K * V / 4; e += 256) {
+            for (int e = threadIdx.x; e < K * V / 4; e += NT) {
                 const int i = e / (V / 4), j4 = (e - i * (V / 4)) * 4;
                 const float4 v = *reinterpret_cast<const float4*>(Sb + static_cast<int64_t>(i) * V + j4);
                 *reinterpret_cast<float*>(sm + L::Bm + sw128_off(j4 + 0, i, V)) = tf32_rn(v.x);
@@ -413,20 +416,20 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
         // previous item's MMAs, has completed)
         if (it + 1 < i1) issue_a(it + 1, buf ^ 1);
         else cp_async_commit();
-        // this thread's token and HALF columns of o, loaded while A is rounded and the MMAs run
+        // this thread's token and COLS columns of o, loaded while A is rounded and the MMAs run
         const int r = 32 * q + lane;
         const int64_t t = t0 + r;
-        float* orow = o + ((b * T + t) * Hv + h) * V + HALF * ch;
-        float4 ov[HALF / 4];
+        float* orow = o + ((b * T + t) * Hv + h) * V + COLS * cg;
+        float4 ov[COLS / 4];
 #pragma unroll
-        for (int c = 0; c < HALF / 4; ++c)
+        for (int c = 0; c < COLS / 4; ++c)
             ov[c] = t < T ? *reinterpret_cast<const float4*>(orow + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
         cp_async_wait<1>();
         {   // round this thread's own chunks of the current buffer to TF32
             uint8_t* a = sm + L::A + buf * L::A_BYTES;
 #pragma unroll
             for (int u = 0; u < CPT; ++u) {
-                const int e = u * 256 + threadIdx.x;
+                const int e = u * NT + threadIdx.x;
                 const int r = e / (K / 4), c4 = (e - r * (K / 4)) * 4;
                 float4* p = reinterpret_cast<float4*>(a + sw128_off(r, c4, kTcTok));
                 const float4 v = *p;
@@ -452,20 +455,22 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
         }
         phase ^= 1;
         tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < HALF / 32; ++cc) {
-            uint32_t x[32];
-            tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + HALF * ch + 32 * cc, x);
+        {
+            uint32_t x[COLS];
+            if constexpr (COLS == 32)
+                tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + COLS * cg, x);
+            else
+                tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + COLS * cg, x);
             tmem_wait_ld();
             if (t < T) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float4 y = ov[8 * cc + c];
+                for (int c = 0; c < COLS / 4; ++c) {
+                    float4 y = ov[c];
                     y.x += __uint_as_float(x[4 * c + 0]);
                     y.y += __uint_as_float(x[4 * c + 1]);
                     y.z += __uint_as_float(x[4 * c + 2]);
                     y.w += __uint_as_float(x[4 * c + 3]);
-                    *reinterpret_cast<float4*>(orow + 32 * cc + 4 * c) = y;
+                    *reinterpret_cast<float4*>(orow + 4 * c) = y;
                     mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))));
                 }
             }
@@ -475,14 +480,14 @@ __global__ void __launch_bounds__(256, 1) scan_correct_tc_kernel(const float* __
     }
     cp_async_wait<0>();
     if (o_amax) {
-        __shared__ unsigned int wmax[8];
+        __shared__ unsigned int wmax[NT / 32];
         const unsigned int wm = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
         if (lane == 0) wmax[warp] = wm;
         __syncthreads();
         if (threadIdx.x == 0) {
             unsigned int bm = wmax[0];
 #pragma unroll
-            for (int i = 1; i < 8; ++i) bm = bm > wmax[i] ? bm : wmax[i];
+            for (int i = 1; i < NT / 32; ++i) bm = bm > wmax[i] ? bm : wmax[i];
             atomicMax(o_amax, bm);
         }
     }
@@ -515,7 +520,7 @@ nvfp4_status launch_correct_tc(const float* m, const float* S_in, float* o, int 
     const int64_t slots = num_sms();
     const int per_cta = static_cast<int>((n_items + slots - 1) / slots);
     const unsigned grid = static_cast<unsigned>((n_items + per_cta - 1) / per_cta);
-    const cudaError_t e = launch_pdl(scan_correct_tc_kernel<K, V>, dim3(grid), dim3(256), smem, st, m, S_in, o, T,
+    const cudaError_t e = launch_pdl(scan_correct_tc_kernel<K, V>, dim3(grid), dim3(512), smem, st, m, S_in, o, T,
                                      Hv, n_items, per_cta, o_amax, err);
     if (e != cudaSuccess) return cuda_fail(e, "scan correct launch");
     return NVFP4_OK;
