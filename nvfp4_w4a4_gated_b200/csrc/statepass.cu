@@ -57,17 +57,17 @@ __global__ void __launch_bounds__(256) identity_fill_kernel(float* __restrict__ 
 // per (n, 32 columns) carries its K x 32 slice through the whole chain in
 // shared memory.  P[j+1][n] (K x K) is copied asynchronously into the second of
 // two shared buffers while step j computes; rows are padded by 4 floats so the
-// four consecutive rows a warp reads at once fall in different banks.  4K
-// threads; thread (tr, tc) owns rows tr and tr + K/2 and columns 4 tc .. 4 tc + 3.
+// four consecutive rows a warp reads at once fall in different banks.  Thread
+// (tr, tc) of 256 owns rows tr + 32 r (r < K / 32) and columns 4 tc .. 4 tc + 3.
 constexpr int kChainCols = 32;
 template <int K>
-__global__ void __launch_bounds__(4 * K, 1) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
-                                                               const float* S_in, float* S_out, int m,
-                                                               int64_t n_total, int V) {
+__global__ void __launch_bounds__(256, 1) state_chain_kernel(const float* __restrict__ P, const float* S_loc,
+                                                             const float* S_in, float* S_out, int m,
+                                                             int64_t n_total, int V) {
     pdl_wait_and_trigger();
-    constexpr int NT = 4 * K;          // threads
-    constexpr int R = 2;
-    constexpr int RS = K / 2;          // row stride between a thread's rows
+    constexpr int NT = 256;            // threads
+    constexpr int R = K / 32;          // rows per thread
+    constexpr int RS = 32;             // row stride between a thread's rows
     constexpr int PK = K + 4;
     extern __shared__ __align__(16) float smem[];
     float* Pb = smem;                      // [2][K][K + 4]
@@ -154,7 +154,7 @@ nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in,
         attr_done[dev] = true;
     }
     const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / kChainCols),
-                                     dim3(4 * K), smem, st, P, S_loc, S_in, S_out, m, n, V);
+                                     dim3(256), smem, st, P, S_loc, S_in, S_out, m, n, V);
     if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
     return NVFP4_OK;
 }
@@ -315,9 +315,11 @@ nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, 
 // 128-byte-swizzled K-major images and rounded to TF32 (nearest).  One CTA per
 // SM takes a contiguous run of items (tile fastest) and stages S_in^T once per
 // head; the m rows of the next item are copied asynchronously into the other A
-// buffer while the current item's MMAs and epilogue run, and each thread loads
-// its o values before the current A is rounded and multiplied.  Warp w of 16 reads TMEM lanes
-// 32 (w % 4) .. + 31 (its token) and columns V/4 (w / 4) .. + V/4 - 1.  The MMA completion wait is
+// buffer while the current item's MMAs and epilogue run.  The accumulator drains
+// through the current A buffer (warp w of 16 reads TMEM lanes 32 (w % 4) .. + 31,
+// one token each, and columns V/4 (w / 4) .. + V/4 - 1, and writes them as
+// row-swizzled 16-byte chunks), so o is read and written in whole rows; the o
+// loads are issued while the MMAs run.  The MMA completion wait is
 // bounded; on expiry the CTA records kErrTimeoutCorrect and stops.
 __device__ __forceinline__ uint32_t sw128_off(int r, int col, int rows) {
     return static_cast<uint32_t>((col >> 5) * rows * 128 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) +
@@ -333,8 +335,8 @@ constexpr int kTcTok = 128;     // tokens per item (MMA M)
 
 template <int K, int V>
 struct CorrTcLayout {
-    static constexpr uint32_t A_BYTES = kTcTok * K * 4;
-    static constexpr uint32_t A = 0;                           // two [128 tokens x K] images
+    static constexpr uint32_t A_BYTES = kTcTok * (K > V ? K : V) * 4;
+    static constexpr uint32_t A = 0;     // two [128 tokens x K] images; the drained D tile reuses one
     static constexpr uint32_t Bm = A + 2 * A_BYTES;            // [V columns x K] image
     static constexpr uint32_t B_BYTES = V * K * 4;
     static constexpr uint32_t BAR = Bm + B_BYTES;
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(512, 1) scan_correct_tc_kernel(const float* __
     const int64_t i0 = static_cast<int64_t>(blockIdx.x) * per_cta;
     const int64_t i1 = i0 + per_cta < n_items ? i0 + per_cta : n_items;
     const int q = warp & 3, cg = warp >> 2;
-    // this thread's A chunks: e = u * 256 + tid -> row e / (K/4), column 4 (e % (K/4))
+    // this thread's A chunks: e = u * NT + tid -> row e / (K/4), column 4 (e % (K/4))
     auto issue_a = [&](int64_t item, int buf) {
         const int64_t bh = item / tiles, t0 = (item - bh * tiles) * kTcTok;
         const int64_t b = bh / Hv, h = bh - b * Hv;
@@ -416,14 +418,6 @@ __global__ void __launch_bounds__(512, 1) scan_correct_tc_kernel(const float* __
         // previous item's MMAs, has completed)
         if (it + 1 < i1) issue_a(it + 1, buf ^ 1);
         else cp_async_commit();
-        // this thread's token and COLS columns of o, loaded while A is rounded and the MMAs run
-        const int r = 32 * q + lane;
-        const int64_t t = t0 + r;
-        float* orow = o + ((b * T + t) * Hv + h) * V + COLS * cg;
-        float4 ov[COLS / 4];
-#pragma unroll
-        for (int c = 0; c < COLS / 4; ++c)
-            ov[c] = t < T ? *reinterpret_cast<const float4*>(orow + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
         cp_async_wait<1>();
         {   // round this thread's own chunks of the current buffer to TF32
             uint8_t* a = sm + L::A + buf * L::A_BYTES;
@@ -448,6 +442,18 @@ __global__ void __launch_bounds__(512, 1) scan_correct_tc_kernel(const float* __
                             sdesc_kmajor_sw128(bb + (j >> 2) * V * 128 + (j & 3) * 32), IDESC, j > 0 ? 1u : 0u);
             mma_commit(bar);
         }
+        // o of this item in the coalesced mapping (a warp per 512 bytes of rows), loaded
+        // while the MMAs run: chunk e = u NT + tid is row e / (V/4), 16-byte chunk e % (V/4)
+        constexpr int PCH = kTcTok * (V / 4) / NT;
+        float4 ov[PCH];
+#pragma unroll
+        for (int u = 0; u < PCH; ++u) {
+            const int e = u * NT + threadIdx.x;
+            const int rr = e / (V / 4), cc = e - rr * (V / 4);
+            const int64_t tt = t0 + rr;
+            ov[u] = tt < T ? *reinterpret_cast<const float4*>(o + ((b * T + tt) * Hv + h) * V + 4 * cc)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         const bool ok = __syncthreads_and(mbar_wait(bar, phase, err, kErrTimeoutCorrect));
         if (!ok) {
             all_ok = false;
@@ -455,28 +461,42 @@ __global__ void __launch_bounds__(512, 1) scan_correct_tc_kernel(const float* __
         }
         phase ^= 1;
         tc_fence_after();
-        {
+        {   // D rows (thread = token) into the current A buffer, 16-byte chunks XOR-swizzled by row
             uint32_t x[COLS];
             if constexpr (COLS == 32)
                 tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + COLS * cg, x);
             else
                 tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + COLS * cg, x);
             tmem_wait_ld();
-            if (t < T) {
+            const int r = 32 * q + lane;
+            uint8_t* drow = sm + L::A + buf * L::A_BYTES + r * V * 4;
 #pragma unroll
-                for (int c = 0; c < COLS / 4; ++c) {
-                    float4 y = ov[c];
-                    y.x += __uint_as_float(x[4 * c + 0]);
-                    y.y += __uint_as_float(x[4 * c + 1]);
-                    y.z += __uint_as_float(x[4 * c + 2]);
-                    y.w += __uint_as_float(x[4 * c + 3]);
-                    *reinterpret_cast<float4*>(orow + 4 * c) = y;
-                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))));
-                }
+            for (int c = 0; c < COLS / 4; ++c) {
+                const int chunk = (COLS * cg) / 4 + c;
+                *reinterpret_cast<uint4*>(drow + ((chunk ^ (r & 7)) << 4)) =
+                    make_uint4(x[4 * c + 0], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
             }
         }
         tc_fence_before();
-        __syncthreads();    // TMEM read and B free before the next item
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < PCH; ++u) {
+            const int e = u * NT + threadIdx.x;
+            const int rr = e / (V / 4), cc = e - rr * (V / 4);
+            const int64_t tt = t0 + rr;
+            if (tt < T) {
+                const float4 d = *reinterpret_cast<const float4*>(sm + L::A + buf * L::A_BYTES + rr * V * 4 +
+                                                                  ((cc ^ (rr & 7)) << 4));
+                float4 y = ov[u];
+                y.x += d.x;
+                y.y += d.y;
+                y.z += d.z;
+                y.w += d.w;
+                *reinterpret_cast<float4*>(o + ((b * T + tt) * Hv + h) * V + 4 * cc) = y;
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y.x), fabsf(y.y)), fmaxf(fabsf(y.z), fabsf(y.w))));
+            }
+        }
+        __syncthreads();    // the D tile read and B free before the next item
     }
     cp_async_wait<0>();
     if (o_amax) {
