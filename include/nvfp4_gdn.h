@@ -334,7 +334,9 @@ typedef struct {
 typedef struct {
     size_t x_codes, x_sf, x_scale; /* quantised input */
     size_t proj;                   /* float32 [B*T x N_in] fused projection */
-    size_t q_hat, k_hat, g, beta;  /* gate / normalisation outputs */
+    size_t q_hat, k_hat, g, beta;  /* g, beta: the gates; q_hat, k_hat: room for gdn_gates'
+                                      normalised q, k (the layer's scans normalise q and k
+                                      themselves and leave these two regions unwritten) */
     size_t o;                      /* float32 [B*T x Hv*V] scan output */
     size_t o_gated;                /* float32 [B*T x Hv*V] gated output (an empty
                                       region when out_norm is NULL) */

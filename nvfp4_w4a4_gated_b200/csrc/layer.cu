@@ -131,8 +131,6 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     nvfp4_tensor oq{reinterpret_cast<uint8_t*>(ws + L.o_codes), reinterpret_cast<uint8_t*>(ws + L.o_sf),
                     reinterpret_cast<float*>(ws + L.o_scale), BT, HvV};
     float* proj = reinterpret_cast<float*>(ws + L.proj);
-    float* q_hat = reinterpret_cast<float*>(ws + L.q_hat);
-    float* k_hat = reinterpret_cast<float*>(ws + L.k_hat);
     float* g = reinterpret_cast<float*>(ws + L.g);
     float* beta = reinterpret_cast<float*>(ws + L.beta);
     float* o = reinterpret_cast<float*>(ws + L.o);
@@ -154,22 +152,21 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
         qkv = cv;
         ld_qkv = qkv_width(d);
     }
-    // T > 1: the chunked scan reads the raw q, k slices and normalises them while
-    // staging them, so only g and beta are formed here.
-    // T = 1 (decode): the recurrent scan reads normalised q_hat, k_hat.
+    // Both scans read the raw q, k slices and normalise them themselves (the
+    // chunked one while staging a chunk, the recurrent one per token), so only g
+    // and beta are formed here.
     const bool chunked = T > 1;
-    if (!chunked && (s = l2norm_launch(qkv, ld_qkv, BT, d, q_hat, k_hat, st)) != NVFP4_OK) return s;
     if ((s = gate_only_launch(proj, ldp, BT, d, w->A_log, w->dt_bias, g, beta, st)) != NVFP4_OK) return s;
-    const float* q_in = chunked ? qkv : q_hat;
-    const float* k_in = chunked ? qkv + static_cast<int64_t>(d.Hk) * d.K : k_hat;
-    const int64_t ld_qk = chunked ? ld_qkv : static_cast<int64_t>(d.Hk) * d.K;
+    const float* q_in = qkv;
+    const float* k_in = qkv + static_cast<int64_t>(d.Hk) * d.K;
+    const int64_t ld_qk = ld_qkv;
     const float scale = 1.0f / sqrtf(static_cast<float>(d.K));
     // the scan folds max|o| into the quantiser's amax word as it writes o, so the o
     // quantiser runs its quantisation pass only
     unsigned int* o_amax = qw + 2;
     if ((s = scan_launch(q_in, k_in, qkv + 2ll * d.Hk * d.K, ld_qkv, g, beta, B, T, d, scale, form,
                          chunked ? GDN_SCAN_CHUNKED : GDN_SCAN_RECURRENT, state_in, state_out, o, ws + L.scan_ws, st,
-                         o_amax, ld_qk, chunked ? 1 : 0)) != NVFP4_OK)
+                         o_amax, ld_qk, 1)) != NVFP4_OK)
         return s;
     const float* oq_in = o;
     unsigned int* oq_amax = o_amax;

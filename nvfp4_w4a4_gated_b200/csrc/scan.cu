@@ -68,9 +68,13 @@ struct ChunkRec {
 };
 
 // --------------------------------------------------------------- recurrent --
+// q and k rows of token (b, t) at (b*T + t) * ld_qk (+ key head * K); with
+// normalize_qk they are the raw projection slices and are scaled here by
+// 1 / sqrt(sum x^2 + 1e-6) per key head.
 template <int K>
 __global__ void __launch_bounds__(128) scan_recurrent_kernel(
-    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, int64_t ld_v,
+    const float* __restrict__ q, const float* __restrict__ k, int64_t ld_qk, int normalize_qk,
+    const float* __restrict__ v, int64_t ld_v,
     const float* __restrict__ g, const float* __restrict__ beta, int B, int64_t T, int Hk, int Hv, int V, float scale,
     int form, const float* state_in, float* state_out, float* __restrict__ o, unsigned int* __restrict__ o_amax) {
     pdl_wait_and_trigger();
@@ -89,16 +93,34 @@ __global__ void __launch_bounds__(128) scan_recurrent_kernel(
 
     __shared__ float ks[K], qs[K];
     __shared__ float red1[4][32], red2[4][32];
+    __shared__ float inv_norm[2];
     for (int64_t t = 0; t < T; ++t) {
         const int64_t tok = static_cast<int64_t>(b) * T + t;
         if (threadIdx.x < K) {
-            ks[threadIdx.x] = k[(tok * Hk + hk) * K + threadIdx.x];
-            qs[threadIdx.x] = q[(tok * Hk + hk) * K + threadIdx.x];
+            ks[threadIdx.x] = k[tok * ld_qk + static_cast<int64_t>(hk) * K + threadIdx.x];
+            qs[threadIdx.x] = q[tok * ld_qk + static_cast<int64_t>(hk) * K + threadIdx.x];
         }
         const float alpha = expf(g[tok * Hv + h]);
         const float bt = beta[tok * Hv + h];
         const float vj = v[tok * ld_v + static_cast<int64_t>(h) * V + j];
         __syncthreads();
+        if (normalize_qk) {   // warp 0 takes |k|, warp 1 |q|
+            if (w < 2) {
+                const float* src = w == 0 ? ks : qs;
+                float ss = 0.0f;
+#pragma unroll
+                for (int i = lane; i < K; i += 32) ss = fmaf(src[i], src[i], ss);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                if (lane == 0) inv_norm[w] = 1.0f / sqrtf(ss + 1e-6f);
+            }
+            __syncthreads();
+            if (threadIdx.x < K) {
+                ks[threadIdx.x] *= inv_norm[0];
+                qs[threadIdx.x] *= inv_norm[1];
+            }
+            __syncthreads();
+        }
         float p = 0.0f;
 #pragma unroll
         for (int i = 0; i < RW; ++i) p = fmaf(S[i], ks[w * RW + i], p);
@@ -949,15 +971,15 @@ nvfp4_status scan_launch(const float* q, const float* k, const float* v, int64_t
                          const float* s_in, float* s_out, float* o, void* ws, cudaStream_t st,
                          unsigned int* o_amax, int64_t ld_qk, int normalize_qk) {
     const bool chunked = algo == GDN_SCAN_CHUNKED || (algo == GDN_SCAN_AUTO && T > 1);
-    if (!chunked && (normalize_qk || ld_qk != static_cast<int64_t>(d.Hk) * d.K))
-        return fail(NVFP4_ERR_INVALID_ARG, "raw q/k rows need the chunked scan");
     if (!chunked) {
         const unsigned blocks = static_cast<unsigned>(B * d.Hv * (d.V / 32));
         const cudaError_t e =
-            d.K == 128 ? launch_pdl(scan_recurrent_kernel<128>, dim3(blocks), dim3(128), 0, st, q, k, v, ld_v, g, beta,
-                                    B, T, d.Hk, d.Hv, d.V, scale, form, s_in, s_out, o, o_amax)
-                       : launch_pdl(scan_recurrent_kernel<64>, dim3(blocks), dim3(128), 0, st, q, k, v, ld_v, g, beta, B,
-                                    T, d.Hk, d.Hv, d.V, scale, form, s_in, s_out, o, o_amax);
+            d.K == 128 ? launch_pdl(scan_recurrent_kernel<128>, dim3(blocks), dim3(128), 0, st, q, k, ld_qk,
+                                    normalize_qk, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form, s_in, s_out, o,
+                                    o_amax)
+                       : launch_pdl(scan_recurrent_kernel<64>, dim3(blocks), dim3(128), 0, st, q, k, ld_qk,
+                                    normalize_qk, v, ld_v, g, beta, B, T, d.Hk, d.Hv, d.V, scale, form, s_in, s_out, o,
+                                    o_amax);
         if (e != cudaSuccess) return cuda_fail(e, "recurrent scan launch");
         return NVFP4_OK;
     }
