@@ -40,9 +40,10 @@ UNIT = "tokens/s"
 WORKLOAD = "gdn_layer_prefill_B1_T4096_h5120_hk16_hv32_k128_v128"
 NVFP4_OVER_BF16 = 4.0   # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
 
-# launches of this library's kernels per gdn_layer_forward (T > 1): quantise x (amax, quant),
-# in_proj GEMM, gates (norm, gate), scan (prep, sequential), quantise o (amax, quant), out_proj GEMM
-LAUNCHES_PER_STEP = 10
+# launches of this library's kernels per gdn_layer_forward (T > 1), as the ncu launch list
+# shows them: zero the quantiser words, quantise x (one cooperative launch), in_proj GEMM,
+# gates (g, beta), scan (prep, sequential), quantise o (from the scan's amax), out_proj GEMM
+LAUNCHES_PER_STEP = 8
 
 
 def peaks():
