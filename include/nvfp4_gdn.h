@@ -59,7 +59,8 @@ typedef enum {
 typedef void* nvfp4_stream_t; /* cudaStream_t */
 
 enum { NVFP4_DTYPE_BF16 = 0, NVFP4_DTYPE_FP32 = 1 };
-enum { NVFP4_QUANT_COMPUTE_SCALE = 0, NVFP4_QUANT_GIVEN_SCALE = 1 };
+enum { NVFP4_QUANT_COMPUTE_SCALE = 0, NVFP4_QUANT_GIVEN_SCALE = 1, NVFP4_QUANT_AMAX_ONLY = 2,
+       NVFP4_QUANT_FROM_AMAX = 3 };
 enum { GDN_FORM_PAGES = 0, GDN_FORM_STANDARD = 1 };
 enum { GDN_SCAN_AUTO = 0, GDN_SCAN_RECURRENT = 1, GDN_SCAN_CHUNKED = 2 };
 
@@ -124,11 +125,20 @@ NVFP4_API size_t nvfp4_quantize_workspace_size(void);
  *            amax < 2^-100) is computed on the device and written to
  *            *out->global_scale;  NVFP4_QUANT_GIVEN_SCALE: the value already
  *            in *out->global_scale is used (harmonised weight scales).
+ *            The per-tensor scale of a tensor split across GPUs (rows of a
+ *            sequence on several ranks) takes two calls around a collective:
+ *            NVFP4_QUANT_AMAX_ONLY sets workspace word 0 to the float bits of
+ *            max|x| and writes nothing else; after a max all-reduce of that
+ *            word over the ranks (as 32-bit integers: non-negative floats order
+ *            as their bits), NVFP4_QUANT_FROM_AMAX quantises with S formed on
+ *            the device from word 0 as in COMPUTE_SCALE and writes S to
+ *            *out->global_scale.  Each rank's codes and scales then equal
+ *            those of the whole tensor quantised at once.
  *   Per block of 16: sb = E4M3_rn_satfinite(m / (6 S)), m the block amax;
  *   codes = E2M1_rn_satfinite(x * (1 / (E4M3(sb) * S))), all float32 ops
  *   rounded to nearest even; blocks whose E4M3(sb) * S is 0 get code 0.
- *   workspace: device, >= nvfp4_quantize_workspace_size() bytes (required in
- *            COMPUTE_SCALE mode; may be NULL with GIVEN_SCALE).
+ *   workspace: device, >= nvfp4_quantize_workspace_size() bytes, 16-byte
+ *            aligned (required except with GIVEN_SCALE, where it may be NULL).
  * Requirements: rows >= 1, cols >= 64, cols % 64 == 0. */
 NVFP4_API nvfp4_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t rows, int64_t cols, int64_t ld,
                             const nvfp4_tensor* out, int32_t flags, void* workspace,

@@ -22,13 +22,14 @@ __all__ = [
     "gdn_scan", "gdn_scan_noalloc", "gdn_output_gate", "gdn_short_conv", "gdn_layer_forward", "layer_workspace_layout",
     "check_device_error", "gdn_scan_transition", "gdn_state_combine", "gdn_scan_correct", "gdn_scan_span",
     "selftest_wait_timeout", "FORM_PAGES",
-    "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS",
+    "FORM_STANDARD", "SCAN_AUTO", "SCAN_RECURRENT", "SCAN_CHUNKED", "EXPORTED_SYMBOLS", "QUANT_COMPUTE_SCALE",
+    "QUANT_GIVEN_SCALE", "QUANT_AMAX_ONLY", "QUANT_FROM_AMAX",
 ]
 
 FORM_PAGES, FORM_STANDARD = 0, 1
 SCAN_AUTO, SCAN_RECURRENT, SCAN_CHUNKED = 0, 1, 2
 DTYPE_BF16, DTYPE_FP32 = 0, 1
-QUANT_COMPUTE_SCALE, QUANT_GIVEN_SCALE = 0, 1
+QUANT_COMPUTE_SCALE, QUANT_GIVEN_SCALE, QUANT_AMAX_ONLY, QUANT_FROM_AMAX = 0, 1, 2, 3
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA", 5: "TIMEOUT", 6: "WORKSPACE"}
 
@@ -216,9 +217,13 @@ def _scratch(nbytes: int, device) -> torch.Tensor:
 
 
 def nvfp4_quantize(x: torch.Tensor, out: NVFP4Matrix | None = None, given_scale: bool = False, workspace=None,
-                   stream=None) -> NVFP4Matrix:
+                   stream=None, mode: int | None = None) -> NVFP4Matrix:
     """Quantise a bf16 or fp32 CUDA matrix to NVFP4 (the per-tensor scale is
-    computed on the device unless ``given_scale``, which uses ``out.scale``)."""
+    computed on the device unless ``given_scale``, which uses ``out.scale``).
+    ``mode`` QUANT_AMAX_ONLY sets workspace word 0 to max|x| and writes nothing
+    else; QUANT_FROM_AMAX quantises with S formed from workspace word 0 (for a
+    tensor split across ranks: AMAX_ONLY, a max all-reduce of the word, then
+    FROM_AMAX)."""
     assert x.is_cuda and x.dim() == 2 and x.stride(1) == 1
     dtype = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_FP32}[x.dtype]
     rows, cols = x.shape
@@ -226,9 +231,10 @@ def nvfp4_quantize(x: torch.Tensor, out: NVFP4Matrix | None = None, given_scale:
         out = NVFP4Matrix.empty(rows, cols, x.device)
     if workspace is None:
         workspace = _scratch(lib().nvfp4_quantize_workspace_size(), x.device)
+    if mode is None:
+        mode = QUANT_GIVEN_SCALE if given_scale else QUANT_COMPUTE_SCALE
     t = out.c()
-    _check(lib().nvfp4_quantize(_ptr(x), dtype, rows, cols, x.stride(0), ctypes.byref(t),
-                                QUANT_GIVEN_SCALE if given_scale else QUANT_COMPUTE_SCALE, _ptr(workspace),
+    _check(lib().nvfp4_quantize(_ptr(x), dtype, rows, cols, x.stride(0), ctypes.byref(t), mode, _ptr(workspace),
                                 workspace.numel(), _stream(stream)))
     return out
 

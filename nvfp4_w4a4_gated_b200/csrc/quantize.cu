@@ -390,6 +390,16 @@ nvfp4_status quant_dispatch(const T* x, int64_t rows, int64_t cols, int64_t ld, 
     const int64_t atoms = ((rows + 127) / 128) * (cols / 64);
     const int64_t groups_needed = (atoms + kQuantGroups - 1) / kQuantGroups;
     cudaError_t e;
+    if (flags == NVFP4_QUANT_AMAX_ONLY) {   // word 0 := max|x|, nothing else written
+        e = launch_pdl(zero_words_kernel, dim3(1), dim3(32), 0, st, ws, 2);
+        if (e != cudaSuccess) return cuda_fail(e, "zero amax words");
+        int64_t blocks = (rows + 7) / 8;
+        const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+        if (blocks > cap) blocks = cap;
+        e = launch_pdl(amax_kernel<T>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, x, rows, cols, ld, ws);
+        if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+        return NVFP4_OK;
+    }
     if (flags == NVFP4_QUANT_COMPUTE_SCALE || flags == kQuantComputeZeroedWs) {
         if (flags == NVFP4_QUANT_COMPUTE_SCALE) {
             e = launch_pdl(zero_words_kernel, dim3(1), dim3(32), 0, st, ws, 2);
@@ -444,6 +454,7 @@ nvfp4_status zero_words_launch(unsigned int* w, int n, cudaStream_t st) {
 
 // flags: NVFP4_QUANT_COMPUTE_SCALE (amax and quantisation, one cooperative
 // launch; kQuantComputeZeroedWs when the caller has zeroed workspace[0..1]),
+// NVFP4_QUANT_AMAX_ONLY (workspace[0] := max|x| only),
 // NVFP4_QUANT_GIVEN_SCALE (S read from out.global_scale), or
 // kQuantFromAmax (S from the amax word at workspace[0], which a producer such
 // as the scan has filled; the quantisation pass only).
@@ -483,7 +494,8 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t r
     using namespace nvg;
     if (!x) return fail(NVFP4_ERR_INVALID_ARG, "x is null");
     if (x_dtype != NVFP4_DTYPE_BF16 && x_dtype != NVFP4_DTYPE_FP32) return fail(NVFP4_ERR_INVALID_ARG, "bad x_dtype");
-    if (flags != NVFP4_QUANT_COMPUTE_SCALE && flags != NVFP4_QUANT_GIVEN_SCALE)
+    if (flags != NVFP4_QUANT_COMPUTE_SCALE && flags != NVFP4_QUANT_GIVEN_SCALE && flags != NVFP4_QUANT_AMAX_ONLY &&
+        flags != NVFP4_QUANT_FROM_AMAX)
         return fail(NVFP4_ERR_INVALID_ARG, "bad flags");
     nvfp4_status s = validate_tensor(out, "out");
     if (s != NVFP4_OK) return s;
@@ -491,8 +503,9 @@ extern "C" nvfp4_status nvfp4_quantize(const void* x, int32_t x_dtype, int64_t r
     if (ld < cols) return fail(NVFP4_ERR_INVALID_ARG, "ld < cols");
     const int64_t esz = x_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
     if (!aligned16(x) || (ld * esz) % 16) return fail(NVFP4_ERR_MISALIGNED, "x / ld not 16-byte aligned");
-    if (flags == NVFP4_QUANT_COMPUTE_SCALE &&
+    if (flags != NVFP4_QUANT_GIVEN_SCALE &&
         (!workspace || workspace_bytes < nvfp4_quantize_workspace_size() || !aligned16(workspace)))
         return fail(NVFP4_ERR_WORKSPACE, "quantize workspace missing or too small");
-    return quantize_launch(x, x_dtype, rows, cols, ld, *out, flags, workspace, as_stream(stream));
+    return quantize_launch(x, x_dtype, rows, cols, ld, *out, flags == NVFP4_QUANT_FROM_AMAX ? kQuantFromAmax : flags,
+                           workspace, as_stream(stream));
 }

@@ -70,6 +70,11 @@ def test_quantize_validation():
     assert st == 6
     st, _ = _err(L.nvfp4_quantize(FAKE, 0, 64, 256, 256, ctypes.byref(t), 0, FAKE, 256, None))
     assert st == 1  # shape differs from out
+    st, _ = _err(L.nvfp4_quantize(FAKE, 0, 128, 256, 256, ctypes.byref(t), 4, FAKE, 256, None))
+    assert st == 1  # unknown flag
+    for flag in (nv.QUANT_AMAX_ONLY, nv.QUANT_FROM_AMAX):   # the word lives in the workspace
+        st, _ = _err(L.nvfp4_quantize(FAKE, 0, 128, 256, 256, ctypes.byref(t), flag, None, 0, None))
+        assert st == 6
 
 
 def test_gemm_validation():

@@ -115,3 +115,35 @@ def test_quantize_block_maxima_near_e4m3_midpoints(cuda_dev, amax):
     x[:blocks.shape[0]] = blocks
     x = x.reshape(-1, 64)
     _check(f32_device(x), x)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_rows_split_across_ranks_share_the_tensor_scale(cuda_dev, dtype):
+    """A tensor whose rows are split over three (emulated) ranks: each part's
+    amax word (AMAX_ONLY), the max over the parts (what a max all-reduce
+    gives), then each part quantised from that word (FROM_AMAX).  Every part's
+    codes, scales and S must equal the oracle's quantisation of the whole
+    tensor restricted to the part's rows."""
+    rows, cols = 700, 512
+    bits, x = gdn_synth.activations(77, rows, cols, hot="percent")
+    dev = bf16_device(bits) if dtype == "bf16" else f32_device(x)
+    codes, sf, S = oracle.quantize(x)
+    bounds = [0, 129, 130, rows]          # parts of 129, 1 and 570 rows
+    words = []
+    for a, b in zip(bounds, bounds[1:]):
+        ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        nv.nvfp4_quantize(dev[a:b], workspace=ws, mode=nv.QUANT_AMAX_ONLY)
+        words.append(ws)
+    torch.cuda.synchronize()
+    local = [w[:4].view(torch.int32).item() for w in words]
+    for (a, b), lw in zip(zip(bounds, bounds[1:]), local):
+        assert np.int32(lw).view(np.float32) == np.abs(x[a:b]).max()
+    glob = torch.stack([w[:4].view(torch.int32) for w in words]).amax(dim=0)
+    for (a, b), ws in zip(zip(bounds, bounds[1:]), words):
+        ws[:4].view(torch.int32).copy_(glob)
+        q = nv.nvfp4_quantize(dev[a:b], workspace=ws, mode=nv.QUANT_FROM_AMAX)
+        torch.cuda.synchronize()
+        nv.check_device_error()
+        assert q.scale.item() == float(S)
+        assert np.array_equal(q.codes.cpu().numpy(), codes[a:b])
+        assert np.array_equal(q.sf.cpu().numpy(), oracle.sf_linear_to_mma(sf[a:b], b - a, cols))
