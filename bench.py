@@ -232,6 +232,22 @@ def cpu_baseline(sample_tokens: int, seed: int):
 
 
 # ------------------------------------------------------------- our arm -----
+def max_over_ranks(values, dev, distributed: bool):
+    """Each timing as the maximum over the ranks (the slowest rank sets the
+    job's time); unchanged on one rank."""
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
+    if distributed:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_throughput(world: int, tokens_per_rank_step: int, steps: int, total_ms: float):
+    """Whole-job tokens and tokens/s: every rank's tokens over the slowest
+    rank's time (weak scaling: each rank runs the same workload)."""
+    tokens = world * tokens_per_rank_step * steps
+    return tokens, tokens / (total_ms / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import nvfp4_w4a4_gated_b200 as nv
     dev = torch.device("cuda", local_rank)
@@ -348,12 +364,8 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = t_start.elapsed_time(t_end)
 
     # ---- aggregate over ranks: max time
-    tvec = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        torch.distributed.all_reduce(tvec, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms = float(tvec[0]), float(tvec[1])
-    tokens = world * B * T * args.steps
-    value = tokens / (total_ms / 1e3)
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, dist)
+    tokens, value = job_throughput(world, B * T, args.steps, total_ms)
 
     pk = peaks()
     work = stage_work(sh, B, T)

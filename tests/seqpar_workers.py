@@ -79,3 +79,25 @@ def rank_main(rank, world, port, bounds, form, with_state, out_dir):
             f.write(f"{err_o} {err_S}\n")
     finally:
         dist.destroy_process_group()
+
+
+def bench_rank_main(rank, world, port, out_dir):
+    """bench.py's aggregation over gloo ranks: each rank reports its own times;
+    all must come back with the maximum, and the throughput counts every
+    rank's tokens over that time."""
+    import importlib.util
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+        spec = importlib.util.spec_from_file_location("bench_agg", os.path.join(root, "bench.py"))
+        b = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(b)
+        mine = [10.0 + rank, 20.0 - rank]
+        got = b.max_over_ranks(mine, torch.device("cpu"), True)
+        tokens, value = b.job_throughput(world, 4096, 10, got[0])
+        with open(os.path.join(out_dir, f"agg{rank}.txt"), "w") as f:
+            f.write(f"{got[0]} {got[1]} {tokens} {value}\n")
+    finally:
+        dist.destroy_process_group()

@@ -49,3 +49,14 @@ def test_single_process_path_needs_no_process_group():
     outs, S2 = segmented_scan(spans, 2, dims, state_in=torch.from_numpy(S0), ops=ops)
     got = np.concatenate([o.numpy().reshape(2, -1, dims.Hv, dims.V) for o in outs], axis=1)
     assert np.allclose(got, o_ref, atol=1e-12) and np.allclose(S2.numpy(), S_ref, atol=1e-12)
+
+
+def test_bench_aggregation_on_gloo_ranks(tmp_path):
+    """bench.py under N ranks: the max over ranks of each timing and the
+    whole-job throughput (all ranks' tokens over the slowest time)."""
+    world = 2
+    mp.spawn(seqpar_workers.bench_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    for r in range(world):
+        t0, t1, tokens, value = map(float, open(os.path.join(tmp_path, f"agg{r}.txt")).read().split())
+        assert (t0, t1) == (11.0, 20.0)
+        assert tokens == 2 * 4096 * 10 and abs(value - tokens / 0.011) < 1e-6 * value
