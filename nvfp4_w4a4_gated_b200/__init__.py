@@ -128,10 +128,18 @@ def _check(status: int):
         raise NVFP4Error(status, lib().nvfp4_last_error().decode())
 
 
+def _dev_addr(t) -> int:
+    """Device address of a CUDA tensor; a host tensor is refused here, before
+    any kernel could be handed a host pointer."""
+    if not t.is_cuda:
+        raise ValueError("the library takes CUDA tensors; got a tensor on " + str(t.device))
+    return t.data_ptr()
+
+
 def _ptr(t):
     if t is None:
         return None
-    return ctypes.c_void_p(t.data_ptr())
+    return ctypes.c_void_p(_dev_addr(t))
 
 
 def _stream(stream):
@@ -158,7 +166,7 @@ class NVFP4Matrix:
                            torch.empty(1, dtype=torch.float32, device=device), rows, cols)
 
     def c(self) -> _Tensor:
-        return _Tensor(self.codes.data_ptr(), self.sf.data_ptr(), self.scale.data_ptr(), self.rows, self.cols)
+        return _Tensor(_dev_addr(self.codes), _dev_addr(self.sf), _dev_addr(self.scale), self.rows, self.cols)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -189,7 +197,7 @@ class LayerWeights:
     conv_width: int = 4
 
     def c(self) -> _LayerWeights:
-        return _LayerWeights(self.w_in.c(), self.w_out.c(), self.A_log.data_ptr(), self.dt_bias.data_ptr(),
+        return _LayerWeights(self.w_in.c(), self.w_out.c(), _dev_addr(self.A_log), _dev_addr(self.dt_bias),
                              self.dims.c(), self.hidden, _ptr(self.out_norm), _ptr(self.conv_weight),
                              self.conv_width)
 

@@ -251,3 +251,21 @@ def test_state_passing_validation_and_sizes():
     assert st == 1 and "overlap" in msg
     st, _ = _err(L.gdn_scan_correct(FAKE, FAKE, big, 70000, 64, 32, 128, 128, None, None))
     assert st == 2
+
+
+def test_binding_refuses_host_tensors():
+    """A CPU tensor never reaches the library as a pointer: the binding raises
+    on the host before any call (on a GPU machine a host pointer in a kernel would
+    fault)."""
+    import torch
+    import pytest as _pytest
+    x = torch.zeros((64, 128), dtype=torch.float32)
+    with _pytest.raises(ValueError, match="CUDA tensors"):
+        nv._ptr(x)
+    S = torch.zeros((1, 2, 64, 64))
+    with _pytest.raises(ValueError, match="CUDA tensors"):
+        nv.gdn_state_combine(torch.zeros((1, 2, 64, 64)), S, S)
+    m = nv.NVFP4Matrix(torch.zeros((64, 32), dtype=torch.uint8), torch.zeros(512, dtype=torch.uint8),
+                       torch.zeros(1), 64, 64)
+    with _pytest.raises(ValueError, match="CUDA tensors"):
+        m.c()
