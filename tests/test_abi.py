@@ -255,7 +255,7 @@ def test_state_passing_validation_and_sizes():
 
 def test_binding_refuses_host_tensors():
     """A CPU tensor never reaches the library as a pointer: the binding raises
-    on the host before any call (on a GPU machine a host pointer in a kernel would
+    on the host before any call (on a machine with a GPU a host pointer in a kernel would
     fault)."""
     import torch
     import pytest as _pytest
