@@ -17,10 +17,13 @@
  *   - Pointers named in a call are DEVICE pointers owned by the caller unless
  *     the comment says host; the library allocates no device memory.  Scratch
  *     ("workspace") is sized by the matching *_workspace_size() call and
- *     passed in; it must stay valid until the stream reaches the call.
+ *     passed in; it must stay valid until the stream reaches the call.  The
+ *     one exception is gdn_scan_noalloc, which keeps its scratch in a fixed
+ *     array inside the library (see its comment).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *     default stream) and launches only this library's kernels (plus
- *     cudaMemsetAsync of workspace words).
+ *     default stream) and launches only this library's kernels (workspace
+ *     words that must start at zero are cleared by one of them, not by a
+ *     memset).
  *   - Arguments are validated on the host before anything is launched; a
  *     rejected call launches nothing and returns a non-OK status.  The
  *     message of the last failure on the calling host thread is returned by
@@ -179,7 +182,7 @@ NVFP4_API size_t gdn_scan_workspace_size(int32_t B, int64_t T, const gdn_dims* d
  * q_hat, k_hat: device [B x T x Hk x K]; v: device, token (b, t) row at
  * v + (b*T + t) * ld_v, head h at + h*V; g (log alpha), beta: device [B x T x Hv];
  * o: device [B x T x Hv x V]; state_in (NULL = zeros), state_out (NULL = not
- * written): device [B x Hv x K x V].  state_in may equal state_out.
+ * written): device [B x Hv x K x V], 16-byte aligned.  state_in may equal state_out.
  * algo: AUTO (chunked for T > 1, recurrent for T == 1), RECURRENT (token by
  * token), CHUNKED (chunks of 64 tokens, WY/UT form).
  * workspace: device, >= gdn_scan_workspace_size(B, T, dims, algo) bytes. */
@@ -204,8 +207,11 @@ NVFP4_API nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const fl
  *     NVFP4_ERR_WORKSPACE before anything is launched (64 MiB covers, e.g.,
  *     B = 1, 32 value heads of 128 x 128, T <= 896).
  *   - First use: the first call on a device looks up the array's device
- *     address (cudaGetSymbolAddress) with that device current; make that first
- *     call before any stream capture begins.
+ *     address (cudaGetSymbolAddress) with that device current and keeps it for
+ *     the life of the process; make that first call before any stream capture
+ *     begins.  A device reset (cudaDeviceReset, or the primary context being
+ *     destroyed and re-created) invalidates the kept address: do not call this
+ *     function on that device again in the same process.
  *   - Sharing: every call on a device uses the same array and leaves its
  *     contents behind (the chunk preparation overwrites all of it, nothing has
  *     to start at zero).  Calls whose executions overlap on the GPU -- on
@@ -367,7 +373,7 @@ NVFP4_API nvfp4_status gdn_layer_workspace_layout(const gdn_layer_weights* w, in
  * instead of o):
  *   x_bf16: device bf16 [B*T x hidden]; y: device float32 [B*T x hidden].
  *   state_in (NULL = zeros) / state_out (NULL = not written): device float32
- *   [B x Hv x K x V].  form: GDN_FORM_PAGES or GDN_FORM_STANDARD.
+ *   [B x Hv x K x V], 16-byte aligned.  form: GDN_FORM_PAGES or GDN_FORM_STANDARD.
  *   workspace: device, >= the layout's `total` bytes, 256-byte aligned. */
 NVFP4_API nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void* x_bf16, int32_t B, int64_t T,
                                float* y, const float* state_in, float* state_out, int32_t form,

@@ -12,6 +12,7 @@ import ctypes
 import dataclasses
 import math
 import os
+import re
 
 import torch
 
@@ -41,8 +42,20 @@ EXPORTED_SYMBOLS = [
     "gdn_state_combine", "gdn_scan_correct", "gdn_scan_span_workspace_size", "gdn_scan_span",
 ]
 
-# Size of the fixed scratch array gdn_scan_noalloc uses (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
-NOALLOC_MAX_SCRATCH_BYTES = 64 << 20
+
+
+def _header_size_macro(name: str) -> int:
+    """Value of a `#define NAME ((size_t)A << B)` size macro of the C header."""
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4_gdn.h")
+    m = re.search(r"#define\s+" + name + r"\s+\(\(size_t\)\s*(\d+)\s*<<\s*(\d+)\)", open(path).read())
+    if m is None:
+        raise RuntimeError(f"{name} not found in {path}")
+    return int(m.group(1)) << int(m.group(2))
+
+
+# Size of the fixed scratch array gdn_scan_noalloc uses, as the header defines it
+# (GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES).
+NOALLOC_MAX_SCRATCH_BYTES = _header_size_macro("GDN_SCAN_NOALLOC_MAX_SCRATCH_BYTES")
 
 
 class NVFP4Error(RuntimeError):

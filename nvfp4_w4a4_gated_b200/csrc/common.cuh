@@ -7,9 +7,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <utility>
-
+#include <atomic>
+#include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/nvfp4_gdn.h"
 
@@ -24,6 +25,41 @@ unsigned int* device_error_word();
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(nvfp4_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 int num_sms();
+
+// One-time set-up per device (for example raising a kernel's dynamic shared-memory
+// limit), safe under concurrent first calls from several host threads: the first
+// caller on a device runs the set-up under a lock; later callers see the flag
+// without locking.  A failed set-up is retried by the next call.
+struct PerDeviceOnce {
+    std::mutex mu;
+    std::atomic<bool> done[64];
+    PerDeviceOnce() {
+        for (auto& d : done) d.store(false, std::memory_order_relaxed);
+    }
+};
+
+template <typename F>
+nvfp4_status once_per_device(PerDeviceOnce& once, F&& setup) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(NVFP4_ERR_CUDA, "device ordinal outside 0..63");
+    if (once.done[dev].load(std::memory_order_acquire)) return NVFP4_OK;
+    std::lock_guard<std::mutex> lk(once.mu);
+    if (once.done[dev].load(std::memory_order_relaxed)) return NVFP4_OK;
+    const nvfp4_status s = setup();
+    if (s == NVFP4_OK) once.done[dev].store(true, std::memory_order_release);
+    return s;
+}
+
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` once per device.
+template <typename Kern>
+nvfp4_status smem_limit_once(PerDeviceOnce& once, Kern kernel, int bytes, const char* what) {
+    return once_per_device(once, [&]() -> nvfp4_status {
+        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, what);
+    });
+}
 
 // Build a 2-D tiled TMA descriptor over a row-major byte matrix [rows x row_bytes]
 // (row pitch = row_bytes) with a box of box_rows x box_bytes and 128-byte swizzle.

@@ -633,14 +633,10 @@ nvfp4_status launch_gemm_pair(const nvfp4_tensor& A, const nvfp4_tensor& B, floa
     if (s != NVFP4_OK) return s;
     s = make_tmap_f32_sw128(&tc, C, A.rows, B.rows, ldc, 32, 32);
     if (s != NVFP4_OK) return s;
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair smem)");
-        attr_done[dev] = true;
-    }
+    static PerDeviceOnce attr_once;
+    if ((s = smem_limit_once(attr_once, w4a4_gemm_pair_kernel, G::SMEM, "cudaFuncSetAttribute(gemm pair smem)")) !=
+        NVFP4_OK)
+        return s;
     unsigned int* err = device_error_word();
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
@@ -663,15 +659,9 @@ nvfp4_status launch_gemm(const nvfp4_tensor& A, const nvfp4_tensor& B, float* C,
     if (s != NVFP4_OK) return s;
     s = make_tmap_f32_sw128(&tc, C, A.rows, B.rows, ldc, 32, 32);
     if (s != NVFP4_OK) return s;
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
-        attr_done[dev] = true;
-    }
+    static PerDeviceOnce attr_once;
+    if ((s = smem_limit_once(attr_once, w4a4_gemm_kernel<BN>, G::SMEM, "cudaFuncSetAttribute(gemm smem)")) != NVFP4_OK)
+        return s;
     unsigned int* err = device_error_word();
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);

@@ -116,6 +116,8 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     if (!x_bf16 || !y) return fail(NVFP4_ERR_INVALID_ARG, "x / y null");
     if (form != GDN_FORM_PAGES && form != GDN_FORM_STANDARD) return fail(NVFP4_ERR_INVALID_ARG, "bad form");
     if (!aligned16(x_bf16) || !aligned16(y)) return fail(NVFP4_ERR_MISALIGNED, "x / y must be 16-byte aligned");
+    if (!aligned16(state_in) || !aligned16(state_out))
+        return fail(NVFP4_ERR_MISALIGNED, "state_in and state_out must be 16-byte aligned");
     gdn_layer_ws_layout L;
     layout_of(w, B, T, &L);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -135,7 +137,8 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     float* beta = reinterpret_cast<float*>(ws + L.beta);
     float* o = reinterpret_cast<float*>(ws + L.o);
 
-    // quantiser words: [0] x amax, [1] x arrival counter, [2] o amax; one memset
+    // quantiser words: [0] x amax, [1] x arrival counter, [2] o amax, [3] gated-o amax,
+    // zeroed by one small kernel (it chains with its neighbours by programmatic launch)
     unsigned int* qw = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
     if ((s = zero_words_launch(qw, 4, st)) != NVFP4_OK) return s;
     if ((s = quantize_launch(x_bf16, NVFP4_DTYPE_BF16, BT, H, H, xq, kQuantComputeZeroedWs, qw, st)) != NVFP4_OK)

@@ -882,16 +882,14 @@ nvfp4_status launch_chunked_kv(const float* q, const float* k, const float* v, i
     const int NC = static_cast<int>((T + CH - 1) / CH);
     const int prep_smem = sizeof(PrepSmem<K, V>);
     const int seq_smem = SeqLayout<K>::BYTES;
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    static PerDeviceOnce attr_once;
+    nvfp4_status s = once_per_device(attr_once, [&]() -> nvfp4_status {
         cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prep)");
         e = cudaFuncSetAttribute(chunk_seq_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, seq_smem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(seq)");
-        attr_done[dev] = true;
-    }
+        return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "cudaFuncSetAttribute(seq)");
+    });
+    if (s != NVFP4_OK) return s;
     unsigned int* err = device_error_word();
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     uint8_t* recs = static_cast<uint8_t*>(ws);
@@ -1015,6 +1013,8 @@ extern "C" nvfp4_status gdn_scan(const float* q_hat, const float* k_hat, const f
     if (static_cast<int64_t>(B) * T > (int64_t(1) << 31)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "B*T too large");
     if (!aligned16(q_hat) || !aligned16(k_hat) || !aligned16(o) || !aligned16(v) || ld_v % 4)
         return fail(NVFP4_ERR_MISALIGNED, "q_hat, k_hat, v, o must be 16-byte aligned and ld_v % 4 == 0");
+    if (!aligned16(state_in) || !aligned16(state_out))   // the chunked kernel moves the state as float4
+        return fail(NVFP4_ERR_MISALIGNED, "state_in and state_out must be 16-byte aligned");
     const size_t need = scan_workspace_bytes(B, T, *dims, algo);
     if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)))
         return fail(NVFP4_ERR_WORKSPACE, "scan workspace missing, too small or not 256-byte aligned");

@@ -68,6 +68,8 @@ extern "C" nvfp4_status gdn_scan_noalloc(const float* q_hat, const float* k_hat,
     if (static_cast<int64_t>(B) * T > (int64_t(1) << 31)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "B*T too large");
     if (!aligned16(q_hat) || !aligned16(k_hat) || !aligned16(o) || !aligned16(v) || ld_v % 4)
         return fail(NVFP4_ERR_MISALIGNED, "q_hat, k_hat, v, o must be 16-byte aligned and ld_v % 4 == 0");
+    if (!aligned16(state_in) || !aligned16(state_out))   // the chunked kernel moves the state as float4
+        return fail(NVFP4_ERR_MISALIGNED, "state_in and state_out must be 16-byte aligned");
     const size_t need = scan_workspace_bytes(B, T, *dims, GDN_SCAN_CHUNKED);
     if (need > kNoAllocScratchBytes)
         return fail(NVFP4_ERR_WORKSPACE, "gdn_scan_noalloc: this problem needs " + std::to_string(need) +

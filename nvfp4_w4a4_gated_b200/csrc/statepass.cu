@@ -145,14 +145,9 @@ template <int K>
 nvfp4_status launch_chain(const float* P, const float* S_loc, const float* S_in, float* S_out, int m, int64_t n,
                           int V, cudaStream_t st) {
     constexpr int smem = (2 * K * (K + 4) + K * kChainCols) * 4;
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(state_chain_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chain)");
-        attr_done[dev] = true;
-    }
+    static PerDeviceOnce attr_once;
+    const nvfp4_status s = smem_limit_once(attr_once, state_chain_kernel<K>, smem, "cudaFuncSetAttribute(chain)");
+    if (s != NVFP4_OK) return s;
     const cudaError_t e = launch_pdl(state_chain_kernel<K>, dim3(static_cast<unsigned>(n), V / kChainCols),
                                      dim3(256), smem, st, P, S_loc, S_in, S_out, m, n, V);
     if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
@@ -290,14 +285,9 @@ template <int K, int V>
 nvfp4_status launch_correct(const float* m, const float* S_in, float* o, int B, int64_t T, int Hv,
                             unsigned int* o_amax, cudaStream_t st) {
     constexpr int smem = (K * V + 2 * kCorrTok * K) * 4;
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(scan_correct_kernel<K, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(correct)");
-        attr_done[dev] = true;
-    }
+    static PerDeviceOnce attr_once;
+    const nvfp4_status s = smem_limit_once(attr_once, scan_correct_kernel<K, V>, smem, "cudaFuncSetAttribute(correct)");
+    if (s != NVFP4_OK) return s;
     const int64_t n_items = static_cast<int64_t>(B) * Hv * ((T + kCorrTok - 1) / kCorrTok);
     const int64_t slots = int64_t(num_sms()) * 2;
     const int per_cta = static_cast<int>((n_items + slots - 1) / slots);
@@ -525,15 +515,10 @@ template <int K, int V>
 nvfp4_status launch_correct_tc(const float* m, const float* S_in, float* o, int B, int64_t T, int Hv,
                                unsigned int* o_amax, cudaStream_t st) {
     constexpr int smem = static_cast<int>(CorrTcLayout<K, V>::BYTES);
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(scan_correct_tc_kernel<K, V>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(correct tc)");
-        attr_done[dev] = true;
-    }
+    static PerDeviceOnce attr_once;
+    const nvfp4_status s =
+        smem_limit_once(attr_once, scan_correct_tc_kernel<K, V>, smem, "cudaFuncSetAttribute(correct tc)");
+    if (s != NVFP4_OK) return s;
     unsigned int* err = device_error_word();
     if (!err) return fail(NVFP4_ERR_CUDA, "device error word unavailable");
     const int64_t n_items = static_cast<int64_t>(B) * Hv * ((T + kTcTok - 1) / kTcTok);

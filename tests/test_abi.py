@@ -118,6 +118,25 @@ def test_gates_and_scan_validation():
     assert st == 1
 
 
+def test_scan_refuses_unaligned_state_pointers():
+    """The chunked scan moves the state as 16-byte vectors: an offset state_in or
+    state_out is refused on the host (MISALIGNED), for gdn_scan, the
+    allocation-free variant and the layer."""
+    L = nv.lib()
+    d = nv.GdnDims(16, 32, 128, 128).c()
+    for s_in, s_out in ((FAKE + 4, None), (None, FAKE + 8), (FAKE + 4, FAKE + 4)):
+        st, msg = _err(L.gdn_scan(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 64, ctypes.byref(d), 0.1, 0, 2, s_in, s_out,
+                                  FAKE, FAKE, 1 << 30, None))
+        assert st == 3 and "state" in msg
+        st, msg = _err(L.gdn_scan_noalloc(FAKE, FAKE, FAKE, 4096, FAKE, FAKE, 1, 64, ctypes.byref(d), 0.1, 0, s_in,
+                                          s_out, FAKE, None))
+        assert st == 3 and "state" in msg
+    dims = nv.GdnDims(16, 32, 128, 128)
+    lw = nv._LayerWeights(_tensor(dims.n_in, 5120), _tensor(5120, 4096), FAKE, FAKE, dims.c(), 5120)
+    st, msg = _err(L.gdn_layer_forward(ctypes.byref(lw), FAKE, 1, 64, FAKE, FAKE + 4, None, 0, FAKE, 1 << 40, None))
+    assert st == 3 and "state" in msg
+
+
 def test_layer_layout_and_validation():
     L = nv.lib()
     dims = nv.GdnDims(16, 32, 128, 128)

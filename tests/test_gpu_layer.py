@@ -89,20 +89,36 @@ def test_tiny_layer_out_proj_stage_isolated(cuda_dev):
 
 
 def test_layer_decode_step_chain(cuda_dev):
-    """Decode: T = 1 per call with the state carried; 4 steps equal one call over 4 tokens."""
-    sh, B = gdn_synth.TINY, 3
-    w, _ = _make_layer(sh, 7)
-    bits, _x = gdn_synth.activations(8, B * 4, sh.H, hot="fixed")
-    xs = bf16_device(bits).view(B, 4, sh.H)
+    """Decode: T = 1 per call, B = 3 sequences, the state carried in place over four
+    steps.  Each step is checked against the oracle's layer step taken from the
+    oracle's own carried state: o and the state within the scan bar, the o codes and
+    y at the flip bar of the stage-wise test (each single-token call quantises its
+    own rows with its own per-tensor scale, on both sides)."""
+    sh, B, steps = gdn_synth.TINY, 3, 4
+    w, (W_in, W_out, A_log, dt_bias) = _make_layer(sh, 7)
+    bits, x = gdn_synth.activations(8, B * steps, sh.H, hot="fixed")
+    xs = bf16_device(bits).view(B, steps, sh.H)
+    xh = x.reshape(B, steps, sh.H)
+    Wq_in, Wq_out = oracle.quantize(W_in), oracle.quantize(W_out)
+    W_in_deq, W_out_deq = oracle.dequantize(*Wq_in), oracle.dequantize(*Wq_out)
     S = torch.zeros((B, sh.Hv, sh.K, sh.V), device="cuda")
-    ys = []
-    for t in range(4):
-        xt = xs[:, t].contiguous()
-        y, _, _ = nv.gdn_layer_forward(w, xt, B, 1, state_in=S, state_out=S)
-        ys.append(y)
-    torch.cuda.synchronize()
-    assert all(torch.isfinite(y).all() for y in ys)
-    assert float(S.abs().max()) > 0
+    S_ref = np.zeros((B, sh.Hv, sh.K, sh.V))
+    HvV = sh.Hv * sh.V
+    for t in range(steps):
+        y, ws, lay = nv.gdn_layer_forward(w, xs[:, t].contiguous(), B, 1, state_in=S, state_out=S)
+        torch.cuda.synchronize()
+        nv.check_device_error()
+        ref = oracle.layer_forward(np.ascontiguousarray(xh[:, t]), Wq_in, Wq_out, A_log, dt_bias, B, 1, sh.Hk, sh.Hv,
+                                   sh.K, sh.V, S0=S_ref, stages=True, W_in_deq=W_in_deq, W_out_deq=W_out_deq)
+        o = _view(ws, lay["o"], B * HvV * 4, torch.float32).cpu().numpy().reshape(B, 1, sh.Hv, sh.V)
+        assert rel_fro(o, ref["o"]) <= 2e-3, t
+        assert rel_fro(S.cpu().numpy(), ref["S"]) <= 2e-3, t
+        oc = _view(ws, lay["o_codes"], B * HvV // 2, torch.uint8).cpu().numpy().reshape(B, HvV // 2)
+        flipped = np.mean(oc != ref["oq"][0])
+        assert flipped < 0.02, t
+        assert rel_fro(y.cpu().numpy(), ref["y"]) <= max(2e-2, 0.5 * np.sqrt(flipped)), t
+        S_ref = ref["S"]
+    assert np.linalg.norm(S_ref) > 0
 
 
 def test_full_size_prefill_layer_stage_checks(cuda_dev):

@@ -260,26 +260,93 @@ def test_softplus_closed_forms():
     assert oracle.softplus(800.0) == 800.0
 
 
-def test_gates_ranges_and_library_forms():
-    g = gdn_synth.rng(31)
-    a = g.standard_normal((50, 4)) * 5
-    b = g.standard_normal((50, 4)) * 5
-    A_log, dt_bias = gdn_synth.gate_params(32, 4)
-    gg, beta = oracle.gates(a, b, A_log, dt_bias)
-    alpha = np.exp(gg)
+def test_softplus_limits():
+    """softplus(u) -> u as u -> +inf (the log1p term is below the last bit of u
+    once e^-u < 2^-53 u) and -> e^u as u -> -inf."""
+    for u in (40.0, 60.0, 200.0):
+        assert oracle.softplus(u) == u
+    for u in (-40.0, -60.0, -200.0):
+        assert abs(oracle.softplus(u) / math.exp(u) - 1.0) < 1e-15
+
+
+# The gate heads below: per-head A_log and dt_bias all different and non-zero, so
+# that a dropped or swapped parameter moves every closed form.
+_A_LOG = np.array([math.log(1.5), math.log(4.0), math.log(16.0), -0.75])
+_DT_BIAS = np.array([0.3, -1.2, 2.0, -0.45])
+
+
+def test_gates_closed_form_at_zero_softplus_argument():
+    """Eq.(1) at a + dt_bias = 0: softplus(0) = ln 2, so g = -e^{A_log} ln 2
+    per head (review page, paper sec.2)."""
+    a = np.tile(-_DT_BIAS, (3, 1))
+    g, _ = oracle.gates(a, np.zeros_like(a), _A_LOG, _DT_BIAS)
+    want = -np.exp(_A_LOG) * math.log(2.0)
+    assert np.allclose(g, np.tile(want, (3, 1)), rtol=1e-15, atol=0)
+
+
+def test_gates_closed_form_at_unit_softplus():
+    """a + dt_bias = ln(e - 1) gives softplus = ln(1 + e - 1) = 1, so g = -e^{A_log}
+    and the decay alpha = exp(-e^{A_log}); at A_log = ln 4 that is e^-4."""
+    a = np.tile(math.log(math.e - 1.0) - _DT_BIAS, (2, 1))
+    g, _ = oracle.gates(a, np.zeros_like(a), _A_LOG, _DT_BIAS)
+    assert np.allclose(g, np.tile(-np.exp(_A_LOG), (2, 1)), rtol=1e-14, atol=0)
+    assert abs(math.exp(g[0, 1]) - math.exp(-4.0)) < 1e-15
+
+
+def test_beta_closed_forms():
+    """beta = sigmoid(b): 1/2 at b = 0, 3/4 at b = ln 3, 1/4 at b = -ln 3
+    (1 / (1 + 1/3) and 1 / (1 + 3)), whatever A_log and dt_bias are."""
+    l3 = math.log(3.0)
+    b = np.array([[0.0, l3, -l3, 0.0], [l3, -l3, 0.0, l3]])
+    _, beta = oracle.gates(np.zeros_like(b), b, _A_LOG, _DT_BIAS)
+    want = np.array([[0.5, 0.75, 0.25, 0.5], [0.75, 0.25, 0.5, 0.75]])
+    assert np.allclose(beta, want, rtol=1e-15, atol=0)
+
+
+def test_gates_monotone_and_in_range():
+    """alpha = e^g lies in (0, 1) and strictly decreases as a grows (a larger
+    step forgets more); beta lies in (0, 1) and strictly increases with b."""
+    u = np.linspace(-8.0, 8.0, 161)
+    a = np.repeat(u[:, None], 4, axis=1)
+    g, beta = oracle.gates(a, a, _A_LOG, _DT_BIAS)
+    alpha = np.exp(g)
     assert np.all((alpha > 0) & (alpha < 1)) and np.all((beta > 0) & (beta < 1))
-    ref_g = -np.exp(A_log.astype(np.float64)) * np.logaddexp(0.0, a + dt_bias.astype(np.float64))
-    assert np.allclose(gg, ref_g, rtol=1e-13, atol=0)
-    from scipy.special import expit
-    assert np.allclose(beta, expit(b), rtol=1e-14, atol=0)
+    assert np.all(np.diff(alpha, axis=0) < 0)
+    assert np.all(np.diff(beta, axis=0) > 0)
+
+
+def test_gates_heads_are_independent():
+    """Head h reads only A_log[h] and dt_bias[h]: permuting the heads' parameters
+    together with the columns of a and b permutes the outputs."""
+    g0 = gdn_synth.rng(31)
+    a = g0.standard_normal((20, 4)) * 3
+    b = g0.standard_normal((20, 4)) * 3
+    g, beta = oracle.gates(a, b, _A_LOG, _DT_BIAS)
+    p = np.array([2, 0, 3, 1])
+    gp, bp = oracle.gates(a[:, p], b[:, p], _A_LOG[p], _DT_BIAS[p])
+    assert np.array_equal(gp, g[:, p]) and np.array_equal(bp, beta[:, p])
+
+
+def test_l2norm_closed_forms():
+    """(3, 4, 0, ...) -> (3, 4, 0, ...) / sqrt(25 + eps); a row 1e-4 e_1 shows where
+    eps sits (reading G2, inside the square root): 1e-4 / sqrt(1e-8 + 1e-6),
+    not 1e-4 / (1e-4 + 1e-6); a zero row stays zero."""
+    x = np.zeros((3, 1, 8))
+    x[0, 0, :2] = (3.0, 4.0)
+    x[1, 0, 0] = 1e-4
+    y = oracle.l2norm(x)
+    assert np.allclose(y[0, 0, :2], np.array([3.0, 4.0]) / math.sqrt(25.0 + 1e-6), rtol=1e-15, atol=0)
+    assert abs(y[1, 0, 0] - 1e-4 / math.sqrt(1e-8 + 1e-6)) < 1e-16
+    assert abs(y[1, 0, 0] - 0.0995037190209989) < 1e-15
+    assert np.array_equal(y[2], np.zeros((1, 8)))
 
 
 def test_l2norm_unit_rows():
     x = gdn_synth.gaussian(33, (10, 3, 64))
     y = oracle.l2norm(x)
-    n = np.linalg.norm(x.astype(np.float64), axis=-1, keepdims=True)
-    assert np.allclose(y, x / np.sqrt(n ** 2 + 1e-6), rtol=1e-14)
     assert np.allclose(np.linalg.norm(y, axis=-1), 1.0, atol=1e-6)
+    # each row keeps its direction: y is a positive multiple of x
+    assert np.allclose(y * np.linalg.norm(x.astype(np.float64), axis=-1, keepdims=True), x, rtol=1e-6, atol=0)
 
 
 # -------------------------------------------------------------------- scan --
