@@ -20,6 +20,14 @@ The compute steps are the library's kernels (``gdn_scan_span`` for step 1,
 torch.distributed carries the exchange.  ``ops`` lets the host logic run
 against another implementation of the steps (the multi-rank CPU tests use
 it); the default is the CUDA library and nothing else.
+
+``sequence_parallel_layer`` composes the whole layer forward around the split
+scan.  The pages' NVFP4 format has one FP32 scale per tensor (review page,
+background / paper sec.1), so each quantised activation (x, and o before
+out_proj) takes its scale from the amax of the whole sequence: every rank
+writes the amax of its rows, a max all-reduce joins them, and every rank
+quantises its rows from the joined word, so its codes and block scales are
+the whole tensor's rows.
 """
 from __future__ import annotations
 
@@ -28,7 +36,8 @@ from dataclasses import dataclass
 import torch
 import torch.distributed as dist
 
-from . import FORM_PAGES, SCAN_AUTO, GdnDims, gdn_scan_correct, gdn_scan_span, gdn_state_combine
+from . import (FORM_PAGES, QUANT_AMAX_ONLY, QUANT_FROM_AMAX, SCAN_AUTO, GdnDims, LayerWeights, gdn_gates,
+               gdn_scan_correct, gdn_scan_span, gdn_state_combine, lib, nvfp4_quantize, w4a4_gemm)
 
 
 class CudaSpanOps:
@@ -115,3 +124,86 @@ def segmented_scan(spans, B: int, dims: GdnDims, scale: float | None = None, for
         o, S = span_join(loc, None, None, B, span[5], S, ops)
         outs.append(o)
     return outs, S
+
+
+# ------------------------------------------------------------ the layer --
+class CudaLayerOps(CudaSpanOps):
+    """The layer's steps on the GPU, through the C-ABI library."""
+
+    def amax_word(self, x):
+        """int32 [1] holding the float bits of max|x| (workspace word 0 of an
+        NVFP4_QUANT_AMAX_ONLY quantisation)."""
+        ws = torch.zeros(max(16, lib().nvfp4_quantize_workspace_size()), dtype=torch.uint8, device=x.device)
+        nvfp4_quantize(x, workspace=ws, stream=self.stream, mode=QUANT_AMAX_ONLY)
+        return ws[:4].view(torch.int32)
+
+    def quantize_from_amax(self, x, word):
+        ws = torch.zeros(max(16, lib().nvfp4_quantize_workspace_size()), dtype=torch.uint8, device=x.device)
+        ws[:4].view(torch.int32).copy_(word)
+        return nvfp4_quantize(x, workspace=ws, stream=self.stream, mode=QUANT_FROM_AMAX)
+
+    def gemm(self, a, b):
+        return w4a4_gemm(a, b, stream=self.stream)
+
+    def gates(self, P, w: LayerWeights):
+        """(q_hat, k_hat, v, g, beta) of the fused projection's rows."""
+        d = w.dims
+        q_hat, k_hat, g, beta = gdn_gates(P, d, w.A_log, w.dt_bias, stream=self.stream)
+        c0 = 2 * d.Hk * d.K
+        return q_hat, k_hat, P[:, c0:c0 + d.Hv * d.V], g, beta
+
+
+def _quantize_across(x, ops, group, distributed):
+    """x quantised with the scale of the whole tensor split across the ranks."""
+    word = ops.amax_word(x)
+    if distributed:
+        dist.all_reduce(word, op=dist.ReduceOp.MAX, group=group)   # non-negative floats order as their bits
+    return ops.quantize_from_amax(x, word)
+
+
+def sequence_parallel_layer(w, x, B: int, T: int, form: int = FORM_PAGES, state_in=None, group=None, ops=None):
+    """One GDN layer forward under NVFP4 W4A4 for B sequences whose tokens are
+    split across the ranks of ``group`` in rank order: this rank holds T
+    consecutive tokens of every sequence (x [B*T, hidden], rows (b, t)).  The
+    steps are the layer's: x quantised (with the whole sequence's scale), the
+    fused in_proj, gates and q/k normalisation, the sequence-split scan, o
+    quantised (whole-sequence scale), out_proj.  Every rank passes the same
+    weights and ``state_in`` (None = zero).  Returns (y [B*T, hidden] for the
+    local tokens, the quantised x, the quantised o, the state after the local
+    span).  Collectives, in the same order on every rank: one max all-reduce
+    (x), the scan's two all-gathers, one max all-reduce (o)."""
+    ops = ops or CudaLayerOps()
+    distributed = dist.is_initialized() and dist.get_world_size(group) > 1
+    d = w.dims
+    xq = _quantize_across(x, ops, group, distributed)
+    P = ops.gemm(xq, w.w_in)
+    q_hat, k_hat, v, g, beta = ops.gates(P, w)
+    scale = 1.0 / float(d.K) ** 0.5
+    o, S_end = sequence_parallel_scan(q_hat, k_hat, v, g, beta, B, T, d, scale=scale, form=form, state_in=state_in,
+                                      group=group, ops=ops)
+    oq = _quantize_across(o.reshape(B * T, d.Hv * d.V), ops, group, distributed)
+    return ops.gemm(oq, w.w_out), xq, oq, S_end
+
+
+def segmented_layer(w, xs, B: int, form: int = FORM_PAGES, state_in=None, ops=None):
+    """sequence_parallel_layer's steps on one device, with the spans of every
+    sequence given in order as a list of (x [B*T_i, hidden], T_i): the amax
+    words of all spans first and their maximum in place of the all-reduce, then
+    each span's in_proj and gates, the segmented scan, and the same for o.
+    Returns the list of span outputs y and the final state."""
+    ops = ops or CudaLayerOps()
+    d = w.dims
+
+    def quantize_all(ts):
+        words = [ops.amax_word(t) for t in ts]
+        word = torch.stack(words).amax(dim=0)
+        return [ops.quantize_from_amax(t, word) for t in ts]
+
+    xqs = quantize_all([x for x, _ in xs])
+    spans = []
+    for xq, (_, T) in zip(xqs, xs):
+        q_hat, k_hat, v, g, beta = ops.gates(ops.gemm(xq, w.w_in), w)
+        spans.append((q_hat, k_hat, v, g, beta, T))
+    outs, S = segmented_scan(spans, B, d, scale=1.0 / float(d.K) ** 0.5, form=form, state_in=state_in, ops=ops)
+    oqs = quantize_all([o.reshape(-1, d.Hv * d.V) for o in outs])
+    return [ops.gemm(oq, w.w_out) for oq in oqs], xqs, oqs, S

@@ -101,3 +101,82 @@ def bench_rank_main(rank, world, port, out_dir):
             f.write(f"{got[0]} {got[1]} {tokens} {value}\n")
     finally:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ the layer --
+class OracleLayerOps(OracleSpanOps):
+    """The layer's other steps (quantiser modes, GEMM, gates) restated with the
+    oracle, on CPU tensors, for nvfp4_w4a4_gated_b200.seqpar.sequence_parallel_layer."""
+
+    def amax_word(self, x):
+        a = np.float32(np.max(np.abs(np.asarray(x.numpy(), dtype=np.float32))))
+        return torch.from_numpy(np.array([a], dtype=np.float32).view(np.int32))
+
+    def quantize_from_amax(self, x, word):
+        amax = word.numpy().view(np.float32)
+        S = oracle.global_scale(amax)          # the per-tensor scale of a tensor whose amax is this word
+        return oracle.quantize(np.asarray(x.numpy(), dtype=np.float32), S=S)
+
+    def gemm(self, a, b):
+        return torch.from_numpy(oracle.w4a4_gemm(a, b))
+
+    def gates(self, P, w):
+        d = w.dims
+        q, k, v, _, a, b = oracle.split_projection(P.numpy(), d.Hk, d.Hv, d.K, d.V)
+        g, beta = oracle.gates(a, b, w.A_log, w.dt_bias)
+        n = P.shape[0]
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+        return (t(oracle.l2norm(q.reshape(n, d.Hk, d.K))), t(oracle.l2norm(k.reshape(n, d.Hk, d.K))), t(v), t(g),
+                t(beta))
+
+
+class OracleLayer:
+    """Weights of the layer test: the oracle's quantised in_proj / out_proj."""
+
+    def __init__(self, dims, w_in, w_out, A_log, dt_bias):
+        self.dims, self.w_in, self.w_out, self.A_log, self.dt_bias = dims, w_in, w_out, A_log, dt_bias
+
+
+def layer_problem(form):
+    """One seeded layer shared by every rank: 2 sequences of 90 tokens, hidden 64."""
+    from nvfp4_w4a4_gated_b200 import GdnDims
+    dims = GdnDims(2, 4, 16, 16)
+    B, T, H = 2, 90, 64
+    _, x = gdn_synth.activations(310, B * T, H, hot="fixed")
+    W_in = gdn_synth.weights(311, dims.n_in, H)
+    W_out = gdn_synth.weights(312, H, dims.Hv * dims.V)
+    A_log, dt_bias = gdn_synth.gate_params(313, dims.Hv)
+    S0 = gdn_synth.gaussian(314, (B, dims.Hv, dims.K, dims.V), std=0.5).astype(np.float64)
+    w = OracleLayer(dims, oracle.quantize(W_in), oracle.quantize(W_out), A_log, dt_bias)
+    return w, x, B, T, H, S0
+
+
+def layer_rank_main(rank, world, port, bounds, form, with_state, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from nvfp4_w4a4_gated_b200.seqpar import sequence_parallel_layer
+        w, x, B, T, H, S0 = layer_problem(form)
+        d = w.dims
+        a, e = bounds[rank], bounds[rank + 1]
+        x_loc = np.ascontiguousarray(x.reshape(B, T, H)[:, a:e].reshape(B * (e - a), H))
+        y, xq, oq, S_end = sequence_parallel_layer(w, torch.from_numpy(x_loc), B, e - a, form=form,
+                                                   state_in=torch.from_numpy(S0) if with_state else None,
+                                                   ops=OracleLayerOps())
+        ref = oracle.layer_forward(x, w.w_in, w.w_out, w.A_log, w.dt_bias, B, T, d.Hk, d.Hv, d.K, d.V, form=form,
+                                   S0=S0 if with_state else None, stages=True)
+        rows = lambda m: np.ascontiguousarray(m.reshape(B, T, -1)[:, a:e].reshape(B * (e - a), -1))
+        same_x = (np.array_equal(xq[0], rows(ref["xq"][0])) and np.array_equal(xq[1], rows(ref["xq"][1]))
+                  and np.float32(xq[2]) == np.float32(ref["xq"][2]))
+        same_o = (np.array_equal(oq[0], rows(ref["oq"][0])) and np.array_equal(oq[1], rows(ref["oq"][1]))
+                  and np.float32(oq[2]) == np.float32(ref["oq"][2]))
+        y_ref = rows(ref["y"])
+        err_y = float(np.max(np.abs(y.numpy() - y_ref)) / np.abs(y_ref).max())
+        err_S = 0.0
+        if rank == world - 1:
+            err_S = float(np.max(np.abs(S_end.numpy() - ref["S"])) / np.abs(ref["S"]).max())
+        with open(os.path.join(out_dir, f"layer{rank}.txt"), "w") as f:
+            f.write(f"{int(same_x)} {int(same_o)} {err_y} {err_S}\n")
+    finally:
+        dist.destroy_process_group()

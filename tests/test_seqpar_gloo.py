@@ -60,3 +60,23 @@ def test_bench_aggregation_on_gloo_ranks(tmp_path):
         t0, t1, tokens, value = map(float, open(os.path.join(tmp_path, f"agg{r}.txt")).read().split())
         assert (t0, t1) == (11.0, 20.0)
         assert tokens == 2 * 4096 * 10 and abs(value - tokens / 0.011) < 1e-6 * value
+
+
+@pytest.mark.parametrize("bounds,form,with_state", [
+    ([0, 45, 90], oracle.FORM_PAGES, False),
+    ([0, 10, 11, 90], oracle.FORM_STANDARD, True),     # a one-token span in the middle
+    ([0, 30, 64, 90], oracle.FORM_PAGES, True),
+])
+def test_sequence_parallel_layer_on_gloo_ranks(tmp_path, bounds, form, with_state):
+    """The whole layer with its tokens split across 2 and 3 CPU ranks (the
+    steps are the oracle's): each rank's quantised x and o are the rows of the
+    whole tensors' quantisation, bit for bit (one scale per tensor, from a max
+    all-reduce of the ranks' amax words), and its y rows and the last rank's
+    state equal the oracle's whole-sequence layer."""
+    world = len(bounds) - 1
+    mp.spawn(seqpar_workers.layer_rank_main, args=(world, _free_port(), bounds, form, with_state, str(tmp_path)),
+             nprocs=world, join=True)
+    for r in range(world):
+        same_x, same_o, err_y, err_S = open(os.path.join(tmp_path, f"layer{r}.txt")).read().split()
+        assert same_x == "1" and same_o == "1", (r, same_x, same_o)
+        assert float(err_y) < 1e-12 and float(err_S) < 1e-12, (r, err_y, err_S)
