@@ -2,14 +2,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (one "step"): gdn_layer_forward over B=1, T=4096 tokens of a layer
+Workload (one "step"): gdn_layer_forward over B=1, T=32768 tokens (the
+long-context layer prefill, the largest single-GPU configuration) of a layer
 with hidden 5120, 16 key / 32 value heads, head dims 128 (fused in_proj
 N_in = 12352, out_proj 5120 x 4096), synthetic seeded inputs (outlier-heavy
 bf16 activations, N(0, 0.02) weights quantised once to NVFP4, untimed).  The
 step covers every stage of the path: activation quantisation, fused in_proj
 GEMM, gates + q/k normalisation, chunked delta-rule scan, o quantisation,
-out_proj GEMM.  L2 (126 MB) is flushed by a 256 MB write before every timed
-step; each step is timed with CUDA events on the launching stream.
+out_proj GEMM.  The T=4096 layer prefill is measured the same way and
+reported under its own key.  L2 (126 MB) is flushed by a 256 MB write before
+every timed step; each step is timed with CUDA events on the launching
+stream.
 
 Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
 replica of the workload (the layer does not shard at this size; weak scaling)
@@ -37,7 +40,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GDN-layer W4A4 prefill tokens/s; FP4 GEMM TFLOPS and % NVFP4/HBM roofline"
 UNIT = "tokens/s"
-WORKLOAD = "gdn_layer_prefill_B1_T4096_h5120_hk16_hv32_k128_v128"
+WORKLOAD = "gdn_layer_prefill_B1_T32768_h5120_hk16_hv32_k128_v128"
+HEADLINE_T = 32768
 NVFP4_OVER_BF16 = 4.0   # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
 
 # launches of this library's kernels per gdn_layer_forward (T > 1), as the ncu launch list
@@ -192,10 +196,12 @@ def run_stages(nv, w, x, B, T, ws, lay, y, stream, events=None):
     ev(6)
 
 
-def traffic_for(stage: str):
-    """DRAM bytes per launch of the stage's dominant kernel from the committed
+def traffic_for(stage: str, T: int):
+    """DRAM bytes per launch of the stage's kernels at T tokens from the committed
     ncu summary (profiles/dram_traffic.txt), or None when absent or when the
-    kernel source changed since the counters were taken."""
+    kernel source changed since the counters were taken.  A figure captured at
+    another T is scaled by the tokens processed (the stage's traffic grows in
+    proportion to T: per-chunk records, per-token rows)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -205,8 +211,8 @@ def traffic_for(stage: str):
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     for ln in open(p):
         f = ln.split()
-        if len(f) >= 3 and not ln.startswith("#") and f[0] == stage:
-            return float(f[1]) if f[2] == sha else None
+        if len(f) >= 4 and not ln.startswith("#") and f[0] == stage:
+            return float(f[1]) * T / float(f[3]) if f[2] == sha else None
     return None
 
 
@@ -220,14 +226,15 @@ def cpu_baseline(sample_tokens: int, seed: int):
     A_log, dt_bias = gdn_synth.gate_params(seed + 102, sh.Hv, 0.0, math.log(16.0))
     Wid = oracle.dequantize(*oracle.quantize(W_in))
     Wod = oracle.dequantize(*oracle.quantize(W_out))
-    _, x = gdn_synth.activations(seed, 4096, sh.H, hot="percent")
-    xs = x[:sample_tokens]
+    _, x = gdn_synth.activations(seed, HEADLINE_T, sh.H, hot="percent")
+    xs = np.ascontiguousarray(x[:sample_tokens])
+    del x
     t0 = time.perf_counter()
     oracle.layer_forward(xs, None, None, A_log, dt_bias, 1, sample_tokens, sh.Hk, sh.Hv, sh.K, sh.V, W_in_deq=Wid,
                          W_out_deq=Wod)
     dt = time.perf_counter() - t0
     return {"value": sample_tokens / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"first {sample_tokens} of the 4096 tokens (B=1), full layer width, float64 oracle; "
+            "sample": f"first {sample_tokens} of the {HEADLINE_T} tokens (B=1), full layer width, float64 oracle; "
                       f"weights dequantised before timing", "seconds": dt}
 
 
@@ -248,32 +255,92 @@ def job_throughput(world: int, tokens_per_rank_step: int, steps: int, total_ms: 
     return tokens, tokens / (total_ms / 1e3)
 
 
-def run_ours(args, rank, world, local_rank):
-    import nvfp4_w4a4_gated_b200 as nv
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    dist = world > 1
-    seed = 2 + rank
-    B, T = 1, 4096
-    w, sh = make_layer(dev, seed)
+def spread(ms):
+    return {"min": round(min(ms), 4), "median": round(statistics.median(ms), 4), "max": round(max(ms), 4)}
+
+
+def time_prefill(nv, w, sh, dev, B, T, steps, warmup, flush, stream, seed):
+    """gdn_layer_forward over B x T tokens: `steps` timed steps (L2 flushed before
+    each, CUDA events on the launching stream), then the same step as its six
+    library calls with an event after each (per-stage times)."""
     import gdn_synth
     bits, _ = gdn_synth.activations(seed, B * T, sh.H, hot="percent")
     x = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
     y = torch.empty((B * T, sh.H), dtype=torch.float32, device=dev)
     lay = nv.layer_workspace_layout(w, B, T)
     ws = torch.empty(lay["total"], dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def step():
         nv.gdn_layer_forward(w, x, B, T, y=y, workspace=ws, stream=stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     nv.check_device_error()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    nstage = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        run_stages(nv, w, x, B, T, ws, lay, y, stream, evs[i])
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    names = ["quant_x", "gemm_in", "gates", "scan", "quant_o", "gemm_out"]
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
+                for j, n in enumerate(names)}
+    return dict(x=x, y=y, ws=ws, lay=lay, step_ms=step_ms, stage_ms=stage_ms, names=names)
 
-    # ---- timed region: K steps of gdn_layer_forward, L2 flushed before each
+
+def roofline_of(sh, B, T, stage_ms, pk):
+    """The dominant stage's roofline and every stage's achieved fraction."""
+    work = stage_work(sh, B, T)
+    dom = max(stage_ms, key=stage_ms.get)
+    bound, units = work[dom]
+    if bound == "tensor":
+        peak = pk["bf16_tflops"] * NVFP4_OVER_BF16
+        achieved = units / (stage_ms[dom] / 1e3) / 1e12
+        unit, peak_note = "TFLOP/s", f"{pk['source']} bf16 burst x {NVFP4_OVER_BF16:g} (nominal FP4:BF16)"
+    else:
+        peak = pk["hbm_gbs"]
+        achieved = units / (stage_ms[dom] / 1e3) / 1e9
+        unit, peak_note = "GB/s", f"{pk['source']} HBM copy"
+    stages = {}
+    for n, ms in stage_ms.items():
+        b, u = work[n]
+        if b == "tensor":
+            stages[n] = {"ms": round(ms, 4), "TFLOP/s": round(u / (ms / 1e3) / 1e12, 1),
+                         "frac": round(u / (ms / 1e3) / 1e12 / (pk["bf16_tflops"] * NVFP4_OVER_BF16), 3)}
+        else:
+            stages[n] = {"ms": round(ms, 4), "GB/s": round(u / (ms / 1e3) / 1e9, 1),
+                         "frac": round(u / (ms / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
+    roof = {"bound": bound, "kernel": f"{dom}: {STAGE_KERNELS[dom]}", "achieved": round(achieved, 1),
+            "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+            "traffic": traffic_for(dom, T), "peak_source": peak_note}
+    return roof, stages
+
+
+def run_ours(args, rank, world, local_rank):
+    import nvfp4_w4a4_gated_b200 as nv
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = world > 1
+    seed = 2 + rank
+    B, T = 1, HEADLINE_T
+    w, sh = make_layer(dev, seed)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    pk = peaks()
+
+    # ---- timed region: K steps of gdn_layer_forward at T = 32768, L2 flushed before each
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -282,41 +349,32 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(uuid)
     clocks.start()
     time.sleep(0.3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if dist:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize()
+    run = time_prefill(nv, w, sh, dev, B, T, args.steps, args.warmup, flush, stream, seed)
     if dist:
         torch.distributed.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-
-    # ---- the same step as its six calls, an event after each: per-stage times
-    nstage = 6
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        run_stages(nv, w, x, B, T, ws, lay, y, stream, evs[i])
-    torch.cuda.synchronize()
     clk = clocks.stop()
-    nv.check_device_error()
-    names = ["quant_x", "gemm_in", "gates", "scan", "quant_o", "gemm_out"]
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
-                for j, n in enumerate(names)}
+    total_ms = sum(run["step_ms"])
+    stage_ms = run["stage_ms"]
+    x, y, ws = run["x"], run["y"], run["ws"]
+
+    # ---- the T = 4096 layer prefill, the same measurement (its own key)
+    run4k = time_prefill(nv, w, sh, dev, 1, 4096, args.steps, args.warmup, flush, stream, seed)
+    roof4k, stages4k = roofline_of(sh, 1, 4096, run4k["stage_ms"], pk)
+    prefill_4k = {"workload": "gdn_layer_prefill_B1_T4096_h5120_hk16_hv32_k128_v128",
+                  "value": round(4096 / (statistics.mean(run4k["step_ms"]) / 1e3), 1), "unit": UNIT,
+                  "ms_per_step": round(statistics.mean(run4k["step_ms"]), 4), "ms_spread": spread(run4k["step_ms"]),
+                  "roofline": roof4k, "stages": stages4k}
+    x4k = run4k["x"]
+    del run4k
 
     # ---- standalone GEMM workload (M=8192, N=12288, K=5120), TFLOPS
     gemm = bench_gemm(nv, dev, args.steps, flush, stream)
     # ---- batch-64 decode step (HBM-bound)
     decode = bench_decode(nv, dev, w, sh, args.steps, stream)
-    # ---- the prefill step with the optional output gate
-    gated = bench_gated(nv, dev, w, sh, x, B, T, args.steps, flush, stream)
+    # ---- the T = 4096 prefill step with the optional output gate
+    gated = bench_gated(nv, dev, w, sh, x4k, 1, 4096, args.steps, flush, stream)
     # ---- the 32K-token scan split into eight spans (one sequence-parallel rank's work)
     seqpar = bench_seqpar(nv, dev, args.steps, flush, stream, clk.get("sm_max_mhz"))
 
@@ -366,29 +424,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- aggregate over ranks: max time
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, dist)
     tokens, value = job_throughput(world, B * T, args.steps, total_ms)
-
-    pk = peaks()
-    work = stage_work(sh, B, T)
-    dom = max(stage_ms, key=stage_ms.get)
-    bound, units = work[dom]
-    if bound == "tensor":
-        peak = pk["bf16_tflops"] * NVFP4_OVER_BF16
-        achieved = units / (stage_ms[dom] / 1e3) / 1e12
-        unit, peak_note = "TFLOP/s", f"{pk['source']} bf16 burst x {NVFP4_OVER_BF16:g} (nominal FP4:BF16)"
-    else:
-        peak = pk["hbm_gbs"]
-        achieved = units / (stage_ms[dom] / 1e3) / 1e9
-        unit, peak_note = "GB/s", f"{pk['source']} HBM copy"
-    traffic = traffic_for(dom)
-    stages = {}
-    for n in names:
-        b, u = work[n]
-        if b == "tensor":
-            stages[n] = {"ms": round(stage_ms[n], 4), "TFLOP/s": round(u / (stage_ms[n] / 1e3) / 1e12, 1),
-                         "frac": round(u / (stage_ms[n] / 1e3) / 1e12 / (pk["bf16_tflops"] * NVFP4_OVER_BF16), 3)}
-        else:
-            stages[n] = {"ms": round(stage_ms[n], 4), "GB/s": round(u / (stage_ms[n] / 1e3) / 1e9, 1),
-                         "frac": round(u / (stage_ms[n] / 1e3) / 1e9 / pk["hbm_gbs"], 3)}
+    roof, stages = roofline_of(sh, B, T, stage_ms, pk)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4), "higher_is_better": True,
@@ -396,10 +432,10 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "B": B, "T": T, "hidden": sh.H, "Hk": sh.Hk, "Hv": sh.Hv, "K": sh.K,
                    "V": sh.V, "n_in": sh.n_in, "form": "pages", "scan": "chunked C=64",
                    "l2": "flushed (256 MB write) before every timed step", "replicas": world},
-        "roofline": {"bound": bound, "kernel": f"{dom}: {STAGE_KERNELS[dom]}", "achieved": round(achieved, 1),
-                     "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "peak_source": peak_note},
+        "ms_spread": spread(run["step_ms"]),
+        "roofline": roof,
         "stages": stages,
+        "prefill_T4096": prefill_4k,
         "gemm_standalone": gemm,
         "decode": decode,
         "output_gate": gated,
@@ -698,8 +734,10 @@ def run_reference(args):
     A_log, dt_bias = gdn_synth.gate_params(seed + 102, sh.Hv, 0.0, math.log(16.0))
     Wid = oracle.dequantize(*oracle.quantize(W_in))
     Wod = oracle.dequantize(*oracle.quantize(W_out))
-    _, x = gdn_synth.activations(seed, 4096, sh.H, hot="percent")
-    xs = x[:sample]
+    # the workload's activations (the hot channels depend on the row count), then a prefix
+    _, x = gdn_synth.activations(seed, HEADLINE_T, sh.H, hot="percent")
+    xs = np.ascontiguousarray(x[:sample])
+    del x
 
     def step():
         oracle.layer_forward(xs, None, None, A_log, dt_bias, 1, sample, sh.Hk, sh.Hv, sh.K, sh.V, W_in_deq=Wid,
@@ -716,11 +754,67 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (quantiser exact f32)",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": 1, "T": 4096, "hidden": sh.H, "Hk": sh.Hk, "Hv": sh.Hv,
+            "config": {"workload": WORKLOAD, "B": 1, "T": HEADLINE_T, "hidden": sh.H, "Hk": sh.Hk, "Hv": sh.Hv,
                        "K": sh.K, "V": sh.V, "sample_tokens_per_step": sample},
             "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"first {sample} tokens of the T=4096 workload per step"},
+                             "sample": f"first {sample} tokens of the T={HEADLINE_T} workload per step"},
             "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_studies(args):
+    """The pages' mechanism studies (review page, paper sec.5.2 Table 3, sec.5.3
+    Fig. 1 and Table 6) through the library's kernels on the layer-prefill
+    shapes: the sensitivity replay over the T = 4096 workload, the lockstep
+    trajectories, the impulse and the gate-noise table over the T = 32768
+    workload.  Synthetic inputs and random weights: context, not the pages'
+    numbers (theirs come from a trained model)."""
+    import gdn_synth
+    import nvfp4_w4a4_gated_b200 as nv
+    from nvfp4_w4a4_gated_b200 import studies
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    be = studies.CudaBackend(dev, device_noise=True)
+    sh = gdn_synth.FULL
+    seed = 2
+    W_in = gdn_synth.weights(seed + 100, sh.n_in, sh.H)
+    W_out = gdn_synth.weights(seed + 101, sh.H, sh.Hv * sh.V)
+    dims = nv.GdnDims(sh.Hk, sh.Hv, sh.K, sh.V)
+    _, x4 = gdn_synth.activations(seed, 4096, sh.H, hot="percent")
+    _, x32 = gdn_synth.activations(seed, HEADLINE_T, sh.H, hot="percent")
+    xs4, xs = be.upload(x4), be.upload(x32)
+    del x4, x32
+    # two gate regimes: the layer's own (A_log ~ U(log 1, log 16): decays of a few tokens on
+    # these random weights) and long memory, alpha within ~1e-4 of 1 (horizons of 10^4-10^5
+    # tokens, the regime the pages' trained layers sit in)
+    regimes = {"layer_gates": gdn_synth.gate_params(seed + 102, sh.Hv, 0.0, math.log(16.0)),
+               "long_memory": gdn_synth.gate_params(seed + 103, sh.Hv, math.log(1e-5), math.log(1e-4))}
+    out = {}
+    for name, (A_log, dt_bias) in regimes.items():
+        L = studies.StudyLayer.make(be, W_in, W_out, A_log, dt_bias, dims, sh.H)
+        t1 = studies.sensitivity(be, L, xs4, 1, 4096)
+        t2 = studies.lockstep(be, L, xs, HEADLINE_T, [256, 512, 1024, 2048, 4096, 8192, 16384, 32768],
+                              n_perturbed=11)
+        imp = studies.impulse(be, L, xs, HEADLINE_T, t_imp=1024)
+        t3 = studies.gate_noise(be, L, xs, HEADLINE_T)
+        out[name] = (t1, t2, imp, t3)
+    nv.check_device_error()
+
+    def summary(vals):
+        got = sorted(v for v in vals if v is not None)
+        return {"min": got[0] if got else None, "median": got[len(got) // 2] if got else None,
+                "max": got[-1] if got else None, "not_reached": sum(v is None for v in vals)}
+    res = {"study": "mechanism studies (sensitivity replay, lockstep trajectories, impulse, gate noise)",
+           "data": "synthetic inputs, random weights (N(0, 0.02)); context, not the pages' trained-model numbers",
+           "workloads": {"sensitivity": "gdn_layer_prefill_B1_T4096_h5120_hk16_hv32_k128_v128",
+                         "lockstep_impulse_gate_noise": WORKLOAD}}
+    for name, (t1, t2, imp, t3) in out.items():
+        res[name] = {"sensitivity": t1, "lockstep": t2,
+                     "impulse": {"t_inject": 1024, "size": 0.01, "resolution": imp["resolution"],
+                                 "steps_to_1_over_e": summary(imp["steps_to_1_over_e"]),
+                                 "steps_to_1_over_10": summary(imp["steps_to_1_over_10"]),
+                                 "horizon_1_over_1_minus_alpha": summary(imp["horizon_1_over_1_minus_alpha"])},
+                     "gate_noise": t3}
+    return res
 
 
 def kernel_case(args):
@@ -776,6 +870,18 @@ def kernel_case(args):
         S_in = torch.randn((B, Hv, Kd, Kd), generator=g, device=dev)
         o = torch.randn((B * T, Hv, Kd), generator=g, device=dev)
         fn = lambda: nv.gdn_scan_correct(qm, S_in, o, B, T)
+    elif args.kernel_case == "decode":
+        # one batch-64 decode step of the layer (T = 1, states carried in place)
+        import gdn_synth
+        w, sh = make_layer(dev, 2)
+        Bd = 64
+        S = torch.from_numpy(gdn_synth.gaussian(9, (Bd, sh.Hv, sh.K, sh.V), std=0.3)).to(dev)
+        x = torch.from_numpy(gdn_synth.activations(2000, Bd, sh.H, hot="none")[0].view(np.int16)).to(dev)
+        x = x.view(torch.bfloat16)
+        y = torch.empty((Bd, sh.H), dtype=torch.float32, device=dev)
+        lay = nv.layer_workspace_layout(w, Bd, 1)
+        wsd = torch.empty(lay["total"], dtype=torch.uint8, device=dev)
+        fn = lambda: nv.gdn_layer_forward(w, x, Bd, 1, y=y, state_in=S, state_out=S, workspace=wsd, stream=stream)
     elif args.kernel_case == "statepass":
         # one rank's joining steps over a span of T tokens: seven maps composed, then the correction
         B, T, Hv, Kd = 1, args.T, 32, 128
@@ -813,7 +919,10 @@ def main(argv=None):
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     ap.add_argument("--ref-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct", "statepass"], default=None,
+    ap.add_argument("--study", action="store_true",
+                    help="print the mechanism-study tables (sensitivity replay, lockstep, impulse, gate noise)")
+    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct", "statepass", "decode"],
+                    default=None,
                     help="profile helper: run one kernel on a fixed case and exit")
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
@@ -822,6 +931,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.kernel_case:
         kernel_case(args)
+        return 0
+    if args.study:
+        print(json.dumps(run_studies(args)), flush=True)
         return 0
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))

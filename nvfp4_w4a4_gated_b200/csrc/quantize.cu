@@ -13,6 +13,8 @@
 // If the grid cannot be co-resident, a separate amax launch runs first.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace nvg {
@@ -285,9 +287,13 @@ enum QuantScaleMode : int {
 // group's atoms; after one atomicMax per CTA the CTAs meet at a grid barrier
 // (an arrival counter, so the launch must be cooperative), and pass 2 then
 // quantises the same atoms in reverse order, so the data read last in pass 1
-// (still in L2) is read first.  ws[0] = amax bits, ws[1] = arrival counter, both
-// zero at launch.  The barrier wait is bounded: on expiry the kernel sets
-// kErrTimeoutQuant and carries on with whatever amax it sees.
+// (still in L2) is read first; the very last atom of pass 1 stays in registers
+// across the barrier and is quantised without a second read.  With bf16 input
+// pass 2 loads the next atom before quantising the current one (two atoms in
+// flight per thread); fp32 input has no registers to spare for that.
+// ws[0] = amax bits, ws[1] = arrival counter, both zero at launch.  The barrier
+// wait is bounded: on expiry the kernel sets kErrTimeoutQuant and carries on
+// with whatever amax it sees.
 template <typename T, bool kFindAmax>
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
                                                               int64_t ld, unsigned int* __restrict__ ws,
@@ -302,13 +308,13 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const T* __restric
     const int64_t ngroups = static_cast<int64_t>(gridDim.x) * kQuantGroups;
     __shared__ float s_scale;
     __shared__ unsigned int warp_max[kQuantThreads / 32];
+    AtomRegs<T> cur;   // pass 1's last atom is pass 2's first
 
     if constexpr (kFindAmax) {
         typename AbsMaxOf<T>::type m;
         for (int64_t atom = group; atom < natoms; atom += ngroups) {
-            AtomRegs<T> a;
-            atom_load(x, rows, ld, k_atoms, atom, t, a);
-            atom_absmax(a, m);
+            atom_load(x, rows, ld, k_atoms, atom, t, cur);
+            atom_absmax(cur, m);
         }
         const unsigned int b = __reduce_max_sync(0xffffffffu, __float_as_uint(m.value()));
         if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = b;
@@ -360,11 +366,21 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const T* __restric
     const float y6 = __frcp_rn(d6);
     if (group >= natoms) return;
     const int64_t last = group + ((natoms - 1 - group) / ngroups) * ngroups;
-    for (int64_t atom = kFindAmax ? last : group; kFindAmax ? atom >= group : atom < natoms;
-         atom += kFindAmax ? -ngroups : ngroups) {
-        AtomRegs<T> a;
-        atom_load(x, rows, ld, k_atoms, atom, t, a);
-        atom_quantize_store(a, rows, cols, atom, t, d6, y6, s_inv, codes, sf);
+    const int64_t first = kFindAmax ? last : group, step = kFindAmax ? -ngroups : ngroups;
+    auto in_range = [&](int64_t atom) { return kFindAmax ? atom >= group : atom < natoms; };
+    if constexpr (!kFindAmax) atom_load(x, rows, ld, k_atoms, first, t, cur);
+    constexpr bool kPrefetch = std::is_same<T, __nv_bfloat16>::value;
+    for (int64_t atom = first; in_range(atom); atom += step) {
+        if constexpr (kPrefetch) {
+            AtomRegs<T> nxt;
+            const bool more = in_range(atom + step);
+            if (more) atom_load(x, rows, ld, k_atoms, atom + step, t, nxt);
+            atom_quantize_store(cur, rows, cols, atom, t, d6, y6, s_inv, codes, sf);
+            if (more) cur = nxt;
+        } else {
+            if (atom != first) atom_load(x, rows, ld, k_atoms, atom, t, cur);
+            atom_quantize_store(cur, rows, cols, atom, t, d6, y6, s_inv, codes, sf);
+        }
     }
 }
 

@@ -35,7 +35,7 @@ def test_reference_arm_prints_the_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["warmup"] >= 3 and d["steps"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
-    assert d["config"]["workload"].startswith("gdn_layer_prefill_B1_T4096")
+    assert d["config"]["workload"].startswith("gdn_layer_prefill_B1_T32768")
 
 
 def test_reference_arm_other_ranks_exit_quietly():
@@ -59,6 +59,9 @@ def test_roofline_inputs():
     # stored counters are used only while the kernel source still matches them
     src = os.path.join(ROOT, "nvfp4_w4a4_gated_b200", "csrc", "scan.cu")
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    assert b.traffic_for("scan") == (float(scan[0][1]) if scan[0][2] == sha else None)
-    assert b.traffic_for("gates") is None
+    t0 = int(scan[0][3])
+    assert b.traffic_for("scan", t0) == (float(scan[0][1]) if scan[0][2] == sha else None)
+    # at 8x the tokens, 8x the bytes (the figure is scaled by the tokens processed)
+    assert b.traffic_for("scan", 8 * t0) == (8 * float(scan[0][1]) if scan[0][2] == sha else None)
+    assert b.traffic_for("gates", t0) is None
 
