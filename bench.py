@@ -899,14 +899,27 @@ def kernel_case(args):
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(args.steps):
-        fn()
-    e.record(stream)
-    torch.cuda.synchronize()
+    if args.flush:
+        # L2 written over before each launch; each launch timed on its own
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for s, e in ev:
+            flush.fill_(1)
+            s.record(stream)
+            fn()
+            e.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(s.elapsed_time(e) for s, e in ev) / args.steps
+    else:
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e.record(stream)
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / args.steps
     nv.check_device_error()
-    print(json.dumps({"kernel_case": args.kernel_case, "ms_per_launch": s.elapsed_time(e) / args.steps,
+    print(json.dumps({"kernel_case": args.kernel_case, "ms_per_launch": ms, "l2_flushed": bool(args.flush),
                       "M": args.M, "N": args.N, "K": args.K, "T": args.T}))
 
 
@@ -921,13 +934,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--study", action="store_true",
                     help="print the mechanism-study tables (sensitivity replay, lockstep, impulse, gate noise)")
-    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct", "statepass", "decode"],
+    ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct", "statepass",
+                                              "decode"],
                     default=None,
                     help="profile helper: run one kernel on a fixed case and exit")
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=5120)
     ap.add_argument("--T", type=int, default=4096)
+    ap.add_argument("--flush", action="store_true", help="kernel case: write over L2 before each launch")
     args = ap.parse_args(argv)
     if args.kernel_case:
         kernel_case(args)
