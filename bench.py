@@ -139,61 +139,21 @@ def stage_work(sh, B, T):
     return {
         "quant_x": ("hbm", BT * sh.H * (2 + 0.5 + 1 / 16)),
         "gemm_in": ("tensor", 2.0 * BT * sh.n_in * sh.H),
-        "gates": ("hbm", BT * (2 * HkK * 4 + 2 * sh.Hv * 4 + 2 * HkK * 4 + 2 * sh.Hv * 4)),
+        "gates": ("hbm", BT * (2 * sh.Hv * 4 + 2 * sh.Hv * 4)),   # a, b columns in; g, beta out
         "scan": ("hbm", BT * (2 * HkK * 4 + HvV * 4 + 2 * sh.Hv * 4 + HvV * 4) + 2 * B * sh.Hv * sh.K * sh.V * 4),
         "quant_o": ("hbm", BT * HvV * (4 + 0.5 + 1 / 16)),
         "gemm_out": ("tensor", 2.0 * BT * sh.H * HvV),
     }
 
 
-STAGE_KERNELS = {"quant_x": "quant_kernel<bf16> (+amax)", "gemm_in": "w4a4_gemm_kernel", "gates": "l2norm+gate",
-                 "scan": "chunk_prep_kernel + chunk_seq_kernel", "quant_o": "quant_kernel<f32> (+amax)",
+# the layer's own launches per stage (gdn_layer_forward_timed records an event
+# before each stage): the scan normalises q and k while staging a chunk, the
+# gates kernel forms g and beta only, and o is quantised from the amax word the
+# scan filled
+STAGE_KERNELS = {"quant_x": "zero_words_kernel + quant_kernel<bf16> (amax pass, grid barrier, quantise pass)",
+                 "gemm_in": "w4a4_gemm_kernel", "gates": "gate_kernel (g, beta)",
+                 "scan": "chunk_prep_kernel + chunk_seq_kernel", "quant_o": "quant_kernel<f32> (from the scan's amax)",
                  "gemm_out": "w4a4_gemm_kernel"}
-
-
-def run_stages(nv, w, x, B, T, ws, lay, y, stream, events=None):
-    """The layer forward as its six library calls (the same launches, in the
-    same order, as gdn_layer_forward), optionally with an event after each."""
-    import ctypes
-    L = nv.lib()
-    sh = w.dims
-    base = ws.data_ptr()
-    BT, H, HvV = B * T, w.hidden, sh.Hv * sh.V
-    ldp = (sh.n_in + 3) // 4 * 4
-    xq = nv._Tensor(base + lay["x_codes"], base + lay["x_sf"], base + lay["x_scale"], BT, H)
-    oq = nv._Tensor(base + lay["o_codes"], base + lay["o_sf"], base + lay["o_scale"], BT, HvV)
-    s = ctypes.c_void_p(stream.cuda_stream)
-    P = base + lay["proj"]
-    d = sh.c()
-    win, wout = w.w_in.c(), w.w_out.c()
-
-    def ev(i):
-        if events is not None:
-            events[i].record(stream)
-
-    ev(0)
-    nv._check(L.nvfp4_quantize(ctypes.c_void_p(x.data_ptr()), 0, BT, H, H, ctypes.byref(xq), 0,
-                               ctypes.c_void_p(base + lay["quant_ws"]), 256, s))
-    ev(1)
-    nv._check(L.w4a4_gemm(ctypes.byref(xq), ctypes.byref(win), ctypes.c_void_p(P), ldp, s))
-    ev(2)
-    nv._check(L.gdn_gates(ctypes.c_void_p(P), ldp, BT, ctypes.byref(d), ctypes.c_void_p(w.A_log.data_ptr()),
-                          ctypes.c_void_p(w.dt_bias.data_ptr()), ctypes.c_void_p(base + lay["q_hat"]),
-                          ctypes.c_void_p(base + lay["k_hat"]), ctypes.c_void_p(base + lay["g"]),
-                          ctypes.c_void_p(base + lay["beta"]), s))
-    ev(3)
-    scan_ws = L.gdn_scan_workspace_size(B, T, ctypes.byref(d), 0)
-    nv._check(L.gdn_scan(ctypes.c_void_p(base + lay["q_hat"]), ctypes.c_void_p(base + lay["k_hat"]),
-                         ctypes.c_void_p(P + 2 * sh.Hk * sh.K * 4), ldp, ctypes.c_void_p(base + lay["g"]),
-                         ctypes.c_void_p(base + lay["beta"]), B, T, ctypes.byref(d), 1.0 / math.sqrt(sh.K), 0, 0,
-                         None, None, ctypes.c_void_p(base + lay["o"]), ctypes.c_void_p(base + lay["scan_ws"]),
-                         scan_ws, s))
-    ev(4)
-    nv._check(L.nvfp4_quantize(ctypes.c_void_p(base + lay["o"]), 1, BT, HvV, HvV, ctypes.byref(oq), 0,
-                               ctypes.c_void_p(base + lay["quant_ws"]), 256, s))
-    ev(5)
-    nv._check(L.w4a4_gemm(ctypes.byref(oq), ctypes.byref(wout), ctypes.c_void_p(y.data_ptr()), H, s))
-    ev(6)
 
 
 def traffic_for(stage: str, T: int):
@@ -261,8 +221,9 @@ def spread(ms):
 
 def time_prefill(nv, w, sh, dev, B, T, steps, warmup, flush, stream, seed):
     """gdn_layer_forward over B x T tokens: `steps` timed steps (L2 flushed before
-    each, CUDA events on the launching stream), then the same step as its six
-    library calls with an event after each (per-stage times)."""
+    each, CUDA events on the launching stream), then `steps` more through
+    gdn_layer_forward_timed, which records an event before each of the layer's
+    six stages and after the last (per-stage times of the same launches)."""
     import gdn_synth
     bits, _ = gdn_synth.activations(seed, B * T, sh.H, hot="percent")
     x = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -291,7 +252,7 @@ def time_prefill(nv, w, sh, dev, B, T, steps, warmup, flush, stream, seed):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage + 1)] for _ in range(steps)]
     for i in range(steps):
         flush.zero_()
-        run_stages(nv, w, x, B, T, ws, lay, y, stream, evs[i])
+        nv.gdn_layer_forward(w, x, B, T, y=y, workspace=ws, stream=stream, events=evs[i])
     torch.cuda.synchronize()
     nv.check_device_error()
     names = ["quant_x", "gemm_in", "gates", "scan", "quant_o", "gemm_out"]
@@ -870,6 +831,17 @@ def kernel_case(args):
         S_in = torch.randn((B, Hv, Kd, Kd), generator=g, device=dev)
         o = torch.randn((B * T, Hv, Kd), generator=g, device=dev)
         fn = lambda: nv.gdn_scan_correct(qm, S_in, o, B, T)
+    elif args.kernel_case == "layer":
+        # one layer prefill of T tokens (B = 1), the headline step's launches
+        import gdn_synth
+        w, sh = make_layer(dev, 2)
+        bits, _ = gdn_synth.activations(2000, args.T, sh.H, hot="percent")
+        x = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((args.T, sh.H), dtype=torch.float32, device=dev)
+        lay = nv.layer_workspace_layout(w, 1, args.T)
+        wsl = torch.empty(lay["total"], dtype=torch.uint8, device=dev)
+        S = torch.zeros((1, sh.Hv, sh.K, sh.V), dtype=torch.float32, device=dev)
+        fn = lambda: nv.gdn_layer_forward(w, x, 1, args.T, y=y, state_in=S, state_out=S, workspace=wsl, stream=stream)
     elif args.kernel_case == "decode":
         # one batch-64 decode step of the layer (T = 1, states carried in place)
         import gdn_synth
@@ -935,7 +907,7 @@ def main(argv=None):
     ap.add_argument("--study", action="store_true",
                     help="print the mechanism-study tables (sensitivity replay, lockstep, impulse, gate noise)")
     ap.add_argument("--kernel-case", choices=["gemm", "quant", "scan", "gate", "conv", "correct", "statepass",
-                                              "decode"],
+                                              "decode", "layer"],
                     default=None,
                     help="profile helper: run one kernel on a fixed case and exit")
     ap.add_argument("--M", type=int, default=8192)

@@ -388,6 +388,18 @@ NVFP4_API nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, co
                                                   const float* conv_state_in, float* conv_state_out, int32_t form,
                                                   void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
 
+/* gdn_layer_forward_stateful that also records seven caller-created CUDA
+ * events (cudaEvent_t, passed as void*) on the stream, for per-stage timing of
+ * the layer's own launches: events[i] before stage i (0 quantise x, 1 in_proj,
+ * 2 gates and the optional short convolution, 3 scan, 4 the optional output gate
+ * and quantise o, 5 out_proj) and events[6] after out_proj.  The launches are
+ * those of gdn_layer_forward_stateful; null events or a null handle: status 1. */
+NVFP4_API nvfp4_status gdn_layer_forward_timed(const gdn_layer_weights* w, const void* x_bf16, int32_t B, int64_t T,
+                                               float* y, const float* state_in, float* state_out,
+                                               const float* conv_state_in, float* conv_state_out, int32_t form,
+                                               void* workspace, size_t workspace_bytes, nvfp4_stream_t stream,
+                                               void* const* events);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,6 +40,7 @@ EXPORTED_SYMBOLS = [
     "gdn_scan", "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc", "gdn_output_gate",
     "gdn_short_conv", "gdn_layer_forward_stateful", "gdn_scan_transition_workspace_size", "gdn_scan_transition",
     "gdn_state_combine", "gdn_scan_correct", "gdn_scan_span_workspace_size", "gdn_scan_span",
+    "gdn_layer_forward_timed",
 ]
 
 
@@ -120,6 +121,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_layer_forward.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, i32, P, sz, P]
         L.gdn_layer_forward_stateful.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, P, P, i32, P,
                                                  sz, P]
+        L.gdn_layer_forward_timed.argtypes = [ctypes.POINTER(_LayerWeights), P, i32, i64, P, P, P, P, P, i32, P, sz,
+                                              P, ctypes.POINTER(ctypes.c_void_p)]
         L.gdn_short_conv.argtypes = [P, i64, i32, i64, i32, i32, P, P, P, P, i64, P]
         L.gdn_scan_transition_workspace_size.argtypes = [i32, i64, DP, i32]
         L.gdn_scan_transition_workspace_size.restype = sz
@@ -130,7 +133,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_scan_span.argtypes = [P, P, P, i64, P, P, i32, i64, DP, ctypes.c_float, i32, i32, P, P, P, P, P, sz, P]
         L.gdn_scan_correct.argtypes = [P, P, P, i32, i64, i32, i32, i32, P, P]
         for f in ("nvfp4_check_device_error", "nvfp4_selftest_wait_timeout", "nvfp4_quantize", "w4a4_gemm", "gdn_gates", "gdn_scan",
-                  "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc"):
+                  "gdn_layer_workspace_layout", "gdn_layer_forward", "gdn_scan_noalloc", "gdn_layer_forward_timed"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -422,10 +425,13 @@ def layer_workspace_layout(w: LayerWeights, B: int, T: int) -> dict:
 
 
 def gdn_layer_forward(w: LayerWeights, x: torch.Tensor, B: int, T: int, y=None, state_in=None, state_out=None,
-                      form: int = FORM_PAGES, workspace=None, stream=None, conv_state_in=None, conv_state_out=None):
+                      form: int = FORM_PAGES, workspace=None, stream=None, conv_state_in=None, conv_state_out=None,
+                      events=None):
     """y = GDN layer(x) under NVFP4 W4A4.  x: bf16 [B*T, hidden] on the device.
     conv_state_in / conv_state_out: the short convolution's carried inputs
-    [B, 2 Hk K + Hv V, conv_width - 1] (used only when w.conv_weight is set)."""
+    [B, 2 Hk K + Hv V, conv_width - 1] (used only when w.conv_weight is set).
+    events: optional list of 7 torch.cuda.Event (timing enabled), recorded on the
+    stream around the layer's stages (gdn_layer_forward_timed)."""
     assert x.dtype == torch.bfloat16 and x.is_contiguous()
     if y is None:
         y = torch.empty((B * T, w.hidden), dtype=torch.float32, device=x.device)
@@ -433,6 +439,18 @@ def gdn_layer_forward(w: LayerWeights, x: torch.Tensor, B: int, T: int, y=None, 
     if workspace is None:
         workspace = torch.empty(lay["total"], dtype=torch.uint8, device=x.device)
     lw = w.c()
+    if events is not None:
+        if len(events) != 7:
+            raise ValueError("events: 7 torch.cuda.Event")
+        st = stream if stream is not None else torch.cuda.current_stream(x.device)
+        for ev in events:
+            if ev.cuda_event == 0:   # torch creates the CUDA event on its first record
+                ev.record(st)
+        handles = (ctypes.c_void_p * 7)(*[ev.cuda_event for ev in events])
+        _check(lib().gdn_layer_forward_timed(ctypes.byref(lw), _ptr(x), B, T, _ptr(y), _ptr(state_in),
+                                             _ptr(state_out), _ptr(conv_state_in), _ptr(conv_state_out), form,
+                                             _ptr(workspace), workspace.numel(), _stream(stream), handles))
+        return y, workspace, lay
     _check(lib().gdn_layer_forward_stateful(ctypes.byref(lw), _ptr(x), B, T, _ptr(y), _ptr(state_in), _ptr(state_out),
                                             _ptr(conv_state_in), _ptr(conv_state_out), form, _ptr(workspace),
                                             workspace.numel(), _stream(stream)))

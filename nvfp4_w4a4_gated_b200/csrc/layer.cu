@@ -106,11 +106,16 @@ extern "C" nvfp4_status gdn_layer_forward(const gdn_layer_weights* w, const void
                                       workspace_bytes, stream);
 }
 
-extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, const void* x_bf16, int32_t B,
-                                                   int64_t T, float* y, const float* state_in, float* state_out,
-                                                   const float* conv_state_in, float* conv_state_out, int32_t form,
-                                                   void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
-    using namespace nvg;
+namespace nvg {
+// The layer's launches; with events (an array of kLayerEvents cudaEvent_t), event
+// i is recorded before stage i (quantise x, in_proj, gates and the optional
+// convolution, scan, the optional output gate and quantise o, out_proj) and the
+// last one after out_proj.
+constexpr int kLayerEvents = 7;
+static nvfp4_status layer_forward(const gdn_layer_weights* w, const void* x_bf16, int32_t B, int64_t T, float* y,
+                                  const float* state_in, float* state_out, const float* conv_state_in,
+                                  float* conv_state_out, int32_t form, void* workspace, size_t workspace_bytes,
+                                  nvfp4_stream_t stream, void* const* events) {
     nvfp4_status s = validate_layer(w, B, T);
     if (s != NVFP4_OK) return s;
     if (!x_bf16 || !y) return fail(NVFP4_ERR_INVALID_ARG, "x / y null");
@@ -123,6 +128,11 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return fail(NVFP4_ERR_WORKSPACE, "layer workspace missing, too small or not 256-byte aligned");
     cudaStream_t st = as_stream(stream);
+    auto mark = [&](int i) -> nvfp4_status {
+        if (!events) return NVFP4_OK;
+        const cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+        return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "stage event record");
+    };
     char* ws = static_cast<char*>(workspace);
     const gdn_dims& d = w->dims;
     const int64_t BT = static_cast<int64_t>(B) * T, H = w->hidden, HvV = static_cast<int64_t>(d.Hv) * d.V;
@@ -140,10 +150,13 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     // quantiser words: [0] x amax, [1] x arrival counter, [2] o amax, [3] gated-o amax,
     // zeroed by one small kernel (it chains with its neighbours by programmatic launch)
     unsigned int* qw = reinterpret_cast<unsigned int*>(ws + L.quant_ws);
+    if ((s = mark(0)) != NVFP4_OK) return s;
     if ((s = zero_words_launch(qw, 4, st)) != NVFP4_OK) return s;
     if ((s = quantize_launch(x_bf16, NVFP4_DTYPE_BF16, BT, H, H, xq, kQuantComputeZeroedWs, qw, st)) != NVFP4_OK)
         return s;
+    if ((s = mark(1)) != NVFP4_OK) return s;
     if ((s = gemm_launch(xq, w->w_in, proj, ldp, st)) != NVFP4_OK) return s;
+    if ((s = mark(2)) != NVFP4_OK) return s;
     // q|k|v come from the projection, or from its short convolution when one is set
     const float* qkv = proj;
     int64_t ld_qkv = ldp;
@@ -167,10 +180,12 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     // the scan folds max|o| into the quantiser's amax word as it writes o, so the o
     // quantiser runs its quantisation pass only
     unsigned int* o_amax = qw + 2;
+    if ((s = mark(3)) != NVFP4_OK) return s;
     if ((s = scan_launch(q_in, k_in, qkv + 2ll * d.Hk * d.K, ld_qkv, g, beta, B, T, d, scale, form,
                          chunked ? GDN_SCAN_CHUNKED : GDN_SCAN_RECURRENT, state_in, state_out, o, ws + L.scan_ws, st,
                          o_amax, ld_qk, 1)) != NVFP4_OK)
         return s;
+    if ((s = mark(4)) != NVFP4_OK) return s;
     const float* oq_in = o;
     unsigned int* oq_amax = o_amax;
     if (w->out_norm) {
@@ -183,5 +198,29 @@ extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, c
     }
     if ((s = quantize_launch(oq_in, NVFP4_DTYPE_FP32, BT, HvV, HvV, oq, kQuantFromAmax, oq_amax, st)) != NVFP4_OK)
         return s;
-    return gemm_launch(oq, w->w_out, y, H, st);
+    if ((s = mark(5)) != NVFP4_OK) return s;
+    if ((s = gemm_launch(oq, w->w_out, y, H, st)) != NVFP4_OK) return s;
+    return mark(6);
+}
+}  // namespace nvg
+
+extern "C" nvfp4_status gdn_layer_forward_stateful(const gdn_layer_weights* w, const void* x_bf16, int32_t B,
+                                                   int64_t T, float* y, const float* state_in, float* state_out,
+                                                   const float* conv_state_in, float* conv_state_out, int32_t form,
+                                                   void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+    return nvg::layer_forward(w, x_bf16, B, T, y, state_in, state_out, conv_state_in, conv_state_out, form,
+                              workspace, workspace_bytes, stream, nullptr);
+}
+
+extern "C" nvfp4_status gdn_layer_forward_timed(const gdn_layer_weights* w, const void* x_bf16, int32_t B,
+                                                int64_t T, float* y, const float* state_in, float* state_out,
+                                                const float* conv_state_in, float* conv_state_out, int32_t form,
+                                                void* workspace, size_t workspace_bytes, nvfp4_stream_t stream,
+                                                void* const* events) {
+    using namespace nvg;
+    if (!events) return fail(NVFP4_ERR_INVALID_ARG, "events is null");
+    for (int i = 0; i < kLayerEvents; ++i)
+        if (!events[i]) return fail(NVFP4_ERR_INVALID_ARG, "event handle is null");
+    return layer_forward(w, x_bf16, B, T, y, state_in, state_out, conv_state_in, conv_state_out, form, workspace,
+                         workspace_bytes, stream, events);
 }

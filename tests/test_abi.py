@@ -154,6 +154,14 @@ def test_layer_layout_and_validation():
     assert st == 6
     st, _ = _err(L.gdn_layer_forward(ctypes.byref(lw), FAKE, 1, 4096, FAKE, None, None, 3, FAKE, 1 << 40, None))
     assert st == 1
+    # the timed variant checks its seven event handles before anything else
+    st, msg = _err(L.gdn_layer_forward_timed(ctypes.byref(lw), FAKE, 1, 4096, FAKE, None, None, None, None, 0, FAKE,
+                                             1 << 40, None, None))
+    assert st == 1 and "events" in msg
+    handles = (ctypes.c_void_p * 7)(*([FAKE] * 6 + [None]))
+    st, msg = _err(L.gdn_layer_forward_timed(ctypes.byref(lw), FAKE, 1, 4096, FAKE, None, None, None, None, 0, FAKE,
+                                             1 << 40, None, handles))
+    assert st == 1 and "event" in msg
     del w_in
 
 

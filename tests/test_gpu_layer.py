@@ -182,3 +182,25 @@ def test_o_quantised_from_the_producer_amax_full_size(cuda_dev):
     torch.cuda.synchronize()
     nv.check_device_error()
     _check_o_quantised_exactly(ws, lay, B * T, sh.Hv * sh.V)
+
+
+@pytest.mark.parametrize("B,T", [(2, 100), (3, 1)])
+def test_timed_layer_forward_is_the_same_launches(cuda_dev, B, T):
+    """gdn_layer_forward_timed (the bench's per-stage timing) runs the same
+    launches as gdn_layer_forward: y and the state are bit-identical, and the
+    six stage intervals are ordered and add up to the recorded span."""
+    sh = gdn_synth.TINY
+    bits, _ = gdn_synth.activations(11, B * T, sh.H, hot="percent")
+    w, _ = _make_layer(sh, 11)
+    S0 = f32_device(gdn_synth.gaussian(12, (B, sh.Hv, sh.K, sh.V), std=0.5))
+    x = bf16_device(bits)
+    S1, S2 = torch.empty_like(S0), torch.empty_like(S0)
+    y1, _, _ = nv.gdn_layer_forward(w, x, B, T, state_in=S0, state_out=S1)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    y2, _, _ = nv.gdn_layer_forward(w, x, B, T, state_in=S0, state_out=S2, events=evs)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    assert torch.equal(y1, y2) and torch.equal(S1, S2)
+    parts = [evs[i].elapsed_time(evs[i + 1]) for i in range(6)]
+    assert all(p >= 0.0 for p in parts)
+    assert abs(sum(parts) - evs[0].elapsed_time(evs[6])) <= 1e-3 * max(1.0, sum(parts))
