@@ -256,7 +256,7 @@ def time_prefill(nv, w, sh, dev, B, T, steps, warmup, flush, stream, seed):
     torch.cuda.synchronize()
     nv.check_device_error()
     names = ["quant_x", "gemm_in", "gates", "scan", "quant_o", "gemm_out"]
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
+    stage_ms = {n: statistics.median(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps))
                 for j, n in enumerate(names)}
     return dict(x=x, y=y, ws=ws, lay=lay, step_ms=step_ms, stage_ms=stage_ms, names=names)
 

@@ -108,6 +108,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// base advanced to the next 1024-byte boundary of the shared window, as pointer
+// arithmetic on the shared array itself: a round trip through an integer would hide
+// the shared address space from the compiler and turn every access through the
+// result into a generic one (wider addresses, more registers).
+__device__ __forceinline__ uint8_t* align1024_shared(uint8_t* base) {
+    return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 // 16-byte asynchronous copy global -> shared; with valid == false nothing is
 // read and the destination is zero-filled (src must still be a valid address).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(320, 1)
                      const float* __restrict__ scaleB, int M, int N, int K, unsigned int* __restrict__ err) {
     using G = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = align1024_shared(smem_raw);
     uint8_t* sA = smem;
     uint8_t* sB = sA + G::STAGES * G::A_BYTES;
     uint8_t* sSFA = sB + G::STAGES * G::B_BYTES;
@@ -379,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
                           const float* __restrict__ scaleB, int M, int N, int K, unsigned int* __restrict__ err) {
     using G = CfgPair;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = align1024_shared(smem_raw);
     uint8_t* sA = smem;
     uint8_t* sB = sA + G::STAGES * G::A_BYTES;
     uint8_t* sSFA = sB + G::STAGES * G::B_BYTES;

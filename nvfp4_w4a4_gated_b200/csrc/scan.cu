@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1) chunk_seq_kernel(const uint8_t
     using L = SeqLayout<K>;
     using RC = ChunkRec<K, V>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = align1024_shared(smem_raw);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + kNumSeqBars);
     constexpr int NSL = V / 32;

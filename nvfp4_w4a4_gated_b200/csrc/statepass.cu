@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(512, 1) scan_correct_tc_kernel(const float* __
     constexpr int CPT = kTcTok * K / 4 / NT;        // 16-byte chunks of A per thread
     constexpr int COLS = V / 4;                     // columns per warp
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = align1024_shared(smem_raw);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::BAR + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
