@@ -184,14 +184,21 @@ def test_o_quantised_from_the_producer_amax_full_size(cuda_dev):
     _check_o_quantised_exactly(ws, lay, B * T, sh.Hv * sh.V)
 
 
-@pytest.mark.parametrize("B,T", [(2, 100), (3, 1)])
-def test_timed_layer_forward_is_the_same_launches(cuda_dev, B, T):
+@pytest.mark.parametrize("B,T,block", [(2, 100, False), (3, 1, False), (2, 100, True)])
+def test_timed_layer_forward_is_the_same_launches(cuda_dev, B, T, block):
     """gdn_layer_forward_timed (the bench's per-stage timing) runs the same
     launches as gdn_layer_forward: y and the state are bit-identical, and the
-    six stage intervals are ordered and add up to the recorded span."""
+    six stage intervals are ordered and add up to the recorded span.  With
+    block=True the optional output gate and short convolution are on too (they
+    fall inside the gates and quantise-o stages)."""
     sh = gdn_synth.TINY
     bits, _ = gdn_synth.activations(11, B * T, sh.H, hot="percent")
     w, _ = _make_layer(sh, 11)
+    if block:
+        C = 2 * sh.Hk * sh.K + sh.Hv * sh.V
+        w.out_norm = f32_device(1.0 + 0.1 * gdn_synth.gaussian(13, (sh.V,)))
+        w.conv_weight = f32_device(0.5 * gdn_synth.gaussian(14, (C, 4)))
+        w.conv_width = 4
     S0 = f32_device(gdn_synth.gaussian(12, (B, sh.Hv, sh.K, sh.V), std=0.5))
     x = bf16_device(bits)
     S1, S2 = torch.empty_like(S0), torch.empty_like(S0)
