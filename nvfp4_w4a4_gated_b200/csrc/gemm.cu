@@ -121,6 +121,21 @@ __global__ void __launch_bounds__(320, 1)
     const int kb_total = K / 64;                 // 64-wide k-blocks = scale atoms along K
     const int num_kt = (kb_total + 3) / 4;       // 256-wide k-tiles
     const int sfb_row_blocks = (N + 127) / 128;
+    // Tile order: the smaller operand stays in L2 while the larger one streams once.
+    // With M > N (the layer's long prefills: A of 32768 x 5120 against a weight of
+    // 12352 x 5120) the n tiles of one m run back to back, so each A tile is read
+    // while it is hot and the weight is the operand that is reused; otherwise the m
+    // tiles of one n do.
+    const bool n_fast = M > N;
+    auto tile_mn = [&](int tile, int& m_idx, int& n_idx) {
+        if (n_fast) {
+            m_idx = tile / num_n;
+            n_idx = tile - m_idx * num_n;
+        } else {
+            n_idx = tile / num_m;
+            m_idx = tile - n_idx * num_m;
+        }
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < G::STAGES; ++s) {
@@ -152,7 +167,8 @@ __global__ void __launch_bounds__(320, 1)
             // ---------------------------------------------------- producer --
             uint32_t stage = 0, phase = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-                const int m_idx = tile % num_m, n_idx = tile / num_m;
+                int m_idx, n_idx;
+                tile_mn(tile, m_idx, n_idx);
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, err, kErrTimeoutTma)) goto producer_done;
                     const int nkb = min(4, kb_total - kt * 4);
@@ -291,7 +307,8 @@ __global__ void __launch_bounds__(320, 1)
         float* stg = sStage + (warp - 2) * 2 * 32 * 32;
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            const int m_idx = tile % num_m, n_idx = tile / num_m;
+            int m_idx, n_idx;
+            tile_mn(tile, m_idx, n_idx);
             const int buf = local & 1;
             if (!mbar_wait(acc_full, local & 1, err, kErrTimeoutEpi)) break;
             tc_fence_after();
