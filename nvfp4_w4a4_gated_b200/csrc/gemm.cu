@@ -305,6 +305,9 @@ __global__ void __launch_bounds__(320, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const float alpha = __fmul_rn(*scaleA, *scaleB);
         float* stg = sStage + (warp - 2) * 2 * 32 * 32;
+        // C is a stream that no later tile reads: its lines leave L2 first, so the
+        // operand that is reused keeps its place
+        const uint64_t c_policy = l2_policy_evict_first();
         int local = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int m_idx, n_idx;
@@ -327,7 +330,7 @@ __global__ void __launch_bounds__(320, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 const int col0 = n_idx * BN + chunk_col(ci) * 32;
-                if (lane == 0 && row0 < M && col0 < N) tma_store_2d(&tmC, tile, col0, row0);
+                if (lane == 0 && row0 < M && col0 < N) tma_store_2d_hint(&tmC, tile, col0, row0, c_policy);
                 if (lane == 0) bulk_commit();
             };
             // the chunks the next tile's accumulator reuses go to registers first, so the
