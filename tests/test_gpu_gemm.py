@@ -54,6 +54,8 @@ def _run(Aq, Bq, M, N, K, ldc=None):
     (384, 768, 1024),     # several tiles in both dimensions
     (1, 64, 64),          # smallest legal problem
     (1000, 1536, 640),    # many tiles per CTA
+    (1000, 520, 256),     # M > N: the n tiles of one m tile run back to back; ragged in both
+    (640, 384, 512),      # M > N, whole tiles
 ])
 def test_gemm_matches_oracle(cuda_dev, variant, M, N, K):
     Aq, Bq = _operands(M + N + K, M, N, K)

@@ -147,6 +147,37 @@ def test_full_size_prefill_layer_stage_checks(cuda_dev):
     assert torch.isfinite(y).all() and torch.isfinite(S_out).all()
 
 
+def test_prefill_T32768_projections_sampled_rows(cuda_dev):
+    """The T = 32768 layer prefill as the benchmark runs it (one call).  Both GEMMs
+    have M > N there, so the n tiles of one m tile run back to back.  On sampled
+    rows: x codes bit-exact; P against the float64 product of the oracle-quantised
+    operands; y against the oracle's product of the GPU's o, quantised under the
+    GPU's o scale, with W_out (the o codes themselves are checked bit for bit by
+    the o-quantiser tests)."""
+    sh, B, T = gdn_synth.FULL, 1, 32768
+    bits, x = gdn_synth.activations(3, B * T, sh.H, hot="percent")
+    w, (W_in, W_out, _, _) = _make_layer(sh, 3)
+    y, ws, lay = nv.gdn_layer_forward(w, bf16_device(bits), B, T)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    BT, H, n_in, HvV = B * T, sh.H, sh.n_in, sh.Hv * sh.V
+    ldp = (n_in + 3) // 4 * 4
+    rows = np.unique(np.concatenate([np.arange(4), gdn_synth.rng(9).integers(0, BT, 24), np.arange(BT - 4, BT)]))
+    rows_t = torch.from_numpy(rows).cuda()
+    xq = oracle.quantize(x)
+    xc = _view(ws, lay["x_codes"], BT * H // 2, torch.uint8).view(BT, H // 2)[rows_t].cpu().numpy()
+    assert np.array_equal(xc, xq[0][rows])
+    ref_P = oracle.gemm_nt(oracle.dequantize(xq[0][rows], xq[1][rows], xq[2]), oracle.dequantize(*oracle.quantize(W_in)))
+    P = _view(ws, lay["proj"], BT * ldp * 4, torch.float32).view(BT, ldp)[rows_t, :n_in].cpu().numpy()
+    assert rel_fro(P, ref_P) <= 1e-3
+    o = _view(ws, lay["o"], BT * HvV * 4, torch.float32).view(BT, HvV)[rows_t].cpu().numpy()
+    oS = float(_view(ws, lay["o_scale"], 4, torch.float32).cpu().numpy()[0])
+    ref_y = oracle.gemm_nt(oracle.dequantize(*oracle.quantize(o, S=oS)), oracle.dequantize(*oracle.quantize(W_out)))
+    got_y = y[rows_t].cpu().numpy()
+    assert rel_fro(got_y, ref_y) <= 1e-3
+    assert np.max(np.abs(got_y - ref_y)) <= 1e-3 * np.max(np.abs(ref_y))
+
+
 def _check_o_quantised_exactly(ws, lay, BT, HvV, o_field="o"):
     """The o quantiser in the layer takes its amax from the word the scan (or the
     output gate) filled, and runs only its quantisation pass.  Codes, block scales
