@@ -326,17 +326,6 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
     return d;
 }
 
-// Shared-memory descriptor of one 512-byte scale-factor atom (32 rows x 16
-// bytes, no swizzle, 8-row core matrices 128 bytes apart) for tcgen05.cp.
-__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(1u) << 16;
-    d |= static_cast<uint64_t>(128u >> 4) << 32;
-    d |= static_cast<uint64_t>(1u) << 46;
-    return d;
-}
-
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: E2M1 x E2M1, UE4M3
 // scales (one per 16 elements), both operands K-major, f32 accumulate.
 __host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
@@ -358,12 +347,6 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
-// Copy one 512-byte scale atom (32 rows x 128 bits) from shared memory to TMEM,
-// replicated to the four 32-lane sub-partitions (4 TMEM columns).
-__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 // Pair MMA issued by the even CTA: each CTA supplies its own A rows and half of
 // the B rows from its shared memory; D, and the scale factors, sit in each CTA's TMEM.
 __device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -375,10 +358,6 @@ __device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, u
         "}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
-}
-// Pair scale-atom copy: each CTA's shared memory at this offset -> its own TMEM.
-__device__ __forceinline__ void tmem_cp_sf_atom_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 // Arrive on one mbarrier (possibly in the peer CTA) when this thread's prior pair ops complete.
 __device__ __forceinline__ void mma_commit_pair(uint32_t cluster_addr) {

@@ -699,8 +699,8 @@ nvfp4_status validate_tensor(const nvfp4_tensor* t, const char* name);
 // Kernel choice.  NVFP4_GEMM_VARIANT=pair|single|narrow forces one (tests
 // cover each); by default the single-CTA 128 x 256 kernel takes problems with
 // at least one tile per SM and the 128 x 128 kernel smaller / decode shapes.
-// The CTA-pair kernel (which still moves scales with tcgen05.cp) measured
-// slower and is only used on request.
+// The CTA-pair kernel measured slower (a cross-SM round trip per k-tile on its
+// two-slot scale ring) and is only used on request.
 static int gemm_variant_override() {
     const char* e = getenv("NVFP4_GEMM_VARIANT");
     if (e && !strcmp(e, "pair")) return 1;
