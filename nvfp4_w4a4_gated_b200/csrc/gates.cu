@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) l2norm_kernel(const float* __restrict__ p
     for (int i = 0; i < PER_LANE; ++i) ss = fmaf(v[i], v[i], ss);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = 1.0f / sqrtf(ss + 1e-6f);
+    const float inv = rsqrtf(ss + 1e-6f);
     float* dst = (which == 0 ? q_hat : k_hat) + th * D + lane * PER_LANE;
     if constexpr (PER_LANE == 4) {
         *reinterpret_cast<float4*>(dst) = make_float4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(128) scan_recurrent_kernel(
                 for (int i = lane; i < K; i += 32) ss = fmaf(src[i], src[i], ss);
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                if (lane == 0) inv_norm[w] = 1.0f / sqrtf(ss + 1e-6f);
+                if (lane == 0) inv_norm[w] = rsqrtf(ss + 1e-6f);
             }
             __syncthreads();
             if (threadIdx.x < K) {
@@ -167,6 +167,17 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Four 8 x 4 float32 matrices from shared memory, one 16-byte row address per
+// lane (lanes 8i..8i+7 give the rows of matrix i).  Register i of lane l then
+// holds element (l / 4, l % 4) of matrix i: with the matrices chosen as below this
+// is a TF32 m16n8k8 A fragment (rows +0..7 | +8..15 x columns +0..3 | +4..7), or
+// the B fragments of two 8-column tiles.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const float* p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(p)));
+}
+
 // ------------------------------------------------------ chunk preparation --
 // One CTA (256 threads) per (sequence, chunk, value head).
 template <int K, int V>
@@ -195,11 +206,11 @@ struct PrepSmem {
 // Float offset of element (r, c) of a K, Q or V tile with row stride KS (a
 // multiple of 32).  Bits 2..4 of the column are XORed with ((r & 3) << 3) | (r & 4),
 // which permutes the 4-float groups inside each 32-float segment of a row.  Every
-// access pattern of the tiles is then free of bank conflicts: the TF32 mma.sync A
-// and B fragments read with k along a row (rows grp, columns tig), the B
-// fragments read with k down the columns (rows tig, columns grp), the float2
-// accumulator accesses, and row-contiguous vector accesses.  Aligned 2- and
-// 4-float vectors stay contiguous.
+// access pattern of the tiles is then free of bank conflicts: the ldmatrix reads of
+// TF32 mma.sync fragments with k along a row (eight 16-byte row pieces of eight
+// consecutive rows), the B fragments read with k down the columns (rows tig,
+// columns grp), the float2 accumulator accesses, and row-contiguous vector
+// accesses.  Aligned 2- and 4-float vectors stay contiguous.
 template <int KS>
 __device__ __forceinline__ int tile_off(int r, int c) {
     static_assert(KS % 32 == 0, "tile stride must be a multiple of 32 floats");
@@ -211,6 +222,8 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
                                             const float* __restrict__ s, float* __restrict__ X, int c0, int lane,
                                             Store store) {
     const int grp = lane >> 2, tig = lane & 3;
+    // row and column of this lane's ldmatrix address inside a 16 x 8 A fragment
+    const int fr = (lane & 7) + ((lane >> 3) & 1) * 8, fc = (lane >> 4) * 4;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
         const int r0 = 16 * b;
@@ -228,10 +241,8 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
         }
 #pragma unroll
         for (int k0 = 0; k0 < r0; k0 += 8) {
-            const uint32_t a[4] = {__float_as_uint(Lm[(r0 + grp) * LS + k0 + tig]),
-                                   __float_as_uint(Lm[(r0 + grp + 8) * LS + k0 + tig]),
-                                   __float_as_uint(Lm[(r0 + grp) * LS + k0 + tig + 4]),
-                                   __float_as_uint(Lm[(r0 + grp + 8) * LS + k0 + tig + 4])};
+            uint32_t a[4];
+            ldsm_x4(a, &Lm[(r0 + fr) * LS + k0 + fc]);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const uint32_t bb[2] = {__float_as_uint(X[tile_off<KS>(k0 + tig, c0 + nt * 8 + grp)]),
@@ -255,9 +266,8 @@ __device__ __forceinline__ void block_subst(const float* __restrict__ Lm, const 
         const float* Tbb = Tb + b * 16 * TBS;
 #pragma unroll
         for (int k0 = 0; k0 < 16; k0 += 8) {
-            const uint32_t a[4] = {__float_as_uint(Tbb[grp * TBS + k0 + tig]), __float_as_uint(Tbb[(grp + 8) * TBS + k0 + tig]),
-                                   __float_as_uint(Tbb[grp * TBS + k0 + tig + 4]),
-                                   __float_as_uint(Tbb[(grp + 8) * TBS + k0 + tig + 4])};
+            uint32_t a[4];
+            ldsm_x4(a, &Tbb[fr * TBS + k0 + fc]);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const uint32_t bb[2] = {__float_as_uint(X[tile_off<KS>(r0 + k0 + tig, c0 + nt * 8 + grp)]),
@@ -304,13 +314,19 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
 
     // K, Q rows (zero past the end of the sequence) by asynchronous copies, g and beta;
     // token t's head hk row starts at (b T + t) ld_qk + hk K
-    constexpr int V4 = K / 4;
-    for (int idx = tid; idx < CH * V4; idx += 256) {
-        const int r = idx / V4, c4 = idx - r * V4;
-        const bool valid = r < n;
-        const int64_t off = valid ? (static_cast<int64_t>(b) * T + t0 + r) * ld_qk + static_cast<int64_t>(hk) * K + c4 * 4 : 0;
-        cp_async16(&sm.ks[tile_off<KS>(r, c4 * 4)], k + off, valid);
-        cp_async16(&sm.qs[tile_off<KS>(r, c4 * 4)], q + off, valid);
+    {
+        // each thread copies one 16-byte column piece of every RS-th row
+        constexpr int V4 = K / 4, RS = 256 / V4;
+        const int c4 = tid % V4, r0 = tid / V4;
+        const int64_t step = static_cast<int64_t>(RS) * ld_qk;
+        int64_t off = (static_cast<int64_t>(b) * T + t0 + r0) * ld_qk + static_cast<int64_t>(hk) * K + c4 * 4;
+#pragma unroll
+        for (int r = r0; r < CH; r += RS, off += step) {
+            const bool valid = r < n;
+            const int so = tile_off<KS>(r, c4 * 4);
+            cp_async16(&sm.ks[so], k + (valid ? off : 0), valid);
+            cp_async16(&sm.qs[so], q + (valid ? off : 0), valid);
+        }
     }
     cp_async_commit();
     if (tid < CH) {
@@ -342,7 +358,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
                 for (int i = 0; i < PL; ++i) ss = fmaf(vv[i], vv[i], ss);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                inv = 1.0f / sqrtf(ss + 1e-6f);
+                inv = rsqrtf(ss + 1e-6f);
             }
 #pragma unroll
             for (int i = 0; i < PL; ++i) vv[i] = __uint_as_float(to_tf32(normalize_qk ? vv[i] * inv : vv[i]));
@@ -384,22 +400,27 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
         const int grp = lane >> 2, tig = lane & 3;
         const float* A = warp < 4 ? sm.ks : sm.qs;
         const int r0 = (warp & 3) * 16;
+        // tiles right of this warp's diagonal block are skipped (masked out afterwards):
+        // it takes 8-column tiles 0 .. r0/8 + 1, two per B load
+        const int npairs = (r0 >> 4) + 1;
+        // ldmatrix addresses: A rows r0 + ar, columns + ac; B rows 16 np + br, columns + bc
+        const int ar = r0 + (lane & 7) + ((lane >> 3) & 1) * 8, ac = (lane >> 4) * 4;
+        const int br = (lane & 7) + (lane >> 4) * 8, bc = ((lane >> 3) & 1) * 4;
         float acc[8][4];
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll 4
         for (int k0 = 0; k0 < K; k0 += 8) {
-            const float a[4] = {A[tile_off<KS>(r0 + grp, k0 + tig)], A[tile_off<KS>(r0 + grp + 8, k0 + tig)],
-                                A[tile_off<KS>(r0 + grp, k0 + tig + 4)], A[tile_off<KS>(r0 + grp + 8, k0 + tig + 4)]};
-            const uint32_t ai[4] = {__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
-                                    __float_as_uint(a[3])};
+            uint32_t ai[4];
+            ldsm_x4(ai, &A[tile_off<KS>(ar, k0 + ac)]);
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                // tiles right of this warp's diagonal block are masked out afterwards
-                if (nt * 8 > r0 + 15) continue;
-                const uint32_t bb[2] = {__float_as_uint(sm.ks[tile_off<KS>(nt * 8 + grp, k0 + tig)]),
-                                        __float_as_uint(sm.ks[tile_off<KS>(nt * 8 + grp, k0 + tig + 4)])};
-                mma_tf32(acc[nt], ai, bb);
+            for (int np = 0; np < 4; ++np) {
+                if (np >= npairs) continue;
+                uint32_t bq[4];
+                ldsm_x4(bq, &sm.ks[tile_off<KS>(16 * np + br, k0 + bc)]);
+                const uint32_t b0[2] = {bq[0], bq[1]}, b1[2] = {bq[2], bq[3]};
+                mma_tf32(acc[2 * np], ai, b0);
+                mma_tf32(acc[2 * np + 1], ai, b1);
             }
         }
 #pragma unroll
@@ -445,12 +466,16 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const float* __restrict
     __syncthreads();
     // Q is no longer needed: its tile now receives the V rows (zero past the sequence
     // end); the copies land while the diagonal blocks are inverted
-    constexpr int VV4 = V / 4;
-    for (int idx = tid; idx < CH * VV4; idx += 256) {
-        const int r = idx / VV4, c4 = idx - r * VV4;
-        const bool valid = r < n;
-        const int64_t off = valid ? (static_cast<int64_t>(b) * T + t0 + r) * ld_v + static_cast<int64_t>(h) * V + c4 * 4 : 0;
-        cp_async16(&sm.qs[tile_off<KS>(r, c4 * 4)], v + off, valid);
+    {
+        constexpr int VV4 = V / 4, RS = 256 / VV4;
+        const int c4 = tid % VV4, r0 = tid / VV4;
+        const int64_t step = static_cast<int64_t>(RS) * ld_v;
+        int64_t off = (static_cast<int64_t>(b) * T + t0 + r0) * ld_v + static_cast<int64_t>(h) * V + c4 * 4;
+#pragma unroll
+        for (int r = r0; r < CH; r += RS, off += step) {
+            const bool valid = r < n;
+            cp_async16(&sm.qs[tile_off<KS>(r, c4 * 4)], v + (valid ? off : 0), valid);
+        }
     }
     cp_async_commit();
 
