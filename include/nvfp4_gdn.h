@@ -161,7 +161,8 @@ NVFP4_API nvfp4_status w4a4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* B, f
 /* Gates, Eq.(1) (review page, paper sec.2), and per-head q/k L2 normalisation:
  *   proj: device float32 [n_tokens x ld_proj], the fused projection with
  *         column slices q [Hk*K] | k [Hk*K] | v [Hv*V] | z [Hv*V] | a [Hv] | b [Hv].
- *   q_hat, k_hat: device float32 [n_tokens x Hk x K]: x / sqrt(sum x^2 + 1e-6).
+ *   q_hat, k_hat: device float32 [n_tokens x Hk x K]: x / sqrt(sum x^2 + 1e-6), computed
+ *         as x * rsqrtf(sum x^2 + 1e-6) (the same in the scans' own normalisation).
  *   g:     device float32 [n_tokens x Hv]: -exp(A_log[h]) * softplus(a + dt_bias[h])
  *          (log of the decay alpha), softplus(u) = max(u,0) + log1p(exp(-|u|)).
  *   beta:  device float32 [n_tokens x Hv]: 1 / (1 + exp(-b)).
