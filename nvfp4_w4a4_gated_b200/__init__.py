@@ -449,7 +449,7 @@ def gdn_layer_forward(w: LayerWeights, x: torch.Tensor, B: int, T: int, y=None, 
         handles = (ctypes.c_void_p * 7)(*[ev.cuda_event for ev in events])
         _check(lib().gdn_layer_forward_timed(ctypes.byref(lw), _ptr(x), B, T, _ptr(y), _ptr(state_in),
                                              _ptr(state_out), _ptr(conv_state_in), _ptr(conv_state_out), form,
-                                             _ptr(workspace), workspace.numel(), _stream(stream), handles))
+                                             _ptr(workspace), workspace.numel(), _stream(st), handles))
         return y, workspace, lay
     _check(lib().gdn_layer_forward_stateful(ctypes.byref(lw), _ptr(x), B, T, _ptr(y), _ptr(state_in), _ptr(state_out),
                                             _ptr(conv_state_in), _ptr(conv_state_out), form, _ptr(workspace),
