@@ -1,6 +1,7 @@
 // api.cu -- status plumbing, device error word, TMA descriptor encoding.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -40,16 +41,19 @@ unsigned int* device_error_word() {
 }
 
 int num_sms() {
-    static int cached[64] = {0};
+    // per device; threads may race to fill a slot, and all store the same value
+    static std::atomic<int> cached[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
+    int v = cached[dev].load(std::memory_order_relaxed);
+    if (!v) {
         int n = 0;
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 148;
+        v = n > 0 ? n : 148;
+        cached[dev].store(v, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return v;
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

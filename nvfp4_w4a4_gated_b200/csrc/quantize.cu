@@ -11,6 +11,7 @@
 // in reverse order (their data still in L2), one thread per four 16-element
 // blocks, the scale bytes of an atom stored as four coalesced 128-byte rows.
 // If the grid cannot be co-resident, a separate amax launch runs first.
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include <type_traits>
@@ -386,16 +387,19 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const T* __restric
 
 template <typename T, bool kFindAmax>
 int quant_blocks_per_sm() {
-    static int cached = 0;
-    if (!cached) {
+    // threads may race to fill it, and all store the same value
+    static std::atomic<int> cached{0};
+    int v = cached.load(std::memory_order_relaxed);
+    if (!v) {
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, quant_kernel<T, kFindAmax>, kQuantThreads, 0) !=
                 cudaSuccess ||
             n < 1)
             n = 1;
-        cached = n;
+        v = n;
+        cached.store(v, std::memory_order_relaxed);
     }
-    return cached;
+    return v;
 }
 
 template <typename T>
